@@ -1,0 +1,205 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) forward pass of a Mixture-of-Experts FFN layer.
+ *
+ * The layer (notation of "Основы MoE", section "Как устроен MoE-слой", steps 1-4, and of
+ * the "Mixture-of-Experts : routage et capacité" slides):
+ *
+ *   z   = x . W_g                                  router projection, fp32 logits  [N][E]
+ *   key = z + b            (softmax scoring)       selection keys; b is a per-expert,
+ *       = sigma(z) + b     (sigmoid scoring)       selection-only bias, one set per modality
+ *   T   = the k largest keys, descending, ties to the lower expert index
+ *   g_i = softmax over the selected unbiased z     (softmax, renorm = 1)
+ *       = p_i of the full softmax                  (softmax, renorm = 0: Switch k = 1)
+ *       = s_i / sum_{j in T} s_j                   (sigmoid, renorm = 1)
+ *   capacity C: the assignments to one expert are served in token order, the first C
+ *       are kept, the others dropped (a dropped slot contributes 0; the kept gates are
+ *       not renormalised)
+ *   y_t = sum_{kept i in T} g_i FFN_i(x_t) + FFN_shared(x_t)
+ *   FFN = (SiLU(x W_gate) * (x W_up)) W_down   with an optional clamp of both
+ *         pre-activations to [-clamp, clamp] ("SwiGLU, écrêtée à 10"), or
+ *         max(x W1, 0) W2 (the two-layer ReLU expert of the dataistudio listing).
+ *
+ * Conventions shared by every entry point:
+ *  - All array pointers are caller-owned DEVICE memory unless a parameter says "host".
+ *    The library never allocates device memory; scratch comes from the caller's workspace
+ *    (moe_workspace_size bytes, 256-byte aligned, prepared once by moe_workspace_init).
+ *  - Row-major everywhere.  Weights are stored out-major / K-contiguous (nn.Linear style):
+ *      W_g    [E][d]                      (the math d x E matrix, transposed)
+ *      W_gu   [E+S][2F][d]  SwiGLU        rows [0,F) = W_gate, rows [F,2F) = W_up
+ *             [E+S][F][d]   ReLU          W1
+ *      W_down [E+S][d][F]
+ *    S = n_shared (0 or 1); the shared expert is stored last, at index E.
+ *  - Element types: dtype MOE_DT_BF16 means x, weights, xp, ye and y are bf16 (fp32
+ *    accumulation); MOE_DT_F32 means they are all fp32.  Logits, gates and biases are
+ *    always fp32; ids, counts, offsets, rows are int32; masks and modality flags uint8.
+ *  - Row layout of the per-expert buffers: routed rows of expert e occupy
+ *    [offsets[e], offsets[e+1]) (offsets[E] = M, the kept assignments, M <= N*k); the
+ *    shared expert's row for token t is N*k + t.  So xp has N*k rows, ye has N*k + S*N.
+ *  - Every call is asynchronous and stream-ordered on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).  No call synchronises the host, except
+ *    moe_check_status and moe_forward_host.
+ *  - Errors: host-side checks return a status before anything is enqueued.  Device-side
+ *    findings (bad ids or modality flags, a bounded wait that ran out) are recorded in
+ *    the workspace status word and reported by moe_check_status.  No device code traps.
+ *  - Thread safety: calls on different workspaces may run concurrently; calls sharing a
+ *    workspace must be ordered on one stream.  moe_last_error() is per thread.
+ */
+#ifndef MOE_B200_MOE_H_
+#define MOE_B200_MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* a host-checked argument is wrong; nothing was enqueued */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid request outside what this build implements
+                                (alignment, d or F not a multiple of 8, k > 32, ...) */
+  MOE_ERR_CUDA = 3,          /* a CUDA call or launch failed; see moe_last_error() */
+  MOE_ERR_INVALID_INPUT = 4, /* device-detected: expert id out of range or repeated in a
+                                token, modality flag >= n_bias_sets */
+  MOE_ERR_TIMEOUT = 5        /* device-detected: a bounded wait inside a kernel ran out */
+} moe_status;
+
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_fn;
+typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_RELU = 1 } moe_act;
+typedef enum { MOE_DT_BF16 = 0, MOE_DT_F32 = 1 } moe_dtype;
+
+/* Shapes and options of one layer call. */
+typedef struct {
+  int64_t N;           /* tokens in this call (0 is allowed: every call is a no-op) */
+  int32_t d;           /* model dimension */
+  int32_t E;           /* routed experts, 1..1024 */
+  int32_t k;           /* experts per token, 1..min(E, 32) */
+  int32_t F;           /* hidden dimension of every expert (routed and shared) */
+  int32_t n_shared;    /* always-on shared experts: 0 or 1 */
+  int32_t n_bias_sets; /* 0: no selection bias; >= 1: bias is [n_bias_sets][E], token t
+                          uses set modality[t] (set 0 when modality is NULL) */
+  int32_t score_fn;    /* moe_score_fn */
+  int32_t renorm;      /* 1: gates renormalised over the selected experts; 0: raw score */
+  int32_t act;         /* moe_act */
+  int32_t dtype;       /* moe_dtype */
+  float clamp;         /* > 0: clamp gate and up pre-activations to [-clamp, clamp] */
+  int64_t capacity;    /* C; <= 0 means unlimited */
+} moe_config;
+
+/* Optional routing outputs of moe_forward; every member may be NULL. */
+typedef struct {
+  float* logits;       /* [N][E]  fp32 router logits (z, plus logit_offset) */
+  int32_t* ids;        /* [N][k]  selected experts, descending key */
+  float* gates;        /* [N][k]  gate weights (dropped slots keep their gate value) */
+  int32_t* counts;     /* [E]     kept assignments per expert */
+  int32_t* demand;     /* [E]     assignments per expert before capacity */
+  uint8_t* drop_mask;  /* [N][k]  1 = assignment dropped by capacity */
+  int32_t* offsets;    /* [E+1]   exclusive scan of counts */
+} moe_route_out;
+
+/* Bytes of device workspace a call with this configuration needs (0 on a bad config).
+ * The size depends on N, d, E, k, F, n_shared and dtype only. */
+MOE_API size_t moe_workspace_size(const moe_config* cfg);
+
+/* Zero the workspace header (the device status word).  Call once after allocating. */
+MOE_API moe_status moe_workspace_init(void* ws, moe_stream_t stream);
+
+/* Capacity C = ceil(T * k / E * f) with f = cf_num / cf_den, in exact integer
+ * arithmetic ("Mixture-of-Experts : routage et capacité", section "L'idée — Capacité").
+ * cf_num <= 0 means no limit and returns 0.  Returns -1 on a bad argument.  Host only. */
+MOE_API int64_t moe_capacity(int64_t T, int32_t k, int32_t E, int64_t cf_num, int64_t cf_den);
+
+/* Router and capacity ("Основы MoE", steps 1-3; slides, "L'idée — Capacité").
+ *   logits     [N][E] fp32 input, or NULL: then logits = x . W_g^T (+ logit_offset) are
+ *              computed on the tensor cores (bf16) or in fp32 (MOE_DT_F32)
+ *   x          [N][d], W_g [E][d]: read only when logits == NULL
+ *   logit_offset [E] fp32 or NULL: added to computed logits (enters selection AND gates)
+ *   bias       [n_bias_sets][E] fp32 or NULL (NULL iff n_bias_sets == 0)
+ *   modality   [N] uint8 or NULL (required when n_bias_sets > 1)
+ *   ids [N][k], gates [N][k], counts [E], demand [E], drop_mask [N][k]: outputs
+ *   logits_out [N][E] or NULL: where computed logits are written (else workspace)
+ * Ids, counts, demand and drop_mask are a deterministic function of the fp32 logits. */
+MOE_API moe_status moe_route(const moe_config* cfg, const float* logits, const void* x,
+                     const void* W_g, const float* logit_offset, const float* bias,
+                     const uint8_t* modality, int32_t* ids, float* gates, int32_t* counts,
+                     int32_t* demand, uint8_t* drop_mask, float* logits_out, void* ws,
+                     moe_stream_t stream);
+
+/* Permutation into per-expert contiguous groups (the per-expert gather of the
+ * "Эксперимент на PyTorch" MoE.forward, laid out as the slides' dispatch table).
+ *   ids [N][k] (values checked on the device), drop_mask [N][k] or NULL (none dropped)
+ *   x [N][d] input rows
+ *   offsets [E+1], row_token [N*k] (entries >= M are left untouched),
+ *   slot_row [N][k] (-1 = dropped), xp [N*k][d]: outputs.
+ * Within an expert, rows follow token order. */
+MOE_API moe_status moe_permute(const moe_config* cfg, const int32_t* ids, const uint8_t* drop_mask,
+                       const void* x, int32_t* offsets, int32_t* row_token,
+                       int32_t* slot_row, void* xp, void* ws, moe_stream_t stream);
+
+/* Expert FFNs over the groups: ye[r] = FFN_e(xp[r]) for r in [offsets[e], offsets[e+1]),
+ * and ye[N*k + t] = FFN_shared(x[t]) when n_shared == 1.
+ *   xp [N*k][d], offsets [E+1] (device), x [N][d] (read iff n_shared == 1)
+ *   W_gu, W_down as above; ye [N*k + S*N][d] output.  Rows of ye outside the groups are
+ *   left untouched.  bf16: tcgen05 grouped GEMMs, SwiGLU/ReLU fused in the epilogue,
+ *   hidden activations rounded to bf16 in the workspace. */
+MOE_API moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const int32_t* offsets,
+                          const void* x, const void* W_gu, const void* W_down, void* ye,
+                          void* ws, moe_stream_t stream);
+
+/* Gate-weighted combine back to token order ("Основы MoE", step 4):
+ *   y[t] = sum_{j: slot_row[t][j] >= 0} gates[t][j] ye[slot_row[t][j]]  (+ ye[N*k + t])
+ * summed in fp32 and rounded once.  y [N][d] output. */
+MOE_API moe_status moe_combine(const moe_config* cfg, const void* ye, const int32_t* slot_row,
+                       const float* gates, void* y, moe_stream_t stream);
+
+/* The whole layer: route, capacity, permute, expert FFNs (routed + shared), combine.
+ * Inputs as above; y [N][d] output; route_out may be NULL or have NULL members. */
+MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const void* W_g,
+                       const float* logit_offset, const float* bias,
+                       const uint8_t* modality, const void* W_gu, const void* W_down,
+                       void* y, const moe_route_out* route_out, void* ws,
+                       moe_stream_t stream);
+
+/* moe_forward with x_host and y_host in HOST memory (pinned for full copy speed): copies
+ * x to the workspace, runs the layer, copies y back and synchronises the stream.
+ * Weights, bias, modality and logit_offset are device pointers as in moe_forward. */
+MOE_API moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const void* W_g,
+                            const float* logit_offset, const float* bias,
+                            const uint8_t* modality, const void* W_gu, const void* W_down,
+                            void* y_host, void* ws, moe_stream_t stream);
+
+/* Synchronise `stream`, read and clear the workspace status word.  Returns MOE_OK or the
+ * first device-detected error (MOE_ERR_INVALID_INPUT, MOE_ERR_TIMEOUT) since the last
+ * check; MOE_ERR_CUDA if the stream reports an asynchronous CUDA error. */
+MOE_API moe_status moe_check_status(void* ws, moe_stream_t stream);
+
+/* Text of the last error raised on the calling thread ("" if none). */
+MOE_API const char* moe_last_error(void);
+
+/* Per-launch timing of moe_forward on the calling thread.  After moe_profile_begin(n), the
+ * next n calls of moe_forward / moe_forward_host record a CUDA event on their stream before
+ * their first kernel and after each kernel (the events carry timing; nothing else changes).
+ * moe_profile_end synchronises on the recorded events, writes into launch_ms[i] the total
+ * milliseconds of the i-th launch summed over the recorded calls (i < max_launches), stores
+ * the number of recorded calls in *calls, releases the events and returns the number of
+ * launches per call (or -1 on a CUDA error).  Launch order of a bf16 forward: router GEMM,
+ * top-k, rank pass, scan pass, scatter/gather pass, gate/up GEMM, down GEMM, combine. */
+MOE_API moe_status moe_profile_begin(int32_t max_calls);
+MOE_API int32_t moe_profile_end(float* launch_ms, int32_t max_launches, int32_t* calls);
+
+/* Number of kernel launches the last successful entry point on this thread enqueued. */
+MOE_API int32_t moe_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_MOE_H_ */

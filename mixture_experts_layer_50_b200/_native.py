@@ -1,0 +1,228 @@
+"""ctypes binding of ``libmoe_b200.so`` (the C ABI of include/moe.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.
+Functions keep the C names and take torch tensors (device memory) plus the current torch
+CUDA stream.  There is no fallback: if the library is missing, importing this module
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from fractions import Fraction
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmoe_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m mixture_experts_layer_50_b200.build` "
+        "(nvcc, sm_100a). There is no non-CUDA implementation of this layer.")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_INVALID_INPUT, \
+    MOE_ERR_TIMEOUT = range(6)
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+                3: "MOE_ERR_CUDA", 4: "MOE_ERR_INVALID_INPUT", 5: "MOE_ERR_TIMEOUT"}
+SOFTMAX, SIGMOID = 0, 1
+SWIGLU, RELU = 0, 1
+BF16, F32 = 0, 1
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.moe_last_error().decode("utf-8", "replace")
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}: {msg}")
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("F", ctypes.c_int32), ("n_shared", ctypes.c_int32),
+                ("n_bias_sets", ctypes.c_int32), ("score_fn", ctypes.c_int32),
+                ("renorm", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("clamp", ctypes.c_float), ("capacity", ctypes.c_int64)]
+
+
+class moe_route_out(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("logits", "ids", "gates", "counts", "demand", "drop_mask", "offsets")]
+
+
+_vp, _i32, _i64, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+_cfgp = ctypes.POINTER(moe_config)
+lib.moe_workspace_size.argtypes = [_cfgp]
+lib.moe_workspace_size.restype = _sz
+lib.moe_workspace_init.argtypes = [_vp, _vp]
+lib.moe_capacity.argtypes = [_i64, _i32, _i32, _i64, _i64]
+lib.moe_capacity.restype = _i64
+lib.moe_route.argtypes = [_cfgp] + [_vp] * 14
+lib.moe_permute.argtypes = [_cfgp] + [_vp] * 9
+lib.moe_expert_ffn.argtypes = [_cfgp] + [_vp] * 8
+lib.moe_combine.argtypes = [_cfgp] + [_vp] * 5
+lib.moe_forward.argtypes = [_cfgp] + [_vp] * 11
+lib.moe_forward_host.argtypes = [_cfgp] + [_vp] * 10
+lib.moe_check_status.argtypes = [_vp, _vp]
+lib.moe_profile_begin.argtypes = [_i32]
+lib.moe_profile_begin.restype = ctypes.c_int
+lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)]
+lib.moe_profile_end.restype = _i32
+lib.moe_last_error.restype = ctypes.c_char_p
+lib.moe_last_launch_count.restype = _i32
+for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
+           "moe_forward", "moe_forward_host", "moe_check_status"):
+    getattr(lib, _f).restype = ctypes.c_int
+
+EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
+            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
+            "moe_check_status", "moe_profile_begin", "moe_profile_end", "moe_last_error",
+            "moe_last_launch_count")
+
+
+def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
+                act=SWIGLU, dtype=BF16, clamp=0.0, capacity=0) -> moe_config:
+    return moe_config(int(N), int(d), int(E), int(k), int(F), int(n_shared), int(n_bias_sets),
+                      int(score_fn), int(renorm), int(act), int(dtype), float(clamp),
+                      int(capacity))
+
+
+def config_from_shape(shape, N: Optional[int] = None, capacity: int = 0) -> moe_config:
+    """moe_config for a workloads.LayerShape."""
+    return make_config(shape.N if N is None else N, shape.d, shape.E, shape.k, shape.F,
+                       shape.n_shared, shape.n_bias_sets, shape.score_fn, shape.renorm,
+                       shape.act, shape.dtype, shape.clamp, capacity)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"expected a torch tensor, got {type(t)}")
+    if not t.is_cuda:
+        raise ValueError("tensors passed to the MoE library must live in CUDA memory")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the MoE library must be contiguous")
+    return t.data_ptr()
+
+
+def _host_ptr(t) -> int:
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("host buffers must be contiguous CPU tensors (pinned for speed)")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(st: int, where: str):
+    if st != MOE_OK:
+        raise MoeError(st, where)
+
+
+def moe_workspace_size(cfg: moe_config) -> int:
+    return int(lib.moe_workspace_size(ctypes.byref(cfg)))
+
+
+def moe_workspace_init(ws: torch.Tensor, stream=None):
+    _check(lib.moe_workspace_init(_ptr(ws), _stream(stream)), "moe_workspace_init")
+
+
+def alloc_workspace(cfg: moe_config, device="cuda") -> torch.Tensor:
+    """A zero-initialised workspace (uint8 tensor) for calls with this configuration."""
+    size = moe_workspace_size(cfg)
+    if size == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_workspace_size")
+    ws = torch.empty(size + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    ws = ws[off:off + size]
+    moe_workspace_init(ws)
+    return ws
+
+
+def moe_capacity(T: int, k: int, E: int, cf) -> int:
+    """C = ceil(T k / E * cf); cf None (no limit) gives 0."""
+    if cf is None:
+        return 0
+    f = Fraction(cf)
+    return int(lib.moe_capacity(int(T), int(k), int(E), f.numerator, f.denominator))
+
+
+def moe_route(cfg, *, logits=None, x=None, W_g=None, logit_offset=None, bias=None,
+              modality=None, ids=None, gates=None, counts=None, demand=None, drop_mask=None,
+              logits_out=None, ws, stream=None):
+    st = lib.moe_route(ctypes.byref(cfg), _ptr(logits), _ptr(x), _ptr(W_g), _ptr(logit_offset),
+                       _ptr(bias), _ptr(modality), _ptr(ids), _ptr(gates), _ptr(counts),
+                       _ptr(demand), _ptr(drop_mask), _ptr(logits_out), _ptr(ws),
+                       _stream(stream))
+    _check(st, "moe_route")
+
+
+def moe_permute(cfg, *, ids, drop_mask=None, x, offsets, row_token=None, slot_row, xp, ws,
+                stream=None):
+    st = lib.moe_permute(ctypes.byref(cfg), _ptr(ids), _ptr(drop_mask), _ptr(x), _ptr(offsets),
+                         _ptr(row_token), _ptr(slot_row), _ptr(xp), _ptr(ws), _stream(stream))
+    _check(st, "moe_permute")
+
+
+def moe_expert_ffn(cfg, *, xp, offsets, x=None, W_gu, W_down, ye, ws, stream=None):
+    st = lib.moe_expert_ffn(ctypes.byref(cfg), _ptr(xp), _ptr(offsets), _ptr(x), _ptr(W_gu),
+                            _ptr(W_down), _ptr(ye), _ptr(ws), _stream(stream))
+    _check(st, "moe_expert_ffn")
+
+
+def moe_combine(cfg, *, ye, slot_row, gates, y, stream=None):
+    st = lib.moe_combine(ctypes.byref(cfg), _ptr(ye), _ptr(slot_row), _ptr(gates), _ptr(y),
+                         _stream(stream))
+    _check(st, "moe_combine")
+
+
+def moe_forward(cfg, *, x, W_g, W_gu, W_down, y, logit_offset=None, bias=None, modality=None,
+                route_out: Optional[dict] = None, ws, stream=None):
+    ro = None
+    if route_out:
+        ro = moe_route_out(*[_ptr(route_out.get(n)) for n, _ in moe_route_out._fields_])
+    st = lib.moe_forward(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(logit_offset), _ptr(bias),
+                         _ptr(modality), _ptr(W_gu), _ptr(W_down), _ptr(y),
+                         ctypes.byref(ro) if ro is not None else None, _ptr(ws),
+                         _stream(stream))
+    _check(st, "moe_forward")
+
+
+def moe_forward_host(cfg, *, x_host, W_g, W_gu, W_down, y_host, logit_offset=None, bias=None,
+                     modality=None, ws, stream=None):
+    st = lib.moe_forward_host(ctypes.byref(cfg), _host_ptr(x_host), _ptr(W_g),
+                              _ptr(logit_offset), _ptr(bias), _ptr(modality), _ptr(W_gu),
+                              _ptr(W_down), _host_ptr(y_host), _ptr(ws), _stream(stream))
+    _check(st, "moe_forward_host")
+
+
+def moe_check_status(ws, stream=None) -> int:
+    """Synchronise and return the device status (0 = MOE_OK); clears it."""
+    return int(lib.moe_check_status(_ptr(ws), _stream(stream)))
+
+
+def moe_last_launch_count() -> int:
+    return int(lib.moe_last_launch_count())
+
+
+def moe_profile_begin(max_calls: int):
+    _check(lib.moe_profile_begin(int(max_calls)), "moe_profile_begin")
+
+
+def moe_profile_end(max_launches: int = 16):
+    """(per-launch total ms over the recorded calls, number of recorded calls)."""
+    buf = (ctypes.c_float * max_launches)()
+    calls = _i32(0)
+    n = lib.moe_profile_end(buf, max_launches, ctypes.byref(calls))
+    if n < 0:
+        raise MoeError(MOE_ERR_CUDA, "moe_profile_end")
+    return [float(buf[i]) for i in range(min(n, max_launches))], int(calls.value)

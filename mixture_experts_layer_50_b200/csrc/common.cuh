@@ -1,0 +1,39 @@
+// Device-side helpers shared by the kernels of the MoE layer (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Device status codes (same values as moe_status in include/moe.h).
+enum : int { kStatusOk = 0, kStatusInvalidInput = 4, kStatusTimeout = 5 };
+
+// Record a device-side finding: the first error since the last host check wins.
+__device__ __forceinline__ void report_status(int* status, int code) {
+  if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Token-tile size of the dispatch kernels (tokens ranked by one warp in order).
+constexpr int kRankTile = 128;
+
+}  // namespace moe

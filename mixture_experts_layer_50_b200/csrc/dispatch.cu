@@ -1,0 +1,217 @@
+// Capacity, token dropping and the permutation into per-expert contiguous groups.
+//
+// "Mixture-of-Experts : routage et capacité" slides, "L'idée — Capacité" and "Cas guidé —
+// trace complète": an expert serves its assignments in arrival (token) order, keeps the
+// first C and drops the rest; "Support visuel — Capacité" lays the kept tokens of each
+// expert out in that order.  "Основы MoE", "Эксперимент на PyTorch": the per-expert
+// gather x[rows] that feeds each expert.
+//
+// rank(t, e) = #{t' < t : e in ids[t']} is computed without atomics in three passes, so
+// every output is a deterministic function of ids:
+//   1. one warp per tile of kRankTile tokens walks its tokens in order with per-expert
+//      counters in shared memory (local rank) and writes the tile's histogram;
+//   2. one block scans the histograms over tiles (tile_base) and over experts (offsets),
+//      applying the capacity to the per-expert totals;
+//   3. one block per token: rank = tile_base + local rank, keep iff rank < C, row =
+//      offsets[e] + rank; the token's x row is copied to each kept row (the gather).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+__global__ void __launch_bounds__(32) rank_local_kernel(
+    const int32_t* __restrict__ ids, const uint8_t* __restrict__ drop_mask, int64_t N, int k,
+    int E, int32_t* __restrict__ local_rank, int32_t* __restrict__ tile_hist, int* status) {
+  extern __shared__ int32_t smem[];
+  int32_t* cnt = smem;       // [E]
+  int32_t* sid = smem + E;   // [kRankTile * k]
+  const int lane = threadIdx.x;
+  const int64_t t0 = (int64_t)blockIdx.x * kRankTile;
+  const int ntok = (int)min((int64_t)kRankTile, N - t0);
+  for (int e = lane; e < E; e += 32) cnt[e] = 0;
+  bool bad = false;
+  for (int i = lane; i < ntok * k; i += 32) {
+    int v = ids[t0 * k + i];
+    if (v < 0 || v >= E) {
+      bad = true;
+      v = -1;
+    } else if (drop_mask != nullptr && drop_mask[t0 * k + i]) {
+      v = -1;
+    }
+    sid[i] = v;
+  }
+  __syncwarp();
+  for (int t = 0; t < ntok; ++t) {
+    int v = lane < k ? sid[t * k + lane] : -1;
+    // an expert listed twice by one token: keep the first slot only
+    const unsigned peers = __match_any_sync(0xffffffffu, v);
+    if (v >= 0 && (__ffs(peers) - 1) != lane) {
+      bad = true;
+      v = -1;
+    }
+    int r = -1;
+    if (v >= 0) {
+      r = cnt[v];
+      cnt[v] = r + 1;
+    }
+    if (lane < k) local_rank[(t0 + t) * k + lane] = r;
+    __syncwarp();
+  }
+  if (bad) report_status(status, kStatusInvalidInput);
+  for (int e = lane; e < E; e += 32) tile_hist[(int64_t)blockIdx.x * E + e] = cnt[e];
+}
+
+// One block of 1024 threads.  Warp w owns a contiguous chunk of tiles.
+__global__ void __launch_bounds__(1024) dispatch_scan_kernel(
+    const int32_t* __restrict__ tile_hist, int n_tiles, int E, int64_t C,
+    int32_t* __restrict__ tile_base, int32_t* __restrict__ demand,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
+  extern __shared__ int32_t part[];  // [32][E] chunk sums, then chunk bases
+  __shared__ int32_t warp_tot[32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int per = (n_tiles + 31) / 32;
+  const int c0 = min(w * per, n_tiles), c1 = min(c0 + per, n_tiles);
+  for (int e = lane; e < E; e += 32) {
+    int32_t s = 0;
+    for (int c = c0; c < c1; ++c) s += tile_hist[(int64_t)c * E + e];
+    part[w * E + e] = s;
+  }
+  __syncthreads();
+  // per expert: scan over chunks; the total is the demand, the capped total the count
+  int32_t my_count = 0;
+  const int e_me = threadIdx.x;
+  if (e_me < E) {
+    int32_t run = 0;
+    for (int c = 0; c < 32; ++c) {
+      const int32_t v = part[c * E + e_me];
+      part[c * E + e_me] = run;
+      run += v;
+    }
+    demand[e_me] = run;
+    my_count = (C > 0 && run > C) ? (int32_t)C : run;
+    counts[e_me] = my_count;
+  }
+  // exclusive scan of counts over the experts (E <= 1024: one expert per thread)
+  int32_t incl = my_count;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int32_t v = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    warp_tot[lane] = v;  // inclusive over warps
+  }
+  __syncthreads();
+  const int32_t excl = incl - my_count + (w > 0 ? warp_tot[w - 1] : 0);
+  if (e_me < E) offsets[e_me] = excl;
+  if (e_me == E - 1) offsets[E] = excl + my_count;
+  // per tile bases
+  for (int e = lane; e < E; e += 32) {
+    int32_t run = part[w * E + e];
+    for (int c = c0; c < c1; ++c) {
+      tile_base[(int64_t)c * E + e] = run;
+      run += tile_hist[(int64_t)c * E + e];
+    }
+  }
+}
+
+template <typename V>
+__global__ void __launch_bounds__(128) dispatch_scatter_kernel(
+    const int32_t* __restrict__ ids, const int32_t* __restrict__ local_rank,
+    const int32_t* __restrict__ tile_base, const int32_t* __restrict__ offsets, int k, int E,
+    int64_t C, int32_t* __restrict__ slot_row, int32_t* __restrict__ row_token,
+    uint8_t* __restrict__ drop_mask_out, const V* __restrict__ x, V* __restrict__ xp,
+    int row_vecs) {
+  __shared__ int32_t s_row[32];
+  const int64_t t = blockIdx.x;
+  if (threadIdx.x < k) {
+    const int j = threadIdx.x;
+    const int lr = local_rank[t * k + j];
+    int32_t row = -1;
+    if (lr >= 0) {
+      const int e = ids[t * k + j];
+      const int64_t r = (int64_t)tile_base[(t / kRankTile) * E + e] + lr;
+      if (C <= 0 || r < C) row = offsets[e] + (int32_t)r;
+    }
+    slot_row[t * k + j] = row;
+    if (drop_mask_out != nullptr) drop_mask_out[t * k + j] = row < 0 ? 1 : 0;
+    if (row >= 0 && row_token != nullptr) row_token[row] = (int32_t)t;
+    s_row[j] = row;
+  }
+  if (xp == nullptr) return;
+  __syncthreads();
+  const V* src = x + t * row_vecs;
+  for (int v = threadIdx.x; v < row_vecs; v += blockDim.x) {
+    const V val = src[v];
+    for (int j = 0; j < k; ++j) {
+      const int32_t row = s_row[j];
+      if (row >= 0) xp[(int64_t)row * row_vecs + v] = val;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rank_local(const int32_t* ids, const uint8_t* drop_mask, int64_t N, int k,
+                              int E, int32_t* local_rank, int32_t* tile_hist, int* status,
+                              cudaStream_t stream, int* launches) {
+  if (N == 0) return cudaSuccess;
+  const int64_t tiles = (N + kRankTile - 1) / kRankTile;
+  const size_t smem = sizeof(int32_t) * ((size_t)E + (size_t)kRankTile * k);
+  ++*launches;  // at most (1024 + 128 * 32) ints of shared memory: below the 48 KB default
+  rank_local_kernel<<<(unsigned)tiles, 32, smem, stream>>>(ids, drop_mask, N, k, E, local_rank,
+                                                           tile_hist, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_scan(const int32_t* tile_hist, int64_t N, int E, int64_t C,
+                                 int32_t* tile_base, int32_t* demand, int32_t* counts,
+                                 int32_t* offsets, cudaStream_t stream, int* launches) {
+  const int tiles = (int)((N + kRankTile - 1) / kRankTile);
+  const size_t smem = sizeof(int32_t) * 32 * (size_t)E;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaFuncSetAttribute(dispatch_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         32 * 1024 * (int)sizeof(int32_t));
+    attr_set = true;
+  }
+  ++*launches;
+  dispatch_scan_kernel<<<1, 1024, smem, stream>>>(tile_hist, tiles, E, C, tile_base, demand,
+                                                  counts, offsets);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_rank,
+                                    const int32_t* tile_base, const int32_t* offsets,
+                                    int64_t N, int k, int E, int64_t C, int32_t* slot_row,
+                                    int32_t* row_token, uint8_t* drop_mask_out,
+                                    const void* x, void* xp, int row_bytes,
+                                    cudaStream_t stream, int* launches) {
+  if (N == 0) return cudaSuccess;
+  ++*launches;
+  if (xp != nullptr && row_bytes % 16 == 0) {
+    dispatch_scatter_kernel<uint4><<<(unsigned)N, 128, 0, stream>>>(
+        ids, local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
+        (const uint4*)x, (uint4*)xp, row_bytes / 16);
+  } else if (xp != nullptr) {
+    dispatch_scatter_kernel<uint32_t><<<(unsigned)N, 128, 0, stream>>>(
+        ids, local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
+        (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4);
+  } else {
+    dispatch_scatter_kernel<uint4><<<(unsigned)N, 128, 0, stream>>>(
+        ids, local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
+        nullptr, nullptr, 0);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,615 @@
+// Grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM), fed by TMA.
+//
+// It computes, for every expert group g of variable size (read on the device from
+// offsets[], so no group size ever travels to the host):
+//     out[row0_g + i][n] = epilogue( sum_k A[arow0_g + i][k] * B[g][n][k] )
+// with both operands K-major bf16 and fp32 accumulation in tensor memory.  The same kernel
+// serves the three tensor-core steps of the layer:
+//   * the router projection z = x . W_g (one group, fp32 store, plus a per-expert offset);
+//   * the expert gate/up projection with SiLU(gate) * up (optionally clamped, "SwiGLU,
+//     écrêtée à 10" in the DeepSeek-V4.1-Flash table) or ReLU fused in the epilogue
+//     ("Le compte des paramètres": W_gate, W_up, W_down per expert; dataistudio listing:
+//     max(x W1, 0) W2);
+//   * the expert down projection (plain bf16 store).
+// The shared expert ("Des experts partagés") is one more group whose rows are all tokens.
+//
+// Design (one CTA per SM, persistent over a static round-robin of output tiles):
+//   warp 0      one thread issues TMA loads of 128x64 A tiles and BNx64 B tiles (128-byte
+//               swizzle) into a STAGES-deep ring of shared-memory stages;
+//   warp 1      allocates 2*BN TMEM columns (two accumulators) and one thread issues
+//               tcgen05.mma (M=128, N=BN, K=16) and tcgen05.commit;
+//   warps 2-5   drain an accumulator with tcgen05.ld while the next tile accumulates in
+//               the other one, apply the epilogue, stage rows in shared memory and write
+//               them with coalesced 16-byte stores, masking rows beyond the group and
+//               columns beyond n_out.
+// Tiles are numbered group by group, N-block outer and M-block inner, so the CTAs working
+// at the same time share B panels (weights) and A panels (tokens) through L2.
+// Every wait is bounded (globaltimer); on expiry the kernel records MOE_ERR_TIMEOUT in
+// the status word, lets the other roles stop, drains what it issued and frees TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                 // 64 bf16 = one 128-byte swizzle row
+constexpr int kThreads = 192;
+constexpr int kStageA = BM * BK * 2;   // 16 KB
+constexpr int kStagingPerWarp = 32 * 144;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// ---- mbarrier ------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Wait for the phase of `parity` to complete.  Gives up (false) when another role of the
+// CTA has given up, or after kWaitLimitNs, recording a timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          volatile int* abort_flag, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      report_status(status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// ---- TMA -----------------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// ---- tcgen05 -------------------------------------------------------------------------
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the 128-byte
+// swizzle: rows of 128 bytes, 8-row (1024-byte) swizzle atoms stacked at a 1024-byte
+// stride (SBO); the leading-dimension offset is unused for this layout (set to 1).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) |
+         ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both K-major.
+template <int BN>
+__device__ __forceinline__ constexpr uint32_t idesc_bf16() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                         uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+// Thread i of the warp receives TMEM lane (taddr.lane + i), 32 consecutive columns.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+struct Args {
+  const int32_t* offsets;
+  int n_routed;
+  int has_shared;
+  int shared_rows;
+  int shared_a_row0;
+  int shared_out_row0;
+  int K;
+  int n_out;
+  int up_row0;       // SwiGLU: first W_up row inside a group's B slice
+  float clamp;
+  const float* col_bias;
+  void* out;
+  int64_t ld_out;
+  int* status;
+};
+
+template <int BN, int STAGES>
+struct Layout {
+  static constexpr int kStageB = BN * BK * 2;
+  static constexpr int kOffB = STAGES * kStageA;
+  static constexpr int kOffStaging = kOffB + STAGES * kStageB;
+  static constexpr int kOffBar = kOffStaging + 4 * kStagingPerWarp;
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;       // tmem base, abort flag
+  static constexpr int kOffStart = kOffMisc + 16;               // tile prefix [G + 1]
+  static size_t bytes(int groups) { return 1024 + kOffStart + 4 * (size_t)(groups + 1); }
+};
+
+__device__ __forceinline__ void decode_tile(int tile, const int* s_start, int G, int nt,
+                                            int& g, int& m_blk, int& n_blk) {
+  int lo = 0, hi = G;  // largest g with s_start[g] <= tile
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_start[mid] <= tile) lo = mid; else hi = mid;
+  }
+  g = lo;
+  const int r = tile - s_start[g];
+  const int mt = (s_start[g + 1] - s_start[g]) / nt;
+  n_blk = r / mt;
+  m_blk = r - n_blk * mt;
+}
+
+__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
+
+template <int BN, int EPI, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmAs,
+                        const __grid_constant__ CUtensorMap tmB, const Args p) {
+  using L = Layout<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + L::kOffB;
+  uint8_t* staging = smem + L::kOffStaging;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = bars + 2 * STAGES + 2;
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
+  int* s_start = reinterpret_cast<int*>(smem + L::kOffStart);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.n_routed + p.has_shared;
+  constexpr int kOutPerTile = (EPI == kEpiSwiglu) ? BN / 2 : BN;
+  const int nt = (p.n_out + kOutPerTile - 1) / kOutPerTile;
+  const int nk = (p.K + BK - 1) / BK;
+
+  // ---- tile schedule: per-group tile counts and their prefix, from device offsets ----
+  if (warp == 0) {
+    const int per = (G + 31) / 32;
+    const int g0 = min(lane * per, G), g1 = min(g0 + per, G);
+    int local = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
+      local += ((cnt + BM - 1) / BM) * nt;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int g = g0; g < g1; ++g) {
+      s_start[g] = run;
+      const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
+      run += ((cnt + BM - 1) / BM) * nt;
+    }
+    if (lane == 31) s_start[G] = incl;
+    if (lane == 0) {
+      for (int i = 0; i < STAGES; ++i) {
+        mbar_init(&full[i], 1);
+        mbar_init(&empty[i], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&tfull[i], 1);
+        mbar_init(&tempty[i], 128);
+      }
+      mbar_init(drain, 1);
+      *s_abort = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+  } else if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_tmem)),
+                 "r"(2 * BN));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int total = s_start[G];
+
+  if (warp == 0) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed = 0;  // stages armed so far (for the drain on abort)
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        int g, m_blk, n_blk;
+        decode_tile(tile, s_start, G, nt, g, m_blk, n_blk);
+        const bool sh = g >= p.n_routed;
+        const int a_row = (sh ? p.shared_a_row0 : p.offsets[g]) + m_blk * BM;
+        const CUtensorMap* mA = sh ? &tmAs : &tmA;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[stage], kStageA + L::kStageB);
+          tma_load_2d(sA + stage * kStageA, mA, &full[stage], kb * BK, a_row);
+          uint8_t* b_dst = sB + stage * L::kStageB;
+          if (EPI == kEpiSwiglu) {
+            tma_load_3d(b_dst, &tmB, &full[stage], kb * BK, n_blk * (BN / 2), g);
+            tma_load_3d(b_dst + (BN / 2) * BK * 2, &tmB, &full[stage], kb * BK,
+                        p.up_row0 + n_blk * (BN / 2), g);
+          } else {
+            tma_load_3d(b_dst, &tmB, &full[stage], kb * BK, n_blk * BN, g);
+          }
+          ++armed;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // let the loads already issued land before the CTA leaves
+        for (int i = 0; i < STAGES && i < armed; ++i) {
+          stage = (stage + STAGES - 1) % STAGES;
+          if (stage == STAGES - 1) phase ^= 1;
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&full[stage], phase) && global_timer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      constexpr uint32_t kIdesc = idesc_bf16<BN>();
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], aph ^ 1, s_abort, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, s_abort, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * kStageA);
+          const uint32_t b0 = smem_u32(sB + stage * L::kStageB);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            mma_bf16(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), kIdesc,
+                     (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) mma_commit(&tfull[acc]);
+      }
+      if (!ok) {
+        // wait for the MMAs already issued before TMEM is released
+        mma_commit(drain);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ================= epilogue (warps 2..5) =================
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    uint8_t* stg = staging + (warp - 2) * kStagingPerWarp;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      int g, m_blk, n_blk;
+      decode_tile(tile, s_start, G, nt, g, m_blk, n_blk);
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      // warp-uniform decision: tcgen05.ld below needs all 32 lanes
+      const bool ready = mbar_wait(&tfull[acc], aph, s_abort, p.status);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tc_fence_after();
+      const bool sh = g >= p.n_routed;
+      const int cnt = sh ? p.shared_rows : p.offsets[g + 1] - p.offsets[g];
+      const int64_t out_row0 = (int64_t)(sh ? p.shared_out_row0 : p.offsets[g]) + m_blk * BM;
+      const int rows_valid = min(BM, cnt - m_blk * BM);
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+
+      constexpr int kColsPerChunk = (EPI == kEpiStoreF32) ? 32 : 64;
+      constexpr int kChunks = kOutPerTile / kColsPerChunk;
+#pragma unroll 1
+      for (int c = 0; c < kChunks; ++c) {
+        uint32_t packed[32];
+        if constexpr (EPI == kEpiSwiglu) {
+          float gv[32], uv[32];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            tmem_ld32(t_row + c * 64 + h * 32, gv);
+            tmem_ld32(t_row + BN / 2 + c * 64 + h * 32, uv);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float g0 = gv[2 * i], g1 = gv[2 * i + 1], u0 = uv[2 * i], u1 = uv[2 * i + 1];
+              if (p.clamp > 0.f) {
+                g0 = fminf(fmaxf(g0, -p.clamp), p.clamp);
+                g1 = fminf(fmaxf(g1, -p.clamp), p.clamp);
+                u0 = fminf(fmaxf(u0, -p.clamp), p.clamp);
+                u1 = fminf(fmaxf(u1, -p.clamp), p.clamp);
+              }
+              __nv_bfloat162 hv = __floats2bfloat162_rn(silu_f(g0) * u0, silu_f(g1) * u1);
+              packed[h * 16 + i] = *reinterpret_cast<uint32_t*>(&hv);
+            }
+          }
+        } else if constexpr (EPI == kEpiStoreF32) {
+          float v[32];
+          tmem_ld32(t_row + c * 32, v);
+          tmem_ld_wait();
+          const int col0 = n_blk * BN + c * 32;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float o = v[i];
+            if (p.col_bias != nullptr && col0 + i < p.n_out) o += p.col_bias[col0 + i];
+            packed[i] = __float_as_uint(o);
+          }
+        } else {
+          float v[32];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            tmem_ld32(t_row + c * 64 + h * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float a = v[2 * i], b = v[2 * i + 1];
+              if (EPI == kEpiRelu) {
+                a = fmaxf(a, 0.f);
+                b = fmaxf(b, 0.f);
+              }
+              __nv_bfloat162 hv = __floats2bfloat162_rn(a, b);
+              packed[h * 16 + i] = *reinterpret_cast<uint32_t*>(&hv);
+            }
+          }
+        }
+        if (c == kChunks - 1) {
+          // all TMEM reads of this accumulator are done: hand it back to the MMA warp
+          tc_fence_before();
+          mbar_arrive(&tempty[acc]);
+        }
+        // stage this thread's 128-byte row piece (row stride 144 B: conflict-free)
+        uint4* my = reinterpret_cast<uint4*>(stg + lane * 144);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          my[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        __syncwarp();
+        // coalesced copy-out: 4 rows x 128 bytes per instruction
+        constexpr int kElPerPiece = (EPI == kEpiStoreF32) ? 4 : 8;
+        const int col_base = n_blk * kOutPerTile + c * kColsPerChunk;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int rr = i * 4 + (lane >> 3);
+          const int pc = lane & 7;
+          const int row_in_tile = q * 32 + rr;
+          const int col = col_base + pc * kElPerPiece;
+          if (row_in_tile < rows_valid && col < p.n_out) {
+            const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 144 + pc * 16);
+            const int64_t orow = out_row0 + row_in_tile;
+            if constexpr (EPI == kEpiStoreF32) {
+              float* o = reinterpret_cast<float*>(p.out) + orow * p.ld_out + col;
+              if (col + 4 <= p.n_out) {
+                *reinterpret_cast<uint4*>(o) = val;
+              } else {
+                const float* f = reinterpret_cast<const float*>(&val);
+                for (int e = 0; e < p.n_out - col; ++e) o[e] = f[e];
+              }
+            } else {
+              __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + orow * p.ld_out + col;
+              *reinterpret_cast<uint4*>(o) = val;  // n_out % 8 == 0 (checked on the host)
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(2 * BN));
+  }
+}
+
+// ---- host side -------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor [outer][rows][K] (outer == 0: 2-D [rows][K]); box [box_rows][64], 128B swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, int64_t K, int64_t rows, int64_t outer,
+              int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)rows, (cuuint64_t)(outer > 0 ? outer : 1)};
+  cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)(K * rows * 2)};
+  cuuint32_t box[3] = {(cuuint32_t)BK, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  const cuuint32_t rank = outer > 0 ? 3 : 2;
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides,
+            box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int BN, int EPI, int STAGES>
+cudaError_t launch_t(const GroupedGemm& g, const CUtensorMap& mA, const CUtensorMap& mAs,
+                     const CUtensorMap& mB, cudaStream_t stream, int grid) {
+  using L = Layout<BN, STAGES>;
+  auto kern = grouped_gemm_kernel<BN, EPI, STAGES>;
+  const int groups = g.n_routed + g.has_shared;
+  const size_t smem = L::bytes(groups);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  Args a;
+  a.offsets = g.offsets;
+  a.n_routed = g.n_routed;
+  a.has_shared = g.has_shared;
+  a.shared_rows = (int)g.shared_rows;
+  a.shared_a_row0 = (int)g.shared_a_row0;
+  a.shared_out_row0 = (int)g.shared_out_row0;
+  a.K = g.K;
+  a.n_out = g.n_out;
+  a.up_row0 = g.n_out;
+  a.clamp = g.clamp;
+  a.col_bias = g.col_bias;
+  a.out = g.out;
+  a.ld_out = g.ld_out;
+  a.status = g.status;
+  kern<<<grid, kThreads, smem, stream>>>(mA, mAs, mB, a);
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+
+cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* launches,
+                                const char** why) {
+  using namespace tc;
+  const int groups = g.n_routed + g.has_shared;
+  if (groups == 0) return cudaSuccess;
+  int BN;
+  if (g.epilogue == kEpiStoreF32) {
+    BN = g.n_out <= 32 ? 32 : g.n_out <= 64 ? 64 : g.n_out <= 128 ? 128 : (g.n_out % 256 == 0 || g.n_out > 384) ? 256 : 128;
+  } else {
+    BN = 256;
+  }
+  const int box_b = (g.epilogue == kEpiSwiglu) ? BN / 2 : BN;
+  CUtensorMap mA, mAs, mB;
+  const void* a_ptr = g.a != nullptr ? g.a : g.a_shared;
+  const int64_t a_rows = g.a != nullptr ? g.rows_a : g.rows_a_shared;
+  if (!make_map(&mA, a_ptr, g.K, std::max<int64_t>(a_rows, 1), 0, BM) ||
+      !make_map(&mAs, g.a_shared != nullptr ? g.a_shared : a_ptr, g.K,
+                std::max<int64_t>(g.a_shared != nullptr ? g.rows_a_shared : a_rows, 1), 0, BM) ||
+      !make_map(&mB, g.b, g.K, g.rows_b, g.groups_b, box_b)) {
+    *why = "cuTensorMapEncodeTiled failed (pointer alignment, strides or driver entry point)";
+    return cudaErrorInvalidValue;
+  }
+  // grid: at most one CTA per SM, no more than an upper bound of the tile count
+  const int out_per_tile = (g.epilogue == kEpiSwiglu) ? BN / 2 : BN;
+  const int64_t nt = (g.n_out + out_per_tile - 1) / out_per_tile;
+  int64_t mtiles = 0;
+  if (g.n_routed > 0) mtiles += (g.max_rows_routed + BM - 1) / BM + g.n_routed;
+  if (g.has_shared) mtiles += (g.shared_rows + BM - 1) / BM;
+  const int64_t bound = mtiles * nt;
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), bound));
+  ++*launches;
+  switch (g.epilogue) {
+    case kEpiSwiglu: return launch_t<256, kEpiSwiglu, 4>(g, mA, mAs, mB, stream, grid);
+    case kEpiRelu: return launch_t<256, kEpiRelu, 4>(g, mA, mAs, mB, stream, grid);
+    case kEpiStoreBf16: return launch_t<256, kEpiStoreBf16, 4>(g, mA, mAs, mB, stream, grid);
+    case kEpiStoreF32:
+      switch (BN) {
+        case 32: return launch_t<32, kEpiStoreF32, 8>(g, mA, mAs, mB, stream, grid);
+        case 64: return launch_t<64, kEpiStoreF32, 8>(g, mA, mAs, mB, stream, grid);
+        case 128: return launch_t<128, kEpiStoreF32, 6>(g, mA, mAs, mB, stream, grid);
+        default: return launch_t<256, kEpiStoreF32, 4>(g, mA, mAs, mB, stream, grid);
+      }
+  }
+  *why = "unknown epilogue";
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

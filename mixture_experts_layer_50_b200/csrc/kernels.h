@@ -1,0 +1,92 @@
+// Internal launchers of the MoE layer kernels.  Each returns the cudaError_t of its
+// launch(es) and adds the number of kernels it enqueued to *launches.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ---- routing (route.cu) ---------------------------------------------------------------
+// Scores, selection keys, top-k (descending, ties to the lower index) and gates.
+cudaError_t launch_route_topk(const float* logits, int64_t N, int E, int k, int score_fn,
+                              int renorm, const float* bias, int n_bias_sets,
+                              const uint8_t* modality, int32_t* ids, float* gates,
+                              int* status, cudaStream_t stream, int* launches);
+
+// ---- dispatch (dispatch.cu) -----------------------------------------------------------
+// Pass 1: per token tile, ranks of each assignment among the tile's earlier tokens that
+// chose the same expert, and the tile's per-expert histogram.  Assignments whose
+// drop_mask entry is set (when drop_mask != nullptr), or whose id is invalid, get rank -1.
+cudaError_t launch_rank_local(const int32_t* ids, const uint8_t* drop_mask, int64_t N, int k,
+                              int E, int32_t* local_rank, int32_t* tile_hist, int* status,
+                              cudaStream_t stream, int* launches);
+// Pass 2: scan over tiles and experts: tile_base, demand, counts (capped at C when C > 0)
+// and offsets (exclusive scan of counts, E + 1 entries).
+cudaError_t launch_dispatch_scan(const int32_t* tile_hist, int64_t N, int E, int64_t C,
+                                 int32_t* tile_base, int32_t* demand, int32_t* counts,
+                                 int32_t* offsets, cudaStream_t stream, int* launches);
+// Pass 3: capacity decision, slot rows, row -> token map, drop mask, and (when xp is not
+// null) the gather of x rows into the per-expert layout.
+cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_rank,
+                                    const int32_t* tile_base, const int32_t* offsets,
+                                    int64_t N, int k, int E, int64_t C, int32_t* slot_row,
+                                    int32_t* row_token, uint8_t* drop_mask_out,
+                                    const void* x, void* xp, int row_bytes,
+                                    cudaStream_t stream, int* launches);
+
+// ---- combine (combine.cu) -------------------------------------------------------------
+// y[t] = sum_j gates[t,j] ye[slot_row[t,j]] (+ ye[shared_row0 + t] when shared_row0 >= 0).
+cudaError_t launch_combine(const void* ye, const int32_t* slot_row, const float* gates,
+                           int64_t N, int k, int d, int64_t shared_row0, int is_f32, void* y,
+                           cudaStream_t stream, int* launches);
+
+// ---- fp32 path (simt_f32.cu) ----------------------------------------------------------
+cudaError_t launch_router_f32(const float* x, const float* W_g, const float* logit_offset,
+                              int64_t N, int d, int E, float* logits, cudaStream_t stream,
+                              int* launches);
+// h[r] = act(A_r . W1_e) for every row r of the groups (routed rows from xp, shared rows
+// from x), then ye[r] = h[r] . W2_e.
+cudaError_t launch_ffn_f32(const float* xp, const float* x, const int32_t* offsets,
+                           int64_t N, int k, int d, int E, int F, int n_shared, int act,
+                           float clamp, const float* W_gu, const float* W_down, float* h,
+                           float* ye, cudaStream_t stream, int* launches);
+
+// ---- tensor-core grouped GEMM (gemm_tc.cu) --------------------------------------------
+enum GemmEpilogue : int { kEpiStoreBf16 = 0, kEpiSwiglu = 1, kEpiRelu = 2, kEpiStoreF32 = 3 };
+
+struct GroupedGemm {
+  // A: rows of activations, bf16 [rows_a][K]; routed group e reads rows
+  // [offsets[e], offsets[e+1]).  a_shared: bf16 [rows_a_shared][K], read by the shared
+  // group (rows [shared_a_row0, shared_a_row0 + shared_rows)).
+  const void* a;
+  int64_t rows_a;
+  const void* a_shared;
+  int64_t rows_a_shared;
+  int64_t shared_a_row0;
+  // B: weights bf16 [groups][rows_b][K]; routed group e uses slice e, the shared group
+  // slice n_routed.
+  const void* b;
+  int groups_b;
+  int rows_b;
+  int K;
+  const int32_t* offsets;  // [n_routed + 1] device, or null when n_routed == 0
+  int n_routed;
+  int has_shared;
+  int64_t shared_rows;
+  int64_t shared_out_row0;
+  int n_out;               // output columns (SwiGLU: F, with up rows starting at row F)
+  int epilogue;            // GemmEpilogue
+  float clamp;
+  const float* col_bias;   // [n_out] fp32 added before the store (fp32 store only)
+  void* out;
+  int64_t ld_out;          // elements
+  int64_t rows_out;
+  int64_t max_rows_routed; // upper bound of offsets[n_routed] (grid sizing)
+  int* status;
+};
+
+cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* launches,
+                                const char** why);
+
+}  // namespace moe

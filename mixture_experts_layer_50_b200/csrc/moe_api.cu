@@ -1,0 +1,589 @@
+// C ABI of the MoE layer (declared in include/moe.h): argument checks, the workspace
+// layout, and the order of launches on the caller's stream.  No entry point allocates
+// device memory; none synchronises except moe_check_status and moe_forward_host.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <type_traits>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+thread_local int32_t g_last_launches = 0;
+
+// Launch timing (moe_profile_begin / moe_profile_end).
+struct Profile {
+  int32_t max_calls = 0;
+  int32_t call = -1;          // index of the call being recorded
+  bool recording = false;     // inside a moe_forward call that is being recorded
+  std::vector<std::vector<cudaEvent_t>> ev;
+  bool active() const { return recording && call >= 0 && call < max_calls; }
+};
+thread_local Profile g_prof;
+
+void prof_mark(cudaStream_t st) {
+  if (!g_prof.active()) return;
+  cudaEvent_t e;
+  if (cudaEventCreate(&e) != cudaSuccess) return;
+  cudaEventRecord(e, st);
+  g_prof.ev[g_prof.call].push_back(e);
+}
+void prof_call_begin(cudaStream_t st) {
+  if (g_prof.max_calls <= 0) return;
+  ++g_prof.call;
+  g_prof.recording = true;
+  if (g_prof.active()) {
+    g_prof.ev.emplace_back();
+    prof_mark(st);
+  }
+}
+
+moe_status fail(moe_status s, const char* msg) {
+  g_last_error = msg;
+  return s;
+}
+
+moe_status cuda_fail(cudaError_t e, const char* where) {
+  char buf[256];
+  snprintf(buf, sizeof(buf), "%s: %s", where, cudaGetErrorString(e));
+  g_last_error = buf;
+  return MOE_ERR_CUDA;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Ws {
+  size_t status, logits, ids, gates, local_rank, tile_hist, tile_base, demand, counts, offsets,
+      slot_row, row_token, drop_mask, xp, h, ye, x_stage, y_stage, total;
+};
+
+size_t el_size(const moe_config& c) { return c.dtype == MOE_DT_BF16 ? 2 : 4; }
+
+Ws layout(const moe_config& c) {
+  Ws w;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t N = (size_t)c.N, k = (size_t)c.k, E = (size_t)c.E, d = (size_t)c.d,
+               F = (size_t)c.F, S = (size_t)c.n_shared, el = el_size(c);
+  const size_t Nk = N * k;
+  const size_t tiles = (N + moe::kRankTile - 1) / moe::kRankTile;
+  w.status = take(256);
+  w.logits = take(N * E * 4);
+  w.ids = take(Nk * 4);
+  w.gates = take(Nk * 4);
+  w.local_rank = take(Nk * 4);
+  w.tile_hist = take(tiles * E * 4);
+  w.tile_base = take(tiles * E * 4);
+  w.demand = take(E * 4);
+  w.counts = take(E * 4);
+  w.offsets = take((E + 1) * 4);
+  w.slot_row = take(Nk * 4);
+  w.row_token = take(Nk * 4);
+  w.drop_mask = take(Nk);
+  w.xp = take(Nk * d * el);
+  w.h = take((Nk + S * N) * F * el);
+  w.ye = take((Nk + S * N) * d * el);
+  w.x_stage = take(N * d * el);
+  w.y_stage = take(N * d * el);
+  w.total = off;
+  return w;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status check_cfg(const moe_config* c) {
+  if (c == nullptr) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->N < 0) return fail(MOE_ERR_INVALID_ARG, "N < 0");
+  if (c->d <= 0 || c->F <= 0) return fail(MOE_ERR_INVALID_ARG, "d and F must be positive");
+  if (c->E < 1) return fail(MOE_ERR_INVALID_ARG, "E < 1");
+  if (c->k < 1 || c->k > c->E) return fail(MOE_ERR_INVALID_ARG, "k must be in [1, E]");
+  if (c->E > 1024) return fail(MOE_ERR_UNSUPPORTED, "E > 1024");
+  if (c->k > 32) return fail(MOE_ERR_UNSUPPORTED, "k > 32");
+  if (c->n_shared < 0) return fail(MOE_ERR_INVALID_ARG, "n_shared < 0");
+  if (c->n_shared > 1) return fail(MOE_ERR_UNSUPPORTED, "n_shared > 1");
+  if (c->score_fn != MOE_SCORE_SOFTMAX && c->score_fn != MOE_SCORE_SIGMOID)
+    return fail(MOE_ERR_INVALID_ARG, "unknown score_fn");
+  if (c->renorm != 0 && c->renorm != 1) return fail(MOE_ERR_INVALID_ARG, "renorm must be 0 or 1");
+  if (c->act != MOE_ACT_SWIGLU && c->act != MOE_ACT_RELU)
+    return fail(MOE_ERR_INVALID_ARG, "unknown act");
+  if (c->dtype != MOE_DT_BF16 && c->dtype != MOE_DT_F32)
+    return fail(MOE_ERR_INVALID_ARG, "unknown dtype");
+  if (c->n_bias_sets < 0) return fail(MOE_ERR_INVALID_ARG, "n_bias_sets < 0");
+  if (!(c->clamp == c->clamp)) return fail(MOE_ERR_INVALID_ARG, "clamp is NaN");
+  if (c->dtype == MOE_DT_BF16 && (c->d % 8 != 0 || c->F % 8 != 0))
+    return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d and F multiples of 8");
+  if (c->dtype == MOE_DT_F32 && c->d % 4 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need d a multiple of 4");
+  const int64_t rows = c->N * (int64_t)c->k + c->N * (int64_t)c->n_shared;
+  if (rows > (int64_t)INT32_MAX / 2) return fail(MOE_ERR_UNSUPPORTED, "N*k too large for int32 rows");
+  return MOE_OK;
+}
+
+moe_status check_ws(const moe_config* c, void* ws) {
+  if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(ws, 256)) return fail(MOE_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  (void)c;
+  return MOE_OK;
+}
+
+moe_status need(const void* p, const char* name) {
+  if (p == nullptr) {
+    std::string m = std::string(name) + " is NULL";
+    return fail(MOE_ERR_INVALID_ARG, m.c_str());
+  }
+  if (!aligned(p, 16)) {
+    std::string m = std::string(name) + " must be 16-byte aligned";
+    return fail(MOE_ERR_UNSUPPORTED, m.c_str());
+  }
+  return MOE_OK;
+}
+
+moe_status check_bias(const moe_config* c, const float* bias, const uint8_t* modality) {
+  if (c->n_bias_sets == 0 && bias != nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "bias given but n_bias_sets == 0");
+  if (c->n_bias_sets > 0 && bias == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "n_bias_sets > 0 but bias is NULL");
+  if (c->n_bias_sets > 1 && modality == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "several bias sets need the modality flags");
+  return MOE_OK;
+}
+
+#define MOE_TRY(expr)               \
+  do {                              \
+    const moe_status _s = (expr);   \
+    if (_s != MOE_OK) return _s;    \
+  } while (0)
+#define MOE_CUDA(expr, where)                        \
+  do {                                               \
+    const cudaError_t _e = (expr);                   \
+    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+  } while (0)
+
+// ---- the stages, shared by the split entry points and moe_forward --------------------
+
+moe_status stage_logits(const moe_config& c, const void* x, const void* W_g,
+                        const float* logit_offset, float* logits, int* status,
+                        cudaStream_t st, int* launches) {
+  if (c.N == 0) return MOE_OK;
+  if (c.dtype == MOE_DT_F32) {
+    MOE_CUDA(moe::launch_router_f32((const float*)x, (const float*)W_g, logit_offset, c.N, c.d,
+                                    c.E, logits, st, launches),
+             "router (fp32)");
+    prof_mark(st);
+    return MOE_OK;
+  }
+  moe::GroupedGemm g{};
+  g.a = nullptr;
+  g.a_shared = x;
+  g.rows_a_shared = c.N;
+  g.shared_a_row0 = 0;
+  g.b = W_g;
+  g.groups_b = 1;
+  g.rows_b = c.E;
+  g.K = c.d;
+  g.offsets = nullptr;
+  g.n_routed = 0;
+  g.has_shared = 1;
+  g.shared_rows = c.N;
+  g.shared_out_row0 = 0;
+  g.n_out = c.E;
+  g.epilogue = moe::kEpiStoreF32;
+  g.col_bias = logit_offset;
+  g.out = logits;
+  g.ld_out = c.E;
+  g.rows_out = c.N;
+  g.status = status;
+  const char* why = "router GEMM launch";
+  MOE_CUDA(moe::launch_grouped_gemm(g, st, launches, &why), why);
+  prof_mark(st);
+  return MOE_OK;
+}
+
+moe_status stage_route(const moe_config& c, const float* logits, const float* bias,
+                       const uint8_t* modality, int32_t* ids, float* gates, int* status,
+                       cudaStream_t st, int* launches) {
+  MOE_CUDA(moe::launch_route_topk(logits, c.N, c.E, c.k, c.score_fn, c.renorm, bias,
+                                  c.n_bias_sets, modality, ids, gates, status, st, launches),
+           "top-k routing");
+  prof_mark(st);
+  return MOE_OK;
+}
+
+// Ranks, capacity, offsets, slot rows; gathers x into xp when xp != nullptr.
+moe_status stage_dispatch(const moe_config& c, const Ws& L, void* ws, const int32_t* ids,
+                          const uint8_t* drop_in, int64_t C, int32_t* demand, int32_t* counts,
+                          int32_t* offsets, int32_t* slot_row, int32_t* row_token,
+                          uint8_t* drop_out, const void* x, void* xp, cudaStream_t st,
+                          int* launches) {
+  int* status = at<int>(ws, L.status);
+  MOE_CUDA(moe::launch_rank_local(ids, drop_in, c.N, c.k, c.E, at<int32_t>(ws, L.local_rank),
+                                  at<int32_t>(ws, L.tile_hist), status, st, launches),
+           "rank pass");
+  prof_mark(st);
+  MOE_CUDA(moe::launch_dispatch_scan(at<int32_t>(ws, L.tile_hist), c.N, c.E, C,
+                                     at<int32_t>(ws, L.tile_base), demand, counts, offsets, st,
+                                     launches),
+           "scan pass");
+  prof_mark(st);
+  MOE_CUDA(moe::launch_dispatch_scatter(ids, at<int32_t>(ws, L.local_rank),
+                                        at<int32_t>(ws, L.tile_base), offsets, c.N, c.k, c.E, C,
+                                        slot_row, row_token, drop_out, x, xp,
+                                        (int)(c.d * el_size(c)), st, launches),
+           "scatter pass");
+  prof_mark(st);
+  return MOE_OK;
+}
+
+moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
+                     const int32_t* offsets, const void* x, const void* W_gu,
+                     const void* W_down, void* ye, cudaStream_t st, int* launches) {
+  if (c.N == 0) return MOE_OK;
+  const int64_t Nk = c.N * (int64_t)c.k;
+  if (c.dtype == MOE_DT_F32) {
+    MOE_CUDA(moe::launch_ffn_f32((const float*)xp, (const float*)x, offsets, c.N, c.k, c.d, c.E,
+                                 c.F, c.n_shared, c.act, c.clamp, (const float*)W_gu,
+                                 (const float*)W_down, at<float>(ws, L.h), (float*)ye, st,
+                                 launches),
+             "fp32 expert FFN");
+    prof_mark(st);
+    return MOE_OK;
+  }
+  int* status = at<int>(ws, L.status);
+  void* h = at<char>(ws, L.h);
+  moe::GroupedGemm g1{};
+  g1.a = xp;
+  g1.rows_a = Nk;
+  g1.a_shared = c.n_shared ? x : xp;
+  g1.rows_a_shared = c.n_shared ? c.N : Nk;
+  g1.shared_a_row0 = 0;
+  g1.b = W_gu;
+  g1.groups_b = c.E + c.n_shared;
+  g1.rows_b = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
+  g1.K = c.d;
+  g1.offsets = offsets;
+  g1.n_routed = c.E;
+  g1.has_shared = c.n_shared;
+  g1.shared_rows = c.N;
+  g1.shared_out_row0 = Nk;
+  g1.n_out = c.F;
+  g1.epilogue = c.act == MOE_ACT_SWIGLU ? moe::kEpiSwiglu : moe::kEpiRelu;
+  g1.clamp = c.clamp;
+  g1.out = h;
+  g1.ld_out = c.F;
+  g1.rows_out = Nk + c.n_shared * c.N;
+  g1.max_rows_routed = Nk;
+  g1.status = status;
+  const char* why = "gate/up GEMM launch";
+  MOE_CUDA(moe::launch_grouped_gemm(g1, st, launches, &why), why);
+  prof_mark(st);
+
+  moe::GroupedGemm g2{};
+  g2.a = h;
+  g2.rows_a = Nk + c.n_shared * c.N;
+  g2.a_shared = h;
+  g2.rows_a_shared = g2.rows_a;
+  g2.shared_a_row0 = Nk;
+  g2.b = W_down;
+  g2.groups_b = c.E + c.n_shared;
+  g2.rows_b = c.d;
+  g2.K = c.F;
+  g2.offsets = offsets;
+  g2.n_routed = c.E;
+  g2.has_shared = c.n_shared;
+  g2.shared_rows = c.N;
+  g2.shared_out_row0 = Nk;
+  g2.n_out = c.d;
+  g2.epilogue = moe::kEpiStoreBf16;
+  g2.out = ye;
+  g2.ld_out = c.d;
+  g2.rows_out = g2.rows_a;
+  g2.max_rows_routed = Nk;
+  g2.status = status;
+  why = "down GEMM launch";
+  MOE_CUDA(moe::launch_grouped_gemm(g2, st, launches, &why), why);
+  prof_mark(st);
+  return MOE_OK;
+}
+
+moe_status stage_combine(const moe_config& c, const void* ye, const int32_t* slot_row,
+                         const float* gates, void* y, cudaStream_t st, int* launches) {
+  const int64_t shared_row0 = c.n_shared ? c.N * (int64_t)c.k : -1;
+  MOE_CUDA(moe::launch_combine(ye, slot_row, gates, c.N, c.k, c.d, shared_row0,
+                               c.dtype == MOE_DT_F32, y, st, launches),
+           "combine");
+  prof_mark(st);
+  return MOE_OK;
+}
+
+moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
+                        const float* logit_offset, const float* bias, const uint8_t* modality,
+                        const void* W_gu, const void* W_down, void* y,
+                        const moe_route_out* ro, void* ws, cudaStream_t st, int* launches) {
+  const moe_config& c = *cfg;
+  const Ws L = layout(c);
+  int* status = at<int>(ws, L.status);
+  auto pick = [&](auto* user, size_t off) {
+    using T = std::remove_pointer_t<decltype(user)>;
+    return user != nullptr ? user : at<T>(ws, off);
+  };
+  float* logits = pick(ro ? ro->logits : (float*)nullptr, L.logits);
+  int32_t* ids = pick(ro ? ro->ids : (int32_t*)nullptr, L.ids);
+  float* gates = pick(ro ? ro->gates : (float*)nullptr, L.gates);
+  int32_t* counts = pick(ro ? ro->counts : (int32_t*)nullptr, L.counts);
+  int32_t* demand = pick(ro ? ro->demand : (int32_t*)nullptr, L.demand);
+  uint8_t* drop = pick(ro ? ro->drop_mask : (uint8_t*)nullptr, L.drop_mask);
+  int32_t* offsets = pick(ro ? ro->offsets : (int32_t*)nullptr, L.offsets);
+  void* xp = at<char>(ws, L.xp);
+  void* ye = at<char>(ws, L.ye);
+  prof_call_begin(st);
+  MOE_TRY(stage_logits(c, x, W_g, logit_offset, logits, status, st, launches));
+  MOE_TRY(stage_route(c, logits, bias, modality, ids, gates, status, st, launches));
+  MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, c.capacity, demand, counts, offsets,
+                         at<int32_t>(ws, L.slot_row), at<int32_t>(ws, L.row_token), drop, x,
+                         xp, st, launches));
+  MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, launches));
+  MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, launches));
+  g_prof.recording = false;
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_config* cfg) {
+  if (check_cfg(cfg) != MOE_OK) return 0;
+  return layout(*cfg).total;
+}
+
+moe_status moe_workspace_init(void* ws, moe_stream_t stream) {
+  if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  MOE_CUDA(cudaMemsetAsync(ws, 0, 256, (cudaStream_t)stream), "workspace init");
+  return MOE_OK;
+}
+
+int64_t moe_capacity(int64_t T, int32_t k, int32_t E, int64_t cf_num, int64_t cf_den) {
+  if (cf_num <= 0) return 0;
+  if (T < 0 || k < 1 || E < 1 || cf_den <= 0) return -1;
+  const __int128 p = (__int128)T * k * cf_num;
+  const __int128 q = (__int128)E * cf_den;
+  return (int64_t)((p + q - 1) / q);
+}
+
+moe_status moe_route(const moe_config* cfg, const float* logits, const void* x,
+                     const void* W_g, const float* logit_offset, const float* bias,
+                     const uint8_t* modality, int32_t* ids, float* gates, int32_t* counts,
+                     int32_t* demand, uint8_t* drop_mask, float* logits_out, void* ws,
+                     moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  MOE_TRY(check_bias(cfg, bias, modality));
+  if (logits == nullptr) {
+    MOE_TRY(need(x, "x"));
+    MOE_TRY(need(W_g, "W_g"));
+  }
+  const moe_config& c = *cfg;
+  const Ws L = layout(c);
+  cudaStream_t st = (cudaStream_t)stream;
+  int launches = 0;
+  int* status = at<int>(ws, L.status);
+  const float* z = logits;
+  if (z == nullptr) {
+    float* dst = logits_out != nullptr ? logits_out : at<float>(ws, L.logits);
+    MOE_TRY(stage_logits(c, x, W_g, logit_offset, dst, status, st, &launches));
+    z = dst;
+  }
+  int32_t* ids_p = ids != nullptr ? ids : at<int32_t>(ws, L.ids);
+  float* gates_p = gates != nullptr ? gates : at<float>(ws, L.gates);
+  MOE_TRY(stage_route(c, z, bias, modality, ids_p, gates_p, status, st, &launches));
+  MOE_TRY(stage_dispatch(c, L, ws, ids_p, nullptr, c.capacity,
+                         demand != nullptr ? demand : at<int32_t>(ws, L.demand),
+                         counts != nullptr ? counts : at<int32_t>(ws, L.counts),
+                         at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.slot_row), nullptr,
+                         drop_mask != nullptr ? drop_mask : at<uint8_t>(ws, L.drop_mask),
+                         nullptr, nullptr, st, &launches));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_permute(const moe_config* cfg, const int32_t* ids, const uint8_t* drop_mask,
+                       const void* x, int32_t* offsets, int32_t* row_token,
+                       int32_t* slot_row, void* xp, void* ws, moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  if (ids == nullptr || offsets == nullptr || slot_row == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "ids, offsets and slot_row are required");
+  MOE_TRY(need(x, "x"));
+  MOE_TRY(need(xp, "xp"));
+  const moe_config& c = *cfg;
+  const Ws L = layout(c);
+  int launches = 0;
+  MOE_TRY(stage_dispatch(c, L, ws, ids, drop_mask, 0, at<int32_t>(ws, L.demand),
+                         at<int32_t>(ws, L.counts), offsets, slot_row, row_token, nullptr, x,
+                         xp, (cudaStream_t)stream, &launches));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const int32_t* offsets,
+                          const void* x, const void* W_gu, const void* W_down, void* ye,
+                          void* ws, moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  MOE_TRY(need(xp, "xp"));
+  if (offsets == nullptr) return fail(MOE_ERR_INVALID_ARG, "offsets is NULL");
+  if (cfg->n_shared) MOE_TRY(need(x, "x"));
+  MOE_TRY(need(W_gu, "W_gu"));
+  MOE_TRY(need(W_down, "W_down"));
+  MOE_TRY(need(ye, "ye"));
+  int launches = 0;
+  MOE_TRY(stage_ffn(*cfg, layout(*cfg), ws, xp, offsets, x, W_gu, W_down, ye,
+                    (cudaStream_t)stream, &launches));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* ye, const int32_t* slot_row,
+                       const float* gates, void* y, moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(need(ye, "ye"));
+  MOE_TRY(need(y, "y"));
+  if (slot_row == nullptr || gates == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "slot_row and gates are required");
+  int launches = 0;
+  MOE_TRY(stage_combine(*cfg, ye, slot_row, gates, y, (cudaStream_t)stream, &launches));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_forward(const moe_config* cfg, const void* x, const void* W_g,
+                       const float* logit_offset, const float* bias,
+                       const uint8_t* modality, const void* W_gu, const void* W_down,
+                       void* y, const moe_route_out* route_out, void* ws,
+                       moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  MOE_TRY(check_bias(cfg, bias, modality));
+  MOE_TRY(need(x, "x"));
+  MOE_TRY(need(W_g, "W_g"));
+  MOE_TRY(need(W_gu, "W_gu"));
+  MOE_TRY(need(W_down, "W_down"));
+  MOE_TRY(need(y, "y"));
+  int launches = 0;
+  const moe_status fs = forward_impl(cfg, x, W_g, logit_offset, bias, modality, W_gu, W_down,
+                                     y, route_out, ws, (cudaStream_t)stream, &launches);
+  g_prof.recording = false;
+  MOE_TRY(fs);
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const void* W_g,
+                            const float* logit_offset, const float* bias,
+                            const uint8_t* modality, const void* W_gu, const void* W_down,
+                            void* y_host, void* ws, moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  MOE_TRY(check_bias(cfg, bias, modality));
+  if (x_host == nullptr || y_host == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "x_host and y_host are required");
+  MOE_TRY(need(W_g, "W_g"));
+  MOE_TRY(need(W_gu, "W_gu"));
+  MOE_TRY(need(W_down, "W_down"));
+  const moe_config& c = *cfg;
+  const Ws L = layout(c);
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t bytes = (size_t)c.N * c.d * el_size(c);
+  void* xd = at<char>(ws, L.x_stage);
+  void* yd = at<char>(ws, L.y_stage);
+  int launches = 0;
+  if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, st), "copy x to device");
+  const moe_status fs = forward_impl(cfg, xd, W_g, logit_offset, bias, modality, W_gu, W_down,
+                                     yd, nullptr, ws, st, &launches);
+  g_prof.recording = false;
+  MOE_TRY(fs);
+  if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, st), "copy y to host");
+  MOE_CUDA(cudaStreamSynchronize(st), "synchronise");
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_check_status(void* ws, moe_stream_t stream) {
+  if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t st = (cudaStream_t)stream;
+  MOE_CUDA(cudaStreamSynchronize(st), "asynchronous error");
+  int host = 0;
+  MOE_CUDA(cudaMemcpyAsync(&host, ws, sizeof(int), cudaMemcpyDeviceToHost, st), "read status");
+  MOE_CUDA(cudaMemsetAsync(ws, 0, sizeof(int), st), "clear status");
+  MOE_CUDA(cudaStreamSynchronize(st), "read status");
+  if (host == MOE_ERR_INVALID_INPUT)
+    return fail(MOE_ERR_INVALID_INPUT, "device found an invalid expert id or modality flag");
+  if (host == MOE_ERR_TIMEOUT) return fail(MOE_ERR_TIMEOUT, "a bounded device wait ran out");
+  if (host != 0) return fail(MOE_ERR_CUDA, "unknown device status");
+  return MOE_OK;
+}
+
+moe_status moe_profile_begin(int32_t max_calls) {
+  if (max_calls < 0) return fail(MOE_ERR_INVALID_ARG, "max_calls < 0");
+  for (auto& v : g_prof.ev)
+    for (auto e : v) cudaEventDestroy(e);
+  g_prof = Profile();
+  g_prof.max_calls = max_calls;
+  return MOE_OK;
+}
+
+int32_t moe_profile_end(float* launch_ms, int32_t max_launches, int32_t* calls) {
+  int32_t per_call = 0;
+  bool ok = true;
+  if (launch_ms != nullptr)
+    for (int i = 0; i < max_launches; ++i) launch_ms[i] = 0.f;
+  for (auto& v : g_prof.ev) {
+    if (v.empty()) continue;
+    if (cudaEventSynchronize(v.back()) != cudaSuccess) ok = false;
+    per_call = std::max<int32_t>(per_call, (int32_t)v.size() - 1);
+    for (size_t i = 0; ok && i + 1 < v.size(); ++i) {
+      float ms = 0.f;
+      if (cudaEventElapsedTime(&ms, v[i], v[i + 1]) != cudaSuccess) ok = false;
+      if (launch_ms != nullptr && (int)i < max_launches) launch_ms[i] += ms;
+    }
+  }
+  if (calls != nullptr) *calls = (int32_t)g_prof.ev.size();
+  for (auto& v : g_prof.ev)
+    for (auto e : v) cudaEventDestroy(e);
+  g_prof = Profile();
+  if (!ok) {
+    g_last_error = "moe_profile_end: event timing failed";
+    return -1;
+  }
+  return per_call;
+}
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+int32_t moe_last_launch_count(void) { return g_last_launches; }
+
+}  // extern "C"

@@ -1,0 +1,192 @@
+// Router scores, top-k selection and gates: one warp per token.
+//
+// "Основы MoE" (ai.flicky.cc), section "Как устроен MoE-слой", steps 2-3: p = softmax(z),
+// keep the k largest, g_i = p_i / sum_{j in T} p_j; with k = 1 (Switch) the weight is p_i.
+// DeepSeek-V3 scores with a sigmoid.  "Le groupe d'experts (MoE)", "Étape 1: le routeur"
+// and the DeepSeek-V4.1-Flash "Mixture-of-Experts" page ("L'équilibrage de charge",
+// "l'équilibrage par modalité"): a per-expert bias, one set per modality, is added for
+// the selection only; the gates use the unbiased scores.
+//
+// Selection keys are float32: z + b (softmax) or sigma(z) + b (sigmoid).  The k rounds
+// of a warp arg-max pick the largest key, ties to the lower expert index, so ids come out
+// by descending key.  sigma(z) is evaluated with the exp below, built from Cody & Waite's
+// range reduction and a Taylor polynomial out of correctly rounded float32 operations
+// (explicit _rn intrinsics, never contracted into FMAs), so that sigmoid keys -- and the
+// experts they select -- are reproducible bit for bit on any IEEE float32 machine.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+// e^x for |x| <= 80.  x = n ln2 + r with n = rint(x / ln2); ln2 is split into a 16-bit
+// high part (so n * ln2_hi is exact for |n| < 256) and its float remainder; e^r comes
+// from the degree-7 Taylor polynomial in Horner form; 2^n is applied exactly.
+__device__ __forceinline__ float exp_reduced_taylor(float x) {
+  const float inv_ln2 = 1.4426950408889634f;
+  const float ln2_hi = 45426.0f / 65536.0f;
+  const float ln2_lo = (float)(0.6931471805599453 - 0.693145751953125);
+  const float n = rintf(__fmul_rn(x, inv_ln2));
+  float r = __fsub_rn(x, __fmul_rn(n, ln2_hi));
+  r = __fsub_rn(r, __fmul_rn(n, ln2_lo));
+  float p = 1.0f / 5040.0f;
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f / 720.0f);
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f / 120.0f);
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f / 24.0f);
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f / 6.0f);
+  p = __fadd_rn(__fmul_rn(p, r), 0.5f);
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
+  const int ni = (int)n;  // |ni| <= 116 for |x| <= 80: 2^ni is a normal float
+  return __fmul_rn(p, __int_as_float((ni + 127) << 23));
+}
+
+__device__ __forceinline__ float sigmoid_reproducible(float z) {
+  const float zc = fminf(fmaxf(z, -80.0f), 80.0f);
+  return __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_reduced_taylor(-zc)));
+}
+
+// (key, expert) order used by the selection: larger key first, then lower index.
+__device__ __forceinline__ bool beats(float ka, int ea, float kb, int eb) {
+  return ka > kb || (ka == kb && ea < eb);
+}
+
+template <int J>  // keys per lane: E <= 32 * J
+__global__ void __launch_bounds__(256) route_topk_kernel(
+    const float* __restrict__ logits, int64_t N, int E, int k, int score_fn, int renorm,
+    const float* __restrict__ bias, int n_bias_sets, const uint8_t* __restrict__ modality,
+    int32_t* __restrict__ ids, float* __restrict__ gates, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= N) return;
+  const float* z = logits + t * E;
+  const float* b = nullptr;
+  if (bias != nullptr) {
+    int set = 0;
+    if (modality != nullptr) {
+      set = modality[t];
+      if (set >= n_bias_sets) {
+        if (lane == 0) report_status(status, kStatusInvalidInput);
+        set = 0;
+      }
+    }
+    b = bias + (int64_t)set * E;
+  }
+
+  float key[J], sc[J];
+  float zmax = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = -INFINITY;
+    sc[j] = 0.0f;
+    if (e < E) {
+      const float zz = z[e];
+      zmax = fmaxf(zmax, zz);
+      const float s = (score_fn == 1) ? sigmoid_reproducible(zz) : zz;
+      sc[j] = s;
+      key[j] = (b != nullptr) ? __fadd_rn(s, b[e]) : s;
+    }
+  }
+
+  // k rounds of warp arg-max.  Lane r keeps the r-th selection.
+  uint32_t taken = 0;
+  int my_e = -1;
+  float my_sc = 0.0f;
+  for (int r = 0; r < k; ++r) {
+    float bk = -INFINITY, bs = 0.0f;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && !((taken >> j) & 1u) && (be == 0x7fffffff || key[j] > bk)) {
+        bk = key[j];
+        be = e;
+        bs = sc[j];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+      if (oe != 0x7fffffff && (be == 0x7fffffff || beats(ok, oe, bk, be))) {
+        bk = ok;
+        be = oe;
+        bs = os;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == r) {
+      my_e = be;
+      my_sc = bs;
+    }
+  }
+
+  const bool mine = lane < k;
+  float g;
+  if (score_fn == 0) {
+    if (renorm) {
+      // softmax over the selected logits
+      const float m = warp_max(mine ? my_sc : -INFINITY);
+      const float ex = mine ? expf(my_sc - m) : 0.0f;
+      g = ex / warp_sum(ex);
+    } else {
+      // raw probability of the full softmax
+      const float M = warp_max(zmax);
+      float part = 0.0f;
+#pragma unroll
+      for (int j = 0; j < J; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E) part += expf(z[e] - M);
+      }
+      g = expf(my_sc - M) / warp_sum(part);
+    }
+  } else {
+    if (renorm) {
+      g = my_sc / warp_sum(mine ? my_sc : 0.0f);
+    } else {
+      g = my_sc;
+    }
+  }
+  if (mine) {
+    ids[t * k + lane] = my_e;
+    gates[t * k + lane] = g;
+  }
+}
+
+template <int J>
+cudaError_t launch_j(const float* logits, int64_t N, int E, int k, int score_fn, int renorm,
+                     const float* bias, int n_bias_sets, const uint8_t* modality,
+                     int32_t* ids, float* gates, int* status, cudaStream_t stream) {
+  const int threads = 256;
+  const int64_t blocks = (N * 32 + threads - 1) / threads;
+  route_topk_kernel<J><<<(unsigned)blocks, threads, 0, stream>>>(
+      logits, N, E, k, score_fn, renorm, bias, n_bias_sets, modality, ids, gates, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_route_topk(const float* logits, int64_t N, int E, int k, int score_fn,
+                              int renorm, const float* bias, int n_bias_sets,
+                              const uint8_t* modality, int32_t* ids, float* gates,
+                              int* status, cudaStream_t stream, int* launches) {
+  if (N == 0) return cudaSuccess;
+  ++*launches;
+  const int J = (E + 31) / 32;
+#define MOE_ROUTE_CASE(JJ) \
+  if (J <= JJ)             \
+    return launch_j<JJ>(logits, N, E, k, score_fn, renorm, bias, n_bias_sets, modality, ids, gates, status, stream);
+  MOE_ROUTE_CASE(1)
+  MOE_ROUTE_CASE(2)
+  MOE_ROUTE_CASE(4)
+  MOE_ROUTE_CASE(8)
+  MOE_ROUTE_CASE(12)
+  MOE_ROUTE_CASE(16)
+  MOE_ROUTE_CASE(32)
+#undef MOE_ROUTE_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -1,0 +1,77 @@
+"""MoELayer: a layer's device weights and workspace behind one ``forward`` call."""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _native as nat
+
+
+class MoELayer:
+    """Forward pass of one MoE FFN layer through ``moe_forward``.
+
+    Weights use the library's storage convention (``W_g [E][d]``, ``W_gu [E+S][2F][d]``
+    gate rows then up rows, ``W_down [E+S][d][F]``, shared expert last).  The capacity is
+    recomputed per call from ``capacity_factor`` and the call's token count,
+    C = ceil(N k / E * cf).  The workspace is allocated once for ``max_tokens``.
+    """
+
+    def __init__(self, *, W_g, W_gu, W_down, k, n_shared=0, score_fn=nat.SOFTMAX, renorm=1,
+                 act=nat.SWIGLU, clamp=0.0, bias=None, logit_offset=None,
+                 capacity_factor=None, max_tokens: int, stream=None):
+        self.W_g, self.W_gu, self.W_down = W_g, W_gu, W_down
+        self.E, self.d = W_g.shape
+        self.F = W_down.shape[2]
+        self.k, self.n_shared = k, n_shared
+        self.score_fn, self.renorm, self.act, self.clamp = score_fn, renorm, act, clamp
+        self.bias, self.logit_offset = bias, logit_offset
+        self.n_bias_sets = 0 if bias is None else bias.shape[0]
+        self.capacity_factor = capacity_factor
+        self.dtype = nat.BF16 if W_gu.dtype == torch.bfloat16 else nat.F32
+        self.max_tokens = max_tokens
+        self.ws = nat.alloc_workspace(self.config(max_tokens), device=W_gu.device)
+
+    @classmethod
+    def from_workload(cls, shape, tensors: dict, max_tokens: Optional[int] = None):
+        return cls(W_g=tensors["W_g"], W_gu=tensors["W_gu"], W_down=tensors["W_down"],
+                   k=shape.k, n_shared=shape.n_shared, score_fn=shape.score_fn,
+                   renorm=shape.renorm, act=shape.act, clamp=shape.clamp,
+                   bias=tensors.get("bias"), logit_offset=tensors.get("logit_offset"),
+                   capacity_factor=shape.capacity_factor,
+                   max_tokens=shape.N if max_tokens is None else max_tokens)
+
+    def capacity(self, N: int) -> int:
+        return nat.moe_capacity(N, self.k, self.E, self.capacity_factor)
+
+    def config(self, N: int) -> "nat.moe_config":
+        return nat.make_config(N, self.d, self.E, self.k, self.F, self.n_shared,
+                               self.n_bias_sets, self.score_fn, self.renorm, self.act,
+                               self.dtype, self.clamp, self.capacity(N))
+
+    def _check_tokens(self, N):
+        if N > self.max_tokens:
+            raise ValueError(f"{N} tokens > max_tokens={self.max_tokens} of this layer's workspace")
+
+    def forward(self, x: torch.Tensor, modality=None, y=None, route_out: Optional[dict] = None,
+                stream=None) -> torch.Tensor:
+        N = x.shape[0]
+        self._check_tokens(N)
+        if y is None:
+            y = torch.empty_like(x)
+        nat.moe_forward(self.config(N), x=x, W_g=self.W_g, W_gu=self.W_gu, W_down=self.W_down,
+                        y=y, logit_offset=self.logit_offset, bias=self.bias, modality=modality,
+                        route_out=route_out, ws=self.ws, stream=stream)
+        return y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, modality=None,
+                     stream=None) -> torch.Tensor:
+        N = x_host.shape[0]
+        self._check_tokens(N)
+        nat.moe_forward_host(self.config(N), x_host=x_host, W_g=self.W_g, W_gu=self.W_gu,
+                             W_down=self.W_down, y_host=y_host, logit_offset=self.logit_offset,
+                             bias=self.bias, modality=modality, ws=self.ws, stream=stream)
+        return y_host
+
+    def check_status(self, stream=None) -> int:
+        return nat.moe_check_status(self.ws, stream)

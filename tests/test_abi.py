@@ -1,0 +1,143 @@
+"""The C ABI library: it loads, exports what include/moe.h declares, and rejects bad
+arguments on the host before touching the GPU (so these run without one)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from golden.reader import load
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def nat():
+    from mixture_experts_layer_50_b200 import _native
+    return _native
+
+
+def _declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text, re.M)
+    return names
+
+
+def test_library_exports_every_declared_function(nat):
+    names = _declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(nat.lib, n), n
+    assert set(nat.EXPORTED) <= set(names)
+
+
+def test_config_struct_layout(nat):
+    assert ctypes.sizeof(nat.moe_config) == 64
+    assert nat.moe_config.capacity.offset == 56
+    assert ctypes.sizeof(nat.moe_route_out) == 7 * 8
+
+
+def test_capacity_against_the_slides(nat):
+    g = load("p2_capacity_trace.txt")
+    lib = nat.lib
+    assert lib.moe_capacity(8, 2, 4, 5, 4) == int(g["C_1.25"])
+    assert lib.moe_capacity(8, 2, 4, 1, 1) == int(g["C_1.0"])
+    assert lib.moe_capacity(8, 2, 4, 2, 1) == int(g["C_2.0"])
+    assert lib.moe_capacity(8, 1, 4, 5, 4) == int(g["C_k1"])
+    assert lib.moe_capacity(8, 2, 4, 3, 2) == int(g["C_1.5"])
+    assert lib.moe_capacity(8, 2, 4, 0, 1) == 0          # no limit
+    assert lib.moe_capacity(100, 2, 64, 1, 1) == 4       # exact ceiling of 3.125
+    assert lib.moe_capacity(16384, 2, 64, 5, 4) == 640
+    assert lib.moe_capacity(-1, 2, 4, 1, 1) == -1
+    assert nat.moe_capacity(16384, 1, 64, 1) == 256
+
+
+def _cfg(nat, **kw):
+    base = dict(N=64, d=256, E=8, k=2, F=512)
+    base.update(kw)
+    return nat.make_config(**base)
+
+
+def test_workspace_size(nat):
+    small = nat.moe_workspace_size(_cfg(nat, N=16))
+    big = nat.moe_workspace_size(_cfg(nat, N=4096))
+    assert 0 < small < big
+    # xp (N k d bf16) and ye ((N k + N) d bf16) dominate
+    c = _cfg(nat, N=4096, n_shared=1)
+    assert nat.moe_workspace_size(c) >= 2 * (4096 * 2 * 256 + 4096 * 3 * 256)
+    assert nat.moe_workspace_size(_cfg(nat, k=9)) == 0      # k > E
+    assert nat.moe_workspace_size(_cfg(nat, E=2000)) == 0   # unsupported E
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(k=0), 1), (dict(k=9), 1), (dict(E=0), 1), (dict(N=-1), 1), (dict(d=0), 1),
+    (dict(score_fn=7), 1), (dict(act=3), 1), (dict(dtype=5), 1), (dict(renorm=2), 1),
+    (dict(E=64, k=33), 2), (dict(E=1500, k=2), 2), (dict(n_shared=2), 2), (dict(d=100), 2),
+    (dict(F=12), 2),
+])
+def test_forward_rejects_bad_config_on_host(nat, bad, code):
+    c = _cfg(nat, **bad)
+    fake = ctypes.c_void_p(0x100000)
+    st = nat.lib.moe_forward(ctypes.byref(c), fake, fake, None, None, None, fake, fake, fake,
+                             None, fake, None)
+    assert st == code, nat.lib.moe_last_error()
+    assert nat.lib.moe_last_error()
+
+
+def test_forward_rejects_null_and_unaligned_pointers(nat):
+    c = _cfg(nat)
+    fake = ctypes.c_void_p(0x100000)
+    lib = nat.lib
+    assert lib.moe_forward(ctypes.byref(c), None, fake, None, None, None, fake, fake, fake,
+                           None, fake, None) == nat.MOE_ERR_INVALID_ARG
+    assert b"x is NULL" in lib.moe_last_error()
+    assert lib.moe_forward(ctypes.byref(c), ctypes.c_void_p(0x100001), fake, None, None, None,
+                           fake, fake, fake, None, fake, None) == nat.MOE_ERR_UNSUPPORTED
+    assert lib.moe_forward(ctypes.byref(c), fake, fake, None, None, None, fake, fake, fake,
+                           None, ctypes.c_void_p(0x100010), None) == nat.MOE_ERR_INVALID_ARG
+    assert b"256-byte" in lib.moe_last_error()
+    assert lib.moe_forward(None, fake, fake, None, None, None, fake, fake, fake, None, fake,
+                           None) == nat.MOE_ERR_INVALID_ARG
+
+
+def test_bias_and_modality_rules(nat):
+    fake = ctypes.c_void_p(0x100000)
+    lib = nat.lib
+    c = _cfg(nat, n_bias_sets=2)
+    # two bias sets need the modality flags
+    assert lib.moe_forward(ctypes.byref(c), fake, fake, None, fake, None, fake, fake, fake,
+                           None, fake, None) == nat.MOE_ERR_INVALID_ARG
+    c = _cfg(nat, n_bias_sets=0)
+    assert lib.moe_forward(ctypes.byref(c), fake, fake, None, fake, None, fake, fake, fake,
+                           None, fake, None) == nat.MOE_ERR_INVALID_ARG
+    c = _cfg(nat, n_bias_sets=1)
+    assert lib.moe_route(ctypes.byref(c), fake, None, None, None, None, None, fake, fake, fake,
+                         fake, fake, None, fake, None) == nat.MOE_ERR_INVALID_ARG
+
+
+def test_split_entry_points_validate(nat):
+    fake = ctypes.c_void_p(0x100000)
+    lib = nat.lib
+    c = _cfg(nat)
+    assert lib.moe_permute(ctypes.byref(c), None, None, fake, fake, None, fake, fake, fake,
+                           None) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_expert_ffn(ctypes.byref(c), fake, None, None, fake, fake, fake, fake,
+                              None) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine(ctypes.byref(c), fake, None, fake, fake, None) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_route(ctypes.byref(c), None, None, fake, None, None, None, fake, fake, fake,
+                         fake, fake, None, fake, None) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_forward_host(ctypes.byref(c), None, fake, None, None, None, fake, fake,
+                                fake, fake, None) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_check_status(None, None) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_workspace_init(None, None) == nat.MOE_ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_tensors(nat):
+    import torch
+    c = _cfg(nat)
+    with pytest.raises(ValueError):
+        nat.moe_combine(c, ye=torch.zeros(4), slot_row=torch.zeros(4, dtype=torch.int32),
+                        gates=torch.zeros(4), y=torch.zeros(4))

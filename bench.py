@@ -181,24 +181,31 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(v, world):
+def max_over_ranks(v, world, device="cuda"):
+    """The slowest rank's time: every rank takes part in the same all-reduce."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def make_replica(shape, rank):
-    t = W.make_inputs(shape, device="cuda")
-    if rank > 0:  # same layer weights on every replica, own tokens per rank
-        g = torch.Generator(device="cuda")
+def aggregate_tokens_per_s(tokens_per_rank, world, ms_step_max):
+    """Whole-job throughput: tokens of all ranks over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms_step_max / 1e3)
+
+
+def make_replica(shape, rank, device="cuda"):
+    """The layer's inputs for one replica: the same weights everywhere, own tokens per rank."""
+    t = W.make_inputs(shape, device=device)
+    if rank > 0:
+        g = torch.Generator(device=device)
         g.manual_seed(shape.seed * 1000 + rank)
-        x = torch.empty(t["x"].shape, dtype=torch.float32, device="cuda").normal_(generator=g)
+        x = torch.empty(t["x"].shape, dtype=torch.float32, device=device).normal_(generator=g)
         t["x"] = x.to(t["x"].dtype)
         if "modality" in t:
-            u = torch.empty(shape.N, device="cuda").uniform_(generator=g)
+            u = torch.empty(t["x"].shape[0], device=device).uniform_(generator=g)
             t["modality"] = (u < 0.3).to(torch.uint8)
     return t
 
@@ -242,7 +249,7 @@ def run_ours(args):
     assert layer.check_status() == 0
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
     ms_step = ms_total / args.steps
-    value = shape.N * world / (ms_step / 1e3)
+    value = aggregate_tokens_per_s(shape.N, world, ms_step)
 
     # end to end through the public API with host buffers: H2D of x, the layer, D2H of y
     xh = x.cpu().pin_memory()
@@ -262,16 +269,22 @@ def run_ours(args):
     el = x.element_size()
 
     peaks, peak_src = load_peaks()
+    clocks = clk.summary()
+    # cuBLAS reached bf16_tflops at full clock (burst) and bf16_tflops_sustained once the
+    # power cap pulled the clock down: compare against the regime this run's clock shows
+    burst = (clocks.get("sm_mhz") or 0) >= 0.95 * (clocks.get("sm_max_mhz") or 1e9)
+    tensor_key = "bf16_tflops" if burst else "bf16_tflops_sustained"
+    tensor_peak = peaks[tensor_key]
     per_launch = {n: launch_ms[i] / max(calls, 1) for i, n in enumerate(LAUNCH_NAMES)
                   if i < len(launch_ms)}
     gu_ms = per_launch.get("gemm_gate_up")
-    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     intensity = work["flops_gate_up"] / work["bytes_gate_up"]
     roof = None
     if gu_ms:
         if intensity >= ridge:
             ach = work["flops_gate_up"] / (gu_ms / 1e3) / 1e12
-            peak = peaks["bf16_tflops_sustained"]
+            peak = tensor_peak
             roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": peak, "unit": "TFLOP/s"}
         else:
             ach = work["bytes_gate_up"] / (gu_ms / 1e3) / 1e9
@@ -281,9 +294,9 @@ def run_ours(args):
         roof["traffic"] = read_traffic("gemm_gate_up", args.workload)
         roof["kernel"] = "gemm_gate_up (grouped_gemm_kernel<256, SwiGLU>)"
         roof["ms_per_launch"] = round(gu_ms, 4)
-        roof["peak_source"] = f"{peak_src} ({'bf16_tflops_sustained' if roof['bound'] == 'tensor' else 'hbm_gbs'})"
+        roof["peak_source"] = f"{peak_src} ({tensor_key if roof['bound'] == 'tensor' else 'hbm_gbs'})"
     # whole-layer roofline: time bound = max(F / P, B / BW)
-    t_bound = max(work["flops_layer"] / (peaks["bf16_tflops_sustained"] * 1e12),
+    t_bound = max(work["flops_layer"] / (tensor_peak * 1e12),
                   work["bytes_layer"] / (peaks["hbm_gbs"] * 1e9))
     layer_roof = {"flops": work["flops_layer"], "bytes": work["bytes_layer"],
                   "bound_ms": round(t_bound * 1e3, 4), "frac": round(t_bound * 1e3 / ms_step, 4),
@@ -293,7 +306,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(shape, t, sample_tokens=64)
+        cpu = cpu_baseline(shape, t, sample_tokens=192)
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -310,7 +323,7 @@ def run_ours(args):
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": shape.N * shape.d * el,
                 "d2h_bytes_per_step": shape.N * shape.d * el},
         "gpu_launches": per_step_launches * args.steps,
-        "clocks": clk.summary(),
+        "clocks": clocks,
         "cpu_baseline": cpu,
     }
     if rank == 0:

@@ -309,16 +309,22 @@ def _forward_case(name, N=None, sample=None, tol_rows=None):
     ref, info = O.forward(x64, f64(t["W_g"]), _LazyF64(t["W_gu"]), _LazyF64(t["W_down"]),
                           tokens=tokens, logits=z_o, **{k: v for k, v in kw.items()
                                                         if k != "logit_offset"})
+    # Routing from the GPU's logits may differ from routing on float64 logits only where the
+    # top-k decision sits within the logit discrepancy ("fragile" tokens); with a capacity, a
+    # flip can move the keep/drop boundary of the two experts involved.
     frag = fragile_tokens(z_o, ro["logits"], shape.k, shape.score_fn, kw["bias"], kw["modality"])
     same_tok = (ro["ids"] == info["ids"]).all(1) & (ro["drop_mask"] == info["drop_mask"]).all(1)
     n_diff = int((~same_tok).sum())
     assert n_diff <= 3 * int(frag.sum()), (n_diff, int(frag.sum()))
-    assert frag.mean() < 0.01
+    assert n_diff <= max(2, shape.N // 200), n_diff
     if n_diff == 0:
         np.testing.assert_array_equal(ro["counts"], info["counts"])
         np.testing.assert_array_equal(ro["offsets"], info["offsets"])
     keep = same_tok[tokens]
     assert keep.mean() > 0.9
+    mx, rms = err_stats(host(y)[tokens][keep], ref[keep])
+    print(f"PARITY {name} N={shape.N}: logit err {zerr:.2e}, routing differs on {n_diff} "
+          f"tokens ({int(frag.sum())} fragile), output max err {mx:.2e} x max|ref|, rms {rms:.2e}")
     assert_close_layer(host(y)[tokens][keep], ref[keep])
     assert launches == 8
     return ro

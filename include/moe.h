@@ -177,6 +177,29 @@ MOE_API moe_status moe_forward_host(const moe_config* cfg, const void* x_host, c
                             const uint8_t* modality, const void* W_gu, const void* W_down,
                             void* y_host, void* ws, moe_stream_t stream);
 
+/* moe_route on given logits without a workspace: the same routing and capacity results
+ * (ids, gates, counts, demand, drop_mask) for callers that cannot allocate device memory,
+ * e.g. a plug-in running inside a host process whose memory manager has already reserved
+ * the whole device (a cudaMalloc there fails or breaks the host's budget), or a latency-
+ * critical loop that must not risk the implicit device synchronisation of cudaMalloc.
+ * The pages have no counterpart of this call; it is a deployment convenience.
+ * Scratch: a fixed 4 MiB device array inside the library (every GPU that loads the library
+ * holds it until the process exits).  The call needs 4*(2*N*k + 2*ceil(N/128)*E + E + 1)
+ * bytes of it, each part rounded up to 256; larger requests return MOE_ERR_UNSUPPORTED
+ * (e.g. N = 16384 tokens with k = 8 and E = 256 fits; N = 65536 with k = 8 does not).
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ * with that device current; make that first call before any stream capture.
+ * All calls share the array and it keeps the last call's contents: calls that may overlap
+ * on the GPU (other streams, other host threads) race -- order them on one stream.
+ *   status: optional device int32; device findings (a modality flag >= n_bias_sets) are
+ *           recorded there as in the workspace status word (the caller zeroes it).
+ * Other arguments as in moe_route; cfg->N, E, k, n_bias_sets, score_fn, renorm and
+ * capacity are used.  Allocates nothing (no cudaMalloc/cudaFree, no library allocator). */
+MOE_API moe_status moe_route_static(const moe_config* cfg, const float* logits,
+                                    const float* bias, const uint8_t* modality, int32_t* ids,
+                                    float* gates, int32_t* counts, int32_t* demand,
+                                    uint8_t* drop_mask, int32_t* status, moe_stream_t stream);
+
 /* Synchronise `stream`, read and clear the workspace status word.  Returns MOE_OK or the
  * first device-detected error (MOE_ERR_INVALID_INPUT, MOE_ERR_TIMEOUT) since the last
  * check; MOE_ERR_CUDA if the stream reports an asynchronous CUDA error. */

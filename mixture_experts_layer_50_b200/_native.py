@@ -67,6 +67,7 @@ lib.moe_combine.argtypes = [_cfgp] + [_vp] * 5
 lib.moe_forward.argtypes = [_cfgp] + [_vp] * 11
 lib.moe_forward_host.argtypes = [_cfgp] + [_vp] * 10
 lib.moe_check_status.argtypes = [_vp, _vp]
+lib.moe_route_static.argtypes = [_cfgp] + [_vp] * 10
 lib.moe_profile_begin.argtypes = [_i32]
 lib.moe_profile_begin.restype = ctypes.c_int
 lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)]
@@ -74,13 +75,13 @@ lib.moe_profile_end.restype = _i32
 lib.moe_last_error.restype = ctypes.c_char_p
 lib.moe_last_launch_count.restype = _i32
 for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
-           "moe_forward", "moe_forward_host", "moe_check_status"):
+           "moe_forward", "moe_forward_host", "moe_check_status", "moe_route_static"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
             "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
             "moe_check_status", "moe_profile_begin", "moe_profile_end", "moe_last_error",
-            "moe_last_launch_count")
+            "moe_last_launch_count", "moe_route_static")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -164,6 +165,15 @@ def moe_route(cfg, *, logits=None, x=None, W_g=None, logit_offset=None, bias=Non
                        _ptr(demand), _ptr(drop_mask), _ptr(logits_out), _ptr(ws),
                        _stream(stream))
     _check(st, "moe_route")
+
+
+def moe_route_static(cfg, *, logits, bias=None, modality=None, ids, gates, counts, demand,
+                     drop_mask, status=None, stream=None):
+    """moe_route on given logits without a workspace (scratch in the library's fixed array)."""
+    st = lib.moe_route_static(ctypes.byref(cfg), _ptr(logits), _ptr(bias), _ptr(modality),
+                              _ptr(ids), _ptr(gates), _ptr(counts), _ptr(demand),
+                              _ptr(drop_mask), _ptr(status), _stream(stream))
+    _check(st, "moe_route_static")
 
 
 def moe_permute(cfg, *, ids, drop_mask=None, x, offsets, row_token=None, slot_row, xp, ws,

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <type_traits>
 #include <vector>
@@ -528,6 +529,89 @@ moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const voi
   MOE_TRY(fs);
   if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, st), "copy y to host");
   MOE_CUDA(cudaStreamSynchronize(st), "synchronise");
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+}  // extern "C"
+
+// ---- moe_route_static: routing with its scratch in a fixed device array ---------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB
+// Scratch of moe_route_static.  In host code this name is only a host-side stand-in: the
+// kernels get the device address looked up below.
+__device__ __align__(256) unsigned char g_route_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of g_route_scratch on the current device (looked up once per device).
+moe_status static_scratch(void** out) {
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device ordinal >= 64");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    MOE_CUDA(cudaGetSymbolAddress(&p, g_route_scratch), "cudaGetSymbolAddress(route scratch)");
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_route_static(const moe_config* cfg, const float* logits, const float* bias,
+                            const uint8_t* modality, int32_t* ids, float* gates,
+                            int32_t* counts, int32_t* demand, uint8_t* drop_mask,
+                            int32_t* status, moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_bias(cfg, bias, modality));
+  if (logits == nullptr || ids == nullptr || gates == nullptr || counts == nullptr ||
+      demand == nullptr || drop_mask == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "logits, ids, gates, counts, demand and drop_mask are required");
+  const moe_config& c = *cfg;
+  const size_t Nk = (size_t)c.N * c.k;
+  const size_t tiles = ((size_t)c.N + moe::kRankTile - 1) / moe::kRankTile;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t o_rank = take(Nk * 4), o_hist = take(tiles * c.E * 4),
+               o_base = take(tiles * c.E * 4), o_offs = take(((size_t)c.E + 1) * 4),
+               o_slot = take(Nk * 4);
+  if (off > kStaticScratchBytes) {
+    char buf[160];
+    snprintf(buf, sizeof(buf), "moe_route_static needs %zu bytes of scratch; its static array holds %zu",
+             off, kStaticScratchBytes);
+    return fail(MOE_ERR_UNSUPPORTED, buf);
+  }
+  void* scratch = nullptr;
+  MOE_TRY(static_scratch(&scratch));
+  cudaStream_t st = (cudaStream_t)stream;
+  int launches = 0;
+  MOE_TRY(stage_route(c, logits, bias, modality, ids, gates, status, st, &launches));
+  MOE_CUDA(moe::launch_rank_local(ids, nullptr, c.N, c.k, c.E, at<int32_t>(scratch, o_rank),
+                                  at<int32_t>(scratch, o_hist), status, st, &launches),
+           "rank pass");
+  MOE_CUDA(moe::launch_dispatch_scan(at<int32_t>(scratch, o_hist), c.N, c.E, c.capacity,
+                                     at<int32_t>(scratch, o_base), demand, counts,
+                                     at<int32_t>(scratch, o_offs), st, &launches),
+           "scan pass");
+  MOE_CUDA(moe::launch_dispatch_scatter(ids, at<int32_t>(scratch, o_rank),
+                                        at<int32_t>(scratch, o_base),
+                                        at<int32_t>(scratch, o_offs), c.N, c.k, c.E,
+                                        c.capacity, at<int32_t>(scratch, o_slot), nullptr,
+                                        drop_mask, nullptr, nullptr, 0, st, &launches),
+           "scatter pass");
   g_last_launches = launches;
   return MOE_OK;
 }

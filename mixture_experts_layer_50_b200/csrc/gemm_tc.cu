@@ -30,6 +30,8 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -162,6 +164,67 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---- clusters and the 2-SM (cta_group::2) forms ----------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+// The same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_cta(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+// TMA load into this CTA's shared memory whose byte count completes on the barrier of the
+// pair's first CTA (`bar` is a shared::cluster address there).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar,
+                                                 int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"((uint64_t)map), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+// Arrive on the barrier at this offset in both CTAs of the pair once the issued MMAs finish.
+__device__ __forceinline__ void mma_commit_pair_both(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], m;\n\t}\n" ::"r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_pair_local(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
 struct Args {
   const int32_t* offsets;
   int n_routed;
@@ -191,6 +254,10 @@ struct Layout {
   static size_t bytes(int groups) { return 1024 + kOffStart + 4 * (size_t)(groups + 1); }
 };
 
+// Tile -> (group, M block, N block).  Tiles are numbered group by group; inside a group the
+// operand with the smaller total panel is kept resident in L2 while the other streams: if the
+// group's A rows outnumber its B rows, M blocks are outer and N blocks inner, else the reverse.
+template <int BMT, int BN>
 __device__ __forceinline__ void decode_tile(int tile, const int* s_start, int G, int nt,
                                             int& g, int& m_blk, int& n_blk) {
   int lo = 0, hi = G;  // largest g with s_start[g] <= tile
@@ -201,11 +268,115 @@ __device__ __forceinline__ void decode_tile(int tile, const int* s_start, int G,
   g = lo;
   const int r = tile - s_start[g];
   const int mt = (s_start[g + 1] - s_start[g]) / nt;
-  n_blk = r / mt;
-  m_blk = r - n_blk * mt;
+  if (mt * BMT > nt * BN) {
+    m_blk = r / nt;
+    n_blk = r - m_blk * nt;
+  } else {
+    n_blk = r / mt;
+    m_blk = r - n_blk * mt;
+  }
 }
 
 __device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
+
+// One epilogue warp drains its 32 TMEM lanes (rows row_base + lane of the output tile) of an
+// accumulator: activation, packing, per-warp staging in shared memory, then coalesced 16-byte
+// stores with row and column masks.  `release` runs right after the last TMEM read.
+template <int BN, int EPI, typename Release>
+__device__ __forceinline__ void epilogue_warp(const Args& p, uint32_t t_row, uint8_t* stg,
+                                              int lane, int n_blk, int64_t out_row0,
+                                              int row_base, int rows_valid, Release&& release) {
+  constexpr int kOutPerTile = (EPI == kEpiSwiglu) ? BN / 2 : BN;
+  constexpr int kColsPerChunk = (EPI == kEpiStoreF32) ? 32 : 64;
+  constexpr int kChunks = kOutPerTile / kColsPerChunk;
+#pragma unroll 1
+  for (int c = 0; c < kChunks; ++c) {
+    uint32_t packed[32];
+    if constexpr (EPI == kEpiSwiglu) {
+      float gv[32], uv[32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        tmem_ld32(t_row + c * 64 + h * 32, gv);
+        tmem_ld32(t_row + BN / 2 + c * 64 + h * 32, uv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float g0 = gv[2 * i], g1 = gv[2 * i + 1], u0 = uv[2 * i], u1 = uv[2 * i + 1];
+          if (p.clamp > 0.f) {
+            g0 = fminf(fmaxf(g0, -p.clamp), p.clamp);
+            g1 = fminf(fmaxf(g1, -p.clamp), p.clamp);
+            u0 = fminf(fmaxf(u0, -p.clamp), p.clamp);
+            u1 = fminf(fmaxf(u1, -p.clamp), p.clamp);
+          }
+          __nv_bfloat162 hv = __floats2bfloat162_rn(silu_f(g0) * u0, silu_f(g1) * u1);
+          packed[h * 16 + i] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+      }
+    } else if constexpr (EPI == kEpiStoreF32) {
+      float v[32];
+      tmem_ld32(t_row + c * 32, v);
+      tmem_ld_wait();
+      const int col0 = n_blk * BN + c * 32;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        float o = v[i];
+        if (p.col_bias != nullptr && col0 + i < p.n_out) o += p.col_bias[col0 + i];
+        packed[i] = __float_as_uint(o);
+      }
+    } else {
+      float v[32];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        tmem_ld32(t_row + c * 64 + h * 32, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float a = v[2 * i], b = v[2 * i + 1];
+          if (EPI == kEpiRelu) {
+            a = fmaxf(a, 0.f);
+            b = fmaxf(b, 0.f);
+          }
+          __nv_bfloat162 hv = __floats2bfloat162_rn(a, b);
+          packed[h * 16 + i] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+      }
+    }
+    if (c == kChunks - 1) release();
+    // stage this thread's 128-byte row piece (row stride 144 B: conflict-free)
+    uint4* my = reinterpret_cast<uint4*>(stg + lane * 144);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      my[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+    __syncwarp();
+    // coalesced copy-out: 4 rows x 128 bytes per instruction
+    constexpr int kElPerPiece = (EPI == kEpiStoreF32) ? 4 : 8;
+    const int col_base = n_blk * kOutPerTile + c * kColsPerChunk;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int rr = i * 4 + (lane >> 3);
+      const int pc = lane & 7;
+      const int row_in_tile = row_base + rr;
+      const int col = col_base + pc * kElPerPiece;
+      if (row_in_tile < rows_valid && col < p.n_out) {
+        const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 144 + pc * 16);
+        const int64_t orow = out_row0 + row_in_tile;
+        if constexpr (EPI == kEpiStoreF32) {
+          float* o = reinterpret_cast<float*>(p.out) + orow * p.ld_out + col;
+          if (col + 4 <= p.n_out) {
+            *reinterpret_cast<uint4*>(o) = val;
+          } else {
+            const float* f = reinterpret_cast<const float*>(&val);
+            for (int e = 0; e < p.n_out - col; ++e) o[e] = f[e];
+          }
+        } else {
+          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + orow * p.ld_out + col;
+          *reinterpret_cast<uint4*>(o) = val;  // n_out % 8 == 0 (checked on the host)
+        }
+      }
+    }
+    __syncwarp();
+  }
+}
 
 template <int BN, int EPI, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -290,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         int g, m_blk, n_blk;
-        decode_tile(tile, s_start, G, nt, g, m_blk, n_blk);
+        decode_tile<BM, BN>(tile, s_start, G, nt, g, m_blk, n_blk);
         const bool sh = g >= p.n_routed;
         const int a_row = (sh ? p.shared_a_row0 : p.offsets[g]) + m_blk * BM;
         const CUtensorMap* mA = sh ? &tmAs : &tmA;
@@ -380,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       int g, m_blk, n_blk;
-      decode_tile(tile, s_start, G, nt, g, m_blk, n_blk);
+      decode_tile<BM, BN>(tile, s_start, G, nt, g, m_blk, n_blk);
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       // warp-uniform decision: tcgen05.ld below needs all 32 lanes
@@ -393,99 +564,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rows_valid = min(BM, cnt - m_blk * BM);
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
 
-      constexpr int kColsPerChunk = (EPI == kEpiStoreF32) ? 32 : 64;
-      constexpr int kChunks = kOutPerTile / kColsPerChunk;
-#pragma unroll 1
-      for (int c = 0; c < kChunks; ++c) {
-        uint32_t packed[32];
-        if constexpr (EPI == kEpiSwiglu) {
-          float gv[32], uv[32];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            tmem_ld32(t_row + c * 64 + h * 32, gv);
-            tmem_ld32(t_row + BN / 2 + c * 64 + h * 32, uv);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float g0 = gv[2 * i], g1 = gv[2 * i + 1], u0 = uv[2 * i], u1 = uv[2 * i + 1];
-              if (p.clamp > 0.f) {
-                g0 = fminf(fmaxf(g0, -p.clamp), p.clamp);
-                g1 = fminf(fmaxf(g1, -p.clamp), p.clamp);
-                u0 = fminf(fmaxf(u0, -p.clamp), p.clamp);
-                u1 = fminf(fmaxf(u1, -p.clamp), p.clamp);
-              }
-              __nv_bfloat162 hv = __floats2bfloat162_rn(silu_f(g0) * u0, silu_f(g1) * u1);
-              packed[h * 16 + i] = *reinterpret_cast<uint32_t*>(&hv);
-            }
-          }
-        } else if constexpr (EPI == kEpiStoreF32) {
-          float v[32];
-          tmem_ld32(t_row + c * 32, v);
-          tmem_ld_wait();
-          const int col0 = n_blk * BN + c * 32;
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float o = v[i];
-            if (p.col_bias != nullptr && col0 + i < p.n_out) o += p.col_bias[col0 + i];
-            packed[i] = __float_as_uint(o);
-          }
-        } else {
-          float v[32];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            tmem_ld32(t_row + c * 64 + h * 32, v);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float a = v[2 * i], b = v[2 * i + 1];
-              if (EPI == kEpiRelu) {
-                a = fmaxf(a, 0.f);
-                b = fmaxf(b, 0.f);
-              }
-              __nv_bfloat162 hv = __floats2bfloat162_rn(a, b);
-              packed[h * 16 + i] = *reinterpret_cast<uint32_t*>(&hv);
-            }
-          }
-        }
-        if (c == kChunks - 1) {
-          // all TMEM reads of this accumulator are done: hand it back to the MMA warp
-          tc_fence_before();
-          mbar_arrive(&tempty[acc]);
-        }
-        // stage this thread's 128-byte row piece (row stride 144 B: conflict-free)
-        uint4* my = reinterpret_cast<uint4*>(stg + lane * 144);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          my[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-        __syncwarp();
-        // coalesced copy-out: 4 rows x 128 bytes per instruction
-        constexpr int kElPerPiece = (EPI == kEpiStoreF32) ? 4 : 8;
-        const int col_base = n_blk * kOutPerTile + c * kColsPerChunk;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int rr = i * 4 + (lane >> 3);
-          const int pc = lane & 7;
-          const int row_in_tile = q * 32 + rr;
-          const int col = col_base + pc * kElPerPiece;
-          if (row_in_tile < rows_valid && col < p.n_out) {
-            const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 144 + pc * 16);
-            const int64_t orow = out_row0 + row_in_tile;
-            if constexpr (EPI == kEpiStoreF32) {
-              float* o = reinterpret_cast<float*>(p.out) + orow * p.ld_out + col;
-              if (col + 4 <= p.n_out) {
-                *reinterpret_cast<uint4*>(o) = val;
-              } else {
-                const float* f = reinterpret_cast<const float*>(&val);
-                for (int e = 0; e < p.n_out - col; ++e) o[e] = f[e];
-              }
-            } else {
-              __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + orow * p.ld_out + col;
-              *reinterpret_cast<uint4*>(o) = val;  // n_out % 8 == 0 (checked on the host)
-            }
-          }
-        }
-        __syncwarp();
-      }
+      epilogue_warp<BN, EPI>(p, t_row, stg, lane, n_blk, out_row0, q * 32, rows_valid, [&] {
+        // all TMEM reads of this accumulator are done: hand it back to the MMA warp
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+      });
     }
   }
 
@@ -494,6 +577,236 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(2 * BN));
+  }
+}
+
+// ---- 2-SM variant ------------------------------------------------------------------------
+// A cluster of two CTAs on neighbouring SMs computes 256x256 tiles with tcgen05.mma
+// cta_group::2 (M = 256): CTA r stages rows [128 r, 128 r + 128) of the A tile and half of the
+// B tile (the gate box or the up box for SwiGLU; B rows [128 r, 128 r + 128) otherwise), so
+// each SM moves half the B bytes of the 1-SM kernel per MMA.  Both CTAs' TMA loads complete on
+// the first CTA's barrier; the first CTA issues the MMAs; commits arrive on both CTAs'
+// barriers; each CTA drains its own 128 accumulator rows from its own TMEM.
+template <int STAGES>
+struct Layout2 {
+  static constexpr int kStageA = tc::kStageA;          // 128 rows x 64 (16 KB)
+  static constexpr int kStageB = 128 * BK * 2;         // 128 rows x 64 (16 KB)
+  static constexpr int kOffB = STAGES * kStageA;
+  static constexpr int kOffStaging = kOffB + STAGES * kStageB;
+  static constexpr int kOffBar = kOffStaging + 4 * kStagingPerWarp;
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffStart = kOffMisc + 16;
+  static size_t bytes(int groups) { return 1024 + kOffStart + 4 * (size_t)(groups + 1); }
+};
+
+template <int EPI, int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmAs,
+                            const __grid_constant__ CUtensorMap tmB, const Args p) {
+  constexpr int BN = 256;   // MMA N
+  constexpr int BMT = 256;  // tile rows (128 per CTA)
+  using L = Layout2<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + L::kOffB;
+  uint8_t* staging = smem + L::kOffStaging;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = bars + 2 * STAGES + 2;
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
+  int* s_start = reinterpret_cast<int*>(smem + L::kOffStart);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int G = p.n_routed + p.has_shared;
+  constexpr int kOutPerTile = (EPI == kEpiSwiglu) ? BN / 2 : BN;
+  const int nt = (p.n_out + kOutPerTile - 1) / kOutPerTile;
+  const int nk = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    const int per = (G + 31) / 32;
+    const int g0 = min(lane * per, G), g1 = min(g0 + per, G);
+    int local = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
+      local += ((cnt + BMT - 1) / BMT) * nt;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int g = g0; g < g1; ++g) {
+      s_start[g] = run;
+      const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
+      run += ((cnt + BMT - 1) / BMT) * nt;
+    }
+    if (lane == 31) s_start[G] = incl;
+    if (lane == 0) {
+      for (int i = 0; i < STAGES; ++i) {
+        mbar_init(&full[i], 1);
+        mbar_init(&empty[i], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&tfull[i], 1);
+        mbar_init(&tempty[i], 8);  // one arrive per epilogue warp of both CTAs
+      }
+      mbar_init(drain, 1);
+      *s_abort = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+  } else if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_tmem)),
+                 "r"(2 * BN));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before either signals the other's
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int total = s_start[G];
+
+  if (warp == 0) {
+    // ================= TMA producer (both CTAs) =================
+    if (lane == 0) {
+      const uint32_t full0 = map_to_cta(smem_u32(&full[0]), 0);  // the first CTA's barriers
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed = 0;
+      bool ok = true;
+      auto a_row_of = [&](int g, int m_blk) {
+        const bool sh = g >= p.n_routed;
+        return (sh ? p.shared_a_row0 : p.offsets[g]) + m_blk * BMT + (int)rank * 128;
+      };
+      auto b_row_of = [&](int n_blk) {
+        if (EPI == kEpiSwiglu) return rank == 0 ? n_blk * 128 : p.up_row0 + n_blk * 128;
+        return n_blk * BN + (int)rank * 128;
+      };
+      for (int tile = pair; ok && tile < total; tile += npairs) {
+        int g, m_blk, n_blk;
+        decode_tile<BMT, BN>(tile, s_start, G, nt, g, m_blk, n_blk);
+        const CUtensorMap* mA = g >= p.n_routed ? &tmAs : &tmA;
+        const int a_row = a_row_of(g, m_blk);
+        const int b_row = b_row_of(n_blk);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, p.status)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_expect_tx(&full[stage], 2 * (L::kStageA + L::kStageB));
+          const uint32_t bar = full0 + 8u * (uint32_t)stage;
+          tma_load_2d_pair(sA + stage * L::kStageA, mA, bar, kb * BK, a_row);
+          tma_load_3d_pair(sB + stage * L::kStageB, &tmB, bar, kb * BK, b_row, g);
+          ++armed;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && rank == 0) {
+        for (int i = 0; i < STAGES && i < armed; ++i) {
+          stage = (stage + STAGES - 1) % STAGES;
+          if (stage == STAGES - 1) phase ^= 1;
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&full[stage], phase) && global_timer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer (first CTA of the pair) =================
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                                  ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BMT >> 4) << 24);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; ok && tile < total; tile += npairs, ++it) {
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], aph ^ 1, s_abort, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, s_abort, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + stage * L::kStageA);
+          const uint32_t b0 = smem_u32(sB + stage * L::kStageB);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            mma_bf16_pair(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), kIdesc,
+                          (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit_pair_both(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) mma_commit_pair_both(&tfull[acc]);
+      }
+      if (!ok) {
+        mma_commit_pair_local(drain);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ================= epilogue (warps 2..5 of both CTAs) =================
+    const int q = warp & 3;
+    uint8_t* stg = staging + (warp - 2) * kStagingPerWarp;
+    const uint32_t tempty_first = map_to_cta(smem_u32(&tempty[0]), 0);
+    int it = 0;
+    for (int tile = pair; tile < total; tile += npairs, ++it) {
+      int g, m_blk, n_blk;
+      decode_tile<BMT, BN>(tile, s_start, G, nt, g, m_blk, n_blk);
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      const bool ready = mbar_wait(&tfull[acc], aph, s_abort, p.status);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tc_fence_after();
+      const bool sh = g >= p.n_routed;
+      const int cnt = sh ? p.shared_rows : p.offsets[g + 1] - p.offsets[g];
+      const int64_t out_row0 = (int64_t)(sh ? p.shared_out_row0 : p.offsets[g]) + m_blk * BMT;
+      const int rows_valid = min(BMT, cnt - m_blk * BMT);
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      epilogue_warp<BN, EPI>(p, t_row, stg, lane, n_blk, out_row0, (int)rank * 128 + q * 32,
+                             rows_valid, [&] {
+                               tc_fence_before();
+                               __syncwarp();
+                               if (lane == 0) mbar_arrive_cluster(tempty_first + 8u * (uint32_t)acc);
+                             });
+    }
+  }
+
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the other may still signal its barriers
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(2 * BN));
   }
 }
@@ -535,15 +848,7 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
-template <int BN, int EPI, int STAGES>
-cudaError_t launch_t(const GroupedGemm& g, const CUtensorMap& mA, const CUtensorMap& mAs,
-                     const CUtensorMap& mB, cudaStream_t stream, int grid) {
-  using L = Layout<BN, STAGES>;
-  auto kern = grouped_gemm_kernel<BN, EPI, STAGES>;
-  const int groups = g.n_routed + g.has_shared;
-  const size_t smem = L::bytes(groups);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+Args make_args(const GroupedGemm& g) {
   Args a;
   a.offsets = g.offsets;
   a.n_routed = g.n_routed;
@@ -559,8 +864,43 @@ cudaError_t launch_t(const GroupedGemm& g, const CUtensorMap& mA, const CUtensor
   a.out = g.out;
   a.ld_out = g.ld_out;
   a.status = g.status;
-  kern<<<grid, kThreads, smem, stream>>>(mA, mAs, mB, a);
+  return a;
+}
+
+template <int BN, int EPI, int STAGES>
+cudaError_t launch_t(const GroupedGemm& g, const CUtensorMap& mA, const CUtensorMap& mAs,
+                     const CUtensorMap& mB, cudaStream_t stream, int grid) {
+  auto kern = grouped_gemm_kernel<BN, EPI, STAGES>;
+  const size_t smem = Layout<BN, STAGES>::bytes(g.n_routed + g.has_shared);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, stream>>>(mA, mAs, mB, make_args(g));
   return cudaGetLastError();
+}
+
+template <int EPI, int STAGES>
+cudaError_t launch_2sm(const GroupedGemm& g, const CUtensorMap& mA, const CUtensorMap& mAs,
+                       const CUtensorMap& mB, cudaStream_t stream, int pairs) {
+  auto kern = grouped_gemm_2sm_kernel<EPI, STAGES>;
+  const size_t smem = Layout2<STAGES>::bytes(g.n_routed + g.has_shared);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<2 * pairs, kThreads, smem, stream>>>(mA, mAs, mB, make_args(g));
+  return cudaGetLastError();
+}
+
+// Which kernel a bf16 grouped GEMM uses.  The 2-SM kernel tiles 256 rows per group, so it
+// pays off when groups are large; small groups keep the 1-SM kernel's 128-row tiles.
+// MOE_B200_GEMM_PATH=1sm|2sm overrides the choice (used by the tests to cover both kernels).
+bool use_two_sm(const GroupedGemm& g) {
+  if (g.epilogue == kEpiStoreF32) return false;
+  if (const char* env = std::getenv("MOE_B200_GEMM_PATH")) {
+    if (std::strcmp(env, "1sm") == 0) return false;
+    if (std::strcmp(env, "2sm") == 0) return true;
+  }
+  const int groups = g.n_routed + g.has_shared;
+  const int64_t rows = (g.n_routed > 0 ? g.max_rows_routed : 0) + (g.has_shared ? g.shared_rows : 0);
+  return rows >= 1024LL * groups;
 }
 
 }  // namespace tc
@@ -576,7 +916,8 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
   } else {
     BN = 256;
   }
-  const int box_b = (g.epilogue == kEpiSwiglu) ? BN / 2 : BN;
+  const bool two_sm = use_two_sm(g);
+  const int box_b = two_sm ? 128 : (g.epilogue == kEpiSwiglu) ? BN / 2 : BN;
   CUtensorMap mA, mAs, mB;
   const void* a_ptr = g.a != nullptr ? g.a : g.a_shared;
   const int64_t a_rows = g.a != nullptr ? g.rows_a : g.rows_a_shared;
@@ -596,6 +937,17 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
   const int64_t bound = mtiles * nt;
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), bound));
   ++*launches;
+  if (two_sm) {
+    int64_t mt2 = 0;
+    if (g.n_routed > 0) mt2 += (g.max_rows_routed + 255) / 256 + g.n_routed;
+    if (g.has_shared) mt2 += (g.shared_rows + 255) / 256;
+    const int pairs = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms() / 2, mt2 * nt));
+    switch (g.epilogue) {
+      case kEpiSwiglu: return launch_2sm<kEpiSwiglu, 6>(g, mA, mAs, mB, stream, pairs);
+      case kEpiRelu: return launch_2sm<kEpiRelu, 6>(g, mA, mAs, mB, stream, pairs);
+      default: return launch_2sm<kEpiStoreBf16, 6>(g, mA, mAs, mB, stream, pairs);
+    }
+  }
   switch (g.epilogue) {
     case kEpiSwiglu: return launch_t<256, kEpiSwiglu, 4>(g, mA, mAs, mB, stream, grid);
     case kEpiRelu: return launch_t<256, kEpiRelu, 4>(g, mA, mAs, mB, stream, grid);

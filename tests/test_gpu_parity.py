@@ -180,8 +180,11 @@ FFN_CASES = [
 ]
 
 
+@pytest.mark.parametrize("path", ["1sm", "2sm"])
 @pytest.mark.parametrize("N,d,E,k,F,S,act,clamp", FFN_CASES)
-def test_expert_ffn(N, d, E, k, F, S, act, clamp):
+def test_expert_ffn(N, d, E, k, F, S, act, clamp, path, monkeypatch):
+    # both grouped-GEMM kernels (1-SM 128-row tiles, 2-SM 256-row tiles) on every case
+    monkeypatch.setenv("MOE_B200_GEMM_PATH", path)
     shape = W.LayerShape("t", N=N, d=d, E=E, k=k, F=F, n_shared=S, act=act, clamp=clamp,
                          w_std=0.08, seed=N + d)
     t = W.make_inputs(shape, device="cuda")
@@ -343,6 +346,15 @@ class _LazyF64:
 def test_forward_small_shapes_all_tokens():
     for name, N in (("mixtral-n16", 16), ("dsv3-n64", 64), ("v41flash-n64", 64)):
         _forward_case(name, N=N)
+
+
+def test_forward_large_groups_take_the_2sm_kernel(monkeypatch):
+    # 4096 tokens, 8 experts, top-2: about 1024 rows per expert, so the automatic choice is
+    # the 2-SM kernel; the forced 1-SM run must give the same layer within the bar
+    monkeypatch.delenv("MOE_B200_GEMM_PATH", raising=False)
+    _forward_case("mixtral-n4096", sample=np.r_[0:8, 4090:4096])
+    monkeypatch.setenv("MOE_B200_GEMM_PATH", "1sm")
+    _forward_case("mixtral-n4096", sample=np.r_[0:8, 4090:4096])
 
 
 def test_forward_capacity_configs_reduced():

@@ -46,7 +46,20 @@ def parse_args():
     p.add_argument("--workload", default="mixtral-n16384", choices=sorted(W.PRESETS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--tokens", type=int, default=None,
+                   help="override the workload's token count (profiling a smaller case)")
+    p.add_argument("--experts", type=int, default=None,
+                   help="override the workload's routed expert count (profiling a smaller case)")
     return p.parse_args()
+
+
+def workload_shape(args):
+    shape = W.PRESETS[args.workload]
+    if args.tokens is not None:
+        shape = shape.replace(N=args.tokens)
+    if args.experts is not None:
+        shape = shape.replace(E=args.experts)
+    return shape
 
 
 # ------------------------------------------------------------------------------------------
@@ -216,7 +229,7 @@ def run_ours(args):
 
     world, rank, local = dist_init(args.gpus)
     torch.cuda.set_device(local)
-    shape = W.PRESETS[args.workload]
+    shape = workload_shape(args)
     t = make_replica(shape, rank)
     layer = MoELayer.from_workload(shape, t)
     x, mod = t["x"], t.get("modality")
@@ -240,8 +253,10 @@ def run_ours(args):
     nat.moe_profile_begin(args.steps)
     with ClockSampler(local) as clk:
         ev0.record(stream)
+        h0 = time.perf_counter()
         for _ in range(args.steps):
             layer.forward(x, modality=mod, y=y)
+        host_us = (time.perf_counter() - h0) * 1e6 / args.steps
         ev1.record(stream)
         torch.cuda.synchronize()
     barrier(world)
@@ -323,6 +338,7 @@ def run_ours(args):
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": shape.N * shape.d * el,
                 "d2h_bytes_per_step": shape.N * shape.d * el},
         "gpu_launches": per_step_launches * args.steps,
+        "host_enqueue_us_per_step": round(host_us, 1),
         "clocks": clocks,
         "cpu_baseline": cpu,
     }
@@ -390,7 +406,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    shape = W.PRESETS[args.workload]
+    shape = workload_shape(args)
     t = W.make_inputs(shape, device="cuda" if torch.cuda.is_available() else "cpu")
     import oracle as O
     inp = _oracle_inputs(shape, t)

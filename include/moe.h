@@ -169,6 +169,28 @@ MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const void*
                        void* y, const moe_route_out* route_out, void* ws,
                        moe_stream_t stream);
 
+/* The layer with forced (replayed) routing: caller-supplied ids [N][k] and gates [N][k]
+ * replace the router, the scores and the top-k; capacity, permutation, expert FFNs, the
+ * shared expert and the combine run as in moe_forward ("Le groupe d'experts (MoE)",
+ * exercise "Hard": record the experts that fired, force the same routing later).  ids are
+ * checked on the device: an id outside [0, E) or repeated within a token is dropped and
+ * reported as MOE_ERR_INVALID_INPUT by moe_check_status.  route_out may carry counts,
+ * demand, drop_mask and offsets outputs (its logits, ids and gates members are ignored). */
+MOE_API moe_status moe_forward_routed(const moe_config* cfg, const void* x, const int32_t* ids,
+                                      const float* gates, const void* W_gu, const void* W_down,
+                                      void* y, const moe_route_out* route_out, void* ws,
+                                      moe_stream_t stream);
+
+/* Hash router ("Le groupe d'experts (MoE)", exercise "Medium": deterministic, not learned):
+ * for token id t (token_ids [N], int32), expert e's key is fmix32(t * 0x9E3779B1 + e) with
+ * 32-bit wrap-around, fmix32 being MurmurHash3's finaliser; the k largest keys are selected
+ * (descending) and every gate is 1/k.  Then capacity and counts as in moe_route.
+ * Outputs: ids [N][k], gates [N][k], counts [E], demand [E], drop_mask [N][k] (the last three
+ * may be NULL).  cfg->score_fn, renorm and n_bias_sets are not used. */
+MOE_API moe_status moe_route_hash(const moe_config* cfg, const int32_t* token_ids, int32_t* ids,
+                                  float* gates, int32_t* counts, int32_t* demand,
+                                  uint8_t* drop_mask, void* ws, moe_stream_t stream);
+
 /* moe_forward with x_host and y_host in HOST memory (pinned for full copy speed): copies
  * x to the workspace, runs the layer, copies y back and synchronises the stream.
  * Weights, bias, modality and logit_offset are device pointers as in moe_forward. */

@@ -68,6 +68,8 @@ lib.moe_forward.argtypes = [_cfgp] + [_vp] * 11
 lib.moe_forward_host.argtypes = [_cfgp] + [_vp] * 10
 lib.moe_check_status.argtypes = [_vp, _vp]
 lib.moe_route_static.argtypes = [_cfgp] + [_vp] * 10
+lib.moe_forward_routed.argtypes = [_cfgp] + [_vp] * 9
+lib.moe_route_hash.argtypes = [_cfgp] + [_vp] * 8
 lib.moe_profile_begin.argtypes = [_i32]
 lib.moe_profile_begin.restype = ctypes.c_int
 lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)]
@@ -75,13 +77,15 @@ lib.moe_profile_end.restype = _i32
 lib.moe_last_error.restype = ctypes.c_char_p
 lib.moe_last_launch_count.restype = _i32
 for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
-           "moe_forward", "moe_forward_host", "moe_check_status", "moe_route_static"):
+           "moe_forward", "moe_forward_host", "moe_check_status", "moe_route_static",
+           "moe_forward_routed", "moe_route_hash"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
             "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
             "moe_check_status", "moe_profile_begin", "moe_profile_end", "moe_last_error",
-            "moe_last_launch_count", "moe_route_static")
+            "moe_last_launch_count", "moe_route_static", "moe_forward_routed",
+            "moe_route_hash")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -205,6 +209,28 @@ def moe_forward(cfg, *, x, W_g, W_gu, W_down, y, logit_offset=None, bias=None, m
                          ctypes.byref(ro) if ro is not None else None, _ptr(ws),
                          _stream(stream))
     _check(st, "moe_forward")
+
+
+def moe_forward_routed(cfg, *, x, ids, gates, W_gu, W_down, y, route_out: Optional[dict] = None,
+                       ws, stream=None):
+    """The layer with caller-supplied (forced or replayed) ids and gates."""
+    ro = None
+    if route_out:
+        ro = moe_route_out(*[_ptr(route_out.get(n)) for n, _ in moe_route_out._fields_])
+    st = lib.moe_forward_routed(ctypes.byref(cfg), _ptr(x), _ptr(ids), _ptr(gates), _ptr(W_gu),
+                                _ptr(W_down), _ptr(y),
+                                ctypes.byref(ro) if ro is not None else None, _ptr(ws),
+                                _stream(stream))
+    _check(st, "moe_forward_routed")
+
+
+def moe_route_hash(cfg, *, token_ids, ids, gates, counts=None, demand=None, drop_mask=None, ws,
+                   stream=None):
+    """Deterministic hash routing of token ids, then capacity and counts."""
+    st = lib.moe_route_hash(ctypes.byref(cfg), _ptr(token_ids), _ptr(ids), _ptr(gates),
+                            _ptr(counts), _ptr(demand), _ptr(drop_mask), _ptr(ws),
+                            _stream(stream))
+    _check(st, "moe_route_hash")
 
 
 def moe_forward_host(cfg, *, x_host, W_g, W_gu, W_down, y_host, logit_offset=None, bias=None,

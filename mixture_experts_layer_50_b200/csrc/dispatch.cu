@@ -178,11 +178,15 @@ cudaError_t launch_dispatch_scan(const int32_t* tile_hist, int64_t N, int E, int
                                  int32_t* offsets, cudaStream_t stream, int* launches) {
   const int tiles = (int)((N + kRankTile - 1) / kRankTile);
   const size_t smem = sizeof(int32_t) * 32 * (size_t)E;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaFuncSetAttribute(dispatch_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         32 * 1024 * (int)sizeof(int32_t));
-    attr_set = true;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(dispatch_scan_kernel,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               32 * 1024 * (int)sizeof(int32_t));
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
   ++*launches;
   dispatch_scan_kernel<<<1, 1024, smem, stream>>>(tile_hist, tiles, E, C, tile_base, demand,

@@ -30,6 +30,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -841,11 +842,34 @@ bool make_map(CUtensorMap* m, const void* ptr, int64_t K, int64_t rows, int64_t 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+constexpr int kMaxDev = 64;
+
 int num_sms() {
-  int dev = 0, n = 0;
+  static int cached[kMaxDev] = {};
+  int dev = 0;
   cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
+  if (dev < 0 || dev >= kMaxDev) dev = 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
+// Opt a kernel into the largest dynamic shared memory once per device (the per-launch size is
+// always below it), so launches do not repeat the attribute call.  `done` must be distinct
+// for every kernel: each launch_* instantiation passes its own.
+template <typename Kernel>
+cudaError_t allow_max_smem(Kernel kern, bool (&done)[kMaxDev]) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < kMaxDev && done[dev]) return cudaSuccess;
+  int optin = 0;
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+  if (e == cudaSuccess && dev >= 0 && dev < kMaxDev) done[dev] = true;
+  return e;
 }
 
 Args make_args(const GroupedGemm& g) {
@@ -872,7 +896,8 @@ cudaError_t launch_t(const GroupedGemm& g, const CUtensorMap& mA, const CUtensor
                      const CUtensorMap& mB, cudaStream_t stream, int grid) {
   auto kern = grouped_gemm_kernel<BN, EPI, STAGES>;
   const size_t smem = Layout<BN, STAGES>::bytes(g.n_routed + g.has_shared);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static bool done[kMaxDev] = {};
+  const cudaError_t e = allow_max_smem(kern, done);
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, stream>>>(mA, mAs, mB, make_args(g));
   return cudaGetLastError();
@@ -883,7 +908,8 @@ cudaError_t launch_2sm(const GroupedGemm& g, const CUtensorMap& mA, const CUtens
                        const CUtensorMap& mB, cudaStream_t stream, int pairs) {
   auto kern = grouped_gemm_2sm_kernel<EPI, STAGES>;
   const size_t smem = Layout2<STAGES>::bytes(g.n_routed + g.has_shared);
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static bool done[kMaxDev] = {};
+  const cudaError_t e = allow_max_smem(kern, done);
   if (e != cudaSuccess) return e;
   kern<<<2 * pairs, kThreads, smem, stream>>>(mA, mAs, mB, make_args(g));
   return cudaGetLastError();
@@ -892,15 +918,37 @@ cudaError_t launch_2sm(const GroupedGemm& g, const CUtensorMap& mA, const CUtens
 // Which kernel a bf16 grouped GEMM uses.  The 2-SM kernel tiles 256 rows per group, so it
 // pays off when groups are large; small groups keep the 1-SM kernel's 128-row tiles.
 // MOE_B200_GEMM_PATH=1sm|2sm overrides the choice (used by the tests to cover both kernels).
+const char* path_override() { return std::getenv("MOE_B200_GEMM_PATH"); }
+
 bool use_two_sm(const GroupedGemm& g) {
   if (g.epilogue == kEpiStoreF32) return false;
-  if (const char* env = std::getenv("MOE_B200_GEMM_PATH")) {
-    if (std::strcmp(env, "1sm") == 0) return false;
+  if (const char* env = path_override()) {
+    if (std::strncmp(env, "1sm", 3) == 0) return false;
     if (std::strcmp(env, "2sm") == 0) return true;
   }
   const int groups = g.n_routed + g.has_shared;
   const int64_t rows = (g.n_routed > 0 ? g.max_rows_routed : 0) + (g.has_shared ? g.shared_rows : 0);
   return rows >= 1024LL * groups;
+}
+
+// N width of the 1-SM kernel's tiles.  256 keeps the tensor pipe busiest; when nearly every
+// group fits one 128-row tile the launch streams weights (memory-bound) and the tile count
+// is small, so 128-wide tiles are taken when they leave a clearly smaller idle tail on the
+// last wave.  MOE_B200_GEMM_PATH=1sm128 forces 128.
+int pick_bn_1sm(const GroupedGemm& g) {
+  if (const char* env = path_override())
+    if (std::strcmp(env, "1sm128") == 0) return 128;
+  const int groups = g.n_routed + g.has_shared;
+  const int64_t rows = (g.n_routed > 0 ? g.max_rows_routed : 0) + (g.has_shared ? g.shared_rows : 0);
+  if (rows >= 128LL * groups) return 256;
+  int64_t mtiles = std::min<int64_t>(g.n_routed, g.max_rows_routed);
+  if (g.has_shared) mtiles += (g.shared_rows + BM - 1) / BM;
+  auto tail_eff = [&](int bn) {
+    const int out = g.epilogue == kEpiSwiglu ? bn / 2 : bn;
+    const double waves = (double)(mtiles * ((g.n_out + out - 1) / out)) / num_sms();
+    return waves / std::ceil(waves);
+  };
+  return tail_eff(128) > tail_eff(256) + 0.02 ? 128 : 256;
 }
 
 }  // namespace tc
@@ -911,12 +959,12 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
   const int groups = g.n_routed + g.has_shared;
   if (groups == 0) return cudaSuccess;
   int BN;
+  const bool two_sm = use_two_sm(g);
   if (g.epilogue == kEpiStoreF32) {
     BN = g.n_out <= 32 ? 32 : g.n_out <= 64 ? 64 : g.n_out <= 128 ? 128 : (g.n_out % 256 == 0 || g.n_out > 384) ? 256 : 128;
   } else {
-    BN = 256;
+    BN = two_sm ? 256 : pick_bn_1sm(g);
   }
-  const bool two_sm = use_two_sm(g);
   const int box_b = two_sm ? 128 : (g.epilogue == kEpiSwiglu) ? BN / 2 : BN;
   CUtensorMap mA, mAs, mB;
   const void* a_ptr = g.a != nullptr ? g.a : g.a_shared;
@@ -946,6 +994,13 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
       case kEpiSwiglu: return launch_2sm<kEpiSwiglu, 6>(g, mA, mAs, mB, stream, pairs);
       case kEpiRelu: return launch_2sm<kEpiRelu, 6>(g, mA, mAs, mB, stream, pairs);
       default: return launch_2sm<kEpiStoreBf16, 6>(g, mA, mAs, mB, stream, pairs);
+    }
+  }
+  if (BN == 128 && g.epilogue != kEpiStoreF32) {
+    switch (g.epilogue) {
+      case kEpiSwiglu: return launch_t<128, kEpiSwiglu, 6>(g, mA, mAs, mB, stream, grid);
+      case kEpiRelu: return launch_t<128, kEpiRelu, 6>(g, mA, mAs, mB, stream, grid);
+      default: return launch_t<128, kEpiStoreBf16, 6>(g, mA, mAs, mB, stream, grid);
     }
   }
   switch (g.epilogue) {

@@ -14,6 +14,10 @@ cudaError_t launch_route_topk(const float* logits, int64_t N, int E, int k, int 
                               const uint8_t* modality, int32_t* ids, float* gates,
                               int* status, cudaStream_t stream, int* launches);
 
+// Hash router: ids = the k experts with the largest fmix32(token_id * 0x9E3779B1 + e), gates 1/k.
+cudaError_t launch_route_hash(const int32_t* token_ids, int64_t N, int E, int k, int32_t* ids,
+                              float* gates, cudaStream_t stream, int* launches);
+
 // ---- dispatch (dispatch.cu) -----------------------------------------------------------
 // Pass 1: per token tile, ranks of each assignment among the tile's earlier tokens that
 // chose the same expert, and the tile's per-expert histogram.  Assignments whose

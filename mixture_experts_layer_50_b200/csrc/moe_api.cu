@@ -502,6 +502,62 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* W_g,
   return MOE_OK;
 }
 
+moe_status moe_forward_routed(const moe_config* cfg, const void* x, const int32_t* ids,
+                              const float* gates, const void* W_gu, const void* W_down,
+                              void* y, const moe_route_out* route_out, void* ws,
+                              moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  if (ids == nullptr || gates == nullptr) return fail(MOE_ERR_INVALID_ARG, "ids and gates are required");
+  MOE_TRY(need(x, "x"));
+  MOE_TRY(need(W_gu, "W_gu"));
+  MOE_TRY(need(W_down, "W_down"));
+  MOE_TRY(need(y, "y"));
+  const moe_config& c = *cfg;
+  const Ws L = layout(c);
+  cudaStream_t st = (cudaStream_t)stream;
+  const moe_route_out* ro = route_out;
+  int32_t* counts = (ro && ro->counts) ? ro->counts : at<int32_t>(ws, L.counts);
+  int32_t* demand = (ro && ro->demand) ? ro->demand : at<int32_t>(ws, L.demand);
+  uint8_t* drop = (ro && ro->drop_mask) ? ro->drop_mask : at<uint8_t>(ws, L.drop_mask);
+  int32_t* offsets = (ro && ro->offsets) ? ro->offsets : at<int32_t>(ws, L.offsets);
+  void* xp = at<char>(ws, L.xp);
+  void* ye = at<char>(ws, L.ye);
+  int launches = 0;
+  MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, c.capacity, demand, counts, offsets,
+                         at<int32_t>(ws, L.slot_row), at<int32_t>(ws, L.row_token), drop, x, xp,
+                         st, &launches));
+  MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, &launches));
+  MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, &launches));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_route_hash(const moe_config* cfg, const int32_t* token_ids, int32_t* ids,
+                          float* gates, int32_t* counts, int32_t* demand, uint8_t* drop_mask,
+                          void* ws, moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  if (token_ids == nullptr || ids == nullptr || gates == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "token_ids, ids and gates are required");
+  const moe_config& c = *cfg;
+  const Ws L = layout(c);
+  cudaStream_t st = (cudaStream_t)stream;
+  int launches = 0;
+  MOE_CUDA(moe::launch_route_hash(token_ids, c.N, c.E, c.k, ids, gates, st, &launches),
+           "hash routing");
+  MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, c.capacity,
+                         demand != nullptr ? demand : at<int32_t>(ws, L.demand),
+                         counts != nullptr ? counts : at<int32_t>(ws, L.counts),
+                         at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.slot_row), nullptr,
+                         drop_mask != nullptr ? drop_mask : at<uint8_t>(ws, L.drop_mask),
+                         nullptr, nullptr, st, &launches));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
 moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const void* W_g,
                             const float* logit_offset, const float* bias,
                             const uint8_t* modality, const void* W_gu, const void* W_down,

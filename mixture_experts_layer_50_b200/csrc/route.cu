@@ -166,7 +166,89 @@ cudaError_t launch_j(const float* logits, int64_t N, int E, int k, int score_fn,
   return cudaGetLastError();
 }
 
+// MurmurHash3's 32-bit finaliser (A. Appleby, public domain): a bijection that mixes every
+// input bit into every output bit.
+__device__ __forceinline__ uint32_t fmix32(uint32_t h) {
+  h ^= h >> 16;
+  h *= 0x85ebca6bu;
+  h ^= h >> 13;
+  h *= 0xc2b2ae35u;
+  h ^= h >> 16;
+  return h;
+}
+
+// Hash router ("Le groupe d'experts (MoE)", exercise "Medium": deterministic, not learned).
+// Expert e's key for token id t is fmix32(t * 0x9E3779B1 + e); the k largest keys win (they
+// are distinct within a token), listed by descending key; every gate is 1/k.
+template <int J>
+__global__ void __launch_bounds__(256) hash_topk_kernel(const int32_t* __restrict__ token_ids,
+                                                        int64_t N, int E, int k,
+                                                        int32_t* __restrict__ ids,
+                                                        float* __restrict__ gates) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= N) return;
+  const uint32_t base = (uint32_t)token_ids[t] * 0x9E3779B1u;
+  uint32_t key[J];
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = e < E ? fmix32(base + (uint32_t)e) : 0u;
+  }
+  uint32_t taken = 0;
+  int my_e = -1;
+  for (int r = 0; r < k; ++r) {
+    uint32_t bk = 0;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && !((taken >> j) & 1u) && (be == 0x7fffffff || key[j] > bk)) {
+        bk = key[j];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint32_t ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (oe != 0x7fffffff && (be == 0x7fffffff || ok > bk || (ok == bk && oe < be))) {
+        bk = ok;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == r) my_e = be;
+  }
+  if (lane < k) {
+    ids[t * k + lane] = my_e;
+    gates[t * k + lane] = 1.0f / (float)k;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_route_hash(const int32_t* token_ids, int64_t N, int E, int k, int32_t* ids,
+                              float* gates, cudaStream_t stream, int* launches) {
+  if (N == 0) return cudaSuccess;
+  ++*launches;
+  const int J = (E + 31) / 32;
+  const unsigned blocks = (unsigned)((N * 32 + 255) / 256);
+#define MOE_HASH_CASE(JJ) \
+  if (J <= JJ) {          \
+    hash_topk_kernel<JJ><<<blocks, 256, 0, stream>>>(token_ids, N, E, k, ids, gates); \
+    return cudaGetLastError(); \
+  }
+  MOE_HASH_CASE(1)
+  MOE_HASH_CASE(2)
+  MOE_HASH_CASE(4)
+  MOE_HASH_CASE(8)
+  MOE_HASH_CASE(12)
+  MOE_HASH_CASE(16)
+  MOE_HASH_CASE(32)
+#undef MOE_HASH_CASE
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_route_topk(const float* logits, int64_t N, int E, int k, int score_fn,
                               int renorm, const float* bias, int n_bias_sets,

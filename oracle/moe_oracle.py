@@ -271,18 +271,26 @@ def expert_ffn(xr, W_gu_e, W_down_e, act=SWIGLU, clamp=0.0):
 # ---------------------------------------------------------------------------
 def forward(x, W_g, W_gu, W_down, *, k, E, score_fn=SOFTMAX, renorm=1, act=SWIGLU,
             clamp=0.0, n_shared=0, bias=None, modality=None, logit_offset=None,
-            C=0, logits=None, tokens=None):
+            C=0, logits=None, tokens=None, ids=None, gates=None):
     """y[t] = sum_{kept j} g[t,j] FFN_{ids[t,j]}(x_t) + sum_shared FFN_s(x_t), float64.
 
     ``logits`` (float32 [N][E]) replaces the router projection when given.
+    ``ids`` and ``gates`` ([N][k]) replace the whole router when given: forced or
+    replayed routing ("Le groupe d'experts (MoE)", exercise "Hard": record the experts
+    that fired and force the same routing later); capacity still applies.
     ``tokens`` restricts the expert work and the returned rows to those token
     indices; routing and capacity still see every token.
     Returns (y [len(tokens) or N][d] float64, route dict).
     """
     x64 = np.asarray(x, np.float64)
     N = x64.shape[0]
-    z = router_logits(x64, W_g, logit_offset) if logits is None else np.asarray(logits, np.float32)
-    ids, gates = route(z, k, score_fn, renorm, bias, modality)
+    if ids is not None:
+        z = None
+        ids = np.asarray(ids, np.int32)
+        gates = np.asarray(gates, np.float64)
+    else:
+        z = router_logits(x64, W_g, logit_offset) if logits is None else np.asarray(logits, np.float32)
+        ids, gates = route(z, k, score_fn, renorm, bias, modality)
     disp = dispatch(ids, E, C)
     keep = disp["drop_mask"] == 0
     tok = np.arange(N) if tokens is None else np.asarray(tokens, np.int64)
@@ -299,6 +307,31 @@ def forward(x, W_g, W_gu, W_down, *, k, E, score_fn=SOFTMAX, renorm=1, act=SWIGL
     return y, info
 
 
+def fmix32(h):
+    """The 32-bit finaliser of MurmurHash3 (A. Appleby, public domain): a bijection on
+    32-bit integers that mixes every input bit into every output bit."""
+    h = np.asarray(h, np.uint64) & 0xFFFFFFFF
+    h ^= h >> 16
+    h = (h * 0x85EBCA6B) & 0xFFFFFFFF
+    h ^= h >> 13
+    h = (h * 0xC2B2AE35) & 0xFFFFFFFF
+    h ^= h >> 16
+    return h.astype(np.uint32)
+
+
+def hash_route(token_ids, E, k):
+    """Hash router ("Le groupe d'experts (MoE)", exercise "Medium": deterministic, not
+    learned).  Reading: expert e's key for token id t is fmix32(t * 0x9E3779B1 + e) (32-bit
+    wrap-around); the k largest keys are selected, listed by descending key (the keys of one
+    token are distinct because fmix32 is a bijection); every selected expert gets the gate 1/k.
+    Returns (ids [N][k] int32, gates [N][k] float64)."""
+    t = np.asarray(token_ids, np.int64).astype(np.uint64) & 0xFFFFFFFF
+    e = np.arange(E, dtype=np.uint64)
+    keys = fmix32((t[:, None] * 0x9E3779B1 + e[None, :]) & 0xFFFFFFFF).astype(np.int64)
+    ids = np.argsort(-keys, axis=1, kind="stable")[:, :k].astype(np.int32)
+    return ids, np.full(ids.shape, 1.0 / k)
+
+
 def dense_mixture(x, W_g, W_gu, W_down, *, E, act=SWIGLU, clamp=0.0, logit_offset=None):
     """The dense limit k = E with softmax: y = sum_e p_e FFN_e(x) (P5 "Практика")."""
     x64 = np.asarray(x, np.float64)
@@ -311,5 +344,6 @@ def dense_mixture(x, W_g, W_gu, W_down, *, E, act=SWIGLU, clamp=0.0, logit_offse
 
 __all__ = ["exp_f32", "sigmoid_f32", "router_logits", "softmax64", "selection_keys",
            "topk_ids", "gates_for", "route", "capacity", "dispatch", "load_fractions",
-           "silu", "expert_ffn", "forward", "dense_mixture", "SOFTMAX", "SIGMOID",
+           "silu", "expert_ffn", "forward", "dense_mixture", "fmix32", "hash_route",
+           "SOFTMAX", "SIGMOID",
            "SWIGLU", "RELU"]

@@ -180,10 +180,10 @@ FFN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["1sm", "2sm"])
+@pytest.mark.parametrize("path", ["1sm", "1sm128", "2sm"])
 @pytest.mark.parametrize("N,d,E,k,F,S,act,clamp", FFN_CASES)
 def test_expert_ffn(N, d, E, k, F, S, act, clamp, path, monkeypatch):
-    # both grouped-GEMM kernels (1-SM 128-row tiles, 2-SM 256-row tiles) on every case
+    # every grouped-GEMM variant (1-SM 128x256 and 128x128 tiles, 2-SM 256x256) on every case
     monkeypatch.setenv("MOE_B200_GEMM_PATH", path)
     shape = W.LayerShape("t", N=N, d=d, E=E, k=k, F=F, n_shared=S, act=act, clamp=clamp,
                          w_std=0.08, seed=N + d)

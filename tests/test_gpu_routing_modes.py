@@ -1,0 +1,104 @@
+"""GPU parity of the routing variants: forced (replayed) routing and the hash router
+("Le groupe d'experts (MoE)", exercises "Hard" and "Medium")."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from gpu_util import assert_close_layer, check_status, dev, f64, host
+from mixture_experts_layer_50_b200 import _native as nat
+from mixture_experts_layer_50_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _needs_cuda(cuda_dev):
+    yield
+
+
+def _route_out(N, E, k):
+    return dict(ids=torch.empty((N, k), dtype=torch.int32, device="cuda"),
+                gates=torch.empty((N, k), dtype=torch.float32, device="cuda"),
+                counts=torch.empty(E, dtype=torch.int32, device="cuda"),
+                demand=torch.empty(E, dtype=torch.int32, device="cuda"),
+                drop_mask=torch.empty((N, k), dtype=torch.uint8, device="cuda"),
+                offsets=torch.empty(E + 1, dtype=torch.int32, device="cuda"))
+
+
+def test_replayed_routing_reproduces_the_forward_bit_for_bit():
+    shape = W.PRESETS["v41flash-n64"].replace(N=700, d=512, F=256, E=32, k=4)
+    t = W.make_inputs(shape, device="cuda")
+    C = O.capacity(shape.N, shape.k, shape.E, 1)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    ro = _route_out(shape.N, shape.E, shape.k)
+    y = torch.empty_like(t["x"])
+    nat.moe_forward(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y,
+                    bias=t["bias"], modality=t["modality"], route_out=ro, ws=ws)
+    check_status(ws)
+    # record, then force the same routing
+    y2 = torch.empty_like(y)
+    ro2 = {k_: torch.empty_like(ro[k_]) for k_ in ("counts", "demand", "drop_mask", "offsets")}
+    nat.moe_forward_routed(cfg, x=t["x"], ids=ro["ids"].clone(), gates=ro["gates"].clone(),
+                           W_gu=t["W_gu"], W_down=t["W_down"], y=y2, route_out=ro2, ws=ws)
+    check_status(ws)
+    assert torch.equal(y2, y)
+    for k_ in ro2:
+        assert torch.equal(ro2[k_], ro[k_]), k_
+    assert nat.moe_last_launch_count() == 6
+
+
+@pytest.mark.parametrize("C", [0, 40])
+def test_forced_routing_against_the_oracle(C):
+    shape = W.PRESETS["dsv3-n64"].replace(N=300, d=256, F=384, E=16, k=3)
+    t = W.make_inputs(shape, device="cuda")
+    rng = np.random.default_rng(5)
+    # arbitrary forced routing: k distinct experts per token, arbitrary positive gates
+    ids = np.stack([rng.permutation(shape.E)[:shape.k] for _ in range(shape.N)]).astype(np.int32)
+    gates = rng.uniform(0.1, 1.0, ids.shape).astype(np.float32)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    ro = {"drop_mask": torch.empty((shape.N, shape.k), dtype=torch.uint8, device="cuda")}
+    y = torch.empty_like(t["x"])
+    nat.moe_forward_routed(cfg, x=t["x"], ids=dev(ids), gates=dev(gates), W_gu=t["W_gu"],
+                           W_down=t["W_down"], y=y, route_out=ro, ws=ws)
+    check_status(ws)
+    ref, info = O.forward(f64(t["x"]), None, f64(t["W_gu"]), f64(t["W_down"]), k=shape.k,
+                          E=shape.E, n_shared=shape.n_shared, C=C, ids=ids,
+                          gates=gates.astype(np.float64))
+    np.testing.assert_array_equal(host(ro["drop_mask"]), info["drop_mask"])
+    assert_close_layer(host(y), ref)
+
+
+def test_forced_routing_reports_bad_ids():
+    shape = W.PRESETS["dsv3-n64"].replace(N=64, d=256, F=256, E=8, k=2)
+    t = W.make_inputs(shape, device="cuda")
+    ids = np.tile(np.array([[1, 2]], np.int32), (64, 1))
+    ids[5] = [8, 1]          # out of range: dropped
+    cfg = nat.config_from_shape(shape)
+    ws = nat.alloc_workspace(cfg)
+    y = torch.empty_like(t["x"])
+    nat.moe_forward_routed(cfg, x=t["x"], ids=dev(ids), gates=dev(np.full((64, 2), 0.5, np.float32)),
+                           W_gu=t["W_gu"], W_down=t["W_down"], y=y, ws=ws)
+    assert nat.moe_check_status(ws) == nat.MOE_ERR_INVALID_INPUT
+
+
+@pytest.mark.parametrize("N,E,k,C", [(1000, 64, 2, 0), (4097, 384, 6, 80), (33, 8, 1, 3)])
+def test_hash_router_bit_exact(N, E, k, C):
+    tok = np.random.default_rng(N).integers(0, 2**31 - 1, N).astype(np.int32)
+    cfg = nat.make_config(N, 64, E, k, 64, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    out = dict(ids=torch.empty((N, k), dtype=torch.int32, device="cuda"),
+               gates=torch.empty((N, k), dtype=torch.float32, device="cuda"),
+               counts=torch.empty(E, dtype=torch.int32, device="cuda"),
+               demand=torch.empty(E, dtype=torch.int32, device="cuda"),
+               drop_mask=torch.empty((N, k), dtype=torch.uint8, device="cuda"))
+    nat.moe_route_hash(cfg, token_ids=dev(tok), ws=ws, **out)
+    check_status(ws)
+    ids_o, gates_o = O.hash_route(tok, E, k)
+    d_o = O.dispatch(ids_o, E, C)
+    np.testing.assert_array_equal(host(out["ids"]), ids_o)
+    np.testing.assert_array_equal(host(out["gates"]), gates_o.astype(np.float32))
+    for name in ("counts", "demand", "drop_mask"):
+        np.testing.assert_array_equal(host(out[name]), d_o[name])

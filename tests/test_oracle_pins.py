@@ -391,3 +391,59 @@ def test_logit_offset_enters_selection_and_gates():
     ids, w = O.route(zz, 2)
     assert ids.tolist() == [[0, 1]]
     np.testing.assert_allclose(w[0], sp_softmax([1.5, 1.2]), rtol=1e-7)
+
+
+# --------------------------------------------------------------------------
+# forced (replayed) routing and the hash router ("Le groupe d'experts (MoE)", exercises)
+# --------------------------------------------------------------------------
+def test_forced_routing_reproduces_the_routed_layer_and_closed_forms():
+    rng = np.random.default_rng(21)
+    N, d, E, F = 30, 6, 5, 4
+    x, W_g, W_gu, W_down = _tiny_layer(rng, N, d, E, F, E + 1)
+    y, info = O.forward(x, W_g, W_gu, W_down, k=2, E=E, n_shared=1, C=11)
+    y2, info2 = O.forward(x, None, W_gu, W_down, k=2, E=E, n_shared=1, C=11,
+                          ids=info["ids"], gates=info["gates"])
+    np.testing.assert_array_equal(y2, y)
+    np.testing.assert_array_equal(info2["drop_mask"], info["drop_mask"])
+    # every token forced to expert 3 with gate 1 and no capacity: y = FFN_3(x) + FFN_shared(x)
+    ids = np.full((N, 1), 3, np.int32)
+    y3, _ = O.forward(x, None, W_gu, W_down, k=1, E=E, n_shared=1, ids=ids, gates=np.ones((N, 1)))
+    want = O.expert_ffn(x, W_gu[3], W_down[3]) + O.expert_ffn(x, W_gu[E], W_down[E])
+    np.testing.assert_allclose(y3, want, rtol=1e-13)
+    # and with capacity C the tokens after the C-th keep only the shared expert
+    y4, d4 = O.forward(x, None, W_gu, W_down, k=1, E=E, n_shared=1, ids=ids,
+                       gates=np.ones((N, 1)), C=7)
+    np.testing.assert_allclose(y4[:7], want[:7], rtol=1e-13)
+    np.testing.assert_allclose(y4[7:], O.expert_ffn(x[7:], W_gu[E], W_down[E]), rtol=1e-13)
+    assert d4["drop_mask"][:, 0].tolist() == [0] * 7 + [1] * (N - 7)
+
+
+def test_fmix32_is_a_bijection_with_fixed_points_of_the_definition():
+    v = np.arange(1 << 16, dtype=np.uint64) * 65537          # 65536 distinct 32-bit inputs
+    h = O.fmix32(v)
+    assert np.unique(h).size == v.size
+    assert int(O.fmix32(0)) == 0                             # every step maps 0 to 0
+    # one step written out with Python integers (shift-xor, multiply mod 2^32, ...)
+    a = 0xDEADBEEF
+    a ^= a >> 16
+    a = (a * 0x85EBCA6B) % 2**32
+    a ^= a >> 13
+    a = (a * 0xC2B2AE35) % 2**32
+    a ^= a >> 16
+    assert int(O.fmix32(0xDEADBEEF)) == a
+
+
+def test_hash_route_is_deterministic_distinct_uniform():
+    tok = np.arange(20000, dtype=np.int32) * 7 + 3
+    ids, g = O.hash_route(tok, 64, 2)
+    assert ids.shape == (20000, 2) and (ids[:, 0] != ids[:, 1]).all()
+    np.testing.assert_array_equal(g, 0.5)
+    ids2, _ = O.hash_route(tok, 64, 2)
+    np.testing.assert_array_equal(ids, ids2)
+    counts = np.bincount(ids.ravel(), minlength=64)
+    # uniform load: chi-square with 63 degrees of freedom stays far below 130
+    chi2 = ((counts - counts.mean()) ** 2 / counts.mean()).sum()
+    assert chi2 < 130, chi2
+    # the same token id always lands on the same experts, wherever it sits in the batch
+    ids3, _ = O.hash_route(tok[::-1], 64, 2)
+    np.testing.assert_array_equal(ids3[::-1], ids)

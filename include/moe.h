@@ -107,7 +107,7 @@ typedef struct {
 } moe_route_out;
 
 /* Bytes of device workspace a call with this configuration needs (0 on a bad config).
- * The size depends on N, d, E, k, F, n_shared and dtype only. */
+ * The size depends on N, d, E, k, F, n_shared, n_bias_sets and dtype only. */
 MOE_API size_t moe_workspace_size(const moe_config* cfg);
 
 /* Zero the workspace header (the device status word).  Call once after allocating. */
@@ -190,6 +190,28 @@ MOE_API moe_status moe_forward_routed(const moe_config* cfg, const void* x, cons
 MOE_API moe_status moe_route_hash(const moe_config* cfg, const int32_t* token_ids, int32_t* ids,
                                   float* gates, int32_t* counts, int32_t* demand,
                                   uint8_t* drop_mask, void* ws, moe_stream_t stream);
+
+/* Load-balancing statistics of a routed batch and the aux-loss-free bias update.
+ * ("Основы MoE", "Вспомогательный лосс Switch Transformer"; "Le groupe d'experts (MoE)",
+ * load-balance section; DeepSeek-V4.1-Flash page, "L'équilibrage de charge" and
+ * "l'équilibrage par modalité".)
+ *   logits [N][E] fp32 and ids [N][k] of the batch (e.g. moe_forward's route_out)
+ *   modality [N] uint8: the bias set of each token (required when n_bias_sets > 1)
+ *   f [E]      share of the assignments per expert (sums to 1)
+ *   P [E]      mean router probability per expert: softmax(z), or for sigmoid scoring the
+ *              affinities sigma(z) normalised to sum 1 per token
+ *   aux [1]    E * sum_i f_i P_i (1 when balanced, about E when collapsed; the Switch loss
+ *              is alpha times this)
+ *   set_load [max(1, n_bias_sets)][E] assignments per (bias set, expert)
+ *   bias [n_sets][E] in/out or NULL: each entry moves by +gamma when its expert's load is
+ *              below its set's mean load, -gamma when above, 0 when equal (the pages use
+ *              gamma = 0.001)
+ * Any of f, P, aux, set_load, bias may be NULL.  Deterministic (fixed summation order).
+ * At most 8 bias sets. */
+MOE_API moe_status moe_balance(const moe_config* cfg, const float* logits, const int32_t* ids,
+                               const uint8_t* modality, float* f, float* P, float* aux,
+                               int32_t* set_load, float* bias, float gamma, void* ws,
+                               moe_stream_t stream);
 
 /* moe_forward with x_host and y_host in HOST memory (pinned for full copy speed): copies
  * x to the workspace, runs the layer, copies y back and synchronises the stream.

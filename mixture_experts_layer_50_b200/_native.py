@@ -70,6 +70,7 @@ lib.moe_check_status.argtypes = [_vp, _vp]
 lib.moe_route_static.argtypes = [_cfgp] + [_vp] * 10
 lib.moe_forward_routed.argtypes = [_cfgp] + [_vp] * 9
 lib.moe_route_hash.argtypes = [_cfgp] + [_vp] * 8
+lib.moe_balance.argtypes = [_cfgp] + [_vp] * 8 + [ctypes.c_float, _vp, _vp]
 lib.moe_profile_begin.argtypes = [_i32]
 lib.moe_profile_begin.restype = ctypes.c_int
 lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)]
@@ -78,14 +79,14 @@ lib.moe_last_error.restype = ctypes.c_char_p
 lib.moe_last_launch_count.restype = _i32
 for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
            "moe_forward", "moe_forward_host", "moe_check_status", "moe_route_static",
-           "moe_forward_routed", "moe_route_hash"):
+           "moe_forward_routed", "moe_route_hash", "moe_balance"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
             "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
             "moe_check_status", "moe_profile_begin", "moe_profile_end", "moe_last_error",
             "moe_last_launch_count", "moe_route_static", "moe_forward_routed",
-            "moe_route_hash")
+            "moe_route_hash", "moe_balance")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -231,6 +232,15 @@ def moe_route_hash(cfg, *, token_ids, ids, gates, counts=None, demand=None, drop
                             _ptr(counts), _ptr(demand), _ptr(drop_mask), _ptr(ws),
                             _stream(stream))
     _check(st, "moe_route_hash")
+
+
+def moe_balance(cfg, *, logits, ids, modality=None, f=None, P=None, aux=None, set_load=None,
+                bias=None, gamma=0.001, ws, stream=None):
+    """Balance statistics (f, P, E sum f P, loads per bias set) and the +-gamma bias update."""
+    st = lib.moe_balance(ctypes.byref(cfg), _ptr(logits), _ptr(ids), _ptr(modality), _ptr(f),
+                         _ptr(P), _ptr(aux), _ptr(set_load), _ptr(bias), float(gamma), _ptr(ws),
+                         _stream(stream))
+    _check(st, "moe_balance")
 
 
 def moe_forward_host(cfg, *, x_host, W_g, W_gu, W_down, y_host, logit_offset=None, bias=None,

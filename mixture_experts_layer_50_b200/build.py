@@ -16,7 +16,8 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoe_b200.so")
-SOURCES = ["moe_api.cu", "route.cu", "dispatch.cu", "combine.cu", "gemm_tc.cu", "simt_f32.cu"]
+SOURCES = ["moe_api.cu", "route.cu", "dispatch.cu", "combine.cu", "gemm_tc.cu", "simt_f32.cu",
+           "balance.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 
 NVCC_FLAGS = [

@@ -39,6 +39,16 @@ cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_ran
                                     const void* x, void* xp, int row_bytes,
                                     cudaStream_t stream, int* launches);
 
+// ---- balancing statistics (balance.cu) ------------------------------------------------
+// f [E] share of assignments, P [E] mean router probability, aux = E sum f P, set_load
+// [n_sets][E] assignments per modality set; when bias != nullptr, bias += gamma * sign(mean
+// load - load) per set.  n_sets <= 8.  Any output pointer may be null.
+size_t balance_scratch_bytes(int64_t N, int E, int n_sets);
+cudaError_t launch_balance(const float* logits, const int32_t* ids, const uint8_t* modality,
+                           int64_t N, int E, int k, int score_fn, int n_sets, void* scratch,
+                           float* f, float* P, float* aux, int32_t* set_load, float* bias,
+                           float gamma, cudaStream_t stream, int* launches);
+
 // ---- combine (combine.cu) -------------------------------------------------------------
 // y[t] = sum_j gates[t,j] ye[slot_row[t,j]] (+ ye[shared_row0 + t] when shared_row0 >= 0).
 cudaError_t launch_combine(const void* ye, const int32_t* slot_row, const float* gates,

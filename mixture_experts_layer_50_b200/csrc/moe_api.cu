@@ -64,7 +64,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Ws {
   size_t status, logits, ids, gates, local_rank, tile_hist, tile_base, demand, counts, offsets,
-      slot_row, row_token, drop_mask, xp, h, ye, x_stage, y_stage, total;
+      slot_row, row_token, drop_mask, xp, h, ye, x_stage, y_stage, balance, total;
 };
 
 size_t el_size(const moe_config& c) { return c.dtype == MOE_DT_BF16 ? 2 : 4; }
@@ -99,6 +99,7 @@ Ws layout(const moe_config& c) {
   w.ye = take((Nk + S * N) * d * el);
   w.x_stage = take(N * d * el);
   w.y_stage = take(N * d * el);
+  w.balance = take(moe::balance_scratch_bytes((int64_t)N, (int)E, std::max(1, c.n_bias_sets)));
   w.total = off;
   return w;
 }
@@ -554,6 +555,29 @@ moe_status moe_route_hash(const moe_config* cfg, const int32_t* token_ids, int32
                          at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.slot_row), nullptr,
                          drop_mask != nullptr ? drop_mask : at<uint8_t>(ws, L.drop_mask),
                          nullptr, nullptr, st, &launches));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_balance(const moe_config* cfg, const float* logits, const int32_t* ids,
+                       const uint8_t* modality, float* f, float* P, float* aux,
+                       int32_t* set_load, float* bias, float gamma, void* ws,
+                       moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  if (logits == nullptr || ids == nullptr) return fail(MOE_ERR_INVALID_ARG, "logits and ids are required");
+  const int n_sets = std::max(1, cfg->n_bias_sets);
+  if (n_sets > 8) return fail(MOE_ERR_UNSUPPORTED, "moe_balance handles at most 8 bias sets");
+  if (n_sets > 1 && modality == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "several bias sets need the modality flags");
+  if (!(gamma == gamma)) return fail(MOE_ERR_INVALID_ARG, "gamma is NaN");
+  const Ws L = layout(*cfg);
+  int launches = 0;
+  MOE_CUDA(moe::launch_balance(logits, ids, modality, cfg->N, cfg->E, cfg->k, cfg->score_fn,
+                               n_sets, at<char>(ws, L.balance), f, P, aux, set_load, bias, gamma,
+                               (cudaStream_t)stream, &launches),
+           "balance statistics");
   g_last_launches = launches;
   return MOE_OK;
 }

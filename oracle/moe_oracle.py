@@ -60,8 +60,14 @@ Readings where the pages are silent (each is listed again in the design doc):
       optional per-expert logit offset is added before that rounding (the skewed
       capacity workload).
 
-Parity unpinned: the clamp (R6) beyond unit values, and the whole-layer output
-beyond brute force and closed forms -- no page prints a layer output.
+* R11 the balance statistic's P_i for sigmoid scoring averages the affinities
+      normalised per token to sum 1 (the pages print the formula for softmax only).
+* R12 the bias update compares each expert's load with its set's mean load
+      (total / E) exactly, in integers; gamma = 0.001 (both pages' update rate).
+
+Parity unpinned: the clamp (R6) beyond unit values, the whole-layer output beyond
+brute force and closed forms -- no page prints a layer output -- and the hash
+router (a reading of an exercise, pinned only by bijectivity and uniformity).
 """
 from __future__ import annotations
 
@@ -307,6 +313,55 @@ def forward(x, W_g, W_gu, W_down, *, k, E, score_fn=SOFTMAX, renorm=1, act=SWIGL
     return y, info
 
 
+# ---------------------------------------------------------------------------
+# balancing statistics and the aux-loss-free bias update
+# ---------------------------------------------------------------------------
+def router_probs(logits, score_fn):
+    """Per-token router probabilities over all experts: softmax(z), or for sigmoid scoring
+    the affinities s = sigma(z) normalised to sum 1 (reading R11)."""
+    z = np.asarray(logits, np.float64)
+    if score_fn == SOFTMAX:
+        return softmax64(z)
+    s = 1.0 / (1.0 + np.exp(-z))
+    return s / s.sum(axis=1, keepdims=True)
+
+
+def balance_stats(logits, ids, E, score_fn=SOFTMAX):
+    """Switch balance statistic ("Основы MoE", "Вспомогательный лосс Switch Transformer"):
+    f_i = share of the top-k assignments that went to expert i (sums to 1), P_i = mean
+    router probability of expert i over the tokens, aux = E * sum_i f_i P_i (the loss is
+    alpha * aux).  Returns (f, P, aux) in float64."""
+    ids = np.asarray(ids, np.int64)
+    f = np.bincount(ids.ravel(), minlength=E) / ids.size
+    P = router_probs(logits, score_fn).mean(axis=0)
+    return f, P, float(E * np.sum(f * P))
+
+
+def per_set_load(ids, E, modality=None, n_sets=1):
+    """Assignments per (bias set, expert): token t counts in set modality[t] (set 0 without flags)."""
+    ids = np.asarray(ids, np.int64)
+    sets = np.zeros(ids.shape[0], np.int64) if modality is None else np.asarray(modality, np.int64)
+    load = np.zeros((n_sets, E), np.int64)
+    for m in range(n_sets):
+        load[m] = np.bincount(ids[sets == m].ravel(), minlength=E)
+    return load
+
+
+def bias_update(bias, load, gamma=0.001):
+    """Aux-loss-free balancing ("Le groupe d'experts (MoE)", "Le problème de l'équilibre de la
+    charge"; DeepSeek-V4.1-Flash page, "L'équilibrage de charge" and "l'équilibrage par
+    modalité"): after a step each expert's selection bias moves by -gamma when its load is
+    above the set's mean load, +gamma when below, unchanged when equal; each bias set uses
+    its own loads.  float32 in, float32 out (reading R12: the comparison is exact in
+    integers, load_e * E versus the set's total)."""
+    bias = np.asarray(bias, np.float32)
+    load = np.asarray(load, np.int64)
+    E = load.shape[1]
+    total = load.sum(axis=1, keepdims=True)
+    step = np.sign(total - load * E).astype(np.float32) * np.float32(gamma)
+    return (bias + step).astype(np.float32)
+
+
 def fmix32(h):
     """The 32-bit finaliser of MurmurHash3 (A. Appleby, public domain): a bijection on
     32-bit integers that mixes every input bit into every output bit."""
@@ -345,5 +400,6 @@ def dense_mixture(x, W_g, W_gu, W_down, *, E, act=SWIGLU, clamp=0.0, logit_offse
 __all__ = ["exp_f32", "sigmoid_f32", "router_logits", "softmax64", "selection_keys",
            "topk_ids", "gates_for", "route", "capacity", "dispatch", "load_fractions",
            "silu", "expert_ffn", "forward", "dense_mixture", "fmix32", "hash_route",
+           "router_probs", "balance_stats", "per_set_load", "bias_update",
            "SOFTMAX", "SIGMOID",
            "SWIGLU", "RELU"]

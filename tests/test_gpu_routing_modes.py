@@ -1,5 +1,6 @@
-"""GPU parity of the routing variants: forced (replayed) routing and the hash router
-("Le groupe d'experts (MoE)", exercises "Hard" and "Medium")."""
+"""GPU parity of the routing variants and of the balancing by-products: forced (replayed)
+routing and the hash router ("Le groupe d'experts (MoE)", exercises "Hard" and "Medium"), the
+Switch balance statistic and the aux-loss-free bias update per modality."""
 import numpy as np
 import pytest
 import torch
@@ -102,3 +103,29 @@ def test_hash_router_bit_exact(N, E, k, C):
     np.testing.assert_array_equal(host(out["gates"]), gates_o.astype(np.float32))
     for name in ("counts", "demand", "drop_mask"):
         np.testing.assert_array_equal(host(out[name]), d_o[name])
+
+
+@pytest.mark.parametrize("N,E,k,sf,nb", [(1000, 8, 2, 0, 0), (4096, 384, 6, 1, 2), (777, 64, 1, 0, 1)])
+def test_balance_statistics_and_bias_update(N, E, k, sf, nb):
+    z = W.random_logits(N, E, N + E, scale=1.5)
+    bias = W.random_bias(max(nb, 1), E, 9) if nb else np.zeros((1, E), np.float32)
+    mod = W.random_modality(N, 10) if nb > 1 else None
+    ids, _ = O.route(z, k, sf, 1, bias if nb else None, mod)
+    cfg = nat.make_config(N, 64, E, k, 64, n_bias_sets=nb, score_fn=sf)
+    ws = nat.alloc_workspace(cfg)
+    sets = max(nb, 1)
+    f = torch.empty(E, device="cuda")
+    P = torch.empty(E, device="cuda")
+    aux = torch.empty(1, device="cuda")
+    set_load = torch.empty((sets, E), dtype=torch.int32, device="cuda")
+    b = dev(bias)
+    nat.moe_balance(cfg, logits=dev(z), ids=dev(ids), modality=None if mod is None else dev(mod),
+                    f=f, P=P, aux=aux, set_load=set_load, bias=b, gamma=0.001, ws=ws)
+    check_status(ws)
+    f_o, P_o, aux_o = O.balance_stats(z, ids, E, sf)
+    load_o = O.per_set_load(ids, E, mod, sets)
+    np.testing.assert_array_equal(host(f), f_o.astype(np.float32))
+    np.testing.assert_allclose(host(P), P_o, rtol=1e-5)
+    assert abs(float(aux.item()) - aux_o) <= 1e-5 * aux_o
+    np.testing.assert_array_equal(host(set_load), load_o)
+    np.testing.assert_array_equal(host(b), O.bias_update(bias, load_o, 0.001))

@@ -447,3 +447,51 @@ def test_hash_route_is_deterministic_distinct_uniform():
     # the same token id always lands on the same experts, wherever it sits in the batch
     ids3, _ = O.hash_route(tok[::-1], 64, 2)
     np.testing.assert_array_equal(ids3[::-1], ids)
+
+
+# --------------------------------------------------------------------------
+# balancing statistics and the bias update
+# --------------------------------------------------------------------------
+def test_switch_balance_statistic_printed_example():
+    g = load("p5_aux_loss.txt")
+    E = int(g["N"])
+    f, P = np.array(floats(g["load"])), np.array(floats(g["probs"]))
+    # the statistic as defined: E * sum f_i P_i, here through balance_stats' own arithmetic
+    # by building ids and logits whose f and P are exactly the printed ones
+    ids = np.repeat(np.arange(E), (f * 10).astype(int))[:, None]          # 10 assignments
+    z = np.log(np.tile(P, (len(ids), 1)))                                 # softmax(z) = P
+    f_o, P_o, aux = O.balance_stats(z, ids, E)
+    np.testing.assert_allclose(f_o, f, rtol=1e-12)
+    np.testing.assert_allclose(P_o, P, rtol=1e-12)
+    assert round(aux, 2) == float(g["value"])
+    # uniform router and uniform load give 1; collapse onto one expert gives about E
+    zu = np.zeros((8, E))
+    idu = np.arange(8)[:, None] % E
+    assert O.balance_stats(zu, idu, E)[2] == pytest.approx(float(g["uniform_value"]))
+    zc = np.zeros((8, E)); zc[:, 0] = 50.0
+    assert O.balance_stats(zc, np.zeros((8, 1), int), E)[2] == pytest.approx(E, rel=1e-12)
+
+
+def test_bias_update_on_the_slides_trace_loads():
+    # P2 trace demand 6/4/3/3 (mean 4): E1 overloaded, E2 on target, E3 and E4 underloaded
+    gt, assign, T, E, k = _trace()
+    ids = np.array(assign, np.int32)
+    load = O.per_set_load(ids, E)
+    assert load.tolist() == [[6, 4, 3, 3]]
+    b = O.bias_update(np.zeros((1, E), np.float32), load, 0.001)
+    np.testing.assert_array_equal(b, np.float32([[-0.001, 0.0, 0.001, 0.001]]))
+    # two modality sets are balanced separately
+    mod = np.array([0, 0, 0, 0, 1, 1, 1, 1], np.uint8)
+    load2 = O.per_set_load(ids, E, mod, 2)
+    assert load2.tolist() == [[4, 2, 1, 1], [2, 2, 2, 2]]
+    b2 = O.bias_update(np.zeros((2, E), np.float32), load2, 0.001)
+    np.testing.assert_array_equal(b2[1], 0.0)
+    np.testing.assert_array_equal(b2[0], np.float32([-0.001, 0.0, 0.001, 0.001]))   # mean 2
+
+
+def test_sigmoid_probs_sum_to_one_and_follow_the_affinities():
+    z = np.random.default_rng(2).normal(0, 1, (50, 9))
+    P = O.router_probs(z, O.SIGMOID)
+    np.testing.assert_allclose(P.sum(1), 1.0, rtol=1e-14)
+    s = expit(z)
+    np.testing.assert_allclose(P, s / s.sum(1, keepdims=True), rtol=1e-14)

@@ -213,6 +213,30 @@ MOE_API moe_status moe_balance(const moe_config* cfg, const float* logits, const
                                int32_t* set_load, float* bias, float gamma, void* ws,
                                moe_stream_t stream);
 
+/* The padded dispatch buffer [E][C][d] of "Mixture-of-Experts : routage et capacité"
+ * ("Support visuel — Capacité": capacity as a tensor dimension): slot c of expert e holds the
+ * c-th kept token of e in token order; empty slots are zero rows (row_token_pad = -1).  This is
+ * the layout an expert-parallel all-to-all ships.  Needs cfg->capacity = C > 0.
+ *   ids [N][k], drop_mask [N][k] or NULL (assignments already dropped are skipped), x [N][d]
+ *   offsets_pad [E+1] = e*C, counts [E] (kept per expert, <= C), row_token_pad [E*C] or NULL,
+ *   slot_row [N][k] = e*C + rank or -1, xp_pad [E*C][d]: outputs. */
+MOE_API moe_status moe_permute_padded(const moe_config* cfg, const int32_t* ids,
+                                      const uint8_t* drop_mask, const void* x,
+                                      int32_t* offsets_pad, int32_t* counts,
+                                      int32_t* row_token_pad, int32_t* slot_row, void* xp_pad,
+                                      void* ws, moe_stream_t stream);
+
+/* moe_forward through the padded layout: the expert FFNs run over the E*C padded rows
+ * (empty slots are computed on zero rows and never combined), the shared expert's rows follow
+ * at E*C + t.  Same result as moe_forward.  route_out->offsets, when given, receives the padded
+ * offsets e*C.  Needs cfg->capacity > 0; the workspace of moe_workspace_size covers it. */
+MOE_API moe_status moe_forward_padded(const moe_config* cfg, const void* x, const void* W_g,
+                                      const float* logit_offset, const float* bias,
+                                      const uint8_t* modality, const void* W_gu,
+                                      const void* W_down, void* y,
+                                      const moe_route_out* route_out, void* ws,
+                                      moe_stream_t stream);
+
 /* moe_forward with x_host and y_host in HOST memory (pinned for full copy speed): copies
  * x to the workspace, runs the layer, copies y back and synchronises the stream.
  * Weights, bias, modality and logit_offset are device pointers as in moe_forward. */

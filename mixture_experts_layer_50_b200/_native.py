@@ -71,6 +71,8 @@ lib.moe_route_static.argtypes = [_cfgp] + [_vp] * 10
 lib.moe_forward_routed.argtypes = [_cfgp] + [_vp] * 9
 lib.moe_route_hash.argtypes = [_cfgp] + [_vp] * 8
 lib.moe_balance.argtypes = [_cfgp] + [_vp] * 8 + [ctypes.c_float, _vp, _vp]
+lib.moe_permute_padded.argtypes = [_cfgp] + [_vp] * 10
+lib.moe_forward_padded.argtypes = [_cfgp] + [_vp] * 11
 lib.moe_profile_begin.argtypes = [_i32]
 lib.moe_profile_begin.restype = ctypes.c_int
 lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)]
@@ -79,14 +81,15 @@ lib.moe_last_error.restype = ctypes.c_char_p
 lib.moe_last_launch_count.restype = _i32
 for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
            "moe_forward", "moe_forward_host", "moe_check_status", "moe_route_static",
-           "moe_forward_routed", "moe_route_hash", "moe_balance"):
+           "moe_forward_routed", "moe_route_hash", "moe_balance", "moe_permute_padded",
+           "moe_forward_padded"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
             "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
             "moe_check_status", "moe_profile_begin", "moe_profile_end", "moe_last_error",
             "moe_last_launch_count", "moe_route_static", "moe_forward_routed",
-            "moe_route_hash", "moe_balance")
+            "moe_route_hash", "moe_balance", "moe_permute_padded", "moe_forward_padded")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -241,6 +244,28 @@ def moe_balance(cfg, *, logits, ids, modality=None, f=None, P=None, aux=None, se
                          _ptr(P), _ptr(aux), _ptr(set_load), _ptr(bias), float(gamma), _ptr(ws),
                          _stream(stream))
     _check(st, "moe_balance")
+
+
+def moe_permute_padded(cfg, *, ids, drop_mask=None, x, offsets_pad, counts, row_token_pad=None,
+                       slot_row, xp_pad, ws, stream=None):
+    """The padded [E][C][d] dispatch buffer (capacity as a tensor dimension)."""
+    st = lib.moe_permute_padded(ctypes.byref(cfg), _ptr(ids), _ptr(drop_mask), _ptr(x),
+                                _ptr(offsets_pad), _ptr(counts), _ptr(row_token_pad),
+                                _ptr(slot_row), _ptr(xp_pad), _ptr(ws), _stream(stream))
+    _check(st, "moe_permute_padded")
+
+
+def moe_forward_padded(cfg, *, x, W_g, W_gu, W_down, y, logit_offset=None, bias=None,
+                       modality=None, route_out: Optional[dict] = None, ws, stream=None):
+    """The layer through the padded dispatch layout (needs a capacity)."""
+    ro = None
+    if route_out:
+        ro = moe_route_out(*[_ptr(route_out.get(n)) for n, _ in moe_route_out._fields_])
+    st = lib.moe_forward_padded(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(logit_offset),
+                                _ptr(bias), _ptr(modality), _ptr(W_gu), _ptr(W_down), _ptr(y),
+                                ctypes.byref(ro) if ro is not None else None, _ptr(ws),
+                                _stream(stream))
+    _check(st, "moe_forward_padded")
 
 
 def moe_forward_host(cfg, *, x_host, W_g, W_gu, W_down, y_host, logit_offset=None, bias=None,

@@ -159,7 +159,41 @@ __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
   }
 }
 
+__global__ void pad_offsets_kernel(int E, int64_t C, int32_t* __restrict__ offsets_pad) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e <= E) offsets_pad[e] = (int32_t)(e * C);
+}
+
+// One block per padded row.
+__global__ void __launch_bounds__(128) zero_padding_kernel(
+    const int32_t* __restrict__ counts, int64_t C, uint4* __restrict__ xp_pad, int row_vecs,
+    int32_t* __restrict__ row_token_pad) {
+  const int64_t r = blockIdx.x;
+  const int e = (int)(r / C);
+  if (r - (int64_t)e * C < counts[e]) return;
+  if (threadIdx.x == 0 && row_token_pad != nullptr) row_token_pad[r] = -1;
+  for (int v = threadIdx.x; v < row_vecs; v += blockDim.x) xp_pad[r * row_vecs + v] = make_uint4(0, 0, 0, 0);
+}
+
 }  // namespace
+
+cudaError_t launch_pad_offsets(int E, int64_t C, int32_t* offsets_pad, cudaStream_t stream,
+                               int* launches) {
+  ++*launches;
+  pad_offsets_kernel<<<(E + 1 + 255) / 256, 256, 0, stream>>>(E, C, offsets_pad);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_padding(const int32_t* counts, int E, int64_t C, void* xp_pad,
+                                int row_bytes, int32_t* row_token_pad, cudaStream_t stream,
+                                int* launches) {
+  const int64_t rows = (int64_t)E * C;
+  if (rows == 0) return cudaSuccess;
+  ++*launches;
+  zero_padding_kernel<<<(unsigned)rows, 128, 0, stream>>>(counts, C, (uint4*)xp_pad,
+                                                         row_bytes / 16, row_token_pad);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_rank_local(const int32_t* ids, const uint8_t* drop_mask, int64_t N, int k,
                               int E, int32_t* local_rank, int32_t* tile_hist, int* status,

@@ -49,6 +49,15 @@ cudaError_t launch_balance(const float* logits, const int32_t* ids, const uint8_
                            float* f, float* P, float* aux, int32_t* set_load, float* bias,
                            float gamma, cudaStream_t stream, int* launches);
 
+// Padded layout: offsets_pad[e] = e * C for e <= E.
+cudaError_t launch_pad_offsets(int E, int64_t C, int32_t* offsets_pad, cudaStream_t stream,
+                               int* launches);
+// Zero the empty slots (rows e*C + c with c >= counts[e]) of a padded buffer and mark them
+// -1 in row_token_pad (when not null).
+cudaError_t launch_zero_padding(const int32_t* counts, int E, int64_t C, void* xp_pad,
+                                int row_bytes, int32_t* row_token_pad, cudaStream_t stream,
+                                int* launches);
+
 // ---- combine (combine.cu) -------------------------------------------------------------
 // y[t] = sum_j gates[t,j] ye[slot_row[t,j]] (+ ye[shared_row0 + t] when shared_row0 >= 0).
 cudaError_t launch_combine(const void* ye, const int32_t* slot_row, const float* gates,
@@ -60,9 +69,9 @@ cudaError_t launch_router_f32(const float* x, const float* W_g, const float* log
                               int64_t N, int d, int E, float* logits, cudaStream_t stream,
                               int* launches);
 // h[r] = act(A_r . W1_e) for every row r of the groups (routed rows from xp, shared rows
-// from x), then ye[r] = h[r] . W2_e.
+// from x, starting at row Nk), then ye[r] = h[r] . W2_e.
 cudaError_t launch_ffn_f32(const float* xp, const float* x, const int32_t* offsets,
-                           int64_t N, int k, int d, int E, int F, int n_shared, int act,
+                           int64_t N, int64_t Nk, int d, int E, int F, int n_shared, int act,
                            float clamp, const float* W_gu, const float* W_down, float* h,
                            float* ye, cudaStream_t stream, int* launches);
 

@@ -64,10 +64,13 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Ws {
   size_t status, logits, ids, gates, local_rank, tile_hist, tile_base, demand, counts, offsets,
-      slot_row, row_token, drop_mask, xp, h, ye, x_stage, y_stage, balance, total;
+      slot_row, row_token, drop_mask, xp, h, ye, x_stage, y_stage, balance, offsets_pad, total;
 };
 
 size_t el_size(const moe_config& c) { return c.dtype == MOE_DT_BF16 ? 2 : 4; }
+
+// Rows of the padded dispatch buffer [E][C] (0 without a capacity).
+int64_t padded_rows(const moe_config& c) { return c.capacity > 0 ? (int64_t)c.E * c.capacity : 0; }
 
 Ws layout(const moe_config& c) {
   Ws w;
@@ -80,6 +83,7 @@ Ws layout(const moe_config& c) {
   const size_t N = (size_t)c.N, k = (size_t)c.k, E = (size_t)c.E, d = (size_t)c.d,
                F = (size_t)c.F, S = (size_t)c.n_shared, el = el_size(c);
   const size_t Nk = N * k;
+  const size_t R = std::max(Nk, (size_t)padded_rows(c));  // routed region: compact or padded
   const size_t tiles = (N + moe::kRankTile - 1) / moe::kRankTile;
   w.status = take(256);
   w.logits = take(N * E * 4);
@@ -92,14 +96,15 @@ Ws layout(const moe_config& c) {
   w.counts = take(E * 4);
   w.offsets = take((E + 1) * 4);
   w.slot_row = take(Nk * 4);
-  w.row_token = take(Nk * 4);
+  w.row_token = take(R * 4);
   w.drop_mask = take(Nk);
-  w.xp = take(Nk * d * el);
-  w.h = take((Nk + S * N) * F * el);
-  w.ye = take((Nk + S * N) * d * el);
+  w.xp = take(R * d * el);
+  w.h = take((R + S * N) * F * el);
+  w.ye = take((R + S * N) * d * el);
   w.x_stage = take(N * d * el);
   w.y_stage = take(N * d * el);
   w.balance = take(moe::balance_scratch_bytes((int64_t)N, (int)E, std::max(1, c.n_bias_sets)));
+  w.offsets_pad = take((E + 1) * 4);
   w.total = off;
   return w;
 }
@@ -254,13 +259,16 @@ moe_status stage_dispatch(const moe_config& c, const Ws& L, void* ws, const int3
   return MOE_OK;
 }
 
+// R: rows of the routed region of xp / h / ye (N k for the compact layout, E C for the
+// padded one); the shared expert's rows follow it.
 moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
                      const int32_t* offsets, const void* x, const void* W_gu,
-                     const void* W_down, void* ye, cudaStream_t st, int* launches) {
+                     const void* W_down, void* ye, cudaStream_t st, int* launches,
+                     int64_t R = -1) {
   if (c.N == 0) return MOE_OK;
-  const int64_t Nk = c.N * (int64_t)c.k;
+  const int64_t Nk = R >= 0 ? R : c.N * (int64_t)c.k;
   if (c.dtype == MOE_DT_F32) {
-    MOE_CUDA(moe::launch_ffn_f32((const float*)xp, (const float*)x, offsets, c.N, c.k, c.d, c.E,
+    MOE_CUDA(moe::launch_ffn_f32((const float*)xp, (const float*)x, offsets, c.N, Nk, c.d, c.E,
                                  c.F, c.n_shared, c.act, c.clamp, (const float*)W_gu,
                                  (const float*)W_down, at<float>(ws, L.h), (float*)ye, st,
                                  launches),
@@ -326,8 +334,9 @@ moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
 }
 
 moe_status stage_combine(const moe_config& c, const void* ye, const int32_t* slot_row,
-                         const float* gates, void* y, cudaStream_t st, int* launches) {
-  const int64_t shared_row0 = c.n_shared ? c.N * (int64_t)c.k : -1;
+                         const float* gates, void* y, cudaStream_t st, int* launches,
+                         int64_t R = -1) {
+  const int64_t shared_row0 = c.n_shared ? (R >= 0 ? R : c.N * (int64_t)c.k) : -1;
   MOE_CUDA(moe::launch_combine(ye, slot_row, gates, c.N, c.k, c.d, shared_row0,
                                c.dtype == MOE_DT_F32, y, st, launches),
            "combine");
@@ -578,6 +587,101 @@ moe_status moe_balance(const moe_config* cfg, const float* logits, const int32_t
                                n_sets, at<char>(ws, L.balance), f, P, aux, set_load, bias, gamma,
                                (cudaStream_t)stream, &launches),
            "balance statistics");
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_permute_padded(const moe_config* cfg, const int32_t* ids,
+                              const uint8_t* drop_mask, const void* x, int32_t* offsets_pad,
+                              int32_t* counts, int32_t* row_token_pad, int32_t* slot_row,
+                              void* xp_pad, void* ws, moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  if (cfg->capacity <= 0) return fail(MOE_ERR_INVALID_ARG, "the padded layout needs capacity > 0");
+  if (padded_rows(*cfg) > (int64_t)INT32_MAX / 2) return fail(MOE_ERR_UNSUPPORTED, "E*C too large");
+  if (ids == nullptr || offsets_pad == nullptr || counts == nullptr || slot_row == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "ids, offsets_pad, counts and slot_row are required");
+  MOE_TRY(need(x, "x"));
+  MOE_TRY(need(xp_pad, "xp_pad"));
+  const moe_config& c = *cfg;
+  const Ws L = layout(c);
+  cudaStream_t st = (cudaStream_t)stream;
+  int launches = 0;
+  int* status = at<int>(ws, L.status);
+  MOE_CUDA(moe::launch_rank_local(ids, drop_mask, c.N, c.k, c.E, at<int32_t>(ws, L.local_rank),
+                                  at<int32_t>(ws, L.tile_hist), status, st, &launches),
+           "rank pass");
+  MOE_CUDA(moe::launch_dispatch_scan(at<int32_t>(ws, L.tile_hist), c.N, c.E, c.capacity,
+                                     at<int32_t>(ws, L.tile_base), at<int32_t>(ws, L.demand),
+                                     counts, at<int32_t>(ws, L.offsets), st, &launches),
+           "scan pass");
+  MOE_CUDA(moe::launch_pad_offsets(c.E, c.capacity, offsets_pad, st, &launches), "pad offsets");
+  MOE_CUDA(moe::launch_dispatch_scatter(ids, at<int32_t>(ws, L.local_rank),
+                                        at<int32_t>(ws, L.tile_base), offsets_pad, c.N, c.k, c.E,
+                                        c.capacity, slot_row, row_token_pad, nullptr, x, xp_pad,
+                                        (int)(c.d * el_size(c)), st, &launches),
+           "scatter pass");
+  MOE_CUDA(moe::launch_zero_padding(counts, c.E, c.capacity, xp_pad, (int)(c.d * el_size(c)),
+                                    row_token_pad, st, &launches),
+           "zero padding");
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_forward_padded(const moe_config* cfg, const void* x, const void* W_g,
+                              const float* logit_offset, const float* bias,
+                              const uint8_t* modality, const void* W_gu, const void* W_down,
+                              void* y, const moe_route_out* ro, void* ws,
+                              moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  MOE_TRY(check_bias(cfg, bias, modality));
+  if (cfg->capacity <= 0) return fail(MOE_ERR_INVALID_ARG, "the padded layout needs capacity > 0");
+  if (padded_rows(*cfg) + cfg->N > (int64_t)INT32_MAX / 2) return fail(MOE_ERR_UNSUPPORTED, "E*C too large");
+  MOE_TRY(need(x, "x"));
+  MOE_TRY(need(W_g, "W_g"));
+  MOE_TRY(need(W_gu, "W_gu"));
+  MOE_TRY(need(W_down, "W_down"));
+  MOE_TRY(need(y, "y"));
+  const moe_config& c = *cfg;
+  const Ws L = layout(c);
+  cudaStream_t st = (cudaStream_t)stream;
+  int* status = at<int>(ws, L.status);
+  const int64_t R = padded_rows(c);
+  float* logits = (ro && ro->logits) ? ro->logits : at<float>(ws, L.logits);
+  int32_t* ids = (ro && ro->ids) ? ro->ids : at<int32_t>(ws, L.ids);
+  float* gates = (ro && ro->gates) ? ro->gates : at<float>(ws, L.gates);
+  int32_t* counts = (ro && ro->counts) ? ro->counts : at<int32_t>(ws, L.counts);
+  int32_t* demand = (ro && ro->demand) ? ro->demand : at<int32_t>(ws, L.demand);
+  uint8_t* drop = (ro && ro->drop_mask) ? ro->drop_mask : at<uint8_t>(ws, L.drop_mask);
+  int32_t* offsets_pad = (ro && ro->offsets) ? ro->offsets : at<int32_t>(ws, L.offsets_pad);
+  int32_t* slot_row = at<int32_t>(ws, L.slot_row);
+  int32_t* row_token = at<int32_t>(ws, L.row_token);
+  void* xp = at<char>(ws, L.xp);
+  void* ye = at<char>(ws, L.ye);
+  int launches = 0;
+  MOE_TRY(stage_logits(c, x, W_g, logit_offset, logits, status, st, &launches));
+  MOE_TRY(stage_route(c, logits, bias, modality, ids, gates, status, st, &launches));
+  MOE_CUDA(moe::launch_rank_local(ids, nullptr, c.N, c.k, c.E, at<int32_t>(ws, L.local_rank),
+                                  at<int32_t>(ws, L.tile_hist), status, st, &launches),
+           "rank pass");
+  MOE_CUDA(moe::launch_dispatch_scan(at<int32_t>(ws, L.tile_hist), c.N, c.E, c.capacity,
+                                     at<int32_t>(ws, L.tile_base), demand, counts,
+                                     at<int32_t>(ws, L.offsets), st, &launches),
+           "scan pass");
+  MOE_CUDA(moe::launch_pad_offsets(c.E, c.capacity, offsets_pad, st, &launches), "pad offsets");
+  MOE_CUDA(moe::launch_dispatch_scatter(ids, at<int32_t>(ws, L.local_rank),
+                                        at<int32_t>(ws, L.tile_base), offsets_pad, c.N, c.k, c.E,
+                                        c.capacity, slot_row, row_token, drop, x, xp,
+                                        (int)(c.d * el_size(c)), st, &launches),
+           "scatter pass");
+  MOE_CUDA(moe::launch_zero_padding(counts, c.E, c.capacity, xp, (int)(c.d * el_size(c)),
+                                    row_token, st, &launches),
+           "zero padding");
+  MOE_TRY(stage_ffn(c, L, ws, xp, offsets_pad, x, W_gu, W_down, ye, st, &launches, R));
+  MOE_TRY(stage_combine(c, ye, slot_row, gates, y, st, &launches, R));
   g_last_launches = launches;
   return MOE_OK;
 }

@@ -116,11 +116,10 @@ cudaError_t launch_router_f32(const float* x, const float* W_g, const float* log
 }
 
 cudaError_t launch_ffn_f32(const float* xp, const float* x, const int32_t* offsets,
-                           int64_t N, int k, int d, int E, int F, int n_shared, int act,
+                           int64_t N, int64_t Nk, int d, int E, int F, int n_shared, int act,
                            float clamp, const float* W_gu, const float* W_down, float* h,
                            float* ye, cudaStream_t stream, int* launches) {
   if (N == 0) return cudaSuccess;
-  const int64_t Nk = N * k;
   const int64_t rows = Nk + (n_shared ? N : 0);
   dim3 block(32, 8);
   dim3 g1((unsigned)((rows + 7) / 8), (F + 31) / 32);

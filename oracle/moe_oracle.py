@@ -236,6 +236,25 @@ def dispatch(ids, E: int, C: int = 0):
     }
 
 
+def dispatch_padded(ids, E: int, C: int):
+    """The padded dispatch buffer [E, C, d] of the slides ("Support visuel — Capacité"): slot
+    c of expert e holds the c-th kept token (token order), empty slots stay empty.
+    Returns slot_row [N][k] (e*C + rank, -1 = dropped), row_token [E*C] (-1 = empty slot),
+    counts [E], drop_mask [N][k]."""
+    if C <= 0:
+        raise ValueError("the padded layout needs a capacity")
+    d = dispatch(ids, E, C)
+    ids = np.asarray(ids, np.int64)
+    keep = d["drop_mask"] == 0
+    rank = d["slot_row"] - d["offsets"][ids]           # rank inside the expert, for kept ones
+    slot = np.where(keep, ids * C + rank, -1)
+    row_token = np.full(E * C, -1, np.int64)
+    t_idx = np.broadcast_to(np.arange(ids.shape[0])[:, None], ids.shape)
+    row_token[slot[keep]] = t_idx[keep]
+    return {"slot_row": slot.astype(np.int32), "row_token": row_token.astype(np.int32),
+            "counts": d["counts"], "drop_mask": d["drop_mask"]}
+
+
 def load_fractions(ids, E: int):
     """Per-expert load: bincount/N (P4 listing, sums to k) and count/(T k) (P5, sums to 1)."""
     ids = np.asarray(ids, np.int64)
@@ -398,7 +417,8 @@ def dense_mixture(x, W_g, W_gu, W_down, *, E, act=SWIGLU, clamp=0.0, logit_offse
 
 
 __all__ = ["exp_f32", "sigmoid_f32", "router_logits", "softmax64", "selection_keys",
-           "topk_ids", "gates_for", "route", "capacity", "dispatch", "load_fractions",
+           "topk_ids", "gates_for", "route", "capacity", "dispatch", "dispatch_padded",
+           "load_fractions",
            "silu", "expert_ffn", "forward", "dense_mixture", "fmix32", "hash_route",
            "router_probs", "balance_stats", "per_set_load", "bias_update",
            "SOFTMAX", "SIGMOID",

@@ -129,3 +129,57 @@ def test_balance_statistics_and_bias_update(N, E, k, sf, nb):
     assert abs(float(aux.item()) - aux_o) <= 1e-5 * aux_o
     np.testing.assert_array_equal(host(set_load), load_o)
     np.testing.assert_array_equal(host(b), O.bias_update(bias, load_o, 0.001))
+
+
+def test_padded_dispatch_buffer_matches_the_slides_table():
+    """Capacity as a tensor dimension: the [E, C, d] buffer of the 8-token, 4-expert trace."""
+    from golden.reader import ints, load
+    g = load("p2_capacity_trace.txt")
+    assign = [tuple(int(v) for v in p.split()) for p in g["assign"].split("|")]
+    ids = np.array(assign, np.int32)
+    E, C, d = 4, int(g["C_1.25"]), 64
+    cfg = nat.make_config(8, d, E, 2, 64, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    x = torch.arange(8 * d, dtype=torch.float32).reshape(8, d).to(torch.bfloat16).cuda() + 1
+    offsets_pad = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    row_token = torch.full((E * C,), 77, dtype=torch.int32, device="cuda")
+    slot_row = torch.empty((8, 2), dtype=torch.int32, device="cuda")
+    xp = torch.full((E * C, d), 5.0, dtype=torch.bfloat16, device="cuda")
+    nat.moe_permute_padded(cfg, ids=dev(ids), x=x, offsets_pad=offsets_pad, counts=counts,
+                           row_token_pad=row_token, slot_row=slot_row, xp_pad=xp, ws=ws)
+    check_status(ws)
+    p = O.dispatch_padded(ids, E, C)
+    np.testing.assert_array_equal(host(row_token), p["row_token"])
+    np.testing.assert_array_equal(host(slot_row), p["slot_row"])
+    np.testing.assert_array_equal(host(counts), p["counts"])
+    np.testing.assert_array_equal(host(offsets_pad), np.arange(E + 1) * C)
+    for e in range(E):
+        assert host(row_token)[e * C:e * C + len(ints(g[f"table_E{e}"]))].tolist() == ints(g[f"table_E{e}"])
+    rt = host(row_token)
+    xh = x.cpu()
+    for r in range(E * C):
+        if rt[r] >= 0:
+            assert torch.equal(xp[r].cpu(), xh[rt[r]])
+        else:
+            assert (xp[r].cpu() == 0).all()
+
+
+def test_padded_forward_equals_the_compact_forward():
+    shape = W.PRESETS["capacity-cf1.25"].replace(N=3000, d=512, F=256)
+    t = W.make_inputs(shape, device="cuda")
+    C = O.capacity(shape.N, shape.k, shape.E, shape.capacity_factor)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    y = torch.empty_like(t["x"])
+    yp = torch.empty_like(t["x"])
+    off = torch.empty(shape.E + 1, dtype=torch.int32, device="cuda")
+    nat.moe_forward(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y,
+                    logit_offset=t["logit_offset"], ws=ws)
+    nat.moe_forward_padded(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"],
+                           y=yp, logit_offset=t["logit_offset"], route_out={"offsets": off}, ws=ws)
+    check_status(ws)
+    np.testing.assert_array_equal(host(off), np.arange(shape.E + 1) * C)
+    # the same kernels on the same rows: each output row is computed from the same operands
+    # in the same order, so the two layouts agree to the bit
+    assert torch.equal(yp, y)

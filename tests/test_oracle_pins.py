@@ -495,3 +495,26 @@ def test_sigmoid_probs_sum_to_one_and_follow_the_affinities():
     np.testing.assert_allclose(P.sum(1), 1.0, rtol=1e-14)
     s = expit(z)
     np.testing.assert_allclose(P, s / s.sum(1, keepdims=True), rtol=1e-14)
+
+
+def test_padded_dispatch_buffer_is_the_slides_table():
+    """[E, C, d] buffer with C = 5: rows as printed, '.' = empty slot, t6 rejected."""
+    g, assign, T, E, k = _trace()
+    C = int(g["C_1.25"])
+    ids = np.array(assign, np.int32)
+    p = O.dispatch_padded(ids, E, C)
+    for e in range(E):
+        row = p["row_token"][e * C:(e + 1) * C]
+        printed = ints(g[f"table_E{e}"])
+        assert row[:len(printed)].tolist() == printed
+        assert (row[len(printed):] == -1).all()
+    assert int((p["row_token"] >= 0).sum()) == int(g["filled_1.25"])
+    assert p["row_token"].size == int(g["slots_1.25"])
+    # kept slots point back to their token; t6's first choice is the rejected one
+    for t in range(T):
+        for j in range(k):
+            r = p["slot_row"][t, j]
+            assert (r == -1) == bool(p["drop_mask"][t, j])
+            if r >= 0:
+                assert p["row_token"][r] == t and r // C == ids[t, j]
+    assert p["slot_row"][5, 0] == -1

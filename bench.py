@@ -266,21 +266,26 @@ def run_ours(args):
     ms_step = ms_total / args.steps
     value = aggregate_tokens_per_s(shape.N, world, ms_step)
 
-    # end to end through the public API with host buffers: H2D of x, the layer, D2H of y
+    # end to end through the public API with host buffers: every step copies its tokens in
+    # from pinned host memory and its result back out.  moe_forward_host_batches overlaps
+    # step b+1's copy-in and step b-1's copy-out with step b's layer; the serial call
+    # (copy in, layer, copy out, synchronise) is reported beside it.
     xh = x.cpu().pin_memory()
-    yh = torch.empty_like(xh).pin_memory()
-    for _ in range(min(args.warmup, 3)):
-        layer.forward_host(xh, yh, modality=mod)
+    yhs = [torch.empty_like(xh).pin_memory() for _ in range(2)]
+    layer.forward_host_batches([xh] * 3, [yhs[0], yhs[1], yhs[0]], modality=mod)
     barrier(world)
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    w0 = time.perf_counter()
+    layer.forward_host_batches([xh] * args.steps, [yhs[i % 2] for i in range(args.steps)],
+                               modality=mod)
+    e2e_ms = max_over_ranks((time.perf_counter() - w0) * 1e3, world) / args.steps
+    layer.forward_host(xh, yhs[0], modality=mod)
+    barrier(world)
+    torch.cuda.synchronize()
+    w0 = time.perf_counter()
     for _ in range(args.steps):
-        layer.forward_host(xh, yh, modality=mod)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+        layer.forward_host(xh, yhs[0], modality=mod)
+    serial_ms = max_over_ranks((time.perf_counter() - w0) * 1e3, world) / args.steps
     el = x.element_size()
 
     peaks, peak_src = load_peaks()
@@ -336,7 +341,9 @@ def run_ours(args):
         "launch_ms": {k: round(v, 4) for k, v in per_launch.items()},
         "e2e": {"value": round(shape.N * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": shape.N * shape.d * el,
-                "d2h_bytes_per_step": shape.N * shape.d * el},
+                "d2h_bytes_per_step": shape.N * shape.d * el,
+                "method": "moe_forward_host_batches (copies overlapped), wall clock",
+                "serial_ms_per_step": round(serial_ms, 4)},
         "gpu_launches": per_step_launches * args.steps,
         "host_enqueue_us_per_step": round(host_us, 1),
         "clocks": clocks,

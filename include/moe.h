@@ -268,6 +268,20 @@ MOE_API moe_status moe_route_static(const moe_config* cfg, const float* logits,
                                     float* gates, int32_t* counts, int32_t* demand,
                                     uint8_t* drop_mask, int32_t* status, moe_stream_t stream);
 
+/* A sequence of batches with x and y in HOST memory, pipelined: batch b+1 is copied in on one
+ * copy stream and batch b-1 copied out on another while batch b runs on `stream`, through two
+ * staging pairs in the workspace.  x_host[b] [N][d] and y_host[b] [N][d] are host pointers
+ * (pinned memory lets the copies overlap the layer); modality may be NULL or hold one device
+ * pointer per batch.  Each batch is one layer call of cfg->N tokens (capacity applies per
+ * batch).  Returns after the last batch's result is in host memory.  The two copy streams and
+ * their events are created on first use and kept by the calling thread. */
+MOE_API moe_status moe_forward_host_batches(const moe_config* cfg, int32_t n_batches,
+                                            const void* const* x_host, const void* W_g,
+                                            const float* logit_offset, const float* bias,
+                                            const uint8_t* const* modality, const void* W_gu,
+                                            const void* W_down, void* const* y_host, void* ws,
+                                            moe_stream_t stream);
+
 /* Synchronise `stream`, read and clear the workspace status word.  Returns MOE_OK or the
  * first device-detected error (MOE_ERR_INVALID_INPUT, MOE_ERR_TIMEOUT) since the last
  * check; MOE_ERR_CUDA if the stream reports an asynchronous CUDA error. */

@@ -17,7 +17,7 @@ _NATIVE_NAMES = {
     "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
     "moe_check_status", "moe_last_launch_count", "moe_profile_begin", "moe_profile_end",
     "moe_route_static", "moe_forward_routed", "moe_route_hash", "moe_balance",
-    "moe_permute_padded", "moe_forward_padded", "moe_config", "moe_route_out", "make_config",
+    "moe_permute_padded", "moe_forward_padded", "moe_forward_host_batches", "moe_config", "moe_route_out", "make_config",
     "config_from_shape", "MoeError", "lib", "EXPORTED",
 }
 

@@ -73,6 +73,7 @@ lib.moe_route_hash.argtypes = [_cfgp] + [_vp] * 8
 lib.moe_balance.argtypes = [_cfgp] + [_vp] * 8 + [ctypes.c_float, _vp, _vp]
 lib.moe_permute_padded.argtypes = [_cfgp] + [_vp] * 10
 lib.moe_forward_padded.argtypes = [_cfgp] + [_vp] * 11
+lib.moe_forward_host_batches.argtypes = [_cfgp, _i32] + [_vp] * 10
 lib.moe_profile_begin.argtypes = [_i32]
 lib.moe_profile_begin.restype = ctypes.c_int
 lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)]
@@ -82,14 +83,15 @@ lib.moe_last_launch_count.restype = _i32
 for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
            "moe_forward", "moe_forward_host", "moe_check_status", "moe_route_static",
            "moe_forward_routed", "moe_route_hash", "moe_balance", "moe_permute_padded",
-           "moe_forward_padded"):
+           "moe_forward_padded", "moe_forward_host_batches"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
             "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_forward_host",
             "moe_check_status", "moe_profile_begin", "moe_profile_end", "moe_last_error",
             "moe_last_launch_count", "moe_route_static", "moe_forward_routed",
-            "moe_route_hash", "moe_balance", "moe_permute_padded", "moe_forward_padded")
+            "moe_route_hash", "moe_balance", "moe_permute_padded", "moe_forward_padded",
+            "moe_forward_host_batches")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -274,6 +276,24 @@ def moe_forward_host(cfg, *, x_host, W_g, W_gu, W_down, y_host, logit_offset=Non
                               _ptr(logit_offset), _ptr(bias), _ptr(modality), _ptr(W_gu),
                               _ptr(W_down), _host_ptr(y_host), _ptr(ws), _stream(stream))
     _check(st, "moe_forward_host")
+
+
+def moe_forward_host_batches(cfg, *, x_host: list, W_g, W_gu, W_down, y_host: list,
+                             logit_offset=None, bias=None, modality: Optional[list] = None, ws,
+                             stream=None):
+    """Pipelined host-to-host layer over several batches (copies overlap the layer)."""
+    n = len(x_host)
+    if len(y_host) != n:
+        raise ValueError("x_host and y_host must have the same number of batches")
+    xs = (ctypes.c_void_p * n)(*[_host_ptr(t) for t in x_host])
+    ys = (ctypes.c_void_p * n)(*[_host_ptr(t) for t in y_host])
+    mods = None
+    if modality is not None:
+        mods = (ctypes.c_void_p * n)(*[_ptr(t) for t in modality])
+    st = lib.moe_forward_host_batches(ctypes.byref(cfg), n, xs, _ptr(W_g), _ptr(logit_offset),
+                                      _ptr(bias), mods, _ptr(W_gu), _ptr(W_down), ys, _ptr(ws),
+                                      _stream(stream))
+    _check(st, "moe_forward_host_batches")
 
 
 def moe_check_status(ws, stream=None) -> int:

@@ -241,6 +241,8 @@ struct Args {
   void* out;
   int64_t ld_out;
   int* status;
+  int k_splits;       // > 1: split K; split s writes rows [s * split_rows, ...) of out
+  int64_t split_rows;
 };
 
 template <int BN, int STAGES>
@@ -451,7 +453,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
-  const int total = s_start[G];
+  // with a split K, work item = (output tile, K slice); slices of a tile are adjacent
+  const int ks_n = p.k_splits > 1 ? p.k_splits : 1;
+  const int kper = (nk + ks_n - 1) / ks_n;
+  const int total = s_start[G] * ks_n;
 
   if (warp == 0) {
     // ================= TMA producer =================
@@ -462,11 +467,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         int g, m_blk, n_blk;
-        decode_tile<BM, BN>(tile, s_start, G, nt, g, m_blk, n_blk);
+        decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk);
+        const int kb0 = (tile % ks_n) * kper, kb1 = min(nk, kb0 + kper);
         const bool sh = g >= p.n_routed;
         const int a_row = (sh ? p.shared_a_row0 : p.offsets[g]) + m_blk * BM;
         const CUtensorMap* mA = sh ? &tmAs : &tmA;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, p.status)) {
             ok = false;
             break;
@@ -516,7 +522,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < nk; ++kb) {
+        const int kb0 = (tile % ks_n) * kper, kb1 = min(nk, kb0 + kper);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, s_abort, p.status)) {
             ok = false;
             break;
@@ -527,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             mma_bf16(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), kIdesc,
-                     (kb | kk) != 0 ? 1u : 0u);
+                     (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&empty[stage]);
           if (++stage == STAGES) {
@@ -552,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       int g, m_blk, n_blk;
-      decode_tile<BM, BN>(tile, s_start, G, nt, g, m_blk, n_blk);
+      decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk);
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       // warp-uniform decision: tcgen05.ld below needs all 32 lanes
@@ -561,7 +568,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool sh = g >= p.n_routed;
       const int cnt = sh ? p.shared_rows : p.offsets[g + 1] - p.offsets[g];
-      const int64_t out_row0 = (int64_t)(sh ? p.shared_out_row0 : p.offsets[g]) + m_blk * BM;
+      const int64_t out_row0 = (int64_t)(sh ? p.shared_out_row0 : p.offsets[g]) + m_blk * BM +
+                               (int64_t)(tile % ks_n) * p.split_rows;
       const int rows_valid = min(BM, cnt - m_blk * BM);
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
 
@@ -888,6 +896,8 @@ Args make_args(const GroupedGemm& g) {
   a.out = g.out;
   a.ld_out = g.ld_out;
   a.status = g.status;
+  a.k_splits = g.k_splits > 1 ? g.k_splits : 1;
+  a.split_rows = g.split_rows;
   return a;
 }
 
@@ -921,7 +931,7 @@ cudaError_t launch_2sm(const GroupedGemm& g, const CUtensorMap& mA, const CUtens
 const char* path_override() { return std::getenv("MOE_B200_GEMM_PATH"); }
 
 bool use_two_sm(const GroupedGemm& g) {
-  if (g.epilogue == kEpiStoreF32) return false;
+  if (g.epilogue == kEpiStoreF32 || g.k_splits > 1) return false;
   if (const char* env = path_override()) {
     if (std::strncmp(env, "1sm", 3) == 0) return false;
     if (std::strcmp(env, "2sm") == 0) return true;
@@ -982,7 +992,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
   int64_t mtiles = 0;
   if (g.n_routed > 0) mtiles += (g.max_rows_routed + BM - 1) / BM + g.n_routed;
   if (g.has_shared) mtiles += (g.shared_rows + BM - 1) / BM;
-  const int64_t bound = mtiles * nt;
+  const int64_t bound = mtiles * nt * std::max(1, g.k_splits);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), bound));
   ++*launches;
   if (two_sm) {

@@ -9,8 +9,11 @@ namespace moe {
 
 // ---- routing (route.cu) ---------------------------------------------------------------
 // Scores, selection keys, top-k (descending, ties to the lower index) and gates.
-cudaError_t launch_route_topk(const float* logits, int64_t N, int E, int k, int score_fn,
-                              int renorm, const float* bias, int n_bias_sets,
+// logits = sum over n_parts slices (part_stride elements apart) plus offset (when not null);
+// with n_parts > 1 or an offset the summed logits are written to logits_out (when not null).
+cudaError_t launch_route_topk(const float* logits, int n_parts, int64_t part_stride,
+                              const float* offset, float* logits_out, int64_t N, int E, int k,
+                              int score_fn, int renorm, const float* bias, int n_bias_sets,
                               const uint8_t* modality, int32_t* ids, float* gates,
                               int* status, cudaStream_t stream, int* launches);
 
@@ -107,6 +110,8 @@ struct GroupedGemm {
   int64_t rows_out;
   int64_t max_rows_routed; // upper bound of offsets[n_routed] (grid sizing)
   int* status;
+  int k_splits = 1;        // > 1 (fp32 store only): K split in slices, slice s written at
+  int64_t split_rows = 0;  // out rows [s * split_rows, ...): partial sums, col_bias ignored
 };
 
 cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* launches,

@@ -64,10 +64,15 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Ws {
   size_t status, logits, ids, gates, local_rank, tile_hist, tile_base, demand, counts, offsets,
-      slot_row, row_token, drop_mask, xp, h, ye, x_stage, y_stage, balance, offsets_pad, total;
+      slot_row, row_token, drop_mask, xp, h, ye, x_stage, y_stage, x_stage2, y_stage2, balance,
+      offsets_pad, logit_parts, total;
 };
 
 size_t el_size(const moe_config& c) { return c.dtype == MOE_DT_BF16 ? 2 : 4; }
+
+// Router split-K: at most this many K slices, used for calls of at most kSplitMaxTokens tokens.
+constexpr int kMaxLogitSplits = 16;
+constexpr int64_t kSplitMaxTokens = 512;
 
 // Rows of the padded dispatch buffer [E][C] (0 without a capacity).
 int64_t padded_rows(const moe_config& c) { return c.capacity > 0 ? (int64_t)c.E * c.capacity : 0; }
@@ -103,8 +108,11 @@ Ws layout(const moe_config& c) {
   w.ye = take((R + S * N) * d * el);
   w.x_stage = take(N * d * el);
   w.y_stage = take(N * d * el);
+  w.x_stage2 = take(N * d * el);  // second staging pair: pipelined host batches
+  w.y_stage2 = take(N * d * el);
   w.balance = take(moe::balance_scratch_bytes((int64_t)N, (int)E, std::max(1, c.n_bias_sets)));
   w.offsets_pad = take((E + 1) * 4);
+  w.logit_parts = take(N <= (size_t)kSplitMaxTokens ? (size_t)kMaxLogitSplits * N * E * 4 : 0);
   w.total = off;
   return w;
 }
@@ -186,9 +194,39 @@ moe_status check_bias(const moe_config* c, const float* bias, const uint8_t* mod
 
 // ---- the stages, shared by the split entry points and moe_forward --------------------
 
-moe_status stage_logits(const moe_config& c, const void* x, const void* W_g,
-                        const float* logit_offset, float* logits, int* status,
-                        cudaStream_t st, int* launches) {
+// Where the top-k kernel reads the router logits: `n_parts` split-K slices `part_stride`
+// floats apart that it adds in order (plus `offset`), writing the sums to `final_out`; or, with
+// one part and no offset, the finished logits themselves.
+struct LogitSrc {
+  const float* src;
+  int n_parts;
+  int64_t part_stride;
+  const float* offset;
+  float* final_out;
+};
+
+LogitSrc finished_logits(const float* z) { return LogitSrc{z, 1, 0, nullptr, nullptr}; }
+
+// Number of K slices for the router GEMM: small launches (few 128-token tiles) stream W_g
+// through a handful of CTAs, so their K loop is split over more CTAs (at most
+// kMaxLogitSplits); the partial logits sit in the workspace.
+
+int router_splits(const moe_config& c) {
+  if (c.dtype != MOE_DT_BF16 || c.N == 0 || c.N > kSplitMaxTokens) return 1;
+  const int bn = c.E <= 32 ? 32 : c.E <= 64 ? 64 : c.E <= 128 ? 128 : (c.E % 256 == 0 || c.E > 384) ? 256 : 128;
+  const int64_t tiles = ((c.N + 127) / 128) * ((c.E + bn - 1) / bn);
+  const int nk = (c.d + 63) / 64;
+  int64_t want = 128 / tiles;
+  if (want < 2) return 1;
+  int splits = (int)std::min<int64_t>({want, (int64_t)kMaxLogitSplits, (int64_t)nk});
+  const int per = (nk + splits - 1) / splits;
+  return (nk + per - 1) / per;  // no empty slice
+}
+
+moe_status stage_logits(const moe_config& c, const Ws& L, void* ws, const void* x,
+                        const void* W_g, const float* logit_offset, float* logits, int* status,
+                        cudaStream_t st, int* launches, LogitSrc* out) {
+  *out = finished_logits(logits);
   if (c.N == 0) return MOE_OK;
   if (c.dtype == MOE_DT_F32) {
     MOE_CUDA(moe::launch_router_f32((const float*)x, (const float*)W_g, logit_offset, c.N, c.d,
@@ -218,17 +256,28 @@ moe_status stage_logits(const moe_config& c, const void* x, const void* W_g,
   g.ld_out = c.E;
   g.rows_out = c.N;
   g.status = status;
+  const int splits = router_splits(c);
+  if (splits > 1) {
+    float* parts = at<float>(ws, L.logit_parts);
+    g.k_splits = splits;
+    g.split_rows = c.N;
+    g.col_bias = nullptr;
+    g.out = parts;
+    g.rows_out = c.N * splits;
+    *out = LogitSrc{parts, splits, c.N * (int64_t)c.E, logit_offset, logits};
+  }
   const char* why = "router GEMM launch";
   MOE_CUDA(moe::launch_grouped_gemm(g, st, launches, &why), why);
   prof_mark(st);
   return MOE_OK;
 }
 
-moe_status stage_route(const moe_config& c, const float* logits, const float* bias,
+moe_status stage_route(const moe_config& c, const LogitSrc& z, const float* bias,
                        const uint8_t* modality, int32_t* ids, float* gates, int* status,
                        cudaStream_t st, int* launches) {
-  MOE_CUDA(moe::launch_route_topk(logits, c.N, c.E, c.k, c.score_fn, c.renorm, bias,
-                                  c.n_bias_sets, modality, ids, gates, status, st, launches),
+  MOE_CUDA(moe::launch_route_topk(z.src, z.n_parts, z.part_stride, z.offset, z.final_out, c.N,
+                                  c.E, c.k, c.score_fn, c.renorm, bias, c.n_bias_sets, modality,
+                                  ids, gates, status, st, launches),
            "top-k routing");
   prof_mark(st);
   return MOE_OK;
@@ -365,8 +414,9 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
   void* xp = at<char>(ws, L.xp);
   void* ye = at<char>(ws, L.ye);
   prof_call_begin(st);
-  MOE_TRY(stage_logits(c, x, W_g, logit_offset, logits, status, st, launches));
-  MOE_TRY(stage_route(c, logits, bias, modality, ids, gates, status, st, launches));
+  LogitSrc zsrc;
+  MOE_TRY(stage_logits(c, L, ws, x, W_g, logit_offset, logits, status, st, launches, &zsrc));
+  MOE_TRY(stage_route(c, zsrc, bias, modality, ids, gates, status, st, launches));
   MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, c.capacity, demand, counts, offsets,
                          at<int32_t>(ws, L.slot_row), at<int32_t>(ws, L.row_token), drop, x,
                          xp, st, launches));
@@ -417,11 +467,10 @@ moe_status moe_route(const moe_config* cfg, const float* logits, const void* x,
   cudaStream_t st = (cudaStream_t)stream;
   int launches = 0;
   int* status = at<int>(ws, L.status);
-  const float* z = logits;
-  if (z == nullptr) {
+  LogitSrc z = finished_logits(logits);
+  if (logits == nullptr) {
     float* dst = logits_out != nullptr ? logits_out : at<float>(ws, L.logits);
-    MOE_TRY(stage_logits(c, x, W_g, logit_offset, dst, status, st, &launches));
-    z = dst;
+    MOE_TRY(stage_logits(c, L, ws, x, W_g, logit_offset, dst, status, st, &launches, &z));
   }
   int32_t* ids_p = ids != nullptr ? ids : at<int32_t>(ws, L.ids);
   float* gates_p = gates != nullptr ? gates : at<float>(ws, L.gates);
@@ -662,8 +711,9 @@ moe_status moe_forward_padded(const moe_config* cfg, const void* x, const void* 
   void* xp = at<char>(ws, L.xp);
   void* ye = at<char>(ws, L.ye);
   int launches = 0;
-  MOE_TRY(stage_logits(c, x, W_g, logit_offset, logits, status, st, &launches));
-  MOE_TRY(stage_route(c, logits, bias, modality, ids, gates, status, st, &launches));
+  LogitSrc zsrc;
+  MOE_TRY(stage_logits(c, L, ws, x, W_g, logit_offset, logits, status, st, &launches, &zsrc));
+  MOE_TRY(stage_route(c, zsrc, bias, modality, ids, gates, status, st, &launches));
   MOE_CUDA(moe::launch_rank_local(ids, nullptr, c.N, c.k, c.E, at<int32_t>(ws, L.local_rank),
                                   at<int32_t>(ws, L.tile_hist), status, st, &launches),
            "rank pass");
@@ -713,6 +763,74 @@ moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const voi
   MOE_TRY(fs);
   if (bytes > 0) MOE_CUDA(cudaMemcpyAsync(y_host, yd, bytes, cudaMemcpyDeviceToHost, st), "copy y to host");
   MOE_CUDA(cudaStreamSynchronize(st), "synchronise");
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_forward_host_batches(const moe_config* cfg, int32_t n_batches,
+                                    const void* const* x_host, const void* W_g,
+                                    const float* logit_offset, const float* bias,
+                                    const uint8_t* const* modality, const void* W_gu,
+                                    const void* W_down, void* const* y_host, void* ws,
+                                    moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  if (n_batches < 0) return fail(MOE_ERR_INVALID_ARG, "n_batches < 0");
+  if (n_batches > 0 && (x_host == nullptr || y_host == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "x_host and y_host arrays are required");
+  for (int b = 0; b < n_batches; ++b) {
+    if (x_host[b] == nullptr || y_host[b] == nullptr)
+      return fail(MOE_ERR_INVALID_ARG, "a host batch pointer is NULL");
+    MOE_TRY(check_bias(cfg, bias, modality != nullptr ? modality[b] : nullptr));
+  }
+  if (n_batches == 0) return MOE_OK;
+  MOE_TRY(need(W_g, "W_g"));
+  MOE_TRY(need(W_gu, "W_gu"));
+  MOE_TRY(need(W_down, "W_down"));
+  const moe_config& c = *cfg;
+  const Ws L = layout(c);
+  const size_t bytes = (size_t)c.N * c.d * el_size(c);
+  cudaStream_t main = (cudaStream_t)stream;
+  // two copy streams and the events that chain them to the layer (created once per thread)
+  thread_local cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  thread_local cudaEvent_t ev_in[2], ev_done[2], ev_out[2];
+  thread_local int owner_dev = -1;
+  int dev = 0;
+  MOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  if (copy_in == nullptr || owner_dev != dev) {
+    MOE_CUDA(cudaStreamCreateWithFlags(&copy_in, cudaStreamNonBlocking), "create copy stream");
+    MOE_CUDA(cudaStreamCreateWithFlags(&copy_out, cudaStreamNonBlocking), "create copy stream");
+    for (int i = 0; i < 2; ++i) {
+      MOE_CUDA(cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming), "create event");
+      MOE_CUDA(cudaEventCreateWithFlags(&ev_done[i], cudaEventDisableTiming), "create event");
+      MOE_CUDA(cudaEventCreateWithFlags(&ev_out[i], cudaEventDisableTiming), "create event");
+    }
+    owner_dev = dev;
+  }
+  void* xd[2] = {at<char>(ws, L.x_stage), at<char>(ws, L.x_stage2)};
+  void* yd[2] = {at<char>(ws, L.y_stage), at<char>(ws, L.y_stage2)};
+  int launches = 0;
+  for (int b = 0; b < n_batches; ++b) {
+    const int s = b & 1;
+    // x slot s is free once batch b-2's layer is done; y slot s once its copy-out is done
+    if (b >= 2) MOE_CUDA(cudaStreamWaitEvent(copy_in, ev_done[s], 0), "wait");
+    MOE_CUDA(cudaMemcpyAsync(xd[s], x_host[b], bytes, cudaMemcpyHostToDevice, copy_in), "copy x to device");
+    MOE_CUDA(cudaEventRecord(ev_in[s], copy_in), "record");
+    MOE_CUDA(cudaStreamWaitEvent(main, ev_in[s], 0), "wait");
+    if (b >= 2) MOE_CUDA(cudaStreamWaitEvent(main, ev_out[s], 0), "wait");
+    const moe_status fs = forward_impl(cfg, xd[s], W_g, logit_offset, bias,
+                                       modality != nullptr ? modality[b] : nullptr, W_gu, W_down,
+                                       yd[s], nullptr, ws, main, &launches);
+    g_prof.recording = false;
+    MOE_TRY(fs);
+    MOE_CUDA(cudaEventRecord(ev_done[s], main), "record");
+    MOE_CUDA(cudaStreamWaitEvent(copy_out, ev_done[s], 0), "wait");
+    MOE_CUDA(cudaMemcpyAsync(y_host[b], yd[s], bytes, cudaMemcpyDeviceToHost, copy_out), "copy y to host");
+    MOE_CUDA(cudaEventRecord(ev_out[s], copy_out), "record");
+  }
+  MOE_CUDA(cudaStreamSynchronize(copy_out), "synchronise");
+  MOE_CUDA(cudaStreamSynchronize(main), "synchronise");
   g_last_launches = launches;
   return MOE_OK;
 }
@@ -782,7 +900,8 @@ moe_status moe_route_static(const moe_config* cfg, const float* logits, const fl
   MOE_TRY(static_scratch(&scratch));
   cudaStream_t st = (cudaStream_t)stream;
   int launches = 0;
-  MOE_TRY(stage_route(c, logits, bias, modality, ids, gates, status, st, &launches));
+  MOE_TRY(stage_route(c, finished_logits(logits), bias, modality, ids, gates, status, st,
+                      &launches));
   MOE_CUDA(moe::launch_rank_local(ids, nullptr, c.N, c.k, c.E, at<int32_t>(scratch, o_rank),
                                   at<int32_t>(scratch, o_hist), status, st, &launches),
            "rank pass");

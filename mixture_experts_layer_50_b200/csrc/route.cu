@@ -53,9 +53,11 @@ __device__ __forceinline__ bool beats(float ka, int ea, float kb, int eb) {
 
 template <int J>  // keys per lane: E <= 32 * J
 __global__ void __launch_bounds__(256) route_topk_kernel(
-    const float* __restrict__ logits, int64_t N, int E, int k, int score_fn, int renorm,
-    const float* __restrict__ bias, int n_bias_sets, const uint8_t* __restrict__ modality,
-    int32_t* __restrict__ ids, float* __restrict__ gates, int* status) {
+    const float* __restrict__ logits, int n_parts, int64_t part_stride,
+    const float* __restrict__ offset, float* __restrict__ logits_out, int64_t N, int E, int k,
+    int score_fn, int renorm, const float* __restrict__ bias, int n_bias_sets,
+    const uint8_t* __restrict__ modality, int32_t* __restrict__ ids, float* __restrict__ gates,
+    int* status) {
   const int lane = threadIdx.x & 31;
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= N) return;
@@ -73,15 +75,23 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
     b = bias + (int64_t)set * E;
   }
 
-  float key[J], sc[J];
+  float key[J], sc[J], zv[J];
   float zmax = -INFINITY;
 #pragma unroll
   for (int j = 0; j < J; ++j) {
     const int e = lane + 32 * j;
     key[j] = -INFINITY;
     sc[j] = 0.0f;
+    zv[j] = 0.0f;
     if (e < E) {
-      const float zz = z[e];
+      float zz = z[e];
+      if (n_parts > 1 || offset != nullptr) {
+        // split-K partial logits, added in slice order, then the per-expert offset
+        for (int s = 1; s < n_parts; ++s) zz += z[s * part_stride + e];
+        if (offset != nullptr) zz += offset[e];
+        if (logits_out != nullptr) logits_out[t * E + e] = zz;
+      }
+      zv[j] = zz;
       zmax = fmaxf(zmax, zz);
       const float s = (score_fn == 1) ? sigmoid_reproducible(zz) : zz;
       sc[j] = s;
@@ -138,7 +148,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
 #pragma unroll
       for (int j = 0; j < J; ++j) {
         const int e = lane + 32 * j;
-        if (e < E) part += expf(z[e] - M);
+        if (e < E) part += expf(zv[j] - M);
       }
       g = expf(my_sc - M) / warp_sum(part);
     }
@@ -156,13 +166,15 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
 }
 
 template <int J>
-cudaError_t launch_j(const float* logits, int64_t N, int E, int k, int score_fn, int renorm,
+cudaError_t launch_j(const float* logits, int n_parts, int64_t part_stride, const float* offset,
+                     float* logits_out, int64_t N, int E, int k, int score_fn, int renorm,
                      const float* bias, int n_bias_sets, const uint8_t* modality,
                      int32_t* ids, float* gates, int* status, cudaStream_t stream) {
   const int threads = 256;
   const int64_t blocks = (N * 32 + threads - 1) / threads;
   route_topk_kernel<J><<<(unsigned)blocks, threads, 0, stream>>>(
-      logits, N, E, k, score_fn, renorm, bias, n_bias_sets, modality, ids, gates, status);
+      logits, n_parts, part_stride, offset, logits_out, N, E, k, score_fn, renorm, bias,
+      n_bias_sets, modality, ids, gates, status);
   return cudaGetLastError();
 }
 
@@ -250,8 +262,9 @@ cudaError_t launch_route_hash(const int32_t* token_ids, int64_t N, int E, int k,
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_route_topk(const float* logits, int64_t N, int E, int k, int score_fn,
-                              int renorm, const float* bias, int n_bias_sets,
+cudaError_t launch_route_topk(const float* logits, int n_parts, int64_t part_stride,
+                              const float* offset, float* logits_out, int64_t N, int E, int k,
+                              int score_fn, int renorm, const float* bias, int n_bias_sets,
                               const uint8_t* modality, int32_t* ids, float* gates,
                               int* status, cudaStream_t stream, int* launches) {
   if (N == 0) return cudaSuccess;
@@ -259,7 +272,7 @@ cudaError_t launch_route_topk(const float* logits, int64_t N, int E, int k, int 
   const int J = (E + 31) / 32;
 #define MOE_ROUTE_CASE(JJ) \
   if (J <= JJ)             \
-    return launch_j<JJ>(logits, N, E, k, score_fn, renorm, bias, n_bias_sets, modality, ids, gates, status, stream);
+    return launch_j<JJ>(logits, n_parts, part_stride, offset, logits_out, N, E, k, score_fn, renorm, bias, n_bias_sets, modality, ids, gates, status, stream);
   MOE_ROUTE_CASE(1)
   MOE_ROUTE_CASE(2)
   MOE_ROUTE_CASE(4)

@@ -73,5 +73,16 @@ class MoELayer:
                              bias=self.bias, modality=modality, ws=self.ws, stream=stream)
         return y_host
 
+    def forward_host_batches(self, x_host: list, y_host: list, modality=None, stream=None):
+        """Several host batches with copies overlapped with the layer (pinned buffers)."""
+        N = x_host[0].shape[0]
+        self._check_tokens(N)
+        mods = None if modality is None else [modality] * len(x_host)
+        nat.moe_forward_host_batches(self.config(N), x_host=x_host, W_g=self.W_g, W_gu=self.W_gu,
+                                     W_down=self.W_down, y_host=y_host,
+                                     logit_offset=self.logit_offset, bias=self.bias,
+                                     modality=mods, ws=self.ws, stream=stream)
+        return y_host
+
     def check_status(self, stream=None) -> int:
         return nat.moe_check_status(self.ws, stream)

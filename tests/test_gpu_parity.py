@@ -409,3 +409,21 @@ def test_layer_class_and_determinism():
     y2 = layer.forward(t["x"], modality=t["modality"])
     assert torch.equal(y1, y2)
     assert layer.check_status() == 0
+
+
+def test_pipelined_host_batches_match_device_calls():
+    shape = W.PRESETS["v41flash-n64"].replace(N=333, d=256, F=256, E=24)
+    t = W.make_inputs(shape, device="cuda")
+    cfg = nat.config_from_shape(shape)
+    ws = nat.alloc_workspace(cfg)
+    g = torch.Generator().manual_seed(4)
+    xs = [torch.randn(shape.N, shape.d, generator=g).to(torch.bfloat16).pin_memory() for _ in range(5)]
+    ys = [torch.empty_like(xs[0]).pin_memory() for _ in range(5)]
+    nat.moe_forward_host_batches(cfg, x_host=xs, W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"],
+                                 y_host=ys, bias=t["bias"], modality=[t["modality"]] * 5, ws=ws)
+    check_status(ws)
+    for xb, yb in zip(xs, ys):
+        y = torch.empty((shape.N, shape.d), dtype=torch.bfloat16, device="cuda")
+        nat.moe_forward(cfg, x=xb.cuda(), W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y,
+                        bias=t["bias"], modality=t["modality"], ws=ws)
+        assert torch.equal(y.cpu(), yb)

@@ -312,7 +312,7 @@ def run_ours(args):
             roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s"}
         roof["frac"] = round(ach / peak, 4)
         roof["traffic"] = read_traffic("gemm_gate_up", args.workload)
-        roof["kernel"] = "gemm_gate_up (grouped_gemm_kernel<256, SwiGLU>)"
+        roof["kernel"] = "gemm_gate_up (grouped_gemm_kernel, SwiGLU epilogue)"
         roof["ms_per_launch"] = round(gu_ms, 4)
         roof["peak_source"] = f"{peak_src} ({tensor_key if roof['bound'] == 'tensor' else 'hbm_gbs'})"
     # whole-layer roofline: time bound = max(F / P, B / BW)

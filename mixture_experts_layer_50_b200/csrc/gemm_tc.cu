@@ -926,8 +926,11 @@ cudaError_t launch_2sm(const GroupedGemm& g, const CUtensorMap& mA, const CUtens
 }
 
 // Which kernel a bf16 grouped GEMM uses.  The 2-SM kernel tiles 256 rows per group, so it
-// pays off when groups are large; small groups keep the 1-SM kernel's 128-row tiles.
-// MOE_B200_GEMM_PATH=1sm|2sm overrides the choice (used by the tests to cover both kernels).
+// pays off only when groups are large, and there only for the down projection: for gate/up it
+// ran no faster than the 1-SM kernel while reading its operands from DRAM 2.6x over (5.75 GB vs
+// 2.20 GB on the 16384-token Mixtral-shaped layer), where the 1-SM kernel reads each byte once.
+// Small groups keep the 1-SM kernel's 128-row tiles.
+// MOE_B200_GEMM_PATH=1sm|1sm128|2sm overrides the choice (the tests cover every kernel).
 const char* path_override() { return std::getenv("MOE_B200_GEMM_PATH"); }
 
 bool use_two_sm(const GroupedGemm& g) {
@@ -936,6 +939,7 @@ bool use_two_sm(const GroupedGemm& g) {
     if (std::strncmp(env, "1sm", 3) == 0) return false;
     if (std::strcmp(env, "2sm") == 0) return true;
   }
+  if (g.epilogue != kEpiStoreBf16) return false;
   const int groups = g.n_routed + g.has_shared;
   const int64_t rows = (g.n_routed > 0 ? g.max_rows_routed : 0) + (g.has_shared ? g.shared_rows : 0);
   return rows >= 1024LL * groups;

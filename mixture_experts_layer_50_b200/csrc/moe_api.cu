@@ -145,8 +145,8 @@ moe_status check_cfg(const moe_config* c) {
   if (!(c->clamp == c->clamp)) return fail(MOE_ERR_INVALID_ARG, "clamp is NaN");
   if (c->dtype == MOE_DT_BF16 && (c->d % 8 != 0 || c->F % 8 != 0))
     return fail(MOE_ERR_UNSUPPORTED, "bf16 layers need d and F multiples of 8");
-  if (c->dtype == MOE_DT_F32 && c->d % 4 != 0)
-    return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need d a multiple of 4");
+  if (c->dtype == MOE_DT_F32 && (c->d % 4 != 0 || c->d > 4096 || c->F > 4096))
+    return fail(MOE_ERR_UNSUPPORTED, "fp32 layers need d a multiple of 4, d and F at most 4096");
   const int64_t rows = c->N * (int64_t)c->k + c->N * (int64_t)c->n_shared;
   if (rows > (int64_t)INT32_MAX / 2) return fail(MOE_ERR_UNSUPPORTED, "N*k too large for int32 rows");
   return MOE_OK;

@@ -349,8 +349,9 @@ def test_forward_small_shapes_all_tokens():
 
 
 def test_forward_large_groups_take_the_2sm_kernel(monkeypatch):
-    # 4096 tokens, 8 experts, top-2: about 1024 rows per expert, so the automatic choice is
-    # the 2-SM kernel; the forced 1-SM run must give the same layer within the bar
+    # 4096 tokens, 8 experts, top-2: about 1024 rows per expert, so the automatic choice
+    # takes the 2-SM kernel for the down projection; the forced 1-SM run must give the same
+    # layer within the bar
     monkeypatch.delenv("MOE_B200_GEMM_PATH", raising=False)
     _forward_case("mixtral-n4096", sample=np.r_[0:8, 4090:4096])
     monkeypatch.setenv("MOE_B200_GEMM_PATH", "1sm")
@@ -427,3 +428,34 @@ def test_pipelined_host_batches_match_device_calls():
         nat.moe_forward(cfg, x=xb.cuda(), W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y,
                         bias=t["bias"], modality=t["modality"], ws=ws)
         assert torch.equal(y.cpu(), yb)
+
+
+@pytest.mark.parametrize("N,d,E,k,F,S,act,clamp", [(257, 96, 5, 2, 200, 1, W.SWIGLU, 0.3),
+                                                   (100, 64, 8, 2, 256, 0, W.RELU, 0.0),
+                                                   (33, 1000, 3, 1, 72, 1, W.RELU, 0.0)])
+def test_expert_ffn_fp32(N, d, E, k, F, S, act, clamp):
+    """The fp32 expert path (the toy layer's): ragged d and F, shared expert, clamp."""
+    shape = W.LayerShape("t32", N=N, d=d, E=E, k=k, F=F, n_shared=S, act=act, clamp=clamp,
+                         dtype=W.F32, w_std=0.1, seed=N + d)
+    t = W.make_inputs(shape, device="cuda")
+    ids_o, _ = O.route(W.random_logits(N, E, 3), k)
+    dsp = O.dispatch(ids_o, E, 0)
+    M = int(dsp["offsets"][-1])
+    xp = torch.zeros((N * k, d), dtype=torch.float32, device="cuda")
+    xp[:M] = t["x"][torch.from_numpy(dsp["row_token"]).long().cuda()]
+    ye = torch.zeros((N * k + S * N, d), dtype=torch.float32, device="cuda")
+    cfg = nat.config_from_shape(shape)
+    ws = nat.alloc_workspace(cfg)
+    nat.moe_expert_ffn(cfg, xp=xp, offsets=dev(dsp["offsets"]), x=t["x"], W_gu=t["W_gu"],
+                       W_down=t["W_down"], ye=ye, ws=ws)
+    check_status(ws)
+    x64, Wgu, Wd = f64(t["x"]), f64(t["W_gu"]), f64(t["W_down"])
+    got = host(ye)
+    for e in range(E):
+        a, b = dsp["offsets"][e], dsp["offsets"][e + 1]
+        if b > a:
+            ref = O.expert_ffn(x64[dsp["row_token"][a:b]], Wgu[e], Wd[e], act, clamp)
+            assert np.abs(got[a:b] - ref).max() <= 1e-4
+    if S:
+        ref = O.expert_ffn(x64, Wgu[E], Wd[E], act, clamp)
+        assert np.abs(got[N * k:] - ref).max() <= 1e-4

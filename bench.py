@@ -262,6 +262,22 @@ def run_ours(args):
     barrier(world)
     launch_ms, calls = nat.moe_profile_end(16)
     assert layer.check_status() == 0
+
+    # the same steps replayed from a CUDA graph (one launch per step instead of eight)
+    layer.forward_graphed(x, y, modality=mod)
+    for _ in range(args.warmup):
+        layer.forward_graphed(x, y, modality=mod)
+    barrier(world)
+    torch.cuda.synchronize()
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(args.steps):
+        layer.forward_graphed(x, y, modality=mod)
+    g1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    graph_ms = max_over_ranks(g0.elapsed_time(g1), world) / args.steps
+    assert layer.check_status() == 0
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
     ms_step = ms_total / args.steps
     value = aggregate_tokens_per_s(shape.N, world, ms_step)
@@ -346,6 +362,7 @@ def run_ours(args):
                 "serial_ms_per_step": round(serial_ms, 4)},
         "gpu_launches": per_step_launches * args.steps,
         "host_enqueue_us_per_step": round(host_us, 1),
+        "graph_ms_per_step": round(graph_ms, 4),
         "clocks": clocks,
         "cpu_baseline": cpu,
     }

@@ -34,6 +34,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // Token-tile size of the dispatch kernels (tokens ranked by one warp in order).
-constexpr int kRankTile = 128;
+constexpr int kRankTile = 32;
 
 }  // namespace moe

@@ -201,7 +201,7 @@ cudaError_t launch_rank_local(const int32_t* ids, const uint8_t* drop_mask, int6
   if (N == 0) return cudaSuccess;
   const int64_t tiles = (N + kRankTile - 1) / kRankTile;
   const size_t smem = sizeof(int32_t) * ((size_t)E + (size_t)kRankTile * k);
-  ++*launches;  // at most (1024 + 128 * 32) ints of shared memory: below the 48 KB default
+  ++*launches;  // at most (1024 + kRankTile * 32) ints of shared memory: below the 48 KB default
   rank_local_kernel<<<(unsigned)tiles, 32, smem, stream>>>(ids, drop_mask, N, k, E, local_rank,
                                                            tile_hist, status);
   return cudaGetLastError();

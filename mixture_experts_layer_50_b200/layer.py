@@ -31,6 +31,7 @@ class MoELayer:
         self.dtype = nat.BF16 if W_gu.dtype == torch.bfloat16 else nat.F32
         self.max_tokens = max_tokens
         self.ws = nat.alloc_workspace(self.config(max_tokens), device=W_gu.device)
+        self._graphs = {}
 
     @classmethod
     def from_workload(cls, shape, tensors: dict, max_tokens: Optional[int] = None):
@@ -62,6 +63,24 @@ class MoELayer:
         nat.moe_forward(self.config(N), x=x, W_g=self.W_g, W_gu=self.W_gu, W_down=self.W_down,
                         y=y, logit_offset=self.logit_offset, bias=self.bias, modality=modality,
                         route_out=route_out, ws=self.ws, stream=stream)
+        return y
+
+    def forward_graphed(self, x: torch.Tensor, y: torch.Tensor, modality=None) -> torch.Tensor:
+        """forward() replayed from a CUDA graph: the first call with a given (x, y, modality)
+        captures the layer's launches once (the library's one-time per-device set-up has
+        happened in an eager call first); later calls replay them with one graph launch.
+        The buffers must stay the same; their contents may change between calls."""
+        key = (x.data_ptr(), y.data_ptr(), None if modality is None else modality.data_ptr(),
+               x.shape[0])
+        g = self._graphs.get(key)
+        if g is None:
+            self.forward(x, modality=modality, y=y)          # eager run: one-time set-up
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.forward(x, modality=modality, y=y)
+            self._graphs[key] = g
+        g.replay()
         return y
 
     def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, modality=None,

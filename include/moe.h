@@ -110,7 +110,8 @@ typedef struct {
  * The size depends on N, d, E, k, F, n_shared, n_bias_sets and dtype only. */
 MOE_API size_t moe_workspace_size(const moe_config* cfg);
 
-/* Zero the workspace header (the device status word).  Call once after allocating. */
+/* Zero the workspace header (the device status word and the dispatch scan's ticket
+ * counter).  Call once after allocating; later calls leave the header's counter at zero. */
 MOE_API moe_status moe_workspace_init(void* ws, moe_stream_t stream);
 
 /* Capacity C = ceil(T * k / E * f) with f = cf_num / cf_den, in exact integer
@@ -252,7 +253,7 @@ MOE_API moe_status moe_forward_host(const moe_config* cfg, const void* x_host, c
  * critical loop that must not risk the implicit device synchronisation of cudaMalloc.
  * The pages have no counterpart of this call; it is a deployment convenience.
  * Scratch: a fixed 4 MiB device array inside the library (every GPU that loads the library
- * holds it until the process exits).  The call needs 4*(2*N*k + 2*ceil(N/32)*E + E + 1)
+ * holds it until the process exits).  The call needs 256 + 4*(2*N*k + 2*ceil(N/32)*E + E + 1)
  * bytes of it, each part rounded up to 256; larger requests return MOE_ERR_UNSUPPORTED
  * (e.g. N = 16384 tokens with k = 8 and E = 256 fits; N = 65536 with k = 8 does not).
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress)

@@ -10,8 +10,9 @@
 // every output is a deterministic function of ids:
 //   1. one warp per tile of kRankTile tokens walks its tokens in order with per-expert
 //      counters in shared memory (local rank) and writes the tile's histogram;
-//   2. one block scans the histograms over tiles (tile_base) and over experts (offsets),
-//      applying the capacity to the per-expert totals;
+//   2. one block per 32 experts scans the histograms over tiles (tile_base) and applies the
+//      capacity to the per-expert totals; the last block to finish scans the capped totals
+//      over the experts (offsets);
 //   3. one block per token: rank = tile_base + local rank, keep iff rank < C, row =
 //      offsets[e] + rank; the token's x row is copied to each kept row (the gather).
 #include "common.cuh"
@@ -62,37 +63,60 @@ __global__ void __launch_bounds__(32) rank_local_kernel(
   for (int e = lane; e < E; e += 32) tile_hist[(int64_t)blockIdx.x * E + e] = cnt[e];
 }
 
-// One block of 1024 threads.  Warp w owns a contiguous chunk of tiles.
+// Block b scans the tile histograms of experts [32 b, 32 b + 32): lane = expert, warp w = a
+// contiguous chunk of tiles.  The per-expert totals give demand and the capped counts; the
+// block that arrives last (a ticket taken after its counts are visible) scans the counts over
+// the experts into offsets and puts the ticket counter back to 0.  Every output is a fixed
+// function of the histograms: only which block does the final scan varies.
 __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
     const int32_t* __restrict__ tile_hist, int n_tiles, int E, int64_t C,
     int32_t* __restrict__ tile_base, int32_t* __restrict__ demand,
-    int32_t* __restrict__ counts, int32_t* __restrict__ offsets) {
-  extern __shared__ int32_t part[];  // [32][E] chunk sums, then chunk bases
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* arrive) {
+  __shared__ int32_t part[32][33];  // chunk sums [warp][lane]
   __shared__ int32_t warp_tot[32];
+  __shared__ bool s_last;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
+  const bool has_e = e < E;
   const int per = (n_tiles + 31) / 32;
   const int c0 = min(w * per, n_tiles), c1 = min(c0 + per, n_tiles);
-  for (int e = lane; e < E; e += 32) {
-    int32_t s = 0;
+  int32_t s = 0;
+  if (has_e) {
+#pragma unroll 8
     for (int c = c0; c < c1; ++c) s += tile_hist[(int64_t)c * E + e];
-    part[w * E + e] = s;
   }
+  part[w][lane] = s;
   __syncthreads();
-  // per expert: scan over chunks; the total is the demand, the capped total the count
-  int32_t my_count = 0;
-  const int e_me = threadIdx.x;
-  if (e_me < E) {
-    int32_t run = 0;
-    for (int c = 0; c < 32; ++c) {
-      const int32_t v = part[c * E + e_me];
-      part[c * E + e_me] = run;
+  int32_t run = 0, total = 0;
+  for (int j = 0; j < 32; ++j) {
+    const int32_t v = part[j][lane];
+    run += j < w ? v : 0;
+    total += v;
+  }
+  if (has_e) {
+#pragma unroll 8
+    for (int c = c0; c < c1; ++c) {
+      const int32_t v = tile_hist[(int64_t)c * E + e];
+      tile_base[(int64_t)c * E + e] = run;
       run += v;
     }
-    demand[e_me] = run;
-    my_count = (C > 0 && run > C) ? (int32_t)C : run;
-    counts[e_me] = my_count;
+    if (w == 0) {
+      demand[e] = total;
+      counts[e] = (C > 0 && total > C) ? (int32_t)C : total;
+      __threadfence();
+    }
   }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int32_t ticket = atomicAdd(arrive, 1);
+    s_last = ticket == (int32_t)gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
   // exclusive scan of counts over the experts (E <= 1024: one expert per thread)
+  const int e_me = threadIdx.x;
+  const int32_t my_count = e_me < E ? *((volatile const int32_t*)counts + e_me) : 0;
   int32_t incl = my_count;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -114,14 +138,7 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
   const int32_t excl = incl - my_count + (w > 0 ? warp_tot[w - 1] : 0);
   if (e_me < E) offsets[e_me] = excl;
   if (e_me == E - 1) offsets[E] = excl + my_count;
-  // per tile bases
-  for (int e = lane; e < E; e += 32) {
-    int32_t run = part[w * E + e];
-    for (int c = c0; c < c1; ++c) {
-      tile_base[(int64_t)c * E + e] = run;
-      run += tile_hist[(int64_t)c * E + e];
-    }
-  }
+  if (threadIdx.x == 0) *arrive = 0;
 }
 
 template <typename V>
@@ -209,22 +226,12 @@ cudaError_t launch_rank_local(const int32_t* ids, const uint8_t* drop_mask, int6
 
 cudaError_t launch_dispatch_scan(const int32_t* tile_hist, int64_t N, int E, int64_t C,
                                  int32_t* tile_base, int32_t* demand, int32_t* counts,
-                                 int32_t* offsets, cudaStream_t stream, int* launches) {
+                                 int32_t* offsets, int32_t* arrive, cudaStream_t stream,
+                                 int* launches) {
   const int tiles = (int)((N + kRankTile - 1) / kRankTile);
-  const size_t smem = sizeof(int32_t) * 32 * (size_t)E;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(dispatch_scan_kernel,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               32 * 1024 * (int)sizeof(int32_t));
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
   ++*launches;
-  dispatch_scan_kernel<<<1, 1024, smem, stream>>>(tile_hist, tiles, E, C, tile_base, demand,
-                                                  counts, offsets);
+  dispatch_scan_kernel<<<(E + 31) / 32, 1024, 0, stream>>>(tile_hist, tiles, E, C, tile_base,
+                                                           demand, counts, offsets, arrive);
   return cudaGetLastError();
 }
 

@@ -124,6 +124,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) |
          ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
+// TMEM columns the 1-SM kernel allocates: two BN-column accumulators, rounded up to the
+// power of two the allocator requires (BN = 192 -> 512).
+template <int BN>
+__host__ __device__ constexpr int tmem_cols() {
+  return 2 * BN <= 32 ? 32 : 2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512;
+}
 // Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both K-major.
 template <int BN>
 __device__ __forceinline__ constexpr uint32_t idesc_bf16() {
@@ -280,7 +286,9 @@ __device__ __forceinline__ void decode_tile(int tile, const int* s_start, int G,
   }
 }
 
-__device__ __forceinline__ float silu_f(float a) { return a / (1.0f + __expf(-a)); }
+// SiLU(a) = a * sigmoid(a) with the fast exponential and division (the result is rounded to
+// bf16 right after); for a below about -88 the denominator overflows and the result is 0.
+__device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
 // One epilogue warp drains its 32 TMEM lanes (rows row_base + lane of the output tile) of an
 // accumulator: activation, packing, per-warp staging in shared memory, then coalesced 16-byte
@@ -447,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(s_tmem)),
-                 "r"(2 * BN));
+                 "r"(tmem_cols<BN>()));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   __syncthreads();
@@ -586,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(2 * BN));
+                 "r"(tmem_cols<BN>()));
   }
 }
 
@@ -820,6 +828,345 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---- token-in-N ("swapped") variant ---------------------------------------------------------
+// Groups of a few hundred rows leave most of a 128-row M tile idle in their last tile.  This
+// variant puts the weights in the MMA's M dimension and the group's rows in N, which tcgen05
+// takes in steps of 16:  D[w][t] = sum_k W[w][k] X[t][k].  A tile is (group, weight block,
+// up to 256 of the group's rows).  The weight block is one 128-row M operand built from two
+// 64-row TMA boxes: the gate rows f0..f0+63 and the up rows F+f0..F+f0+63 for SwiGLU, or
+// output columns o0..o0+127 otherwise.  Per MMA the tensor core reads the same operand bytes
+// as the 128x256 tile of the 1-SM kernel.  For SwiGLU the up warps (TMEM lanes 64-127) pass
+// their values through shared memory to the gate warps (lanes 0-63), which apply the
+// activation.  The epilogue transposes 32x32 blocks through shared memory so that
+// out[row][feature] is written with coalesced 16-byte stores.  Tiles inside a group run
+// weight block outer, row block inner.
+constexpr int kSwapRows = 256;      // group rows per tile (MMA N <= 256)
+constexpr int kSwapBox = 128;       // rows per TMA box of the N operand
+constexpr int kSwapWBox = 64;       // rows per TMA box of the weight operand
+constexpr int kSwapStageW = 128 * BK * 2;          // the 128-row weight operand (16 KB)
+constexpr int kSwapStageX = kSwapRows * BK * 2;    // up to 256 group rows (32 KB)
+constexpr int kSwapStagingPerWarp = 32 * 64;       // 32 rows x 32 bf16 features
+// SwiGLU exchange, per chunk of 32 rows and per gate/up warp pair: the gate warp's values of
+// rows 16..31 and the up warp's values of rows 0..15 (fp32), double-buffered over chunks
+constexpr int kSwapXchg = 2 * 2 * 2 * 16 * 32 * 4;
+
+template <int STAGES>
+struct LayoutSwap {
+  static constexpr int kStage = kSwapStageW + kSwapStageX;
+  static constexpr int kOffStaging = STAGES * kStage;
+  static constexpr int kOffXchg = kOffStaging + 4 * kSwapStagingPerWarp;
+  static constexpr int kOffBar = kOffXchg + kSwapXchg;
+  static constexpr int kNumBars = 2 * STAGES + 5;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffStart = kOffMisc + 16;
+  static size_t bytes(int groups) { return 1024 + kOffStart + 4 * (size_t)(groups + 1); }
+};
+
+// Tile -> (group, weight block, row block).  Inside a group the smaller panel stays resident
+// in L2 while the other streams: a group with more rows than weight rows (w_rows) runs row
+// blocks outer and weight blocks inner, any other group the reverse.
+__device__ __forceinline__ void decode_tile_swap(int tile, const int* s_start, int G, int nw,
+                                                 int w_rows, int& g, int& w_blk, int& r_blk) {
+  int lo = 0, hi = G;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_start[mid] <= tile) lo = mid; else hi = mid;
+  }
+  g = lo;
+  const int r = tile - s_start[g];
+  const int rt = (s_start[g + 1] - s_start[g]) / nw;
+  if (rt * kSwapRows > w_rows) {
+    r_blk = r / nw;
+    w_blk = r - r_blk * nw;
+  } else {
+    w_blk = r / rt;
+    r_blk = r - w_blk * rt;
+  }
+}
+
+// Named barrier over the four epilogue warps (id 1; id 0 is __syncthreads).
+__device__ __forceinline__ void epilogue_bar() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+// The same barrier, returning whether any of the 128 threads passed true: the four warps
+// take the same exit decision before they meet at epilogue_bar().
+__device__ __forceinline__ bool epilogue_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
+template <int EPI, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmX,
+                             const __grid_constant__ CUtensorMap tmXs,
+                             const __grid_constant__ CUtensorMap tmW, const Args p) {
+  using L = LayoutSwap<STAGES>;
+  constexpr int kOutPerTile = (EPI == kEpiSwiglu) ? 64 : 128;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* staging = smem + L::kOffStaging;
+  float* xchg = reinterpret_cast<float*>(smem + L::kOffXchg);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = bars + 2 * STAGES + 2;
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
+  int* s_start = reinterpret_cast<int*>(smem + L::kOffStart);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.n_routed + p.has_shared;
+  const int nw = (p.n_out + kOutPerTile - 1) / kOutPerTile;
+  const int w_rows = EPI == kEpiSwiglu ? 2 * p.n_out : p.n_out;
+  const int nk = (p.K + BK - 1) / BK;
+  auto group_rows = [&](int g) {
+    return g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
+  };
+
+  if (warp == 0) {
+    const int per = (G + 31) / 32;
+    const int g0 = min(lane * per, G), g1 = min(g0 + per, G);
+    int local = 0;
+    for (int g = g0; g < g1; ++g) local += ((group_rows(g) + kSwapRows - 1) / kSwapRows) * nw;
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    for (int g = g0; g < g1; ++g) {
+      s_start[g] = run;
+      run += ((group_rows(g) + kSwapRows - 1) / kSwapRows) * nw;
+    }
+    if (lane == 31) s_start[G] = incl;
+    if (lane == 0) {
+      for (int i = 0; i < STAGES; ++i) {
+        mbar_init(&full[i], 1);
+        mbar_init(&empty[i], 1);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&tfull[i], 1);
+        mbar_init(&tempty[i], 128);
+      }
+      mbar_init(drain, 1);
+      *s_abort = 0;
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+  } else if (warp == 1) {
+    // two accumulator buffers of up to 256 columns: 512 columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(s_tmem)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+  const int total = s_start[G];
+
+  if (warp == 0) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        int g, w_blk, r_blk;
+        decode_tile_swap(tile, s_start, G, nw, w_rows, g, w_blk, r_blk);
+        const bool sh = g >= p.n_routed;
+        const int rows = min(kSwapRows, group_rows(g) - r_blk * kSwapRows);
+        const int boxes = (rows + kSwapBox - 1) / kSwapBox;
+        const int x_row = (sh ? p.shared_a_row0 : p.offsets[g]) + r_blk * kSwapRows;
+        const CUtensorMap* mX = sh ? &tmXs : &tmX;
+        const int w_row0 = w_blk * kOutPerTile;
+        const int w_row1 = EPI == kEpiSwiglu ? p.up_row0 + w_blk * 64 : w_row0 + 64;
+        const uint32_t bytes = (uint32_t)(kSwapStageW + boxes * kSwapBox * BK * 2);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + stage * L::kStage;
+          mbar_expect_tx(&full[stage], bytes);
+          tma_load_3d(st, &tmW, &full[stage], kb * BK, w_row0, g);
+          tma_load_3d(st + kSwapWBox * BK * 2, &tmW, &full[stage], kb * BK, w_row1, g);
+          for (int b = 0; b < boxes; ++b)
+            tma_load_2d(st + kSwapStageW + b * kSwapBox * BK * 2, mX, &full[stage], kb * BK,
+                        x_row + b * kSwapBox);
+          ++armed;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        for (int i = 0; i < STAGES && i < armed; ++i) {
+          stage = (stage + STAGES - 1) % STAGES;
+          if (stage == STAGES - 1) phase ^= 1;
+          const uint64_t t0 = global_timer_ns();
+          while (!mbar_try_wait(&full[stage], phase) && global_timer_ns() - t0 < kWaitLimitNs) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
+        int g, w_blk, r_blk;
+        decode_tile_swap(tile, s_start, G, nw, w_rows, g, w_blk, r_blk);
+        const int rows = min(kSwapRows, group_rows(g) - r_blk * kSwapRows);
+        const int n_mma = (rows + 15) & ~15;
+        const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                               ((uint32_t)(n_mma >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], aph ^ 1, s_abort, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + (uint32_t)(acc * 256);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(&full[stage], phase, s_abort, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t s0 = smem_u32(smem + stage * L::kStage);
+          const uint32_t x0 = s0 + kSwapStageW;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            mma_bf16(d0, sw128_desc(s0 + kk * 32), sw128_desc(x0 + kk * 32), idesc,
+                     (kb | kk) != 0 ? 1u : 0u);
+          mma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) mma_commit(&tfull[acc]);
+      }
+      if (!ok) {
+        mma_commit(drain);
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ================= epilogue (warps 2..5) =================
+    const int q = warp & 3;  // TMEM lanes 32q..32q+31 = weight rows 32q + lane of the operand
+    uint8_t* stg = staging + (warp - 2) * kSwapStagingPerWarp;
+    __nv_bfloat16* stg_h = reinterpret_cast<__nv_bfloat16*>(stg);
+    __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(p.out);
+    // SwiGLU: warp q = 0, 1 holds the gate rows of features f0 + 32q + lane, warp q + 2 their up
+    // rows.  Per chunk of 32 group rows the gate warp computes rows 0..15 and the up warp rows
+    // 16..31; each passes the other the half it needs through xchg.
+    const bool up_warp = EPI == kEpiSwiglu && q >= 2;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      int g, w_blk, r_blk;
+      decode_tile_swap(tile, s_start, G, nw, w_rows, g, w_blk, r_blk);
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      const bool ready = mbar_wait(&tfull[acc], aph, s_abort, p.status);
+      // the four warps take the same exit decision (they meet at named barriers below), and
+      // this barrier also separates the previous tile's exchange reads from this tile's writes
+      if (epilogue_any(!ready)) break;
+      tc_fence_after();
+      const bool sh = g >= p.n_routed;
+      const int rows = min(kSwapRows, group_rows(g) - r_blk * kSwapRows);
+      const int64_t out_row0 =
+          (int64_t)(sh ? p.shared_out_row0 : p.offsets[g]) + (int64_t)r_blk * kSwapRows;
+      const int chunks = (rows + 31) / 32;
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
+      for (int c = 0; c < chunks; ++c) {
+        float v[32];
+        tmem_ld32(t_row + c * 32, v);
+        tmem_ld_wait();
+        if (c == chunks - 1) {
+          // every TMEM read of this accumulator is done: hand it back to the MMA warp
+          tc_fence_before();
+          mbar_arrive(&tempty[acc]);
+        }
+        int r0 = 0, nr = 32;  // this warp's rows of the chunk
+        if constexpr (EPI == kEpiSwiglu) {
+          float* xb = xchg + ((c & 1) * 2 + (q & 1)) * 1024;  // [gate 16..31 | up 0..15]
+          if (!up_warp) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) xb[i * 32 + lane] = v[16 + i];
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) xb[512 + i * 32 + lane] = v[i];
+          }
+          epilogue_bar();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float gg = up_warp ? xb[i * 32 + lane] : v[i];
+            float uu = up_warp ? v[16 + i] : xb[512 + i * 32 + lane];
+            if (p.clamp > 0.f) {
+              gg = fminf(fmaxf(gg, -p.clamp), p.clamp);
+              uu = fminf(fmaxf(uu, -p.clamp), p.clamp);
+            }
+            v[i] = silu_f(gg) * uu;
+          }
+          r0 = up_warp ? 16 : 0;
+          nr = 16;
+        } else if (EPI == kEpiRelu) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = fmaxf(v[i], 0.f);
+        }
+        // transpose: staging row r holds the warp's 32 features of group row c*32 + r0 + r
+        // (64-byte rows: the stores below and the 16-byte reads are conflict-free)
+#pragma unroll
+        for (int r = 0; r < 32; ++r)
+          if (r < nr) stg_h[r * 32 + lane] = __float2bfloat16_rn(v[r]);
+        __syncwarp();
+        const int feat0 = w_blk * kOutPerTile + (q & (EPI == kEpiSwiglu ? 1 : 3)) * 32;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = i * 8 + (lane >> 2);
+          const int piece = lane & 3;
+          const int col = feat0 + piece * 8;
+          const int grow = c * 32 + r0 + r;
+          if (r < nr && grow < rows && col < p.n_out) {
+            const uint4 val = *reinterpret_cast<const uint4*>(stg + r * 64 + piece * 16);
+            *reinterpret_cast<uint4*>(outp + (out_row0 + grow) * p.ld_out + col) = val;
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(512));
+  }
+}
+
 // ---- host side -------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -925,13 +1272,46 @@ cudaError_t launch_2sm(const GroupedGemm& g, const CUtensorMap& mA, const CUtens
   return cudaGetLastError();
 }
 
+template <int EPI, int STAGES>
+cudaError_t launch_swap(const GroupedGemm& g, const CUtensorMap& mX, const CUtensorMap& mXs,
+                        const CUtensorMap& mW, cudaStream_t stream, int grid) {
+  auto kern = grouped_gemm_swap_kernel<EPI, STAGES>;
+  const size_t smem = LayoutSwap<STAGES>::bytes(g.n_routed + g.has_shared);
+  static bool done[kMaxDev] = {};
+  const cudaError_t e = allow_max_smem(kern, done);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, stream>>>(mX, mXs, mW, make_args(g));
+  return cudaGetLastError();
+}
+
 // Which kernel a bf16 grouped GEMM uses.  The 2-SM kernel tiles 256 rows per group, so it
 // pays off only when groups are large, and there only for the down projection: for gate/up it
 // ran no faster than the 1-SM kernel while reading its operands from DRAM 2.6x over (5.75 GB vs
 // 2.20 GB on the 16384-token Mixtral-shaped layer), where the 1-SM kernel reads each byte once.
 // Small groups keep the 1-SM kernel's 128-row tiles.
-// MOE_B200_GEMM_PATH=1sm|1sm128|2sm overrides the choice (the tests cover every kernel).
+// MOE_B200_GEMM_PATH=1sm|1sm128|2sm|swap overrides the choice (the tests cover every kernel).
 const char* path_override() { return std::getenv("MOE_B200_GEMM_PATH"); }
+
+// Average rows of a routed group, as the caller estimates it (the true sizes stay on the
+// device).  The token-in-N kernel is taken only on request (MOE_B200_GEMM_PATH=swap): it
+// pads a DeepSeek-V3-shaped prefill to 1.02x the MMA rows where 128-row tiles pad to 1.20x,
+// yet measured 17-20 % slower there (and 6 % slower on the capacity configs), so the
+// automatic choice keeps the 1-SM and 2-SM kernels.
+constexpr int64_t kSwapMaxRows = 0;
+
+int64_t avg_group_rows(const GroupedGemm& g) {
+  if (g.rows_per_group_hint >= 0) return g.rows_per_group_hint;
+  return g.n_routed > 0 ? g.max_rows_routed / g.n_routed : g.shared_rows;
+}
+
+bool use_swap(const GroupedGemm& g) {
+  if (g.epilogue == kEpiStoreF32 || g.k_splits > 1) return false;
+  if (const char* env = path_override()) {
+    if (std::strcmp(env, "swap") == 0) return true;
+    if (std::strncmp(env, "1sm", 3) == 0 || std::strcmp(env, "2sm") == 0) return false;
+  }
+  return g.n_routed > 0 && avg_group_rows(g) < kSwapMaxRows;
+}
 
 bool use_two_sm(const GroupedGemm& g) {
   if (g.epilogue == kEpiStoreF32 || g.k_splits > 1) return false;
@@ -941,7 +1321,8 @@ bool use_two_sm(const GroupedGemm& g) {
   }
   if (g.epilogue != kEpiStoreBf16) return false;
   const int groups = g.n_routed + g.has_shared;
-  const int64_t rows = (g.n_routed > 0 ? g.max_rows_routed : 0) + (g.has_shared ? g.shared_rows : 0);
+  const int64_t rows = (g.n_routed > 0 ? avg_group_rows(g) * g.n_routed : 0) +
+                       (g.has_shared ? g.shared_rows : 0);
   return rows >= 1024LL * groups;
 }
 
@@ -967,15 +1348,58 @@ int pick_bn_1sm(const GroupedGemm& g) {
 
 }  // namespace tc
 
+// N width of the fp32-store (router) tiles: the fewest padded columns, then the wider tile.
+int router_tile_n(int n_out) {
+  if (n_out <= 32) return 32;
+  if (n_out <= 64) return 64;
+  if (n_out <= 128) return 128;
+  if (n_out <= 192) return 192;
+  int best = 256;
+  int64_t best_cols = (n_out + 255) / 256 * 256;
+  for (int bn : {192, 128}) {
+    const int64_t cols = (int64_t)(n_out + bn - 1) / bn * bn;
+    if (cols < best_cols) {
+      best = bn;
+      best_cols = cols;
+    }
+  }
+  return best;
+}
+
 cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* launches,
                                 const char** why) {
   using namespace tc;
   const int groups = g.n_routed + g.has_shared;
   if (groups == 0) return cudaSuccess;
+  if (use_swap(g)) {
+    CUtensorMap mX, mXs, mW;
+    const void* x_ptr = g.a != nullptr ? g.a : g.a_shared;
+    const int64_t x_rows = g.a != nullptr ? g.rows_a : g.rows_a_shared;
+    if (!make_map(&mX, x_ptr, g.K, std::max<int64_t>(x_rows, 1), 0, kSwapBox) ||
+        !make_map(&mXs, g.a_shared != nullptr ? g.a_shared : x_ptr, g.K,
+                  std::max<int64_t>(g.a_shared != nullptr ? g.rows_a_shared : x_rows, 1), 0,
+                  kSwapBox) ||
+        !make_map(&mW, g.b, g.K, g.rows_b, g.groups_b, kSwapWBox)) {
+      *why = "cuTensorMapEncodeTiled failed (pointer alignment, strides or driver entry point)";
+      return cudaErrorInvalidValue;
+    }
+    const int out_per_tile = g.epilogue == kEpiSwiglu ? 64 : 128;
+    const int64_t nw = (g.n_out + out_per_tile - 1) / out_per_tile;
+    int64_t rtiles = 0;
+    if (g.n_routed > 0) rtiles += (g.max_rows_routed + kSwapRows - 1) / kSwapRows + g.n_routed;
+    if (g.has_shared) rtiles += (g.shared_rows + kSwapRows - 1) / kSwapRows;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), rtiles * nw));
+    ++*launches;
+    switch (g.epilogue) {
+      case kEpiSwiglu: return launch_swap<kEpiSwiglu, 4>(g, mX, mXs, mW, stream, grid);
+      case kEpiRelu: return launch_swap<kEpiRelu, 4>(g, mX, mXs, mW, stream, grid);
+      default: return launch_swap<kEpiStoreBf16, 4>(g, mX, mXs, mW, stream, grid);
+    }
+  }
   int BN;
   const bool two_sm = use_two_sm(g);
   if (g.epilogue == kEpiStoreF32) {
-    BN = g.n_out <= 32 ? 32 : g.n_out <= 64 ? 64 : g.n_out <= 128 ? 128 : (g.n_out % 256 == 0 || g.n_out > 384) ? 256 : 128;
+    BN = router_tile_n(g.n_out);
   } else {
     BN = two_sm ? 256 : pick_bn_1sm(g);
   }
@@ -1026,6 +1450,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
         case 32: return launch_t<32, kEpiStoreF32, 8>(g, mA, mAs, mB, stream, grid);
         case 64: return launch_t<64, kEpiStoreF32, 8>(g, mA, mAs, mB, stream, grid);
         case 128: return launch_t<128, kEpiStoreF32, 6>(g, mA, mAs, mB, stream, grid);
+        case 192: return launch_t<192, kEpiStoreF32, 5>(g, mA, mAs, mB, stream, grid);
         default: return launch_t<256, kEpiStoreF32, 4>(g, mA, mAs, mB, stream, grid);
       }
   }

@@ -32,7 +32,8 @@ cudaError_t launch_rank_local(const int32_t* ids, const uint8_t* drop_mask, int6
 // and offsets (exclusive scan of counts, E + 1 entries).
 cudaError_t launch_dispatch_scan(const int32_t* tile_hist, int64_t N, int E, int64_t C,
                                  int32_t* tile_base, int32_t* demand, int32_t* counts,
-                                 int32_t* offsets, cudaStream_t stream, int* launches);
+                                 int32_t* offsets, int32_t* arrive, cudaStream_t stream,
+                                 int* launches);
 // Pass 3: capacity decision, slot rows, row -> token map, drop mask, and (when xp is not
 // null) the gather of x rows into the per-expert layout.
 cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_rank,
@@ -109,6 +110,8 @@ struct GroupedGemm {
   int64_t ld_out;          // elements
   int64_t rows_out;
   int64_t max_rows_routed; // upper bound of offsets[n_routed] (grid sizing)
+  int64_t rows_per_group_hint = -1;  // >= 0: the caller's estimate of a routed group's
+                                     // rows (kernel choice); else max_rows_routed / n_routed
   int* status;
   int k_splits = 1;        // > 1 (fp32 store only): K split in slices, slice s written at
   int64_t split_rows = 0;  // out rows [s * split_rows, ...): partial sums, col_bias ignored
@@ -116,5 +119,7 @@ struct GroupedGemm {
 
 cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* launches,
                                 const char** why);
+// N width of the tiles of an fp32-store GEMM with n_out columns (the router).
+int router_tile_n(int n_out);
 
 }  // namespace moe

@@ -70,9 +70,9 @@ struct Ws {
 
 size_t el_size(const moe_config& c) { return c.dtype == MOE_DT_BF16 ? 2 : 4; }
 
-// Router split-K: at most this many K slices, used for calls of at most kSplitMaxTokens tokens.
+// Router split-K: at most this many K slices.
 constexpr int kMaxLogitSplits = 16;
-constexpr int64_t kSplitMaxTokens = 512;
+int router_splits(const moe_config& c);
 
 // Rows of the padded dispatch buffer [E][C] (0 without a capacity).
 int64_t padded_rows(const moe_config& c) { return c.capacity > 0 ? (int64_t)c.E * c.capacity : 0; }
@@ -112,7 +112,8 @@ Ws layout(const moe_config& c) {
   w.y_stage2 = take(N * d * el);
   w.balance = take(moe::balance_scratch_bytes((int64_t)N, (int)E, std::max(1, c.n_bias_sets)));
   w.offsets_pad = take((E + 1) * 4);
-  w.logit_parts = take(N <= (size_t)kSplitMaxTokens ? (size_t)kMaxLogitSplits * N * E * 4 : 0);
+  const int splits = router_splits(c);
+  w.logit_parts = take(splits > 1 ? (size_t)splits * N * E * 4 : 0);
   w.total = off;
   return w;
 }
@@ -121,6 +122,10 @@ template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
 }
+
+// Ticket counter of the dispatch scan: an int in the zeroed 256-byte status region (the
+// status word is at byte 0); every scan leaves it at zero.
+int32_t* arrive_counter(void* ws, const Ws& L) { return at<int32_t>(ws, L.status + 128); }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -207,13 +212,14 @@ struct LogitSrc {
 
 LogitSrc finished_logits(const float* z) { return LogitSrc{z, 1, 0, nullptr, nullptr}; }
 
-// Number of K slices for the router GEMM: small launches (few 128-token tiles) stream W_g
-// through a handful of CTAs, so their K loop is split over more CTAs (at most
-// kMaxLogitSplits); the partial logits sit in the workspace.
+// Number of K slices for the router GEMM: a launch with few output tiles (few 128-token
+// tiles, or one tile column) would run on a fraction of the SMs, so its K loop is split over
+// more CTAs (about 128 work items, at most kMaxLogitSplits slices); the partial logits sit
+// in the workspace and the top-k kernel adds them in slice order.
 
 int router_splits(const moe_config& c) {
-  if (c.dtype != MOE_DT_BF16 || c.N == 0 || c.N > kSplitMaxTokens) return 1;
-  const int bn = c.E <= 32 ? 32 : c.E <= 64 ? 64 : c.E <= 128 ? 128 : (c.E % 256 == 0 || c.E > 384) ? 256 : 128;
+  if (c.dtype != MOE_DT_BF16 || c.N == 0) return 1;
+  const int bn = moe::router_tile_n(c.E);
   const int64_t tiles = ((c.N + 127) / 128) * ((c.E + bn - 1) / bn);
   const int nk = (c.d + 63) / 64;
   int64_t want = 128 / tiles;
@@ -295,8 +301,8 @@ moe_status stage_dispatch(const moe_config& c, const Ws& L, void* ws, const int3
            "rank pass");
   prof_mark(st);
   MOE_CUDA(moe::launch_dispatch_scan(at<int32_t>(ws, L.tile_hist), c.N, c.E, C,
-                                     at<int32_t>(ws, L.tile_base), demand, counts, offsets, st,
-                                     launches),
+                                     at<int32_t>(ws, L.tile_base), demand, counts, offsets,
+                                     arrive_counter(ws, L), st, launches),
            "scan pass");
   prof_mark(st);
   MOE_CUDA(moe::launch_dispatch_scatter(ids, at<int32_t>(ws, L.local_rank),
@@ -349,6 +355,9 @@ moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
   g1.ld_out = c.F;
   g1.rows_out = Nk + c.n_shared * c.N;
   g1.max_rows_routed = Nk;
+  // kernel choice from the configuration alone, so the compact and the padded layouts of
+  // the same call take the same kernels
+  g1.rows_per_group_hint = c.N * (int64_t)c.k / c.E;
   g1.status = status;
   const char* why = "gate/up GEMM launch";
   MOE_CUDA(moe::launch_grouped_gemm(g1, st, launches, &why), why);
@@ -375,6 +384,7 @@ moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
   g2.ld_out = c.d;
   g2.rows_out = g2.rows_a;
   g2.max_rows_routed = Nk;
+  g2.rows_per_group_hint = g1.rows_per_group_hint;
   g2.status = status;
   why = "down GEMM launch";
   MOE_CUDA(moe::launch_grouped_gemm(g2, st, launches, &why), why);
@@ -663,7 +673,8 @@ moe_status moe_permute_padded(const moe_config* cfg, const int32_t* ids,
            "rank pass");
   MOE_CUDA(moe::launch_dispatch_scan(at<int32_t>(ws, L.tile_hist), c.N, c.E, c.capacity,
                                      at<int32_t>(ws, L.tile_base), at<int32_t>(ws, L.demand),
-                                     counts, at<int32_t>(ws, L.offsets), st, &launches),
+                                     counts, at<int32_t>(ws, L.offsets),
+                                     arrive_counter(ws, L), st, &launches),
            "scan pass");
   MOE_CUDA(moe::launch_pad_offsets(c.E, c.capacity, offsets_pad, st, &launches), "pad offsets");
   MOE_CUDA(moe::launch_dispatch_scatter(ids, at<int32_t>(ws, L.local_rank),
@@ -719,7 +730,8 @@ moe_status moe_forward_padded(const moe_config* cfg, const void* x, const void* 
            "rank pass");
   MOE_CUDA(moe::launch_dispatch_scan(at<int32_t>(ws, L.tile_hist), c.N, c.E, c.capacity,
                                      at<int32_t>(ws, L.tile_base), demand, counts,
-                                     at<int32_t>(ws, L.offsets), st, &launches),
+                                     at<int32_t>(ws, L.offsets), arrive_counter(ws, L), st,
+                                     &launches),
            "scan pass");
   MOE_CUDA(moe::launch_pad_offsets(c.E, c.capacity, offsets_pad, st, &launches), "pad offsets");
   MOE_CUDA(moe::launch_dispatch_scatter(ids, at<int32_t>(ws, L.local_rank),
@@ -887,6 +899,9 @@ moe_status moe_route_static(const moe_config* cfg, const float* logits, const fl
     off = align_up(off + bytes, 256);
     return o;
   };
+  // o_arrive: the scan's ticket counter; zero when the module loads, and every scan leaves
+  // it at zero
+  const size_t o_arrive = take(256);
   const size_t o_rank = take(Nk * 4), o_hist = take(tiles * c.E * 4),
                o_base = take(tiles * c.E * 4), o_offs = take(((size_t)c.E + 1) * 4),
                o_slot = take(Nk * 4);
@@ -907,7 +922,8 @@ moe_status moe_route_static(const moe_config* cfg, const float* logits, const fl
            "rank pass");
   MOE_CUDA(moe::launch_dispatch_scan(at<int32_t>(scratch, o_hist), c.N, c.E, c.capacity,
                                      at<int32_t>(scratch, o_base), demand, counts,
-                                     at<int32_t>(scratch, o_offs), st, &launches),
+                                     at<int32_t>(scratch, o_offs),
+                                     at<int32_t>(scratch, o_arrive), st, &launches),
            "scan pass");
   MOE_CUDA(moe::launch_dispatch_scatter(ids, at<int32_t>(scratch, o_rank),
                                         at<int32_t>(scratch, o_base),

@@ -104,6 +104,34 @@ def test_route_full_size_v41flash_and_zipf_capacity():
         assert int(got["drop_mask"].sum()) > 0
 
 
+@pytest.mark.parametrize("N,d,E", [(16, 256, 8), (300, 512, 160), (1000, 256, 384),
+                                   (8192, 512, 256), (777, 136, 1024), (4096, 256, 8)])
+def test_router_gemm_logits(N, d, E):
+    """z = x . W_g on the tensor cores (tile widths 32 to 256, split K for few tiles) against
+    float64, element by element, within an fp32 accumulation bound."""
+    g = torch.Generator().manual_seed(N + E)
+    x = torch.randn(N, d, generator=g).to(torch.bfloat16)
+    W_g = (0.05 * torch.randn(E, d, generator=g)).to(torch.bfloat16)
+    cfg = nat.make_config(N, d, E, 2, 64)
+    ws = nat.alloc_workspace(cfg)
+    z = torch.empty((N, E), dtype=torch.float32, device="cuda")
+    out = dict(ids=torch.empty((N, 2), dtype=torch.int32, device="cuda"),
+               gates=torch.empty((N, 2), dtype=torch.float32, device="cuda"),
+               counts=torch.empty(E, dtype=torch.int32, device="cuda"),
+               demand=torch.empty(E, dtype=torch.int32, device="cuda"),
+               drop_mask=torch.empty((N, 2), dtype=torch.uint8, device="cuda"))
+    nat.moe_route(cfg, x=x.cuda(), W_g=W_g.cuda(), logits_out=z, ws=ws, **out)
+    check_status(ws)
+    x64, w64 = f64(x), f64(W_g)
+    z_o = O.router_logits(x64, w64)
+    bound = 1e-4 * (np.abs(x64) @ np.abs(w64).T) + 1e-30
+    err = np.abs(host(z).astype(np.float64) - z_o)
+    assert (err <= bound).all(), float((err / bound).max())
+    # the routing of those logits, bit for bit
+    assert_route_equal({k_: host(v) for k_, v in out.items()}, host(z), 2, O.SOFTMAX, 1, None,
+                       None, E, 0)
+
+
 def test_route_reports_bad_modality_flag():
     N, E = 64, 8
     z = W.random_logits(N, E, 5)
@@ -180,10 +208,11 @@ FFN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["1sm", "1sm128", "2sm"])
+@pytest.mark.parametrize("path", ["1sm", "1sm128", "2sm", "swap"])
 @pytest.mark.parametrize("N,d,E,k,F,S,act,clamp", FFN_CASES)
 def test_expert_ffn(N, d, E, k, F, S, act, clamp, path, monkeypatch):
-    # every grouped-GEMM variant (1-SM 128x256 and 128x128 tiles, 2-SM 256x256) on every case
+    # every grouped-GEMM variant (1-SM 128x256 and 128x128 tiles, 2-SM 256x256, and the
+    # token-in-N kernel with weights in M) on every case
     monkeypatch.setenv("MOE_B200_GEMM_PATH", path)
     shape = W.LayerShape("t", N=N, d=d, E=E, k=k, F=F, n_shared=S, act=act, clamp=clamp,
                          w_std=0.08, seed=N + d)
@@ -212,6 +241,38 @@ def test_expert_ffn(N, d, E, k, F, S, act, clamp, path, monkeypatch):
     got = host(ye)
     rows = np.r_[0:M, N * k:N * k + S * N]
     assert_close_layer(got[rows], ref[rows])
+
+
+@pytest.mark.parametrize("path", ["1sm", "swap"])
+def test_expert_ffn_group_sizes_around_the_tile_edges(path, monkeypatch):
+    """Groups of 0, 1, 15, 16, 17, 31, 32, 33, 127, 128, 129, 255, 256, 257 rows: the token-in-N
+    kernel rounds a group's last row block up to 16 rows and loads it in 32-row boxes; the
+    1-SM kernel pads to 128-row tiles."""
+    monkeypatch.setenv("MOE_B200_GEMM_PATH", path)
+    sizes = [0, 1, 15, 16, 17, 31, 32, 33, 127, 128, 129, 255, 256, 257]
+    E, k, d, F = len(sizes), 1, 256, 384
+    N = sum(sizes)
+    shape = W.LayerShape("t", N=N, d=d, E=E, k=k, F=F, n_shared=1, act=W.SWIGLU, clamp=0.0,
+                         w_std=0.08, seed=11)
+    t = W.make_inputs(shape, device="cuda")
+    ids = np.repeat(np.arange(E, dtype=np.int32), sizes)[np.random.default_rng(3).permutation(N)]
+    dsp = O.dispatch(ids[:, None], E, 0)
+    np.testing.assert_array_equal(dsp["counts"], sizes)
+    xp = t["x"][torch.from_numpy(dsp["row_token"]).long().cuda()].contiguous()
+    ye = torch.zeros((N * k + N, d), dtype=torch.bfloat16, device="cuda")
+    cfg = nat.config_from_shape(shape)
+    ws = nat.alloc_workspace(cfg)
+    nat.moe_expert_ffn(cfg, xp=xp, offsets=dev(dsp["offsets"]), x=t["x"], W_gu=t["W_gu"],
+                       W_down=t["W_down"], ye=ye, ws=ws)
+    check_status(ws)
+    x64, Wgu, Wd = f64(t["x"]), f64(t["W_gu"]), f64(t["W_down"])
+    ref = np.zeros((2 * N, d))
+    for e in range(E):
+        a, b = dsp["offsets"][e], dsp["offsets"][e + 1]
+        if b > a:
+            ref[a:b] = O.expert_ffn(x64[dsp["row_token"][a:b]], Wgu[e], Wd[e], W.SWIGLU, 0.0)
+    ref[N:] = O.expert_ffn(x64, Wgu[E], Wd[E], W.SWIGLU, 0.0)
+    assert_close_layer(host(ye), ref)
 
 
 # ---------------------------------------------------------------------------------------

@@ -64,10 +64,20 @@ Readings where the pages are silent (each is listed again in the design doc):
       normalised per token to sum 1 (the pages print the formula for softmax only).
 * R12 the bias update compares each expert's load with its set's mean load
       (total / E) exactly, in integers; gamma = 0.001 (both pages' update rate).
+* R13 overflow policy "report" (P2 table "Politiques de débordement quand E1 reçoit
+      6 tokens pour C = 5", row "Report sur E2/E3": the token is handled by its
+      third-best score).  After the capacity pass, a token's i-th dropped slot (slot
+      order, i = 0, 1, ...) is offered its (k+i)-th best expert by selection key (the
+      third best for top-2).  Offers to one expert are served in token order, then
+      slot order, while the expert's kept count plus the offers it took stays below
+      C; an offer that finds no room leaves the slot dropped.  The gates are those of
+      R4 over the token's final slot list (a moved slot takes its new expert's score;
+      a slot still dropped stays in the list and contributes 0, as in R5).
 
 Parity unpinned: the clamp (R6) beyond unit values, the whole-layer output beyond
-brute force and closed forms -- no page prints a layer output -- and the hash
-router (a reading of an exercise, pinned only by bijectivity and uniformity).
+brute force and closed forms -- no page prints a layer output -- the hash
+router (a reading of an exercise, pinned only by bijectivity and uniformity), and
+the "report" overflow policy (R13) beyond the slides' one-token example.
 """
 from __future__ import annotations
 
@@ -236,6 +246,64 @@ def dispatch(ids, E: int, C: int = 0):
     }
 
 
+def dispatch_masked(ids, E: int, drop_mask):
+    """The contiguous per-expert layout of the assignments not marked in ``drop_mask``
+    (no capacity of its own): kept rows expert by expert, token order inside an expert.
+    Returns the same keys as ``dispatch``; ``demand`` counts the kept assignments."""
+    ids = np.asarray(ids, np.int64)
+    keep = np.asarray(drop_mask) == 0
+    N, k = ids.shape
+    counts = np.zeros(E, np.int64)
+    np.add.at(counts, ids[keep], 1)
+    offsets = np.zeros(E + 1, np.int64)
+    offsets[1:] = np.cumsum(counts)
+    slot_row = np.full((N, k), -1, np.int64)
+    row_token = np.full(int(offsets[-1]), -1, np.int64)
+    fill = offsets[:-1].copy()
+    for t in range(N):                 # token order, then slot order
+        for j in range(k):
+            if keep[t, j]:
+                e = ids[t, j]
+                slot_row[t, j] = fill[e]
+                row_token[fill[e]] = t
+                fill[e] += 1
+    return {"demand": counts.astype(np.int32), "counts": counts.astype(np.int32),
+            "offsets": offsets.astype(np.int32), "row_token": row_token.astype(np.int32),
+            "slot_row": slot_row.astype(np.int32), "drop_mask": (~keep).astype(np.uint8)}
+
+
+def route_reroute(logits, k, C, score_fn=SOFTMAX, renorm=1, bias=None, modality=None):
+    """Routing under the "report" overflow policy (reading R13).
+
+    Returns (ids [N][k] int32: the final expert of every slot, gates [N][k] float64,
+    drop_mask [N][k] uint8: slots still dropped, rerouted [N][k] uint8: slots moved to
+    another expert, first: the ``dispatch`` result of the plain capacity pass)."""
+    keys = selection_keys(logits, score_fn, bias, modality)
+    N, E = keys.shape
+    order = topk_ids(keys, min(E, 2 * k))      # descending key, lower index on ties
+    ids = order[:, :k].astype(np.int32).copy()
+    first = dispatch(ids, E, C)
+    drop = first["drop_mask"].astype(bool).copy()
+    rerouted = np.zeros((N, k), bool)
+    kept = first["counts"].astype(np.int64)
+    taken = np.zeros(E, np.int64)
+    for t in range(N):                         # token order
+        i = 0
+        for j in range(k):                     # slot order
+            if not drop[t, j]:
+                continue
+            if k + i < order.shape[1]:
+                e = int(order[t, k + i])
+                if kept[e] + taken[e] < C:
+                    taken[e] += 1
+                    ids[t, j] = e
+                    drop[t, j] = False
+                    rerouted[t, j] = True
+            i += 1
+    gates = gates_for(logits, ids, score_fn, renorm)
+    return ids, gates, drop.astype(np.uint8), rerouted.astype(np.uint8), first
+
+
 def dispatch_padded(ids, E: int, C: int):
     """The padded dispatch buffer [E, C, d] of the slides ("Support visuel — Capacité"): slot
     c of expert e holds the c-th kept token (token order), empty slots stay empty.
@@ -296,7 +364,7 @@ def expert_ffn(xr, W_gu_e, W_down_e, act=SWIGLU, clamp=0.0):
 # ---------------------------------------------------------------------------
 def forward(x, W_g, W_gu, W_down, *, k, E, score_fn=SOFTMAX, renorm=1, act=SWIGLU,
             clamp=0.0, n_shared=0, bias=None, modality=None, logit_offset=None,
-            C=0, logits=None, tokens=None, ids=None, gates=None):
+            C=0, logits=None, tokens=None, ids=None, gates=None, overflow="drop"):
     """y[t] = sum_{kept j} g[t,j] FFN_{ids[t,j]}(x_t) + sum_shared FFN_s(x_t), float64.
 
     ``logits`` (float32 [N][E]) replaces the router projection when given.
@@ -305,6 +373,8 @@ def forward(x, W_g, W_gu, W_down, *, k, E, score_fn=SOFTMAX, renorm=1, act=SWIGL
     that fired and force the same routing later); capacity still applies.
     ``tokens`` restricts the expert work and the returned rows to those token
     indices; routing and capacity still see every token.
+    ``overflow="reroute"`` applies the "report" overflow policy (reading R13) to the
+    router's choice instead of dropping.
     Returns (y [len(tokens) or N][d] float64, route dict).
     """
     x64 = np.asarray(x, np.float64)
@@ -313,10 +383,19 @@ def forward(x, W_g, W_gu, W_down, *, k, E, score_fn=SOFTMAX, renorm=1, act=SWIGL
         z = None
         ids = np.asarray(ids, np.int32)
         gates = np.asarray(gates, np.float64)
+    elif overflow == "reroute":
+        z = router_logits(x64, W_g, logit_offset) if logits is None else np.asarray(logits, np.float32)
+        ids, gates, drop, rerouted, first = route_reroute(z, k, C, score_fn, renorm, bias,
+                                                          modality)
     else:
         z = router_logits(x64, W_g, logit_offset) if logits is None else np.asarray(logits, np.float32)
         ids, gates = route(z, k, score_fn, renorm, bias, modality)
-    disp = dispatch(ids, E, C)
+    if overflow == "reroute" and ids is not None and z is not None:
+        disp = dispatch_masked(ids, E, drop)
+        disp["demand"] = first["demand"]
+        disp["rerouted"] = rerouted
+    else:
+        disp = dispatch(ids, E, C)
     keep = disp["drop_mask"] == 0
     tok = np.arange(N) if tokens is None else np.asarray(tokens, np.int64)
     y = np.zeros((tok.size, x64.shape[1]), np.float64)
@@ -418,6 +497,7 @@ def dense_mixture(x, W_g, W_gu, W_down, *, E, act=SWIGLU, clamp=0.0, logit_offse
 
 __all__ = ["exp_f32", "sigmoid_f32", "router_logits", "softmax64", "selection_keys",
            "topk_ids", "gates_for", "route", "capacity", "dispatch", "dispatch_padded",
+           "dispatch_masked", "route_reroute",
            "load_fractions",
            "silu", "expert_ffn", "forward", "dense_mixture", "fmix32", "hash_route",
            "router_probs", "balance_stats", "per_set_load", "bias_update",

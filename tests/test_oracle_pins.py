@@ -518,3 +518,111 @@ def test_padded_dispatch_buffer_is_the_slides_table():
             if r >= 0:
                 assert p["row_token"][r] == t and r // C == ids[t, j]
     assert p["slot_row"][5, 0] == -1
+
+
+# --------------------------------------------------------------------------
+# overflow policy "report" (slides, "Politiques de débordement"; reading R13)
+# --------------------------------------------------------------------------
+def test_report_policy_on_the_slides_trace():
+    g, assign, T, E, k = _trace()
+    C = int(g["C_1.25"])
+    z = _trace_logits(assign, E)
+    z[5, 3] = -1.0          # t6 = t1's logits on E1..E3; E4 below them
+    ids, gates, drop, rerouted, first = O.route_reroute(z, k, C)
+    assert first["drop_mask"].sum() == 1 and first["drop_mask"][5, 0] == 1
+    t6_new = int(g["report_t6_expert"])
+    assert ids[5].tolist() == [t6_new, 1]          # slot 0 (E1) moved to E3, E2 kept
+    assert drop.sum() == 0 and rerouted.sum() == 1 and rerouted[5, 0] == 1
+    assert (np.delete(ids, 5, axis=0) == np.delete(np.array(assign), 5, axis=0)).all()
+    layout = O.dispatch_masked(ids, E, drop)
+    assert layout["counts"].tolist() == [5, 4, 4, 3]
+    # gates over t6's final list {E3, E2} from the printed exponentials 1.221 and 6.050
+    e = floats(load("p2_router_example.txt")["exp"])
+    np.testing.assert_allclose(gates[5], [e[2] / (e[1] + e[2]), e[1] / (e[1] + e[2])], atol=1e-3)
+    # the other tokens keep their 0.574 / 0.426
+    np.testing.assert_allclose(np.round(gates[0], 3), [0.574, 0.426])
+
+
+def test_report_policy_without_overflow_is_plain_routing():
+    rng = np.random.default_rng(21)
+    z = rng.normal(0, 1.5, (300, 16)).astype(np.float32)
+    for C in (0, 1000):
+        ids, gates, drop, rerouted, _ = O.route_reroute(z, 3, C)
+        ids_r, gates_r = O.route(z, 3)
+        assert (ids == ids_r).all() and not drop.any() and not rerouted.any()
+        np.testing.assert_array_equal(gates, gates_r)
+
+
+def test_report_policy_closed_form_one_hot_expert():
+    # every token ranks the experts 0 > 1 > 2 > 3; k = 1, C = 3: tokens 0-2 keep expert 0,
+    # tokens 3-5 are moved to expert 1 (their second best), tokens 6-9 find it full: dropped
+    z = np.tile(np.array([[3.0, 2.0, 1.0, 0.0]], np.float32), (10, 1))
+    ids, gates, drop, rerouted, _ = O.route_reroute(z, 1, 3)
+    assert ids[:, 0].tolist() == [0, 0, 0, 1, 1, 1, 0, 0, 0, 0]   # a refused slot keeps its id
+    assert drop[:, 0].tolist() == [0] * 6 + [1] * 4
+    assert rerouted[:, 0].tolist() == [0, 0, 0, 1, 1, 1, 0, 0, 0, 0]
+    # renorm over a single slot: the gate is 1 whether the slot moved or not
+    np.testing.assert_allclose(gates[:, 0], 1.0)
+    # Switch gate (renorm = 0): the moved slot takes expert 1's own probability
+    _, g0, _, _, _ = O.route_reroute(z, 1, 3, renorm=0)
+    p = sp_softmax(z[0].astype(np.float64))
+    np.testing.assert_allclose(g0[:3, 0], p[0])
+    np.testing.assert_allclose(g0[3:6, 0], p[1])
+    np.testing.assert_allclose(g0[6:, 0], p[0])     # refused: still expert 0's slot, output 0
+
+
+def test_report_policy_invariants_random():
+    rng = np.random.default_rng(22)
+    N, E, k = 400, 12, 3
+    z = (rng.normal(0, 1, (N, E)) + np.linspace(2, -2, E)[None, :]).astype(np.float32)
+    bias = rng.uniform(-0.1, 0.1, (1, E)).astype(np.float32)
+    for sf in (O.SOFTMAX, O.SIGMOID):
+        C = O.capacity(N, k, E, 1)
+        ids, gates, drop, rerouted, first = O.route_reroute(z, k, C, sf, 1, bias if sf else None)
+        keys = O.selection_keys(z, sf, bias if sf else None)
+        order = O.topk_ids(keys, 2 * k)
+        lay = O.dispatch_masked(ids, E, drop)
+        assert (lay["counts"] <= C).all()
+        assert lay["counts"].sum() >= first["counts"].sum()
+        for t in range(N):
+            assert len(set(ids[t].tolist())) == k          # experts stay distinct per token
+            i = 0
+            for j in range(k):
+                if first["drop_mask"][t, j]:
+                    if rerouted[t, j]:
+                        assert ids[t, j] == order[t, k + i]
+                    else:
+                        assert drop[t, j] and ids[t, j] == order[t, j]
+                    i += 1
+                else:
+                    assert ids[t, j] == order[t, j] and not drop[t, j]
+        # every expert that refused an offer is full
+        for t in range(N):
+            for j in range(k):
+                if drop[t, j]:
+                    i = int(first["drop_mask"][t, :j].sum())
+                    if k + i < E:
+                        assert lay["counts"][order[t, k + i]] == C
+
+
+def test_forward_with_report_policy_matches_hand_sum():
+    g, assign, T, E, k = _trace()
+    rng = np.random.default_rng(23)
+    d, F = 4, 3
+    x = rng.normal(0, 1, (T, d))
+    W_gu = rng.normal(0, 0.5, (E + 1, 2 * F, d))
+    W_down = rng.normal(0, 0.5, (E + 1, d, F))
+    z = _trace_logits(assign, E)
+    z[5, 3] = -1.0
+    y, info = O.forward(x, None, W_gu, W_down, k=k, E=E, n_shared=1, C=int(g["C_1.25"]),
+                        logits=z, overflow="reroute")
+
+    def ffn(e, v):
+        gg = W_gu[e, :F] @ v
+        uu = W_gu[e, F:] @ v
+        return W_down[e] @ (gg / (1 + np.exp(-gg)) * uu)
+    e3 = math.exp(0.2) / (math.exp(0.2) + math.exp(1.8))
+    np.testing.assert_allclose(y[5], e3 * ffn(2, x[5]) + (1 - e3) * ffn(1, x[5]) + ffn(E, x[5]),
+                               rtol=1e-6)
+    assert info["drop_mask"].sum() == 0 and info["rerouted"].sum() == 1
+    assert info["demand"].tolist() == [6, 4, 3, 3]

@@ -35,6 +35,11 @@ from mixture_experts_layer_50_b200 import workloads as W  # noqa: E402
 METRIC = "MoE-layer fwd tokens/s and % of bf16 tensor (prefill) or HBM (decode) roofline"
 LAUNCH_NAMES = ["router_gemm", "route_topk", "rank_local", "dispatch_scan", "scatter_gather",
                 "gemm_gate_up", "gemm_down", "combine"]
+# with the "report" overflow policy: the capacity pass, the offers and the final layout
+LAUNCH_NAMES_REROUTE = ["router_gemm", "route_topk", "rank_local", "dispatch_scan",
+                        "capacity_pass", "reroute_offer", "rank_offers", "scan_offers",
+                        "reroute_accept", "rank_final", "scan_final", "scatter_gather",
+                        "gemm_gate_up", "gemm_down", "combine"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -46,6 +51,8 @@ def parse_args():
     p.add_argument("--workload", default="mixtral-n16384", choices=sorted(W.PRESETS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--overflow", default="drop", choices=["drop", "reroute"],
+                   help="capacity overflow policy: drop, or the slides' 'report' (reroute)")
     p.add_argument("--tokens", type=int, default=None,
                    help="override the workload's token count (profiling a smaller case)")
     p.add_argument("--experts", type=int, default=None,
@@ -231,10 +238,11 @@ def run_ours(args):
     torch.cuda.set_device(local)
     shape = workload_shape(args)
     t = make_replica(shape, rank)
-    layer = MoELayer.from_workload(shape, t)
+    layer = MoELayer.from_workload(shape, t, overflow=args.overflow)
     x, mod = t["x"], t.get("modality")
     y = torch.empty_like(x)
     stream = torch.cuda.current_stream()
+    names = LAUNCH_NAMES_REROUTE if args.overflow == "reroute" and shape.capacity_factor else LAUNCH_NAMES
 
     # routing statistics of this batch (untimed), for the algorithmic work
     counts = torch.empty(shape.E, dtype=torch.int32, device="cuda")
@@ -314,7 +322,7 @@ def run_ours(args):
     burst = (clocks.get("sm_mhz") or 0) >= 0.95 * (clocks.get("sm_max_mhz") or 1e9)
     tensor_key = "bf16_tflops" if burst else "bf16_tflops_sustained"
     tensor_peak = peaks[tensor_key]
-    per_launch = {n: launch_ms[i] / max(calls, 1) for i, n in enumerate(LAUNCH_NAMES)
+    per_launch = {n: launch_ms[i] / max(calls, 1) for i, n in enumerate(names)
                   if i < len(launch_ms)}
     gu_ms = per_launch.get("gemm_gate_up")
     ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -352,8 +360,9 @@ def run_ours(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
         if shape.dtype == W.BF16 else "f32", "data": "synthetic (seeded N(0,0.02) weights, N(0,1) tokens)",
-        "config": {"workload": workload_desc(shape), "tokens_per_gpu": shape.N,
-                   "global_batch": shape.N * world,
+        "config": {"workload": workload_desc(shape)
+                   + (" overflow=reroute" if args.overflow == "reroute" else ""),
+                   "tokens_per_gpu": shape.N, "global_batch": shape.N * world,
                    "l2": f"inputs larger than L2 ({shape.weight_bytes() / 1e9:.2f} GB of weights per step)",
                    "parallelism": f"replicas x{world} (no data-path collective)"},
         "roofline": roof, "layer_roofline": layer_roof,
@@ -361,7 +370,9 @@ def run_ours(args):
         "e2e": {"value": round(shape.N * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": shape.N * shape.d * el,
                 "d2h_bytes_per_step": shape.N * shape.d * el,
-                "method": "moe_forward_host_batches (copies overlapped), wall clock",
+                "method": "moe_forward_host_batches (copies overlapped), wall clock"
+                if args.overflow == "drop" else
+                "pinned-host copies + moe_forward_reroute + copy back, one stream, wall clock",
                 "serial_ms_per_step": round(serial_ms, 4)},
         "gpu_launches": per_step_launches * args.steps,
         "host_enqueue_us_per_step": round(host_us, 1),

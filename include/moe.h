@@ -182,6 +182,38 @@ MOE_API moe_status moe_forward_routed(const moe_config* cfg, const void* x, cons
                                       void* y, const moe_route_out* route_out, void* ws,
                                       moe_stream_t stream);
 
+/* Overflow policy "report" ("Mixture-of-Experts : routage et capacité" slides, table
+ * "Politiques de débordement quand E1 reçoit 6 tokens pour C = 5", row "Report sur E2/E3": the
+ * rejected token is handled by its third-best score).  Routing and capacity as in moe_route,
+ * then a token's i-th dropped slot (slot order, i = 0, 1, ...) is offered the token's
+ * (k+i)-th best expert by selection key; the offers to one expert are served in token order,
+ * then slot order, while its kept count plus the offers it took stays below C; a slot whose
+ * offer finds no room stays dropped and keeps its expert id.  Gates are recomputed over each
+ * token's final slot list as in moe_route (a moved slot takes its new expert's unbiased
+ * score; a slot still dropped stays in the list and contributes 0).  With capacity <= 0
+ * nothing overflows and the result is moe_route's.
+ * Outputs: ids [N][k] (final experts), gates [N][k], counts [E] (kept assignments after the
+ * policy), demand [E] (the router's assignments per expert before capacity), drop_mask
+ * [N][k] (slots still dropped), rerouted [N][k] uint8 or NULL (1 = slot moved).  Requires
+ * k <= 16 (MOE_ERR_UNSUPPORTED otherwise).  Other arguments as in moe_route. */
+MOE_API moe_status moe_route_reroute(const moe_config* cfg, const float* logits, const void* x,
+                                     const void* W_g, const float* logit_offset,
+                                     const float* bias, const uint8_t* modality, int32_t* ids,
+                                     float* gates, int32_t* counts, int32_t* demand,
+                                     uint8_t* drop_mask, uint8_t* rerouted, float* logits_out,
+                                     void* ws, moe_stream_t stream);
+
+/* moe_forward with the "report" overflow policy of moe_route_reroute: the kept and moved
+ * slots are permuted, run through their experts and combined as in moe_forward.  route_out
+ * members as in moe_forward (counts after the policy, demand before capacity, drop_mask =
+ * slots still dropped); rerouted [N][k] uint8 or NULL.  Requires k <= 16. */
+MOE_API moe_status moe_forward_reroute(const moe_config* cfg, const void* x, const void* W_g,
+                                       const float* logit_offset, const float* bias,
+                                       const uint8_t* modality, const void* W_gu,
+                                       const void* W_down, void* y,
+                                       const moe_route_out* route_out, uint8_t* rerouted,
+                                       void* ws, moe_stream_t stream);
+
 /* Hash router ("Le groupe d'experts (MoE)", exercise "Medium": deterministic, not learned):
  * for token id t (token_ids [N], int32), expert e's key is fmix32(t * 0x9E3779B1 + e) with
  * 32-bit wrap-around, fmix32 being MurmurHash3's finaliser; the k largest keys are selected

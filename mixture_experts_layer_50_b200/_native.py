@@ -74,6 +74,8 @@ lib.moe_balance.argtypes = [_cfgp] + [_vp] * 8 + [ctypes.c_float, _vp, _vp]
 lib.moe_permute_padded.argtypes = [_cfgp] + [_vp] * 10
 lib.moe_forward_padded.argtypes = [_cfgp] + [_vp] * 11
 lib.moe_forward_host_batches.argtypes = [_cfgp, _i32] + [_vp] * 10
+lib.moe_route_reroute.argtypes = [_cfgp] + [_vp] * 15
+lib.moe_forward_reroute.argtypes = [_cfgp] + [_vp] * 12
 lib.moe_profile_begin.argtypes = [_i32]
 lib.moe_profile_begin.restype = ctypes.c_int
 lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)]
@@ -83,7 +85,8 @@ lib.moe_last_launch_count.restype = _i32
 for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
            "moe_forward", "moe_forward_host", "moe_check_status", "moe_route_static",
            "moe_forward_routed", "moe_route_hash", "moe_balance", "moe_permute_padded",
-           "moe_forward_padded", "moe_forward_host_batches"):
+           "moe_forward_padded", "moe_forward_host_batches", "moe_route_reroute",
+           "moe_forward_reroute"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
@@ -91,7 +94,7 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_rou
             "moe_check_status", "moe_profile_begin", "moe_profile_end", "moe_last_error",
             "moe_last_launch_count", "moe_route_static", "moe_forward_routed",
             "moe_route_hash", "moe_balance", "moe_permute_padded", "moe_forward_padded",
-            "moe_forward_host_batches")
+            "moe_forward_host_batches", "moe_route_reroute", "moe_forward_reroute")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -215,6 +218,32 @@ def moe_forward(cfg, *, x, W_g, W_gu, W_down, y, logit_offset=None, bias=None, m
                          ctypes.byref(ro) if ro is not None else None, _ptr(ws),
                          _stream(stream))
     _check(st, "moe_forward")
+
+
+def moe_route_reroute(cfg, *, logits=None, x=None, W_g=None, logit_offset=None, bias=None,
+                      modality=None, ids=None, gates=None, counts=None, demand=None,
+                      drop_mask=None, rerouted=None, logits_out=None, ws, stream=None):
+    """Routing with the "report" overflow policy: a dropped slot goes to the token's next-best
+    expert while that expert has room."""
+    st = lib.moe_route_reroute(ctypes.byref(cfg), _ptr(logits), _ptr(x), _ptr(W_g),
+                               _ptr(logit_offset), _ptr(bias), _ptr(modality), _ptr(ids),
+                               _ptr(gates), _ptr(counts), _ptr(demand), _ptr(drop_mask),
+                               _ptr(rerouted), _ptr(logits_out), _ptr(ws), _stream(stream))
+    _check(st, "moe_route_reroute")
+
+
+def moe_forward_reroute(cfg, *, x, W_g, W_gu, W_down, y, logit_offset=None, bias=None,
+                        modality=None, route_out: Optional[dict] = None, rerouted=None, ws,
+                        stream=None):
+    """The layer with the "report" overflow policy instead of dropping."""
+    ro = None
+    if route_out:
+        ro = moe_route_out(*[_ptr(route_out.get(n)) for n, _ in moe_route_out._fields_])
+    st = lib.moe_forward_reroute(ctypes.byref(cfg), _ptr(x), _ptr(W_g), _ptr(logit_offset),
+                                 _ptr(bias), _ptr(modality), _ptr(W_gu), _ptr(W_down), _ptr(y),
+                                 ctypes.byref(ro) if ro is not None else None, _ptr(rerouted),
+                                 _ptr(ws), _stream(stream))
+    _check(st, "moe_forward_reroute")
 
 
 def moe_forward_routed(cfg, *, x, ids, gates, W_gu, W_down, y, route_out: Optional[dict] = None,

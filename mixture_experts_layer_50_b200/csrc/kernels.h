@@ -15,7 +15,20 @@ cudaError_t launch_route_topk(const float* logits, int n_parts, int64_t part_str
                               const float* offset, float* logits_out, int64_t N, int E, int k,
                               int score_fn, int renorm, const float* bias, int n_bias_sets,
                               const uint8_t* modality, int32_t* ids, float* gates,
-                              int* status, cudaStream_t stream, int* launches);
+                              int* status, cudaStream_t stream, int* launches,
+                              int k_extra = 0, int32_t* cand = nullptr,
+                              float* cand_val = nullptr);
+// Overflow policy "report": offers of the dropped slots to the next-best candidates, and the
+// decision on them (csrc/reroute.cu).
+cudaError_t launch_reroute_offer(const int32_t* ids, const uint8_t* drop1, const int32_t* cand,
+                                 int64_t N, int k, int32_t* offer, uint8_t* not_offer,
+                                 cudaStream_t stream, int* launches);
+cudaError_t launch_reroute_accept(int32_t* ids, const uint8_t* drop1, const int32_t* offer,
+                                  const uint8_t* not_offer, const int32_t* local_rank,
+                                  const int32_t* tile_base, const int32_t* counts1,
+                                  const float* cand_val, int64_t N, int E, int k, int64_t C,
+                                  int score_fn, int renorm, float* gates, uint8_t* drop_out,
+                                  uint8_t* rerouted, cudaStream_t stream, int* launches);
 
 // Hash router: ids = the k experts with the largest fmix32(token_id * 0x9E3779B1 + e), gates 1/k.
 cudaError_t launch_route_hash(const int32_t* token_ids, int64_t N, int E, int k, int32_t* ids,

@@ -65,7 +65,8 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 struct Ws {
   size_t status, logits, ids, gates, local_rank, tile_hist, tile_base, demand, counts, offsets,
       slot_row, row_token, drop_mask, xp, h, ye, x_stage, y_stage, x_stage2, y_stage2, balance,
-      offsets_pad, logit_parts, total;
+      offsets_pad, logit_parts, rr_cand, rr_val, rr_drop1, rr_offer, rr_not_offer, rr_counts1,
+      rr_scratch, total;
 };
 
 size_t el_size(const moe_config& c) { return c.dtype == MOE_DT_BF16 ? 2 : 4; }
@@ -114,6 +115,14 @@ Ws layout(const moe_config& c) {
   w.offsets_pad = take((E + 1) * 4);
   const int splits = router_splits(c);
   w.logit_parts = take(splits > 1 ? (size_t)splits * N * E * 4 : 0);
+  // overflow policy "report": next-best candidates, their gate values, the first pass
+  w.rr_cand = take(Nk * 4);
+  w.rr_val = take(2 * Nk * 4);
+  w.rr_drop1 = take(Nk);
+  w.rr_offer = take(Nk * 4);
+  w.rr_not_offer = take(Nk);
+  w.rr_counts1 = take(E * 4);
+  w.rr_scratch = take(3 * (E + 1) * 4);
   w.total = off;
   return w;
 }
@@ -314,6 +323,58 @@ moe_status stage_dispatch(const moe_config& c, const Ws& L, void* ws, const int3
   return MOE_OK;
 }
 
+// Routing under the overflow policy "report" ("Mixture-of-Experts : routage et capacité",
+// table "Politiques de débordement", row "Report sur E2/E3"): the top-k kernel also lists each
+// token's next k candidates; a plain capacity pass finds the dropped slots; each dropped slot
+// is offered the token's next unused candidate; the offers are ranked per expert in token
+// order like the first pass and taken while the expert has room; the gates are recomputed
+// over the final slot list.  Writes ids and gates (final), demand (first pass), drop_out
+// (slots still dropped) and rerouted (optional).  Uses the workspace's rank arrays and slot_row.
+moe_status stage_route_reroute(const moe_config& c, const Ws& L, void* ws, const LogitSrc& z,
+                               const float* bias, const uint8_t* modality, int32_t* ids,
+                               float* gates, int32_t* demand, uint8_t* drop_out,
+                               uint8_t* rerouted, cudaStream_t st, int* launches) {
+  int* status = at<int>(ws, L.status);
+  int32_t* cand = at<int32_t>(ws, L.rr_cand);
+  float* val = at<float>(ws, L.rr_val);
+  uint8_t* drop1 = at<uint8_t>(ws, L.rr_drop1);
+  int32_t* offer = at<int32_t>(ws, L.rr_offer);
+  uint8_t* not_offer = at<uint8_t>(ws, L.rr_not_offer);
+  int32_t* counts1 = at<int32_t>(ws, L.rr_counts1);
+  int32_t* scratch = at<int32_t>(ws, L.rr_scratch);  // [3][E + 1]
+  const int64_t E1 = c.E + 1;
+  MOE_CUDA(moe::launch_route_topk(z.src, z.n_parts, z.part_stride, z.offset, z.final_out, c.N,
+                                  c.E, c.k, c.score_fn, c.renorm, bias, c.n_bias_sets, modality,
+                                  ids, gates, status, st, launches, c.k, cand, val),
+           "top-k routing with candidates");
+  prof_mark(st);
+  // first pass: the plain capacity decision
+  MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, c.capacity, demand, counts1, scratch,
+                         at<int32_t>(ws, L.slot_row), nullptr, drop1, nullptr, nullptr, st,
+                         launches));
+  // offers to the next-best candidates, ranked per expert in token order
+  MOE_CUDA(moe::launch_reroute_offer(ids, drop1, cand, c.N, c.k, offer, not_offer, st, launches),
+           "reroute offers");
+  prof_mark(st);
+  MOE_CUDA(moe::launch_rank_local(offer, not_offer, c.N, c.k, c.E, at<int32_t>(ws, L.local_rank),
+                                  at<int32_t>(ws, L.tile_hist), status, st, launches),
+           "rank pass (offers)");
+  prof_mark(st);
+  MOE_CUDA(moe::launch_dispatch_scan(at<int32_t>(ws, L.tile_hist), c.N, c.E, 0,
+                                     at<int32_t>(ws, L.tile_base), scratch + E1,
+                                     scratch + 2 * E1, scratch, arrive_counter(ws, L), st,
+                                     launches),
+           "scan pass (offers)");
+  prof_mark(st);
+  MOE_CUDA(moe::launch_reroute_accept(ids, drop1, offer, not_offer, at<int32_t>(ws, L.local_rank),
+                                      at<int32_t>(ws, L.tile_base), counts1, val, c.N, c.E, c.k,
+                                      c.capacity, c.score_fn, c.renorm, gates, drop_out,
+                                      rerouted, st, launches),
+           "reroute decision");
+  prof_mark(st);
+  return MOE_OK;
+}
+
 // R: rows of the routed region of xp / h / ye (N k for the compact layout, E C for the
 // padded one); the shared expert's rows follow it.
 moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
@@ -406,7 +467,8 @@ moe_status stage_combine(const moe_config& c, const void* ye, const int32_t* slo
 moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
                         const float* logit_offset, const float* bias, const uint8_t* modality,
                         const void* W_gu, const void* W_down, void* y,
-                        const moe_route_out* ro, void* ws, cudaStream_t st, int* launches) {
+                        const moe_route_out* ro, void* ws, cudaStream_t st, int* launches,
+                        bool reroute = false, uint8_t* rerouted = nullptr) {
   const moe_config& c = *cfg;
   const Ws L = layout(c);
   int* status = at<int>(ws, L.status);
@@ -426,10 +488,23 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
   prof_call_begin(st);
   LogitSrc zsrc;
   MOE_TRY(stage_logits(c, L, ws, x, W_g, logit_offset, logits, status, st, launches, &zsrc));
-  MOE_TRY(stage_route(c, zsrc, bias, modality, ids, gates, status, st, launches));
-  MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, c.capacity, demand, counts, offsets,
-                         at<int32_t>(ws, L.slot_row), at<int32_t>(ws, L.row_token), drop, x,
-                         xp, st, launches));
+  if (reroute && c.capacity > 0) {
+    // final slots after the overflow policy; the capacity is already met, so the dispatch
+    // below only lays the kept slots out (its demand output is scratch: demand keeps the
+    // router's first-pass demand)
+    MOE_TRY(stage_route_reroute(c, L, ws, zsrc, bias, modality, ids, gates, demand, drop,
+                                rerouted, st, launches));
+    MOE_TRY(stage_dispatch(c, L, ws, ids, drop, 0, at<int32_t>(ws, L.rr_scratch), counts,
+                           offsets, at<int32_t>(ws, L.slot_row), at<int32_t>(ws, L.row_token),
+                           drop, x, xp, st, launches));
+  } else {
+    MOE_TRY(stage_route(c, zsrc, bias, modality, ids, gates, status, st, launches));
+    MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, c.capacity, demand, counts, offsets,
+                           at<int32_t>(ws, L.slot_row), at<int32_t>(ws, L.row_token), drop, x,
+                           xp, st, launches));
+    if (rerouted != nullptr && c.N > 0)
+      MOE_CUDA(cudaMemsetAsync(rerouted, 0, (size_t)c.N * c.k, st), "clear rerouted flags");
+  }
   MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, launches));
   MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, launches));
   g_prof.recording = false;
@@ -495,6 +570,55 @@ moe_status moe_route(const moe_config* cfg, const float* logits, const void* x,
   return MOE_OK;
 }
 
+moe_status moe_route_reroute(const moe_config* cfg, const float* logits, const void* x,
+                             const void* W_g, const float* logit_offset, const float* bias,
+                             const uint8_t* modality, int32_t* ids, float* gates,
+                             int32_t* counts, int32_t* demand, uint8_t* drop_mask,
+                             uint8_t* rerouted, float* logits_out, void* ws,
+                             moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  MOE_TRY(check_bias(cfg, bias, modality));
+  if (cfg->k > 16) return fail(MOE_ERR_UNSUPPORTED, "the report overflow policy needs k <= 16");
+  if (logits == nullptr) {
+    MOE_TRY(need(x, "x"));
+    MOE_TRY(need(W_g, "W_g"));
+  }
+  const moe_config& c = *cfg;
+  if (c.capacity <= 0) {
+    // no capacity: nothing overflows, plain routing
+    MOE_TRY(moe_route(cfg, logits, x, W_g, logit_offset, bias, modality, ids, gates, counts,
+                      demand, drop_mask, logits_out, ws, stream));
+    if (rerouted != nullptr && c.N > 0)
+      MOE_CUDA(cudaMemsetAsync(rerouted, 0, (size_t)c.N * c.k, (cudaStream_t)stream),
+               "clear rerouted flags");
+    return MOE_OK;
+  }
+  const Ws L = layout(c);
+  cudaStream_t st = (cudaStream_t)stream;
+  int launches = 0;
+  int* status = at<int>(ws, L.status);
+  LogitSrc z = finished_logits(logits);
+  if (logits == nullptr) {
+    float* dst = logits_out != nullptr ? logits_out : at<float>(ws, L.logits);
+    MOE_TRY(stage_logits(c, L, ws, x, W_g, logit_offset, dst, status, st, &launches, &z));
+  }
+  int32_t* ids_p = ids != nullptr ? ids : at<int32_t>(ws, L.ids);
+  float* gates_p = gates != nullptr ? gates : at<float>(ws, L.gates);
+  uint8_t* drop_p = drop_mask != nullptr ? drop_mask : at<uint8_t>(ws, L.drop_mask);
+  MOE_TRY(stage_route_reroute(c, L, ws, z, bias, modality, ids_p, gates_p,
+                              demand != nullptr ? demand : at<int32_t>(ws, L.demand), drop_p,
+                              rerouted, st, &launches));
+  // kept assignments per expert after the policy
+  MOE_TRY(stage_dispatch(c, L, ws, ids_p, drop_p, 0, at<int32_t>(ws, L.rr_scratch),
+                         counts != nullptr ? counts : at<int32_t>(ws, L.counts),
+                         at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.slot_row), nullptr, drop_p,
+                         nullptr, nullptr, st, &launches));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
 moe_status moe_permute(const moe_config* cfg, const int32_t* ids, const uint8_t* drop_mask,
                        const void* x, int32_t* offsets, int32_t* row_token,
                        int32_t* slot_row, void* xp, void* ws, moe_stream_t stream) {
@@ -544,6 +668,31 @@ moe_status moe_combine(const moe_config* cfg, const void* ye, const int32_t* slo
     return fail(MOE_ERR_INVALID_ARG, "slot_row and gates are required");
   int launches = 0;
   MOE_TRY(stage_combine(*cfg, ye, slot_row, gates, y, (cudaStream_t)stream, &launches));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_forward_reroute(const moe_config* cfg, const void* x, const void* W_g,
+                               const float* logit_offset, const float* bias,
+                               const uint8_t* modality, const void* W_gu, const void* W_down,
+                               void* y, const moe_route_out* route_out, uint8_t* rerouted,
+                               void* ws, moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  MOE_TRY(check_bias(cfg, bias, modality));
+  if (cfg->k > 16) return fail(MOE_ERR_UNSUPPORTED, "the report overflow policy needs k <= 16");
+  MOE_TRY(need(x, "x"));
+  MOE_TRY(need(W_g, "W_g"));
+  MOE_TRY(need(W_gu, "W_gu"));
+  MOE_TRY(need(W_down, "W_down"));
+  MOE_TRY(need(y, "y"));
+  int launches = 0;
+  const moe_status fs = forward_impl(cfg, x, W_g, logit_offset, bias, modality, W_gu, W_down,
+                                     y, route_out, ws, (cudaStream_t)stream, &launches, true,
+                                     rerouted);
+  g_prof.recording = false;
+  MOE_TRY(fs);
   g_last_launches = launches;
   return MOE_OK;
 }

@@ -57,7 +57,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
     const float* __restrict__ offset, float* __restrict__ logits_out, int64_t N, int E, int k,
     int score_fn, int renorm, const float* __restrict__ bias, int n_bias_sets,
     const uint8_t* __restrict__ modality, int32_t* __restrict__ ids, float* __restrict__ gates,
-    int* status) {
+    int* status, int k_extra, int32_t* __restrict__ cand, float* __restrict__ cand_val) {
   const int lane = threadIdx.x & 31;
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= N) return;
@@ -99,11 +99,13 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
     }
   }
 
-  // k rounds of warp arg-max.  Lane r keeps the r-th selection.
+  // k rounds of warp arg-max (k + k_extra when the next-best candidates are asked for, at
+  // most E).  Lane r keeps the r-th selection.
+  const int rounds = cand != nullptr ? min(E, k + k_extra) : k;
   uint32_t taken = 0;
   int my_e = -1;
   float my_sc = 0.0f;
-  for (int r = 0; r < k; ++r) {
+  for (int r = 0; r < rounds; ++r) {
     float bk = -INFINITY, bs = 0.0f;
     int be = 0x7fffffff;
 #pragma unroll
@@ -163,18 +165,26 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
     ids[t * k + lane] = my_e;
     gates[t * k + lane] = g;
   }
+  if (cand != nullptr) {
+    // candidates k .. k + k_extra - 1 (-1 past E), and per selection the value the gates are
+    // computed from: the unbiased score (renorm) or the raw gate (no renorm)
+    if (lane >= k && lane < k + k_extra) cand[t * k_extra + (lane - k)] = lane < rounds ? my_e : -1;
+    if (lane < k + k_extra)
+      cand_val[t * (k + k_extra) + lane] = lane < rounds ? (renorm ? my_sc : g) : 0.0f;
+  }
 }
 
 template <int J>
 cudaError_t launch_j(const float* logits, int n_parts, int64_t part_stride, const float* offset,
                      float* logits_out, int64_t N, int E, int k, int score_fn, int renorm,
                      const float* bias, int n_bias_sets, const uint8_t* modality,
-                     int32_t* ids, float* gates, int* status, cudaStream_t stream) {
+                     int32_t* ids, float* gates, int* status, int k_extra, int32_t* cand,
+                     float* cand_val, cudaStream_t stream) {
   const int threads = 256;
   const int64_t blocks = (N * 32 + threads - 1) / threads;
   route_topk_kernel<J><<<(unsigned)blocks, threads, 0, stream>>>(
       logits, n_parts, part_stride, offset, logits_out, N, E, k, score_fn, renorm, bias,
-      n_bias_sets, modality, ids, gates, status);
+      n_bias_sets, modality, ids, gates, status, k_extra, cand, cand_val);
   return cudaGetLastError();
 }
 
@@ -266,13 +276,15 @@ cudaError_t launch_route_topk(const float* logits, int n_parts, int64_t part_str
                               const float* offset, float* logits_out, int64_t N, int E, int k,
                               int score_fn, int renorm, const float* bias, int n_bias_sets,
                               const uint8_t* modality, int32_t* ids, float* gates,
-                              int* status, cudaStream_t stream, int* launches) {
+                              int* status, cudaStream_t stream, int* launches, int k_extra,
+                              int32_t* cand, float* cand_val) {
   if (N == 0) return cudaSuccess;
+  if (cand != nullptr && k + k_extra > 32) return cudaErrorInvalidValue;
   ++*launches;
   const int J = (E + 31) / 32;
 #define MOE_ROUTE_CASE(JJ) \
   if (J <= JJ)             \
-    return launch_j<JJ>(logits, n_parts, part_stride, offset, logits_out, N, E, k, score_fn, renorm, bias, n_bias_sets, modality, ids, gates, status, stream);
+    return launch_j<JJ>(logits, n_parts, part_stride, offset, logits_out, N, E, k, score_fn, renorm, bias, n_bias_sets, modality, ids, gates, status, k_extra, cand, cand_val, stream);
   MOE_ROUTE_CASE(1)
   MOE_ROUTE_CASE(2)
   MOE_ROUTE_CASE(4)

@@ -64,7 +64,7 @@ Readings where the pages are silent (each is listed again in the design doc):
       normalised per token to sum 1 (the pages print the formula for softmax only).
 * R12 the bias update compares each expert's load with its set's mean load
       (total / E) exactly, in integers; gamma = 0.001 (both pages' update rate).
-* R13 overflow policy "report" (P2 table "Politiques de débordement quand E1 reçoit
+* R14 overflow policy "report" (P2 table "Politiques de débordement quand E1 reçoit
       6 tokens pour C = 5", row "Report sur E2/E3": the token is handled by its
       third-best score).  After the capacity pass, a token's i-th dropped slot (slot
       order, i = 0, 1, ...) is offered its (k+i)-th best expert by selection key (the
@@ -77,7 +77,7 @@ Readings where the pages are silent (each is listed again in the design doc):
 Parity unpinned: the clamp (R6) beyond unit values, the whole-layer output beyond
 brute force and closed forms -- no page prints a layer output -- the hash
 router (a reading of an exercise, pinned only by bijectivity and uniformity), and
-the "report" overflow policy (R13) beyond the slides' one-token example.
+the "report" overflow policy (R14) beyond the slides' one-token example.
 """
 from __future__ import annotations
 
@@ -273,7 +273,7 @@ def dispatch_masked(ids, E: int, drop_mask):
 
 
 def route_reroute(logits, k, C, score_fn=SOFTMAX, renorm=1, bias=None, modality=None):
-    """Routing under the "report" overflow policy (reading R13).
+    """Routing under the "report" overflow policy (reading R14).
 
     Returns (ids [N][k] int32: the final expert of every slot, gates [N][k] float64,
     drop_mask [N][k] uint8: slots still dropped, rerouted [N][k] uint8: slots moved to
@@ -373,7 +373,7 @@ def forward(x, W_g, W_gu, W_down, *, k, E, score_fn=SOFTMAX, renorm=1, act=SWIGL
     that fired and force the same routing later); capacity still applies.
     ``tokens`` restricts the expert work and the returned rows to those token
     indices; routing and capacity still see every token.
-    ``overflow="reroute"`` applies the "report" overflow policy (reading R13) to the
+    ``overflow="reroute"`` applies the "report" overflow policy (reading R14) to the
     router's choice instead of dropping.
     Returns (y [len(tokens) or N][d] float64, route dict).
     """

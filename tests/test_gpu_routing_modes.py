@@ -1,6 +1,8 @@
 """GPU parity of the routing variants and of the balancing by-products: forced (replayed)
 routing and the hash router ("Le groupe d'experts (MoE)", exercises "Hard" and "Medium"), the
 Switch balance statistic and the aux-loss-free bias update per modality."""
+from fractions import Fraction
+
 import numpy as np
 import pytest
 import torch
@@ -183,3 +185,150 @@ def test_padded_forward_equals_the_compact_forward():
     # the same kernels on the same rows: each output row is computed from the same operands
     # in the same order, so the two layouts agree to the bit
     assert torch.equal(yp, y)
+
+
+# ---------------------------------------------------------------------------------------
+# overflow policy "report" (slides, "Politiques de débordement", row "Report sur E2/E3")
+# ---------------------------------------------------------------------------------------
+def _gpu_reroute(cfg, z, bias=None, mod=None):
+    N, E, k = cfg.N, cfg.E, cfg.k
+    ws = nat.alloc_workspace(cfg)
+    out = dict(ids=torch.empty((N, k), dtype=torch.int32, device="cuda"),
+               gates=torch.empty((N, k), dtype=torch.float32, device="cuda"),
+               counts=torch.empty(E, dtype=torch.int32, device="cuda"),
+               demand=torch.empty(E, dtype=torch.int32, device="cuda"),
+               drop_mask=torch.empty((N, k), dtype=torch.uint8, device="cuda"),
+               rerouted=torch.empty((N, k), dtype=torch.uint8, device="cuda"))
+    nat.moe_route_reroute(cfg, logits=dev(z), bias=None if bias is None else dev(bias),
+                          modality=None if mod is None else dev(mod), ws=ws, **out)
+    check_status(ws)
+    return {k_: host(v) for k_, v in out.items()}
+
+
+def _assert_reroute_equal(got, z, k, sf, rn, bias, mod, E, C):
+    ids_o, gates_o, drop_o, rr_o, first = O.route_reroute(z, k, C, sf, rn, bias, mod)
+    np.testing.assert_array_equal(got["ids"], ids_o)
+    np.testing.assert_array_equal(got["drop_mask"], drop_o)
+    np.testing.assert_array_equal(got["rerouted"], rr_o)
+    np.testing.assert_array_equal(got["demand"], first["demand"])
+    np.testing.assert_array_equal(got["counts"], O.dispatch_masked(ids_o, E, drop_o)["counts"])
+    rel = np.abs(got["gates"] - gates_o) / np.maximum(np.abs(gates_o), 1e-30)
+    assert rel.max() <= 1e-5, rel.max()
+    return rr_o
+
+
+@pytest.mark.parametrize("N,E,k,sf,rn,nb,cf", [
+    (3000, 64, 2, 0, 1, 0, 1),            # Zipf-skewed softmax top-2, cf = 1: many moves
+    (2000, 32, 4, 1, 1, 2, 1),            # sigmoid + two bias sets, top-4
+    (4096, 64, 1, 0, 0, 0, 1),            # Switch: raw probability gates
+    (1000, 8, 6, 0, 1, 0, 1),             # 2k > E: the last candidates do not exist
+    (777, 40, 16, 1, 1, 1, 1),            # k = 16, the largest the policy takes
+])
+def test_reroute_routing_bit_exact(N, E, k, sf, rn, nb, cf):
+    z = W.random_logits(N, E, N + k, scale=1.5)
+    z = (z + W.zipf_logit_offsets(E)[None, :] * (sf == 0)).astype(np.float32)
+    bias = W.random_bias(nb, E, N) if nb else None
+    mod = W.random_modality(N, N + 1) if nb > 1 else None
+    C = O.capacity(N, k, E, cf)
+    cfg = nat.make_config(N, 64, E, k, 64, n_bias_sets=nb, score_fn=sf, renorm=rn, capacity=C)
+    got = _gpu_reroute(cfg, z, bias, mod)
+    rr = _assert_reroute_equal(got, z, k, sf, rn, bias, mod, E, C)
+    assert rr.sum() > 0
+
+
+def test_reroute_on_the_slides_trace():
+    from golden.reader import load
+    g = load("p2_capacity_trace.txt")
+    assign = [tuple(int(v) for v in p.split()) for p in g["assign"].split("|")]
+    z = np.full((8, 4), 0.2, np.float32)
+    for t, (a, b) in enumerate(assign):
+        z[t, a], z[t, b] = 2.1, 1.8
+    z[5, 3] = -1.0
+    cfg = nat.make_config(8, 64, 4, 2, 64, capacity=int(g["C_1.25"]))
+    got = _gpu_reroute(cfg, z)
+    assert got["ids"][5].tolist() == [int(g["report_t6_expert"]), 1]
+    assert got["counts"].tolist() == [5, 4, 4, 3] and got["drop_mask"].sum() == 0
+    _assert_reroute_equal(got, z, 2, O.SOFTMAX, 1, None, None, 4, int(g["C_1.25"]))
+
+
+def test_reroute_forward_against_the_oracle():
+    shape = W.PRESETS["capacity-cf1"].replace(N=2048, d=256, F=256)
+    t = W.make_inputs(shape, device="cuda")
+    C = O.capacity(shape.N, shape.k, shape.E, shape.capacity_factor)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    N, k, E = shape.N, shape.k, shape.E
+    ro = dict(logits=torch.empty((N, E), device="cuda"),
+              ids=torch.empty((N, k), dtype=torch.int32, device="cuda"),
+              drop_mask=torch.empty((N, k), dtype=torch.uint8, device="cuda"),
+              counts=torch.empty(E, dtype=torch.int32, device="cuda"))
+    rr = torch.empty((N, k), dtype=torch.uint8, device="cuda")
+    y = torch.empty_like(t["x"])
+    nat.moe_forward_reroute(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y,
+                            logit_offset=t["logit_offset"], route_out=ro, rerouted=rr, ws=ws)
+    check_status(ws)
+    z = host(ro["logits"])
+    sample = np.r_[0:40, 2000:2048]
+    ref, info = O.forward(f64(t["x"]), None, _Lazy(t["W_gu"]), _Lazy(t["W_down"]), k=k, E=E,
+                          n_shared=shape.n_shared, C=C, logits=z, tokens=sample,
+                          overflow="reroute")
+    np.testing.assert_array_equal(host(ro["ids"]), info["ids"])
+    np.testing.assert_array_equal(host(ro["drop_mask"]), info["drop_mask"])
+    np.testing.assert_array_equal(host(rr), info["rerouted"])
+    np.testing.assert_array_equal(host(ro["counts"]), info["counts"])
+    assert info["rerouted"].sum() > 0
+    assert_close_layer(host(y)[sample], ref)
+
+
+def test_reroute_without_capacity_is_the_plain_forward():
+    shape = W.PRESETS["dsv3-n64"].replace(N=300, d=256, F=256, E=16, k=4)
+    t = W.make_inputs(shape, device="cuda")
+    cfg = nat.config_from_shape(shape, capacity=0)
+    ws = nat.alloc_workspace(cfg)
+    y1, y2 = torch.empty_like(t["x"]), torch.empty_like(t["x"])
+    rr = torch.full((shape.N, shape.k), 7, dtype=torch.uint8, device="cuda")
+    nat.moe_forward(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y1,
+                    bias=t["bias"], ws=ws)
+    nat.moe_forward_reroute(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"],
+                            y=y2, bias=t["bias"], rerouted=rr, ws=ws)
+    check_status(ws)
+    assert torch.equal(y1, y2) and int(rr.sum()) == 0
+
+
+def test_reroute_refuses_k_above_16():
+    cfg = nat.make_config(64, 64, 40, 17, 64, capacity=10)
+    ws = nat.alloc_workspace(cfg)
+    with pytest.raises(nat.MoeError) as e:
+        nat.moe_route_reroute(cfg, logits=dev(np.zeros((64, 40), np.float32)),
+                              ids=torch.empty((64, 17), dtype=torch.int32, device="cuda"),
+                              gates=torch.empty((64, 17), device="cuda"), ws=ws)
+    assert e.value.status == nat.MOE_ERR_UNSUPPORTED
+
+
+class _Lazy:
+    def __init__(self, t):
+        self.t = t
+
+    def __getitem__(self, e):
+        return f64(self.t[e])
+
+
+def test_layer_with_reroute_policy_device_and_host_buffers():
+    from mixture_experts_layer_50_b200 import MoELayer
+    shape = W.PRESETS["switch-cf1"].replace(N=1024, d=256, F=256)
+    t = W.make_inputs(shape, device="cuda")
+    layer = MoELayer.from_workload(shape, t, overflow="reroute")
+    C = layer.capacity(shape.N)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    y_ref = torch.empty_like(t["x"])
+    nat.moe_forward_reroute(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"],
+                            y=y_ref, logit_offset=t["logit_offset"], ws=ws)
+    check_status(ws)
+    assert torch.equal(layer.forward(t["x"]), y_ref)
+    xh = t["x"].cpu().pin_memory()
+    yh = [torch.empty_like(xh).pin_memory() for _ in range(2)]
+    layer.forward_host(xh, yh[0])
+    layer.forward_host_batches([xh, xh], yh)
+    assert torch.equal(yh[0], y_ref.cpu()) and torch.equal(yh[1], y_ref.cpu())
+    assert layer.check_status() == 0

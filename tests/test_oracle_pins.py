@@ -521,7 +521,7 @@ def test_padded_dispatch_buffer_is_the_slides_table():
 
 
 # --------------------------------------------------------------------------
-# overflow policy "report" (slides, "Politiques de débordement"; reading R13)
+# overflow policy "report" (slides, "Politiques de débordement"; reading R14)
 # --------------------------------------------------------------------------
 def test_report_policy_on_the_slides_trace():
     g, assign, T, E, k = _trace()

@@ -22,6 +22,10 @@ __device__ __forceinline__ void accum_bf16x8(float (&acc)[8], const uint4& v, fl
   }
 }
 
+// KMAX >= k bounds the slots so that the k row loads of a vector are issued together
+// before the sums (KMAX = 0: any k, one load after the other).  Either way the sum runs in
+// slot order and then adds the shared row, so every KMAX gives the same bits.
+template <int KMAX>
 __global__ void __launch_bounds__(128) combine_bf16_kernel(
     const uint4* __restrict__ ye, const int32_t* __restrict__ slot_row,
     const float* __restrict__ gates, int k, int vecs, int64_t shared_row0,
@@ -36,11 +40,24 @@ __global__ void __launch_bounds__(128) combine_bf16_kernel(
   __syncthreads();
   for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < k; ++j) {
-      const int32_t r = s_row[j];
-      if (r >= 0) accum_bf16x8(acc, ye[(int64_t)r * vecs + v], s_g[j]);
+    if constexpr (KMAX > 0) {
+      uint4 rows[KMAX];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j < k && s_row[j] >= 0) rows[j] = ye[(int64_t)s_row[j] * vecs + v];
+      uint4 sh = make_uint4(0u, 0u, 0u, 0u);
+      if (shared_row0 >= 0) sh = ye[(shared_row0 + t) * vecs + v];
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j)
+        if (j < k && s_row[j] >= 0) accum_bf16x8(acc, rows[j], s_g[j]);
+      if (shared_row0 >= 0) accum_bf16x8(acc, sh, 1.0f);
+    } else {
+      for (int j = 0; j < k; ++j) {
+        const int32_t r = s_row[j];
+        if (r >= 0) accum_bf16x8(acc, ye[(int64_t)r * vecs + v], s_g[j]);
+      }
+      if (shared_row0 >= 0) accum_bf16x8(acc, ye[(shared_row0 + t) * vecs + v], 1.0f);
     }
-    if (shared_row0 >= 0) accum_bf16x8(acc, ye[(shared_row0 + t) * vecs + v], 1.0f);
     uint4 o;
     __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
 #pragma unroll
@@ -96,8 +113,17 @@ cudaError_t launch_combine(const void* ye, const int32_t* slot_row, const float*
     combine_f32_kernel<<<(unsigned)N, 128, 0, stream>>>((const float4*)ye, slot_row, gates, k,
                                                         d / 4, shared_row0, (float4*)y);
   } else {
-    combine_bf16_kernel<<<(unsigned)N, 128, 0, stream>>>((const uint4*)ye, slot_row, gates, k,
-                                                         d / 8, shared_row0, (uint4*)y);
+    const uint4* src = (const uint4*)ye;
+    uint4* dst = (uint4*)y;
+    const unsigned blocks = (unsigned)N;
+    if (k <= 2)
+      combine_bf16_kernel<2><<<blocks, 128, 0, stream>>>(src, slot_row, gates, k, d / 8, shared_row0, dst);
+    else if (k <= 4)
+      combine_bf16_kernel<4><<<blocks, 128, 0, stream>>>(src, slot_row, gates, k, d / 8, shared_row0, dst);
+    else if (k <= 8)
+      combine_bf16_kernel<8><<<blocks, 128, 0, stream>>>(src, slot_row, gates, k, d / 8, shared_row0, dst);
+    else
+      combine_bf16_kernel<0><<<blocks, 128, 0, stream>>>(src, slot_row, gates, k, d / 8, shared_row0, dst);
   }
   return cudaGetLastError();
 }

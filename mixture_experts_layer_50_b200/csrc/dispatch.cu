@@ -166,6 +166,10 @@ __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
   }
   if (xp == nullptr) return;
   __syncthreads();
+  // a token whose slots were all dropped is not read at all
+  bool any = false;
+  for (int j = 0; j < k; ++j) any |= s_row[j] >= 0;
+  if (!any) return;
   const V* src = x + t * row_vecs;
   for (int v = threadIdx.x; v < row_vecs; v += blockDim.x) {
     const V val = src[v];

@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(256) balance_tile_kernel(
     const float* __restrict__ logits, const int32_t* __restrict__ ids,
     const uint8_t* __restrict__ modality, int64_t N, int E, int k, int score_fn, int n_sets,
     float* __restrict__ part_p, int32_t* __restrict__ part_load) {
+  pdl_wait();
   extern __shared__ float sm[];
   float* s_m = sm;                                   // [kTile] per-token max (softmax)
   float* s_inv = sm + kTile;                         // [kTile] 1 / normaliser
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(1024) balance_final_kernel(
     int64_t N, int E, int k, int n_sets, float* __restrict__ f, float* __restrict__ P,
     float* __restrict__ aux, int32_t* __restrict__ set_load, float* __restrict__ bias,
     float gamma) {
+  pdl_wait();
   __shared__ float s_fp[1024];
   __shared__ int64_t s_red[1024];
   __shared__ int64_t s_tot[kMaxSets];
@@ -142,13 +144,13 @@ cudaError_t launch_balance(const float* logits, const int32_t* ids, const uint8_
   int32_t* part_load = reinterpret_cast<int32_t*>(part_p + (size_t)tiles * E);
   if (tiles > 0) {
     const size_t smem = sizeof(float) * 2 * kTile + sizeof(int32_t) * (size_t)n_sets * E;
-    balance_tile_kernel<<<tiles, 256, smem, stream>>>(logits, ids, modality, N, E, k, score_fn,
+    launch_pdl(balance_tile_kernel, tiles, 256, smem, stream, logits, ids, modality, N, E, k, score_fn,
                                                       n_sets, part_p, part_load);
     ++*launches;
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  balance_final_kernel<<<1, 1024, 0, stream>>>(part_p, part_load, tiles, N, E, k, n_sets, f, P,
+  launch_pdl(balance_final_kernel, 1, 1024, 0, stream, part_p, part_load, tiles, N, E, k, n_sets, f, P,
                                                aux, set_load, bias, gamma);
   ++*launches;
   return cudaGetLastError();

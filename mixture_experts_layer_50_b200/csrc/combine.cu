@@ -30,6 +30,7 @@ __global__ void __launch_bounds__(128) combine_bf16_kernel(
     const uint4* __restrict__ ye, const int32_t* __restrict__ slot_row,
     const float* __restrict__ gates, int k, int vecs, int64_t shared_row0,
     uint4* __restrict__ y) {
+  pdl_wait();
   __shared__ int32_t s_row[33];
   __shared__ float s_g[33];
   const int64_t t = blockIdx.x;
@@ -70,6 +71,7 @@ __global__ void __launch_bounds__(128) combine_f32_kernel(
     const float4* __restrict__ ye, const int32_t* __restrict__ slot_row,
     const float* __restrict__ gates, int k, int vecs, int64_t shared_row0,
     float4* __restrict__ y) {
+  pdl_wait();
   __shared__ int32_t s_row[33];
   __shared__ float s_g[33];
   const int64_t t = blockIdx.x;
@@ -110,20 +112,20 @@ cudaError_t launch_combine(const void* ye, const int32_t* slot_row, const float*
   if (N == 0) return cudaSuccess;
   ++*launches;
   if (is_f32) {
-    combine_f32_kernel<<<(unsigned)N, 128, 0, stream>>>((const float4*)ye, slot_row, gates, k,
+    launch_pdl(combine_f32_kernel, (unsigned)N, 128, 0, stream, (const float4*)ye, slot_row, gates, k,
                                                         d / 4, shared_row0, (float4*)y);
   } else {
     const uint4* src = (const uint4*)ye;
     uint4* dst = (uint4*)y;
     const unsigned blocks = (unsigned)N;
     if (k <= 2)
-      combine_bf16_kernel<2><<<blocks, 128, 0, stream>>>(src, slot_row, gates, k, d / 8, shared_row0, dst);
+      launch_pdl(combine_bf16_kernel<2>, blocks, 128, 0, stream, src, slot_row, gates, k, d / 8, shared_row0, dst);
     else if (k <= 4)
-      combine_bf16_kernel<4><<<blocks, 128, 0, stream>>>(src, slot_row, gates, k, d / 8, shared_row0, dst);
+      launch_pdl(combine_bf16_kernel<4>, blocks, 128, 0, stream, src, slot_row, gates, k, d / 8, shared_row0, dst);
     else if (k <= 8)
-      combine_bf16_kernel<8><<<blocks, 128, 0, stream>>>(src, slot_row, gates, k, d / 8, shared_row0, dst);
+      launch_pdl(combine_bf16_kernel<8>, blocks, 128, 0, stream, src, slot_row, gates, k, d / 8, shared_row0, dst);
     else
-      combine_bf16_kernel<0><<<blocks, 128, 0, stream>>>(src, slot_row, gates, k, d / 8, shared_row0, dst);
+      launch_pdl(combine_bf16_kernel<0>, blocks, 128, 0, stream, src, slot_row, gates, k, d / 8, shared_row0, dst);
   }
   return cudaGetLastError();
 }

@@ -36,4 +36,32 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Token-tile size of the dispatch kernels (tokens ranked by one warp in order).
 constexpr int kRankTile = 32;
 
+// Programmatic dependent launch.  Every kernel of the library is launched with programmatic
+// stream serialisation (launch_pdl), so the GPU may schedule it while its predecessor on the
+// stream is still running; pdl_wait() returns once that predecessor has completed and its
+// memory is visible, and every kernel calls it before touching global memory.  The chain
+// stays transitive because each kernel waits before it finishes.  pdl_release() lets the
+// successor be scheduled before this grid ends (the persistent GEMMs call it once their
+// last loads are issued); without it the successor is released at exit.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 }  // namespace moe

@@ -24,6 +24,7 @@ namespace {
 __global__ void __launch_bounds__(32) rank_local_kernel(
     const int32_t* __restrict__ ids, const uint8_t* __restrict__ drop_mask, int64_t N, int k,
     int E, int32_t* __restrict__ local_rank, int32_t* __restrict__ tile_hist, int* status) {
+  pdl_wait();
   extern __shared__ int32_t smem[];
   int32_t* cnt = smem;       // [E]
   int32_t* sid = smem + E;   // [kRankTile * k]
@@ -72,6 +73,7 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
     const int32_t* __restrict__ tile_hist, int n_tiles, int E, int64_t C,
     int32_t* __restrict__ tile_base, int32_t* __restrict__ demand,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* arrive) {
+  pdl_wait();
   __shared__ int32_t part[32][33];  // chunk sums [warp][lane]
   __shared__ int32_t warp_tot[32];
   __shared__ bool s_last;
@@ -148,6 +150,7 @@ __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
     int64_t C, int32_t* __restrict__ slot_row, int32_t* __restrict__ row_token,
     uint8_t* __restrict__ drop_mask_out, const V* __restrict__ x, V* __restrict__ xp,
     int row_vecs) {
+  pdl_wait();
   __shared__ int32_t s_row[32];
   const int64_t t = blockIdx.x;
   if (threadIdx.x < k) {
@@ -181,6 +184,7 @@ __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
 }
 
 __global__ void pad_offsets_kernel(int E, int64_t C, int32_t* __restrict__ offsets_pad) {
+  pdl_wait();
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e <= E) offsets_pad[e] = (int32_t)(e * C);
 }
@@ -189,6 +193,7 @@ __global__ void pad_offsets_kernel(int E, int64_t C, int32_t* __restrict__ offse
 __global__ void __launch_bounds__(128) zero_padding_kernel(
     const int32_t* __restrict__ counts, int64_t C, uint4* __restrict__ xp_pad, int row_vecs,
     int32_t* __restrict__ row_token_pad) {
+  pdl_wait();
   const int64_t r = blockIdx.x;
   const int e = (int)(r / C);
   if (r - (int64_t)e * C < counts[e]) return;
@@ -201,7 +206,7 @@ __global__ void __launch_bounds__(128) zero_padding_kernel(
 cudaError_t launch_pad_offsets(int E, int64_t C, int32_t* offsets_pad, cudaStream_t stream,
                                int* launches) {
   ++*launches;
-  pad_offsets_kernel<<<(E + 1 + 255) / 256, 256, 0, stream>>>(E, C, offsets_pad);
+  launch_pdl(pad_offsets_kernel, (E + 1 + 255) / 256, 256, 0, stream, E, C, offsets_pad);
   return cudaGetLastError();
 }
 
@@ -211,7 +216,7 @@ cudaError_t launch_zero_padding(const int32_t* counts, int E, int64_t C, void* x
   const int64_t rows = (int64_t)E * C;
   if (rows == 0) return cudaSuccess;
   ++*launches;
-  zero_padding_kernel<<<(unsigned)rows, 128, 0, stream>>>(counts, C, (uint4*)xp_pad,
+  launch_pdl(zero_padding_kernel, (unsigned)rows, 128, 0, stream, counts, C, (uint4*)xp_pad,
                                                          row_bytes / 16, row_token_pad);
   return cudaGetLastError();
 }
@@ -223,7 +228,7 @@ cudaError_t launch_rank_local(const int32_t* ids, const uint8_t* drop_mask, int6
   const int64_t tiles = (N + kRankTile - 1) / kRankTile;
   const size_t smem = sizeof(int32_t) * ((size_t)E + (size_t)kRankTile * k);
   ++*launches;  // at most (1024 + kRankTile * 32) ints of shared memory: below the 48 KB default
-  rank_local_kernel<<<(unsigned)tiles, 32, smem, stream>>>(ids, drop_mask, N, k, E, local_rank,
+  launch_pdl(rank_local_kernel, (unsigned)tiles, 32, smem, stream, ids, drop_mask, N, k, E, local_rank,
                                                            tile_hist, status);
   return cudaGetLastError();
 }
@@ -234,7 +239,7 @@ cudaError_t launch_dispatch_scan(const int32_t* tile_hist, int64_t N, int E, int
                                  int* launches) {
   const int tiles = (int)((N + kRankTile - 1) / kRankTile);
   ++*launches;
-  dispatch_scan_kernel<<<(E + 31) / 32, 1024, 0, stream>>>(tile_hist, tiles, E, C, tile_base,
+  launch_pdl(dispatch_scan_kernel, (E + 31) / 32, 1024, 0, stream, tile_hist, tiles, E, C, tile_base,
                                                            demand, counts, offsets, arrive);
   return cudaGetLastError();
 }
@@ -248,15 +253,15 @@ cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_ran
   if (N == 0) return cudaSuccess;
   ++*launches;
   if (xp != nullptr && row_bytes % 16 == 0) {
-    dispatch_scatter_kernel<uint4><<<(unsigned)N, 128, 0, stream>>>(
+    launch_pdl(dispatch_scatter_kernel<uint4>, (unsigned)N, 128, 0, stream, 
         ids, local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
         (const uint4*)x, (uint4*)xp, row_bytes / 16);
   } else if (xp != nullptr) {
-    dispatch_scatter_kernel<uint32_t><<<(unsigned)N, 128, 0, stream>>>(
+    launch_pdl(dispatch_scatter_kernel<uint32_t>, (unsigned)N, 128, 0, stream, 
         ids, local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
         (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4);
   } else {
-    dispatch_scatter_kernel<uint4><<<(unsigned)N, 128, 0, stream>>>(
+    launch_pdl(dispatch_scatter_kernel<uint4>, (unsigned)N, 128, 0, stream, 
         ids, local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
         nullptr, nullptr, 0);
   }

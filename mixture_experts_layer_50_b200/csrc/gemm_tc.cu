@@ -394,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmAs,
                         const __grid_constant__ CUtensorMap tmB, const Args p) {
+  pdl_wait();
   using L = Layout<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -502,6 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // every load of this CTA is issued: the next kernel on the stream may be scheduled
+      pdl_release();
       if (!ok) {
         // let the loads already issued land before the CTA leaves
         for (int i = 0; i < STAGES && i < armed; ++i) {
@@ -623,6 +626,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA,
                             const __grid_constant__ CUtensorMap tmAs,
                             const __grid_constant__ CUtensorMap tmB, const Args p) {
+  pdl_wait();
   constexpr int BN = 256;   // MMA N
   constexpr int BMT = 256;  // tile rows (128 per CTA)
   using L = Layout2<STAGES>;
@@ -734,6 +738,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
       }
+      pdl_release();
       if (!ok && rank == 0) {
         for (int i = 0; i < STAGES && i < armed; ++i) {
           stage = (stage + STAGES - 1) % STAGES;
@@ -908,6 +913,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmX,
                              const __grid_constant__ CUtensorMap tmXs,
                              const __grid_constant__ CUtensorMap tmW, const Args p) {
+  pdl_wait();
   using L = LayoutSwap<STAGES>;
   constexpr int kOutPerTile = (EPI == kEpiSwiglu) ? 64 : 128;
   extern __shared__ uint8_t smem_raw[];
@@ -1013,6 +1019,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      pdl_release();
       if (!ok) {
         for (int i = 0; i < STAGES && i < armed; ++i) {
           stage = (stage + STAGES - 1) % STAGES;
@@ -1256,7 +1263,7 @@ cudaError_t launch_t(const GroupedGemm& g, const CUtensorMap& mA, const CUtensor
   static bool done[kMaxDev] = {};
   const cudaError_t e = allow_max_smem(kern, done);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(mA, mAs, mB, make_args(g));
+  launch_pdl(kern, grid, kThreads, smem, stream, mA, mAs, mB, make_args(g));
   return cudaGetLastError();
 }
 
@@ -1268,7 +1275,7 @@ cudaError_t launch_2sm(const GroupedGemm& g, const CUtensorMap& mA, const CUtens
   static bool done[kMaxDev] = {};
   const cudaError_t e = allow_max_smem(kern, done);
   if (e != cudaSuccess) return e;
-  kern<<<2 * pairs, kThreads, smem, stream>>>(mA, mAs, mB, make_args(g));
+  launch_pdl(kern, 2 * pairs, kThreads, smem, stream, mA, mAs, mB, make_args(g));
   return cudaGetLastError();
 }
 
@@ -1280,7 +1287,7 @@ cudaError_t launch_swap(const GroupedGemm& g, const CUtensorMap& mX, const CUten
   static bool done[kMaxDev] = {};
   const cudaError_t e = allow_max_smem(kern, done);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kThreads, smem, stream>>>(mX, mXs, mW, make_args(g));
+  launch_pdl(kern, grid, kThreads, smem, stream, mX, mXs, mW, make_args(g));
   return cudaGetLastError();
 }
 

@@ -23,6 +23,7 @@ __global__ void reroute_offer_kernel(const int32_t* __restrict__ ids,
                                      const uint8_t* __restrict__ drop1,
                                      const int32_t* __restrict__ cand, int64_t N, int k,
                                      int32_t* __restrict__ offer, uint8_t* __restrict__ not_offer) {
+  pdl_wait();
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (t >= N) return;
   int i = 0;
@@ -52,6 +53,7 @@ __global__ void __launch_bounds__(256) reroute_accept_kernel(
     const int32_t* __restrict__ counts1, const float* __restrict__ cand_val, int64_t N, int E,
     int k, int64_t C, int score_fn, int renorm, float* __restrict__ gates,
     uint8_t* __restrict__ drop_out, uint8_t* __restrict__ rerouted) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= N) return;
@@ -103,7 +105,7 @@ cudaError_t launch_reroute_offer(const int32_t* ids, const uint8_t* drop1, const
                                  cudaStream_t stream, int* launches) {
   if (N == 0) return cudaSuccess;
   ++*launches;
-  reroute_offer_kernel<<<(unsigned)((N + 255) / 256), 256, 0, stream>>>(ids, drop1, cand, N, k,
+  launch_pdl(reroute_offer_kernel, (unsigned)((N + 255) / 256), 256, 0, stream, ids, drop1, cand, N, k,
                                                                        offer, not_offer);
   return cudaGetLastError();
 }
@@ -116,7 +118,7 @@ cudaError_t launch_reroute_accept(int32_t* ids, const uint8_t* drop1, const int3
                                   uint8_t* rerouted, cudaStream_t stream, int* launches) {
   if (N == 0) return cudaSuccess;
   ++*launches;
-  reroute_accept_kernel<<<(unsigned)((N * 32 + 255) / 256), 256, 0, stream>>>(
+  launch_pdl(reroute_accept_kernel, (unsigned)((N * 32 + 255) / 256), 256, 0, stream, 
       ids, drop1, offer, not_offer, local_rank, tile_base, counts1, cand_val, N, E, k, C,
       score_fn, renorm, gates, drop_out, rerouted);
   return cudaGetLastError();

@@ -43,7 +43,8 @@ __device__ __forceinline__ float exp_reduced_taylor(float x) {
 
 __device__ __forceinline__ float sigmoid_reproducible(float z) {
   const float zc = fminf(fmaxf(z, -80.0f), 80.0f);
-  return __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_reduced_taylor(-zc)));
+  // the correctly rounded reciprocal: the same bits as the correctly rounded 1 / y
+  return __frcp_rn(__fadd_rn(1.0f, exp_reduced_taylor(-zc)));
 }
 
 // (key, expert) order used by the selection: larger key first, then lower index.
@@ -58,6 +59,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
     int score_fn, int renorm, const float* __restrict__ bias, int n_bias_sets,
     const uint8_t* __restrict__ modality, int32_t* __restrict__ ids, float* __restrict__ gates,
     int* status, int k_extra, int32_t* __restrict__ cand, float* __restrict__ cand_val) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= N) return;
@@ -182,7 +184,7 @@ cudaError_t launch_j(const float* logits, int n_parts, int64_t part_stride, cons
                      float* cand_val, cudaStream_t stream) {
   const int threads = 256;
   const int64_t blocks = (N * 32 + threads - 1) / threads;
-  route_topk_kernel<J><<<(unsigned)blocks, threads, 0, stream>>>(
+  launch_pdl(route_topk_kernel<J>, (unsigned)blocks, threads, 0, stream, 
       logits, n_parts, part_stride, offset, logits_out, N, E, k, score_fn, renorm, bias,
       n_bias_sets, modality, ids, gates, status, k_extra, cand, cand_val);
   return cudaGetLastError();
@@ -207,6 +209,7 @@ __global__ void __launch_bounds__(256) hash_topk_kernel(const int32_t* __restric
                                                         int64_t N, int E, int k,
                                                         int32_t* __restrict__ ids,
                                                         float* __restrict__ gates) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= N) return;
@@ -258,7 +261,7 @@ cudaError_t launch_route_hash(const int32_t* token_ids, int64_t N, int E, int k,
   const unsigned blocks = (unsigned)((N * 32 + 255) / 256);
 #define MOE_HASH_CASE(JJ) \
   if (J <= JJ) {          \
-    hash_topk_kernel<JJ><<<blocks, 256, 0, stream>>>(token_ids, N, E, k, ids, gates); \
+    launch_pdl(hash_topk_kernel<JJ>, blocks, 256, 0, stream, token_ids, N, E, k, ids, gates); \
     return cudaGetLastError(); \
   }
   MOE_HASH_CASE(1)

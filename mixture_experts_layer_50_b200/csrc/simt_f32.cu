@@ -14,6 +14,7 @@ __global__ void __launch_bounds__(256) router_f32_kernel(const float* __restrict
                                                          const float* __restrict__ off,
                                                          int64_t N, int d, int E,
                                                          float* __restrict__ logits) {
+  pdl_wait();
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= N * E) return;
   const int64_t t = idx / E;
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(256) ffn_up_f32_kernel(
     const float* __restrict__ xp, const float* __restrict__ x, const int32_t* __restrict__ offsets,
     int64_t N, int64_t Nk, int d, int E, int F, int n_shared, int act, float clamp,
     const float* __restrict__ W_gu, float* __restrict__ h) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int f0 = blockIdx.y * 32;
@@ -114,6 +116,7 @@ __global__ void __launch_bounds__(256) ffn_down_f32_kernel(
     const float* __restrict__ h, const float* __restrict__ xp, const float* __restrict__ x,
     const int32_t* __restrict__ offsets, int64_t N, int64_t Nk, int d, int E, int F,
     int n_shared, const float* __restrict__ W_down, float* __restrict__ ye) {
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int c0 = blockIdx.y * 32;
@@ -140,14 +143,14 @@ template <int NV>
 void launch_up(dim3 g, cudaStream_t st, const float* xp, const float* x, const int32_t* offsets,
                int64_t N, int64_t Nk, int d, int E, int F, int n_shared, int act, float clamp,
                const float* W_gu, float* h) {
-  ffn_up_f32_kernel<NV><<<g, 256, 0, st>>>(xp, x, offsets, N, Nk, d, E, F, n_shared, act, clamp,
+  launch_pdl(ffn_up_f32_kernel<NV>, g, 256, 0, st, xp, x, offsets, N, Nk, d, E, F, n_shared, act, clamp,
                                            W_gu, h);
 }
 template <int NV>
 void launch_down(dim3 g, cudaStream_t st, const float* h, const float* xp, const float* x,
                  const int32_t* offsets, int64_t N, int64_t Nk, int d, int E, int F,
                  int n_shared, const float* W_down, float* ye) {
-  ffn_down_f32_kernel<NV><<<g, 256, 0, st>>>(h, xp, x, offsets, N, Nk, d, E, F, n_shared,
+  launch_pdl(ffn_down_f32_kernel<NV>, g, 256, 0, st, h, xp, x, offsets, N, Nk, d, E, F, n_shared,
                                              W_down, ye);
 }
 
@@ -166,7 +169,7 @@ cudaError_t launch_router_f32(const float* x, const float* W_g, const float* log
   if (N == 0) return cudaSuccess;
   ++*launches;
   const int64_t total = N * E;
-  router_f32_kernel<<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(x, W_g, logit_offset,
+  launch_pdl(router_f32_kernel, (unsigned)((total + 255) / 256), 256, 0, stream, x, W_g, logit_offset,
                                                                          N, d, E, logits);
   return cudaGetLastError();
 }

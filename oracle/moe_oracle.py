@@ -27,7 +27,7 @@ Sources (page title, section):
   (steps 1-4 and the numeric example), "Практика" (the ``topk_route``
   contract), "Эксперимент на PyTorch".
 
-Readings where the pages are silent (each is listed again in the design doc):
+Readings where the pages are silent:
 
 * R1  top-k keys: softmax scoring selects on ``z + b`` (the raw logit, plus the
       selection bias when there is one, as P1's ``route`` does); with no bias

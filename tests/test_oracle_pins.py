@@ -261,8 +261,8 @@ def test_load_fractions_sum():
     z = np.random.default_rng(1).normal(0, 1, (1000, 8)).astype(np.float32)
     ids, _ = O.route(z, 2)
     per_n, per_tk = O.load_fractions(ids, 8)
-    assert per_n.sum() == pytest.approx(2.0, abs=1e-12)      # P4: bincount / N sums to k
-    assert per_tk.sum() == pytest.approx(1.0, abs=1e-12)     # P5: count / (T k) sums to 1
+    assert per_n.sum() == pytest.approx(2.0, abs=1e-12)      # dataistudio "Mixture of Experts": bincount / N sums to k
+    assert per_tk.sum() == pytest.approx(1.0, abs=1e-12)     # "Основы MoE": count / (T k) sums to 1
 
 
 # --------------------------------------------------------------------------
@@ -308,7 +308,7 @@ def _tiny_layer(rng, N, d, E, F, G, act=O.SWIGLU):
 
 
 def test_dense_limit_k_equals_E():
-    """k = E with softmax turns the layer into the dense mixture of all experts (P5 Практика)."""
+    """k = E with softmax turns the layer into the dense mixture of all experts ("Основы MoE", "Практика")."""
     rng = np.random.default_rng(7)
     N, d, E, F = 9, 6, 5, 4
     x, W_g, W_gu, W_down = _tiny_layer(rng, N, d, E, F, E)
@@ -473,7 +473,7 @@ def test_switch_balance_statistic_printed_example():
 
 
 def test_bias_update_on_the_slides_trace_loads():
-    # P2 trace demand 6/4/3/3 (mean 4): E1 overloaded, E2 on target, E3 and E4 underloaded
+    # the slides' trace ("Cas guidé"): demand 6/4/3/3 (mean 4): E1 overloaded, E2 on target, E3 and E4 underloaded
     gt, assign, T, E, k = _trace()
     ids = np.array(assign, np.int32)
     load = O.per_set_load(ids, E)

@@ -315,6 +315,15 @@ MOE_API moe_status moe_forward_host_batches(const moe_config* cfg, int32_t n_bat
                                             const void* W_down, void* const* y_host, void* ws,
                                             moe_stream_t stream);
 
+/* Failure-detection self-test (the pages have no counterpart): one device thread waits, with
+ * the same bounded wait the GEMM pipelines use, on a barrier that nothing ever completes.  The
+ * wait runs out after limit_ns (0 .. 1e9; a backstop poll count ends it too if the GPU timer
+ * stalls) and records MOE_ERR_TIMEOUT in the workspace status word, which moe_check_status
+ * then reports -- the path a stalled pipeline takes.  The kernel ends normally: the context
+ * stays usable.  Asynchronous on `stream`; MOE_ERR_INVALID_ARG for a NULL ws or a limit
+ * outside the range. */
+MOE_API moe_status moe_selftest_wait_timeout(void* ws, int64_t limit_ns, moe_stream_t stream);
+
 /* Synchronise `stream`, read and clear the workspace status word.  Returns MOE_OK or the
  * first device-detected error (MOE_ERR_INVALID_INPUT, MOE_ERR_TIMEOUT) since the last
  * check; MOE_ERR_CUDA if the stream reports an asynchronous CUDA error. */

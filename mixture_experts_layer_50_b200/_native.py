@@ -75,6 +75,7 @@ lib.moe_permute_padded.argtypes = [_cfgp] + [_vp] * 10
 lib.moe_forward_padded.argtypes = [_cfgp] + [_vp] * 11
 lib.moe_forward_host_batches.argtypes = [_cfgp, _i32] + [_vp] * 10
 lib.moe_route_reroute.argtypes = [_cfgp] + [_vp] * 15
+lib.moe_selftest_wait_timeout.argtypes = [_vp, _i64, _vp]
 lib.moe_forward_reroute.argtypes = [_cfgp] + [_vp] * 12
 lib.moe_profile_begin.argtypes = [_i32]
 lib.moe_profile_begin.restype = ctypes.c_int
@@ -86,7 +87,7 @@ for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "
            "moe_forward", "moe_forward_host", "moe_check_status", "moe_route_static",
            "moe_forward_routed", "moe_route_hash", "moe_balance", "moe_permute_padded",
            "moe_forward_padded", "moe_forward_host_batches", "moe_route_reroute",
-           "moe_forward_reroute"):
+           "moe_forward_reroute", "moe_selftest_wait_timeout"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
@@ -94,7 +95,8 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_rou
             "moe_check_status", "moe_profile_begin", "moe_profile_end", "moe_last_error",
             "moe_last_launch_count", "moe_route_static", "moe_forward_routed",
             "moe_route_hash", "moe_balance", "moe_permute_padded", "moe_forward_padded",
-            "moe_forward_host_batches", "moe_route_reroute", "moe_forward_reroute")
+            "moe_forward_host_batches", "moe_route_reroute", "moe_forward_reroute",
+            "moe_selftest_wait_timeout")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -323,6 +325,12 @@ def moe_forward_host_batches(cfg, *, x_host: list, W_g, W_gu, W_down, y_host: li
                                       _ptr(bias), mods, _ptr(W_gu), _ptr(W_down), ys, _ptr(ws),
                                       _stream(stream))
     _check(st, "moe_forward_host_batches")
+
+
+def moe_selftest_wait_timeout(ws, limit_ns: int, stream=None):
+    """A bounded device wait on a barrier nothing completes: records MOE_ERR_TIMEOUT."""
+    _check(lib.moe_selftest_wait_timeout(_ptr(ws), int(limit_ns), _stream(stream)),
+           "moe_selftest_wait_timeout")
 
 
 def moe_check_status(ws, stream=None) -> int:

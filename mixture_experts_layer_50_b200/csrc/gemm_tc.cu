@@ -75,16 +75,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Polls after which a wait gives up even if the global timer did not advance (a backstop:
+// each poll takes well over 20 ns, so this is more than a second).
+constexpr uint64_t kWaitMaxPolls = 50000000ull;
+
 // Wait for the phase of `parity` to complete.  Gives up (false) when another role of the
-// CTA has given up, or after kWaitLimitNs, recording a timeout.
+// CTA has given up, or after limit_ns, recording a timeout.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag, int* status) {
+                                          volatile int* abort_flag, int* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  while (true) {
+  for (uint64_t polls = 0;; ++polls) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns || polls > kWaitMaxPolls) {
       *abort_flag = 1;
       report_status(status, kStatusTimeout);
       return false;
@@ -1174,6 +1179,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---- failure-detection self-test --------------------------------------------------------
+// One thread waits, with the GEMMs' bounded wait, on an mbarrier that nothing ever completes:
+// the wait runs out after limit_ns and records MOE_ERR_TIMEOUT in the status word, as a
+// stalled GEMM pipeline would.  out[0] = 1 if the wait (wrongly) succeeded, else 0.
+__global__ void wait_selftest_kernel(int* status, uint64_t limit_ns, int* out) {
+  pdl_wait();
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(&bar, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  const bool ok = mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+  if (out != nullptr) out[0] = ok ? 1 : 0;
+  asm volatile("mbarrier.inval.shared::cta.b64 [%0];" ::"r"(smem_u32(&bar)) : "memory");
+}
+
 // ---- host side -------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -1354,6 +1376,13 @@ int pick_bn_1sm(const GroupedGemm& g) {
 }
 
 }  // namespace tc
+
+cudaError_t launch_wait_selftest(int* status, uint64_t limit_ns, int* out, cudaStream_t stream,
+                                 int* launches) {
+  ++*launches;
+  launch_pdl(tc::wait_selftest_kernel, 1, 32, 0, stream, status, limit_ns, out);
+  return cudaGetLastError();
+}
 
 // N width of the fp32-store (router) tiles: the fewest padded columns, then the wider tile.
 int router_tile_n(int n_out) {

@@ -134,5 +134,8 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
                                 const char** why);
 // N width of the tiles of an fp32-store GEMM with n_out columns (the router).
 int router_tile_n(int n_out);
+// Failure-detection self-test: a bounded wait on a barrier nothing completes (gemm_tc.cu).
+cudaError_t launch_wait_selftest(int* status, uint64_t limit_ns, int* out, cudaStream_t stream,
+                                 int* launches);
 
 }  // namespace moe

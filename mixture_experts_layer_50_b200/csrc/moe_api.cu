@@ -1084,6 +1084,18 @@ moe_status moe_route_static(const moe_config* cfg, const float* logits, const fl
   return MOE_OK;
 }
 
+moe_status moe_selftest_wait_timeout(void* ws, int64_t limit_ns, moe_stream_t stream) {
+  g_last_launches = 0;
+  if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  if (limit_ns < 0 || limit_ns > 1000000000) return fail(MOE_ERR_INVALID_ARG, "limit_ns outside 0 .. 1e9");
+  int launches = 0;
+  MOE_CUDA(moe::launch_wait_selftest(static_cast<int*>(ws), (uint64_t)limit_ns, nullptr,
+                                     (cudaStream_t)stream, &launches),
+           "wait self-test");
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
 moe_status moe_check_status(void* ws, moe_stream_t stream) {
   if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
   cudaStream_t st = (cudaStream_t)stream;

@@ -141,3 +141,11 @@ def test_binding_refuses_host_tensors(nat):
     with pytest.raises(ValueError):
         nat.moe_combine(c, ye=torch.zeros(4), slot_row=torch.zeros(4, dtype=torch.int32),
                         gates=torch.zeros(4), y=torch.zeros(4))
+
+
+def test_wait_selftest_validates_on_host(nat):
+    lib = nat.lib
+    assert lib.moe_selftest_wait_timeout(None, 1000, None) == nat.MOE_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(256)
+    assert lib.moe_selftest_wait_timeout(fake, -1, None) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_selftest_wait_timeout(fake, 2_000_000_000, None) == nat.MOE_ERR_INVALID_ARG

@@ -4,6 +4,7 @@ Routing, capacity and the permutation are compared bit for bit; gates at 1e-5 re
 expert outputs and the layer output at max|err| <= 2e-2 max|ref| for bf16 GEMMs (1e-4
 absolute for the fp32 toy layer).  Sizes span several tiles with ragged tails.
 """
+import time
 from fractions import Fraction
 
 import numpy as np
@@ -537,3 +538,59 @@ def test_graph_replay_matches_eager_forward():
     layer.forward_graphed(t["x"], y)
     assert torch.equal(y, layer.forward(t["x"]))
     assert layer.check_status() == 0
+
+
+def test_bounded_wait_runs_out_and_the_context_stays_usable():
+    """Failure detection without a fault: a device wait on a barrier that nothing completes
+    gives up after 2 ms, the status word reports MOE_ERR_TIMEOUT, and the next layer call on
+    the same context runs normally."""
+    shape = W.PRESETS["mixtral-n16"].replace(d=256, F=256, N=64)
+    t = W.make_inputs(shape, device="cuda")
+    cfg = nat.config_from_shape(shape)
+    ws = nat.alloc_workspace(cfg)
+    t0 = time.perf_counter()
+    nat.moe_selftest_wait_timeout(ws, 2_000_000)
+    assert nat.moe_check_status(ws) == nat.MOE_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    assert nat.moe_check_status(ws) == 0          # cleared by the read
+    y = torch.empty_like(t["x"])
+    nat.moe_forward(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y, ws=ws)
+    check_status(ws)
+    assert torch.isfinite(y.float()).all()
+
+
+def _random_shape(seed):
+    r = np.random.default_rng(1000 + seed)
+    E = int(r.integers(1, 80))
+    k = int(r.integers(1, min(E, 8) + 1))
+    act = W.SWIGLU if r.random() < 0.7 else W.RELU
+    sf = int(r.random() < 0.4)
+    nb = int(r.integers(0, 3)) if sf == 1 else 0
+    cf = [None, Fraction(1), Fraction(5, 4), Fraction(1, 2)][int(r.integers(0, 4))]
+    return W.LayerShape(f"random-{seed}", N=int(r.integers(1, 600)), d=8 * int(r.integers(4, 65)),
+                        E=E, k=k, F=8 * int(r.integers(4, 65)), n_shared=int(r.random() < 0.5),
+                        score_fn=sf, renorm=int(r.random() < 0.85) if k == 1 else 1, act=act,
+                        clamp=float(r.choice([0.0, 0.0, 0.5, 3.0])), n_bias_sets=nb,
+                        capacity_factor=cf, zipf_skew=bool(r.random() < 0.3), w_std=0.05,
+                        seed=seed)
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_forward_random_configurations(seed):
+    """Seeded random layers (d, E, k, F, shared expert, score function, renorm, bias sets,
+    activation, clamp, capacity, skew): routing bit-exact and the output within the bar,
+    against the oracle fed the GPU's logits."""
+    shape = _random_shape(seed)
+    t = W.make_inputs(shape, device="cuda")
+    C = O.capacity(shape.N, shape.k, shape.E, shape.capacity_factor)
+    y, ro, launches = _run_forward(shape, t, C)
+    kw = _oracle_kwargs(shape, t, C)
+    kw.pop("logit_offset")
+    ref, info = O.forward(f64(t["x"]), None, _LazyF64(t["W_gu"]), _LazyF64(t["W_down"]),
+                          logits=ro["logits"], **kw)
+    for name in ("ids", "drop_mask", "counts", "demand", "offsets"):
+        np.testing.assert_array_equal(ro[name], info[name], err_msg=f"{shape} {name}")
+    rel = np.abs(ro["gates"] - info["gates"]) / np.maximum(np.abs(info["gates"]), 1e-30)
+    assert rel.max() <= 1e-5, (shape, rel.max())
+    assert_close_layer(host(y), ref)
+    assert launches == 8

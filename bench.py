@@ -167,7 +167,7 @@ class ClockSampler:
 
 def read_traffic(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary, if its kernel source is unchanged."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload.replace('-', '_')}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()

@@ -53,3 +53,24 @@ def test_two_cpu_ranks_replicas_and_max_timing():
 def test_aggregate_value():
     import bench
     assert bench.aggregate_tokens_per_s(16384, 4, 10.0) == pytest.approx(16384 * 4 / 0.01)
+
+
+def test_traffic_is_read_only_for_the_measured_kernel_source(tmp_path, monkeypatch):
+    """roofline.traffic comes from the committed ncu summary of the workload, and only while
+    the kernel source still hashes to the one the counters were taken on."""
+    import hashlib
+    import bench
+    src = os.path.join(bench.ROOT, "mixture_experts_layer_50_b200", "csrc", "gemm_tc.cu")
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (tmp_path / "mixture_experts_layer_50_b200" / "csrc").mkdir(parents=True)
+    (tmp_path / "mixture_experts_layer_50_b200" / "csrc" / "gemm_tc.cu").write_bytes(open(src, "rb").read())
+    (prof / "gemm_gate_up_mixtral_n16384.md").write_text(
+        f"x\ntraffic_bytes_per_launch: 3.1e9\nkernel_source_sha256: {digest}\n")
+    (prof / "gemm_gate_up_mixtral_n4096.md").write_text(
+        "traffic_bytes_per_launch: 2.0e9\nkernel_source_sha256: 00\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.read_traffic("gemm_gate_up", "mixtral-n16384") == 3.1e9
+    assert bench.read_traffic("gemm_gate_up", "mixtral-n4096") is None    # stale counters
+    assert bench.read_traffic("gemm_gate_up", "dsv3-n8192") is None       # no capture

@@ -377,12 +377,16 @@ __device__ __forceinline__ void epilogue_warp(const Args& p, uint32_t t_row, uin
         const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 144 + pc * 16);
         const int64_t orow = out_row0 + row_in_tile;
         if constexpr (EPI == kEpiStoreF32) {
+          // fp32 rows of n_out = E columns: a 16-byte store only where the row stride and the
+          // base keep it 16-byte aligned (E a multiple of 4), else element by element
           float* o = reinterpret_cast<float*>(p.out) + orow * p.ld_out + col;
-          if (col + 4 <= p.n_out) {
+          const bool vec = (p.ld_out & 3) == 0 && (reinterpret_cast<uintptr_t>(p.out) & 15) == 0;
+          if (vec && col + 4 <= p.n_out) {
             *reinterpret_cast<uint4*>(o) = val;
           } else {
             const float* f = reinterpret_cast<const float*>(&val);
-            for (int e = 0; e < p.n_out - col; ++e) o[e] = f[e];
+            const int n = min(4, p.n_out - col);
+            for (int e = 0; e < n; ++e) o[e] = f[e];
           }
         } else {
           __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + orow * p.ld_out + col;

@@ -106,10 +106,12 @@ def test_route_full_size_v41flash_and_zipf_capacity():
 
 
 @pytest.mark.parametrize("N,d,E", [(16, 256, 8), (300, 512, 160), (1000, 256, 384),
-                                   (8192, 512, 256), (777, 136, 1024), (4096, 256, 8)])
+                                   (8192, 512, 256), (777, 136, 1024), (4096, 256, 8),
+                                   (122, 272, 17), (300, 64, 5), (64, 128, 33)])
 def test_router_gemm_logits(N, d, E):
-    """z = x . W_g on the tensor cores (tile widths 32 to 256, split K for few tiles) against
-    float64, element by element, within an fp32 accumulation bound."""
+    """z = x . W_g on the tensor cores (tile widths 32 to 256, split K for few tiles, E not a
+    multiple of 4 so that logit rows are not 16-byte aligned) against float64, element by
+    element, within an fp32 accumulation bound."""
     g = torch.Generator().manual_seed(N + E)
     x = torch.randn(N, d, generator=g).to(torch.bfloat16)
     W_g = (0.05 * torch.randn(E, d, generator=g)).to(torch.bfloat16)

@@ -596,3 +596,67 @@ def test_forward_random_configurations(seed):
     assert rel.max() <= 1e-5, (shape, rel.max())
     assert_close_layer(host(y), ref)
     assert launches == 8
+
+
+def _random_shape_wide(seed):
+    r = np.random.default_rng(5000 + seed)
+    fp32 = r.random() < 0.2
+    E = int(r.integers(1, 300))
+    k = int(r.integers(1, min(E, 16) + 1))
+    act = W.SWIGLU if r.random() < 0.7 else W.RELU
+    sf = int(r.random() < 0.5)
+    nb = int(r.integers(0, 3)) if sf == 1 else 0
+    cf = [None, Fraction(1), Fraction(5, 4), Fraction(1, 2), Fraction(3, 1)][int(r.integers(0, 5))]
+    step = 4 if fp32 else 8
+    return W.LayerShape(f"wide-{seed}", N=int(r.integers(1, 2000)),
+                        d=step * int(r.integers(2, 512 // step + 1)), E=E, k=k,
+                        F=step * int(r.integers(2, 512 // step + 1)),
+                        n_shared=int(r.random() < 0.5), score_fn=sf,
+                        renorm=int(r.random() < 0.7) if k == 1 else 1, act=act,
+                        clamp=float(r.choice([0.0, 0.0, 1.0, 10.0])), n_bias_sets=nb,
+                        capacity_factor=cf, zipf_skew=bool(r.random() < 0.3), w_std=0.05,
+                        dtype=W.F32 if fp32 else W.BF16, seed=seed)
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_forward_random_configurations_wide(seed):
+    """Wider random layers: up to 300 experts and k = 16, up to 2000 tokens (a sample of rows
+    checked), the fp32 path, and the "report" overflow policy on a third of the capacity
+    cases; routing bit-exact and the output within the bar against the oracle."""
+    shape = _random_shape_wide(seed)
+    reroute = shape.capacity_factor is not None and np.random.default_rng(seed).random() < 0.4
+    t = W.make_inputs(shape, device="cuda")
+    N, E, k = shape.N, shape.E, shape.k
+    C = O.capacity(N, k, E, shape.capacity_factor)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    ro = dict(logits=torch.empty((N, E), dtype=torch.float32, device="cuda"),
+              ids=torch.empty((N, k), dtype=torch.int32, device="cuda"),
+              gates=torch.empty((N, k), dtype=torch.float32, device="cuda"),
+              counts=torch.empty(E, dtype=torch.int32, device="cuda"),
+              demand=torch.empty(E, dtype=torch.int32, device="cuda"),
+              drop_mask=torch.empty((N, k), dtype=torch.uint8, device="cuda"),
+              offsets=torch.empty(E + 1, dtype=torch.int32, device="cuda"))
+    y = torch.empty_like(t["x"])
+    fwd = nat.moe_forward_reroute if reroute else nat.moe_forward
+    fwd(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y,
+        logit_offset=t.get("logit_offset"), bias=t.get("bias"), modality=t.get("modality"),
+        route_out=ro, ws=ws)
+    check_status(ws)
+    ro = {kk: host(v) for kk, v in ro.items()}
+    kw = _oracle_kwargs(shape, t, C)
+    kw.pop("logit_offset")
+    rows = np.arange(N) if N <= 400 else np.unique(np.r_[0:32, N - 32:N,
+                                                          np.random.default_rng(seed).integers(0, N, 64)])
+    ref, info = O.forward(f64(t["x"]), None, _LazyF64(t["W_gu"]), _LazyF64(t["W_down"]),
+                          logits=ro["logits"], tokens=rows,
+                          overflow="reroute" if reroute else "drop", **kw)
+    for name in ("ids", "drop_mask", "counts", "demand", "offsets"):
+        np.testing.assert_array_equal(ro[name], info[name], err_msg=f"{shape} {name}")
+    rel = np.abs(ro["gates"] - info["gates"]) / np.maximum(np.abs(info["gates"]), 1e-30)
+    assert rel.max() <= 1e-5, (shape, rel.max())
+    got = host(y)[rows].astype(np.float64)
+    if shape.dtype == W.F32:
+        assert np.abs(got - ref).max() <= 1e-4 * max(1.0, np.abs(ref).max()), shape
+    else:
+        assert_close_layer(got, ref)

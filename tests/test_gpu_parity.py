@@ -660,3 +660,43 @@ def test_forward_random_configurations_wide(seed):
         assert np.abs(got - ref).max() <= 1e-4 * max(1.0, np.abs(ref).max()), shape
     else:
         assert_close_layer(got, ref)
+
+
+@pytest.mark.parametrize("sf,nb,cf", [(0, 0, None), (1, 2, Fraction(1, 2))])
+def test_forward_largest_expert_count_and_k(sf, nb, cf):
+    """E = 1024 routed experts with k = 32 (the largest the ABI takes), plus a shared expert."""
+    shape = W.LayerShape("max", N=200, d=64, E=1024, k=32, F=64, n_shared=1, score_fn=sf,
+                         n_bias_sets=nb, capacity_factor=cf, w_std=0.05, seed=77)
+    t = W.make_inputs(shape, device="cuda")
+    C = O.capacity(shape.N, shape.k, shape.E, cf)
+    y, ro, launches = _run_forward(shape, t, C)
+    kw = _oracle_kwargs(shape, t, C)
+    kw.pop("logit_offset")
+    ref, info = O.forward(f64(t["x"]), None, _LazyF64(t["W_gu"]), _LazyF64(t["W_down"]),
+                          logits=ro["logits"], **kw)
+    for name in ("ids", "drop_mask", "counts", "demand", "offsets"):
+        np.testing.assert_array_equal(ro[name], info[name], err_msg=name)
+    assert_close_layer(host(y), ref)
+    assert launches == 8
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_route_random_configurations_bit_exact(seed):
+    """Random routing problems on given fp32 logits (up to 1024 experts, k up to 32, capacity
+    or none, ties from quantised logits): ids, counts, demand and drop mask bit-exact, gates
+    within 1e-5."""
+    r = np.random.default_rng(9000 + seed)
+    N = int(r.integers(1, 5000))
+    E = int(r.integers(1, 1025))
+    k = int(r.integers(1, min(E, 32) + 1))
+    sf = int(r.random() < 0.5)
+    rn = int(r.random() < 0.8) if k == 1 else 1
+    nb = int(r.integers(0, 3))
+    C = 0 if r.random() < 0.3 else int(r.integers(1, max(2, N * k // E + 2)))
+    q = float(r.choice([0.0, 0.0, 0.25]))
+    z = W.random_logits(N, E, seed + 31, scale=float(r.uniform(0.5, 3.0)), quantum=q)
+    bias = W.random_bias(nb, E, seed + 32) if nb else None
+    mod = W.random_modality(N, seed + 33) if nb > 1 else None
+    cfg = nat.make_config(N, 64, E, k, 64, n_bias_sets=nb, score_fn=sf, renorm=rn, capacity=C)
+    got = gpu_route(cfg, z, bias, mod)
+    assert_route_equal(got, z, k, sf, rn, bias, mod, E, C)

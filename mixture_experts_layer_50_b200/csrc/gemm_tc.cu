@@ -254,6 +254,7 @@ struct Args {
   int* status;
   int k_splits;       // > 1: split K; split s writes rows [s * split_rows, ...) of out
   int64_t split_rows;
+  int m64_tails;      // 1-SM kernel: a tile with at most 64 valid rows issues M = 64 MMAs
 };
 
 template <int BN, int STAGES>
@@ -529,6 +530,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================= MMA issuer =================
     if (lane == 0) {
       constexpr uint32_t kIdesc = idesc_bf16<BN>();
+      // M = 64: the same descriptor with the M field halved
+      constexpr uint32_t kIdesc64 = (kIdesc & ~(0x1Fu << 24)) | ((uint32_t)(64 >> 4) << 24);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -536,6 +539,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
+        int g, m_blk, n_blk;
+        decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk);
+        const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
+        const uint32_t idesc = (p.m64_tails && cnt - m_blk * BM <= 64) ? kIdesc64 : kIdesc;
         if (!mbar_wait(&tempty[acc], aph ^ 1, s_abort, p.status)) {
           ok = false;
           break;
@@ -553,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b0 = smem_u32(sB + stage * L::kStageB);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            mma_bf16(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), kIdesc,
+            mma_bf16(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc,
                      (kb > kb0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&empty[stage]);
@@ -592,8 +599,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                (int64_t)(tile % ks_n) * p.split_rows;
       const int rows_valid = min(BM, cnt - m_blk * BM);
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      // an M = 64 accumulator holds rows 16q .. 16q + 15 in lanes 32q .. 32q + 15
+      const bool m64 = p.m64_tails && rows_valid <= 64;
+      const int row_base = m64 ? q * 16 : q * 32;
+      const int rows_w = m64 ? min(rows_valid, q * 16 + 16) : rows_valid;
 
-      epilogue_warp<BN, EPI>(p, t_row, stg, lane, n_blk, out_row0, q * 32, rows_valid, [&] {
+      epilogue_warp<BN, EPI>(p, t_row, stg, lane, n_blk, out_row0, row_base, rows_w, [&] {
         // all TMEM reads of this accumulator are done: hand it back to the MMA warp
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
@@ -1278,6 +1289,8 @@ Args make_args(const GroupedGemm& g) {
   a.status = g.status;
   a.k_splits = g.k_splits > 1 ? g.k_splits : 1;
   a.split_rows = g.split_rows;
+  const char* m64 = std::getenv("MOE_B200_M64_TAILS");
+  a.m64_tails = (m64 != nullptr && std::strcmp(m64, "0") == 0) ? 0 : 1;
   return a;
 }
 

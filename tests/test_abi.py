@@ -149,3 +149,30 @@ def test_wait_selftest_validates_on_host(nat):
     fake = ctypes.c_void_p(256)
     assert lib.moe_selftest_wait_timeout(fake, -1, None) == nat.MOE_ERR_INVALID_ARG
     assert lib.moe_selftest_wait_timeout(fake, 2_000_000_000, None) == nat.MOE_ERR_INVALID_ARG
+
+
+def _build_c_client(out_dir):
+    """Compile and link tests/c_abi_forward.c (plain C99) against the library."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    here = os.path.dirname(os.path.abspath(__file__))
+    root = os.path.dirname(here)
+    pkg = os.path.join(root, "mixture_experts_layer_50_b200")
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    exe = os.path.join(str(out_dir), "c_abi_forward")
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-O2",
+           os.path.join(here, "c_abi_forward.c"), "-I", os.path.join(root, "include"),
+           "-I", os.path.join(cuda, "include"), "-L", pkg, "-lmoe_b200",
+           "-L", os.path.join(cuda, "lib64"), "-lcudart", f"-Wl,-rpath,{pkg}",
+           f"-Wl,-rpath,{os.path.join(cuda, 'lib64')}", "-o", exe]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    return exe
+
+
+def test_header_is_plain_c_and_a_c_client_links(tmp_path):
+    """include/moe.h compiles as C99 and a C program links against libmoe_b200.so alone."""
+    exe = _build_c_client(tmp_path)
+    assert os.path.exists(exe)

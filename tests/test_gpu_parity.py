@@ -700,3 +700,14 @@ def test_route_random_configurations_bit_exact(seed):
     cfg = nat.make_config(N, 64, E, k, 64, n_bias_sets=nb, score_fn=sf, renorm=rn, capacity=C)
     got = gpu_route(cfg, z, bias, mod)
     assert_route_equal(got, z, k, sf, rn, bias, mod, E, C)
+
+
+def test_c_client_fused_forward_equals_split_calls(tmp_path):
+    """A plain C program runs moe_forward and route -> permute -> expert_ffn -> combine on
+    the same layer and finds the same routing and the same output bits."""
+    import subprocess
+    from test_abi import _build_c_client
+    exe = _build_c_client(tmp_path)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "moe_forward == route/permute/expert_ffn/combine" in r.stdout

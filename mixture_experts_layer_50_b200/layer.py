@@ -100,7 +100,9 @@ class MoELayer:
             self.forward(x, modality=modality, y=y)          # eager run: one-time set-up
             torch.cuda.synchronize()
             g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
+            # thread-local capture: CUDA calls of other threads (a process group's
+            # watchdog, pinned-memory workers) do not invalidate the capture
+            with torch.cuda.graph(g, capture_error_mode="thread_local"):
                 self.forward(x, modality=modality, y=y)
             self._graphs[key] = g
         g.replay()

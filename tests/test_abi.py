@@ -13,6 +13,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def nat():
+    from conftest import ensure_library
+    ensure_library()
     from mixture_experts_layer_50_b200 import _native
     return _native
 
@@ -158,6 +160,8 @@ def _build_c_client(out_dir):
     gcc = shutil.which("gcc")
     if gcc is None:
         pytest.skip("gcc not available")
+    from conftest import ensure_library
+    ensure_library()
     here = os.path.dirname(os.path.abspath(__file__))
     root = os.path.dirname(here)
     pkg = os.path.join(root, "mixture_experts_layer_50_b200")

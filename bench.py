@@ -232,6 +232,16 @@ def make_replica(shape, rank, device="cuda"):
 
 
 def run_ours(args):
+    from mixture_experts_layer_50_b200 import build as _build
+    if int(os.environ.get("LOCAL_RANK", "0")) == 0:
+        _build.ensure_built()
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        # the other ranks wait for the library local rank 0 builds
+        lib = _build.LIB
+        for _ in range(6000):
+            if os.path.exists(lib):
+                break
+            time.sleep(0.1)
     from mixture_experts_layer_50_b200 import _native as nat
     from mixture_experts_layer_50_b200.layer import MoELayer
 

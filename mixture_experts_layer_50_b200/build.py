@@ -57,11 +57,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", LIB, *objs]
+        # link to a temporary name and rename: a process that sees the library sees all of it
+        tmp = f"{LIB}.{os.getpid()}.tmp"
+        cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
+        os.replace(tmp, LIB)
     return LIB
+
+
+def ensure_built() -> str:
+    """Build the library if it is not there yet (a fresh checkout carries no .so)."""
+    return LIB if os.path.exists(LIB) else build()
 
 
 if __name__ == "__main__":

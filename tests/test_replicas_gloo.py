@@ -74,3 +74,31 @@ def test_traffic_is_read_only_for_the_measured_kernel_source(tmp_path, monkeypat
     assert bench.read_traffic("gemm_gate_up", "mixtral-n16384") == 3.1e9
     assert bench.read_traffic("gemm_gate_up", "mixtral-n4096") is None    # stale counters
     assert bench.read_traffic("gemm_gate_up", "dsv3-n8192") is None       # no capture
+
+
+def test_algorithmic_work_of_the_roofline():
+    """F_alg and B_alg behind roofline and layer_roofline, against the closed forms:
+    F = 2 (M + S N) 3 d F + 2 N d E and B = touched experts' weights + router + x and y."""
+    import numpy as np
+    import bench
+    from mixture_experts_layer_50_b200 import workloads as W
+    s = W.PRESETS["mixtral-n16384"]
+    w = bench.algorithmic_work(s, np.full(8, 4096))
+    assert w["M"] == 32768 and w["touched"] == 8
+    assert w["flops_layer"] == 2 * 32768 * 3 * 4096 * 14336 + 2 * 16384 * 4096 * 8
+    assert w["flops_gate_up"] == 2 * 32768 * 4096 * 2 * 14336
+    assert w["bytes_layer"] == 2 * (8 * 3 * 4096 * 14336 + 8 * 4096 + 2 * 16384 * 4096)
+    # the gate/up launch: W_gate|W_up of the touched experts, x rows in, h rows out
+    assert w["bytes_gate_up"] == 2 * (8 * 2 * 14336 * 4096 + 32768 * 4096 + 32768 * 14336)
+    # decode: 16 tokens touch 7 experts; the shared expert of a V3-shaped layer counts in
+    w = bench.algorithmic_work(s.replace(N=16), np.array([5, 4, 6, 3, 5, 4, 5, 0]))
+    assert w["touched"] == 7
+    assert w["bytes_layer"] == 2 * (7 * 3 * 4096 * 14336 + 8 * 4096 + 2 * 16 * 4096)
+    v3 = W.PRESETS["dsv3-n64"]
+    counts = np.zeros(256, np.int64)
+    counts[:200] = 2
+    counts[200:256:4] = 1
+    w = bench.algorithmic_work(v3, counts)
+    rows = int(counts.sum()) + 64
+    assert w["flops_gate_up"] == 2 * rows * 7168 * 2 * 2048
+    assert w["bytes_layer"] == 2 * ((w["touched"] + 1) * 3 * 7168 * 2048 + 256 * 7168 + 2 * 64 * 7168)

@@ -352,6 +352,7 @@ def run_ours(args):
     per_launch = {n: launch_ms[i] / max(calls, 1) for i, n in enumerate(names)
                   if i < len(launch_ms)}
     gu_ms = per_launch.get("gemm_gate_up")
+    gu_kernel, down_kernel = nat.moe_ffn_kernels(layer.config(shape.N))
     # a short run has few clock samples: a gate/up launch faster than the sustained peak
     # allows ran at burst clocks, whatever the samples say
     if gu_ms and work["flops_gate_up"] / (gu_ms / 1e3) / 1e12 > peaks["bf16_tflops_sustained"]:
@@ -373,8 +374,7 @@ def run_ours(args):
         roof["frac"] = round(ach / peak, 4)
         roof["traffic"] = read_traffic("gemm_gate_up", args.workload)
         act = "SwiGLU" if shape.act == W.SWIGLU else "ReLU"
-        roof["kernel"] = (f"gemm_gate_up (grouped_gemm_kernel, {act} epilogue)"
-                          if shape.dtype == W.BF16 else f"gemm_gate_up (ffn_up_f32_kernel, {act})")
+        roof["kernel"] = f"gemm_gate_up: {gu_kernel}, {act} epilogue"
         roof["ms_per_launch"] = round(gu_ms, 4)
         roof["peak_source"] = f"{peak_src} ({tensor_key if roof['bound'] == 'tensor' else 'hbm_gbs'})"
     # whole-layer roofline: time bound = max(F / P, B / BW)
@@ -406,6 +406,7 @@ def run_ours(args):
                    "parallelism": f"replicas x{world} (no data-path collective)"},
         "roofline": roof, "layer_roofline": layer_roof,
         "launch_ms": {k: round(v, 4) for k, v in per_launch.items()},
+        "ffn_kernels": {"gate_up": gu_kernel, "down": down_kernel},
         "e2e": {"value": round(shape.N * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": shape.N * shape.d * el,
                 "d2h_bytes_per_step": shape.N * shape.d * el,

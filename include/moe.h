@@ -156,6 +156,16 @@ MOE_API moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const i
                           const void* x, const void* W_gu, const void* W_down, void* ye,
                           void* ws, moe_stream_t stream);
 
+/* Names of the kernels moe_expert_ffn (and every forward call) launches for the gate/up and
+ * the down projections of cfg.  The choice is made on the host from the configuration alone
+ * (N, k, E, d, F, act, dtype, n_shared, and the device's SM count and L2 size), so this call
+ * answers without device memory: a bf16 layer takes the 1-SM grouped GEMM (128x256 or 128x128
+ * tiles) or the 2-SM grouped GEMM (256x256 tiles on two SMs) per projection; an fp32 layer
+ * the SIMT kernels.  Each non-NULL buffer receives at most len bytes, NUL included (the
+ * name is truncated to fit).  MOE_ERR_INVALID_ARG for a bad cfg or len == 0 with a buffer;
+ * MOE_ERR_UNSUPPORTED for a configuration the forward calls reject. */
+MOE_API moe_status moe_ffn_kernels(const moe_config* cfg, char* gate_up, char* down, size_t len);
+
 /* Gate-weighted combine back to token order ("Основы MoE", step 4):
  *   y[t] = sum_{j: slot_row[t][j] >= 0} gates[t][j] ye[slot_row[t][j]]  (+ ye[N*k + t])
  * summed in fp32 and rounded once.  y [N][d] output. */

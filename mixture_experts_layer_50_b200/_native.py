@@ -77,6 +77,7 @@ lib.moe_forward_host_batches.argtypes = [_cfgp, _i32] + [_vp] * 10
 lib.moe_route_reroute.argtypes = [_cfgp] + [_vp] * 15
 lib.moe_selftest_wait_timeout.argtypes = [_vp, _i64, _vp]
 lib.moe_forward_reroute.argtypes = [_cfgp] + [_vp] * 12
+lib.moe_ffn_kernels.argtypes = [_cfgp, ctypes.c_char_p, ctypes.c_char_p, ctypes.c_size_t]
 lib.moe_profile_begin.argtypes = [_i32]
 lib.moe_profile_begin.restype = ctypes.c_int
 lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)]
@@ -87,7 +88,7 @@ for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "
            "moe_forward", "moe_forward_host", "moe_check_status", "moe_route_static",
            "moe_forward_routed", "moe_route_hash", "moe_balance", "moe_permute_padded",
            "moe_forward_padded", "moe_forward_host_batches", "moe_route_reroute",
-           "moe_forward_reroute", "moe_selftest_wait_timeout"):
+           "moe_forward_reroute", "moe_selftest_wait_timeout", "moe_ffn_kernels"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
@@ -96,7 +97,7 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_rou
             "moe_last_launch_count", "moe_route_static", "moe_forward_routed",
             "moe_route_hash", "moe_balance", "moe_permute_padded", "moe_forward_padded",
             "moe_forward_host_batches", "moe_route_reroute", "moe_forward_reroute",
-            "moe_selftest_wait_timeout")
+            "moe_selftest_wait_timeout", "moe_ffn_kernels")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -325,6 +326,14 @@ def moe_forward_host_batches(cfg, *, x_host: list, W_g, W_gu, W_down, y_host: li
                                       _ptr(bias), mods, _ptr(W_gu), _ptr(W_down), ys, _ptr(ws),
                                       _stream(stream))
     _check(st, "moe_forward_host_batches")
+
+
+def moe_ffn_kernels(cfg) -> tuple:
+    """Names of the kernels the gate/up and the down projections of cfg launch (host only)."""
+    gu = ctypes.create_string_buffer(128)
+    dn = ctypes.create_string_buffer(128)
+    _check(lib.moe_ffn_kernels(ctypes.byref(cfg), gu, dn, 128), "moe_ffn_kernels")
+    return gu.value.decode(), dn.value.decode()
 
 
 def moe_selftest_wait_timeout(ws, limit_ns: int, stream=None):

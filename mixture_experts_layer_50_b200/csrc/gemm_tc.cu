@@ -1256,6 +1256,19 @@ int num_sms() {
   return cached[dev];
 }
 
+int64_t l2_bytes() {
+  static int64_t cached[kMaxDev] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= kMaxDev) dev = 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrL2CacheSize, dev);
+    cached[dev] = n > 0 ? n : (126LL << 20);
+  }
+  return cached[dev];
+}
+
 // Opt a kernel into the largest dynamic shared memory once per device (the per-launch size is
 // always below it), so launches do not repeat the attribute call.  `done` must be distinct
 // for every kernel: each launch_* instantiation passes its own.
@@ -1359,17 +1372,39 @@ bool use_swap(const GroupedGemm& g) {
   return g.n_routed > 0 && avg_group_rows(g) < kSwapMaxRows;
 }
 
+// Rows of a group as the 1-SM kernel computes them: 128-row tiles, the last one an M = 64
+// tile when it holds at most 64 rows.
+int64_t one_sm_rows(int64_t r) {
+  const int64_t full = r / BM * BM, rem = r - full;
+  return full + (rem == 0 ? 0 : rem <= 64 ? 64 : BM);
+}
+
+// The 2-SM kernel (256-row tiles, each SM staging half of B) halves the operand bytes that
+// cross from L2 to the SMs per MMA, which is what keeps the 1-SM kernel's tensor pipe from
+// running full (its 128x256 tile needs about 96 B per clock per SM), but it computes more
+// padding rows: a routed group of r rows takes ceil(r / 256) tiles of 256 rows there, against
+// 128-row tiles with an M = 64 last tile on the 1-SM kernel, 96 more rows on average when r
+// is spread evenly modulo 256.  It is taken when that padding is at most a quarter of the
+// rows, estimated from the caller's rows per group.  Measured on one B200: the capacity and
+// Switch layers (padding estimate 1/8 and 3/16) gain 2-6 % per step, the Mixtral-shaped down
+// projection (1/64 to 3/32) gains, and the V3/V4.1-shaped prefill (1/3) loses.  For gate/up
+// the weight panel of one expert must also fit in a quarter of L2: with the Mixtral-shaped
+// 235 MB panels the 2-SM kernel missed L2 more (2.99 vs 1.95 GB from DRAM at 4096 tokens)
+// and was 0-9 % slower, while the 1-SM kernel reads each weight byte once.
 bool use_two_sm(const GroupedGemm& g) {
   if (g.epilogue == kEpiStoreF32 || g.k_splits > 1) return false;
   if (const char* env = path_override()) {
     if (std::strncmp(env, "1sm", 3) == 0) return false;
     if (std::strcmp(env, "2sm") == 0) return true;
   }
-  if (g.epilogue != kEpiStoreBf16) return false;
-  const int groups = g.n_routed + g.has_shared;
-  const int64_t rows = (g.n_routed > 0 ? avg_group_rows(g) * g.n_routed : 0) +
-                       (g.has_shared ? g.shared_rows : 0);
-  return rows >= 1024LL * groups;
+  const int64_t routed = g.n_routed > 0 ? avg_group_rows(g) * g.n_routed : 0;
+  const int64_t shared = g.has_shared ? g.shared_rows : 0;
+  if (routed + shared <= 0) return false;
+  int64_t extra = 96LL * g.n_routed;
+  if (shared > 0) extra += (shared + 255) / 256 * 256 - one_sm_rows(shared);
+  if (4 * extra > routed + shared) return false;
+  if (g.epilogue == kEpiStoreBf16) return true;
+  return (int64_t)g.rows_b * g.K * 2 <= l2_bytes() / 4;
 }
 
 // N width of the 1-SM kernel's tiles.  256 keeps the tensor pipe busiest; when nearly every
@@ -1417,6 +1452,26 @@ int router_tile_n(int n_out) {
     }
   }
   return best;
+}
+
+// The kernel launch_grouped_gemm takes for g, by the same host-side decisions in the same
+// order (device attributes only; no device memory is touched).
+const char* grouped_gemm_kernel_name(const GroupedGemm& g) {
+  using namespace tc;
+  if (g.n_routed + g.has_shared == 0) return "none";
+  if (use_swap(g)) return "grouped_gemm_swap_kernel (token-in-N)";
+  if (g.epilogue == kEpiStoreF32) {
+    switch (router_tile_n(g.n_out)) {
+      case 32: return "grouped_gemm_kernel (1-SM, 128x32 fp32 tiles)";
+      case 64: return "grouped_gemm_kernel (1-SM, 128x64 fp32 tiles)";
+      case 128: return "grouped_gemm_kernel (1-SM, 128x128 fp32 tiles)";
+      case 192: return "grouped_gemm_kernel (1-SM, 128x192 fp32 tiles)";
+      default: return "grouped_gemm_kernel (1-SM, 128x256 fp32 tiles)";
+    }
+  }
+  if (use_two_sm(g)) return "grouped_gemm_2sm_kernel (2-SM, 256x256 tiles)";
+  return pick_bn_1sm(g) == 128 ? "grouped_gemm_kernel (1-SM, 128x128 tiles)"
+                               : "grouped_gemm_kernel (1-SM, 128x256 tiles)";
 }
 
 cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* launches,

@@ -132,6 +132,8 @@ struct GroupedGemm {
 
 cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* launches,
                                 const char** why);
+// Name of the kernel launch_grouped_gemm launches for g (host only).
+const char* grouped_gemm_kernel_name(const GroupedGemm& g);
 // N width of the tiles of an fp32-store GEMM with n_out columns (the router).
 int router_tile_n(int n_out);
 // Failure-detection self-test: a bounded wait on a barrier nothing completes (gemm_tc.cu).

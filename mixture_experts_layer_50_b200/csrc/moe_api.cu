@@ -10,6 +10,7 @@
 #include <mutex>
 #include <string>
 #include <type_traits>
+#include <utility>
 #include <vector>
 
 #include "../../include/moe.h"
@@ -375,6 +376,67 @@ moe_status stage_route_reroute(const moe_config& c, const Ws& L, void* ws, const
   return MOE_OK;
 }
 
+// The two grouped GEMMs of the expert FFN (bf16).  Nk: rows of the routed region; the shared
+// expert's N rows follow it.  The kernel choice depends on the configuration alone (not on
+// the pointers), so moe_ffn_kernels can name it without any device memory, and the compact
+// and the padded layouts of the same call take the same kernels.
+moe::GroupedGemm gate_up_gemm(const moe_config& c, int64_t Nk, const void* xp, const void* x,
+                              const void* W_gu, const int32_t* offsets, void* h, int* status) {
+  moe::GroupedGemm g{};
+  g.a = xp;
+  g.rows_a = Nk;
+  g.a_shared = c.n_shared ? x : xp;
+  g.rows_a_shared = c.n_shared ? c.N : Nk;
+  g.shared_a_row0 = 0;
+  g.b = W_gu;
+  g.groups_b = c.E + c.n_shared;
+  g.rows_b = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
+  g.K = c.d;
+  g.offsets = offsets;
+  g.n_routed = c.E;
+  g.has_shared = c.n_shared;
+  g.shared_rows = c.N;
+  g.shared_out_row0 = Nk;
+  g.n_out = c.F;
+  g.epilogue = c.act == MOE_ACT_SWIGLU ? moe::kEpiSwiglu : moe::kEpiRelu;
+  g.clamp = c.clamp;
+  g.out = h;
+  g.ld_out = c.F;
+  g.rows_out = Nk + c.n_shared * c.N;
+  g.max_rows_routed = Nk;
+  g.rows_per_group_hint = c.N * (int64_t)c.k / c.E;
+  g.status = status;
+  return g;
+}
+
+moe::GroupedGemm down_gemm(const moe_config& c, int64_t Nk, const void* h, const void* W_down,
+                           const int32_t* offsets, void* ye, int* status) {
+  moe::GroupedGemm g{};
+  g.a = h;
+  g.rows_a = Nk + c.n_shared * c.N;
+  g.a_shared = h;
+  g.rows_a_shared = g.rows_a;
+  g.shared_a_row0 = Nk;
+  g.b = W_down;
+  g.groups_b = c.E + c.n_shared;
+  g.rows_b = c.d;
+  g.K = c.F;
+  g.offsets = offsets;
+  g.n_routed = c.E;
+  g.has_shared = c.n_shared;
+  g.shared_rows = c.N;
+  g.shared_out_row0 = Nk;
+  g.n_out = c.d;
+  g.epilogue = moe::kEpiStoreBf16;
+  g.out = ye;
+  g.ld_out = c.d;
+  g.rows_out = g.rows_a;
+  g.max_rows_routed = Nk;
+  g.rows_per_group_hint = c.N * (int64_t)c.k / c.E;
+  g.status = status;
+  return g;
+}
+
 // R: rows of the routed region of xp / h / ye (N k for the compact layout, E C for the
 // padded one); the shared expert's rows follow it.
 moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
@@ -394,59 +456,12 @@ moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
   }
   int* status = at<int>(ws, L.status);
   void* h = at<char>(ws, L.h);
-  moe::GroupedGemm g1{};
-  g1.a = xp;
-  g1.rows_a = Nk;
-  g1.a_shared = c.n_shared ? x : xp;
-  g1.rows_a_shared = c.n_shared ? c.N : Nk;
-  g1.shared_a_row0 = 0;
-  g1.b = W_gu;
-  g1.groups_b = c.E + c.n_shared;
-  g1.rows_b = c.act == MOE_ACT_SWIGLU ? 2 * c.F : c.F;
-  g1.K = c.d;
-  g1.offsets = offsets;
-  g1.n_routed = c.E;
-  g1.has_shared = c.n_shared;
-  g1.shared_rows = c.N;
-  g1.shared_out_row0 = Nk;
-  g1.n_out = c.F;
-  g1.epilogue = c.act == MOE_ACT_SWIGLU ? moe::kEpiSwiglu : moe::kEpiRelu;
-  g1.clamp = c.clamp;
-  g1.out = h;
-  g1.ld_out = c.F;
-  g1.rows_out = Nk + c.n_shared * c.N;
-  g1.max_rows_routed = Nk;
-  // kernel choice from the configuration alone, so the compact and the padded layouts of
-  // the same call take the same kernels
-  g1.rows_per_group_hint = c.N * (int64_t)c.k / c.E;
-  g1.status = status;
+  const moe::GroupedGemm g1 = gate_up_gemm(c, Nk, xp, x, W_gu, offsets, h, status);
   const char* why = "gate/up GEMM launch";
   MOE_CUDA(moe::launch_grouped_gemm(g1, st, launches, &why), why);
   prof_mark(st);
 
-  moe::GroupedGemm g2{};
-  g2.a = h;
-  g2.rows_a = Nk + c.n_shared * c.N;
-  g2.a_shared = h;
-  g2.rows_a_shared = g2.rows_a;
-  g2.shared_a_row0 = Nk;
-  g2.b = W_down;
-  g2.groups_b = c.E + c.n_shared;
-  g2.rows_b = c.d;
-  g2.K = c.F;
-  g2.offsets = offsets;
-  g2.n_routed = c.E;
-  g2.has_shared = c.n_shared;
-  g2.shared_rows = c.N;
-  g2.shared_out_row0 = Nk;
-  g2.n_out = c.d;
-  g2.epilogue = moe::kEpiStoreBf16;
-  g2.out = ye;
-  g2.ld_out = c.d;
-  g2.rows_out = g2.rows_a;
-  g2.max_rows_routed = Nk;
-  g2.rows_per_group_hint = g1.rows_per_group_hint;
-  g2.status = status;
+  const moe::GroupedGemm g2 = down_gemm(c, Nk, h, W_down, offsets, ye, status);
   why = "down GEMM launch";
   MOE_CUDA(moe::launch_grouped_gemm(g2, st, launches, &why), why);
   prof_mark(st);
@@ -655,6 +670,30 @@ moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const int32_t* 
   MOE_TRY(stage_ffn(*cfg, layout(*cfg), ws, xp, offsets, x, W_gu, W_down, ye,
                     (cudaStream_t)stream, &launches));
   g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_ffn_kernels(const moe_config* cfg, char* gate_up, char* down, size_t len) {
+  MOE_TRY(check_cfg(cfg));
+  if (len == 0 && (gate_up != nullptr || down != nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "len is 0");
+  const moe_config& c = *cfg;
+  const char* gu = "ffn_up_f32_kernel (SIMT fp32)";
+  const char* dn = "ffn_down_f32_kernel (SIMT fp32)";
+  if (c.dtype == MOE_DT_BF16) {
+    const int64_t Nk = c.N * (int64_t)c.k;
+    gu = moe::grouped_gemm_kernel_name(
+        gate_up_gemm(c, Nk, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr));
+    dn = moe::grouped_gemm_kernel_name(
+        down_gemm(c, Nk, nullptr, nullptr, nullptr, nullptr, nullptr));
+  }
+  if (c.N == 0) gu = dn = "none";
+  for (auto [buf, name] : {std::pair<char*, const char*>{gate_up, gu}, {down, dn}}) {
+    if (buf == nullptr) continue;
+    const size_t n = std::min(len - 1, std::strlen(name));
+    std::memcpy(buf, name, n);
+    buf[n] = '\0';
+  }
   return MOE_OK;
 }
 

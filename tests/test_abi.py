@@ -180,3 +180,34 @@ def test_header_is_plain_c_and_a_c_client_links(tmp_path):
     """include/moe.h compiles as C99 and a C program links against libmoe_b200.so alone."""
     exe = _build_c_client(tmp_path)
     assert os.path.exists(exe)
+
+
+def test_ffn_kernel_choice(nat):
+    """Which grouped GEMM each preset layer takes, decided on the host from the configuration
+    (with no GPU the device attributes fall back to 148 SMs and 126 MB of L2, the B200's)."""
+    from mixture_experts_layer_50_b200 import workloads as W
+    one_256, one_128 = "1-SM, 128x256 tiles", "1-SM, 128x128 tiles"
+    two = "2-SM, 256x256 tiles"
+    want = {
+        "mixtral-n16": (one_128, one_256), "mixtral-n256": (one_128, one_256),
+        # gate/up: 235 MB weight panels per expert stay on the 1-SM kernel
+        "mixtral-n4096": (one_256, two), "mixtral-n16384": (one_256, two),
+        # ~256 rows per expert: 256-row tiles would pad a third more rows
+        "dsv3-n64": (one_256, one_256), "dsv3-n8192": (one_256, one_256),
+        "v41flash-n64": (one_256, one_256), "v41flash-n16384": (one_256, one_256),
+        # the shared expert's 16384 rows dominate; 11.5 MB panels
+        "capacity-cf1": (two, two), "capacity-cfinf": (two, two),
+        "switch-cf1": (two, two), "switch-cfinf": (two, two),
+    }
+    for name, (gu, dn) in want.items():
+        got = nat.moe_ffn_kernels(nat.config_from_shape(W.PRESETS[name]))
+        assert gu in got[0] and dn in got[1], (name, got)
+    toy = nat.moe_ffn_kernels(nat.config_from_shape(W.PRESETS["toy"]))
+    assert "f32" in toy[0] and "f32" in toy[1]
+    assert nat.moe_ffn_kernels(_cfg(nat, N=0)) == ("none", "none")
+    # truncation keeps the terminating NUL; bad arguments are refused on the host
+    buf = ctypes.create_string_buffer(8)
+    assert nat.lib.moe_ffn_kernels(ctypes.byref(_cfg(nat)), buf, None, 8) == 0
+    assert buf.value == b"grouped"
+    assert nat.lib.moe_ffn_kernels(ctypes.byref(_cfg(nat)), buf, None, 0) == nat.MOE_ERR_INVALID_ARG
+    assert nat.lib.moe_ffn_kernels(ctypes.byref(_cfg(nat, k=9)), buf, None, 8) == nat.MOE_ERR_INVALID_ARG

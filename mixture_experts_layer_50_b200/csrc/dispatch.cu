@@ -13,8 +13,8 @@
 //   2. one block per 32 experts scans the histograms over tiles (tile_base) and applies the
 //      capacity to the per-expert totals; the last block to finish scans the capped totals
 //      over the experts (offsets);
-//   3. one block per token: rank = tile_base + local rank, keep iff rank < C, row =
-//      offsets[e] + rank; the token's x row is copied to each kept row (the gather).
+//   3. one block (or one warp) per token: rank = tile_base + local rank, keep iff rank < C,
+//      row = offsets[e] + rank; the token's x row is copied to each kept row (the gather).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -143,6 +143,10 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
   if (threadIdx.x == 0) *arrive = 0;
 }
 
+// One block per token.  Thread j < k resolves slot j's row with two rounds of loads (local
+// rank and expert together, then the expert's tile base and offset together: a local rank
+// >= 0 implies a valid expert, set by the rank pass), then the block copies the token's row
+// to each kept slot, two vectors in flight per thread.
 template <typename V>
 __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
     const int32_t* __restrict__ ids, const int32_t* __restrict__ local_rank,
@@ -156,11 +160,14 @@ __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
   if (threadIdx.x < k) {
     const int j = threadIdx.x;
     const int lr = local_rank[t * k + j];
+    const int e_raw = ids[t * k + j];
+    const int e = lr >= 0 ? e_raw : 0;
+    const int64_t base = tile_base[(t / kRankTile) * E + e];
+    const int32_t off = offsets[e];
     int32_t row = -1;
     if (lr >= 0) {
-      const int e = ids[t * k + j];
-      const int64_t r = (int64_t)tile_base[(t / kRankTile) * E + e] + lr;
-      if (C <= 0 || r < C) row = offsets[e] + (int32_t)r;
+      const int64_t r = base + lr;
+      if (C <= 0 || r < C) row = off + (int32_t)r;
     }
     slot_row[t * k + j] = row;
     if (drop_mask_out != nullptr) drop_mask_out[t * k + j] = row < 0 ? 1 : 0;
@@ -174,11 +181,74 @@ __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
   for (int j = 0; j < k; ++j) any |= s_row[j] >= 0;
   if (!any) return;
   const V* src = x + t * row_vecs;
-  for (int v = threadIdx.x; v < row_vecs; v += blockDim.x) {
-    const V val = src[v];
+  const int step = blockDim.x;
+  for (int v = threadIdx.x; v < row_vecs; v += 2 * step) {
+    const bool two = v + step < row_vecs;
+    const V a = src[v];
+    V b{};
+    if (two) b = src[v + step];
     for (int j = 0; j < k; ++j) {
       const int32_t row = s_row[j];
-      if (row >= 0) xp[(int64_t)row * row_vecs + v] = val;
+      if (row < 0) continue;
+      V* dst = xp + (int64_t)row * row_vecs;
+      dst[v] = a;
+      if (two) dst[v + step] = b;
+    }
+  }
+}
+
+// The same work with one warp per token and kScatterWarps tokens per block: for many tokens
+// with small rows it launches 8x fewer blocks and keeps 64 tokens in flight per SM instead of
+// 16 (the capacity layer, 16384 tokens of 4 KB rows: 16.5 -> 10.6 us); with few tokens or
+// large rows the block-per-token kernel spreads the copies over more SMs and warps.
+constexpr int kScatterWarps = 8;
+constexpr int kScatterUnroll = 4;
+
+template <typename V>
+__global__ void __launch_bounds__(32 * kScatterWarps, 8) dispatch_scatter_warp_kernel(
+    const int32_t* __restrict__ ids, const int32_t* __restrict__ local_rank,
+    const int32_t* __restrict__ tile_base, const int32_t* __restrict__ offsets, int64_t N,
+    int k, int E, int64_t C, int32_t* __restrict__ slot_row, int32_t* __restrict__ row_token,
+    uint8_t* __restrict__ drop_mask_out, const V* __restrict__ x, V* __restrict__ xp,
+    int row_vecs) {
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * kScatterWarps + (threadIdx.x >> 5);
+  if (t >= N) return;  // warp-uniform
+  int32_t row = -1;
+  if (lane < k) {
+    const int lr = local_rank[t * k + lane];
+    const int e_raw = ids[t * k + lane];
+    const int e = lr >= 0 ? e_raw : 0;
+    const int64_t base = tile_base[(t / kRankTile) * E + e];
+    const int32_t off = offsets[e];
+    if (lr >= 0) {
+      const int64_t r = base + lr;
+      if (C <= 0 || r < C) row = off + (int32_t)r;
+    }
+    slot_row[t * k + lane] = row;
+    if (drop_mask_out != nullptr) drop_mask_out[t * k + lane] = row < 0 ? 1 : 0;
+    if (row >= 0 && row_token != nullptr) row_token[row] = (int32_t)t;
+  }
+  if (xp == nullptr) return;
+  if (__ballot_sync(0xffffffffu, row >= 0) == 0u) return;
+  const V* src = x + t * row_vecs;
+  for (int v0 = 0; v0 < row_vecs; v0 += 32 * kScatterUnroll) {
+    V val[kScatterUnroll];
+#pragma unroll
+    for (int u = 0; u < kScatterUnroll; ++u) {
+      const int v = v0 + u * 32 + lane;
+      if (v < row_vecs) val[u] = src[v];
+    }
+    for (int j = 0; j < k; ++j) {
+      const int32_t r = __shfl_sync(0xffffffffu, row, j);
+      if (r < 0) continue;
+      V* dst = xp + (int64_t)r * row_vecs;
+#pragma unroll
+      for (int u = 0; u < kScatterUnroll; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < row_vecs) dst[v] = val[u];
+      }
     }
   }
 }
@@ -252,18 +322,39 @@ cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_ran
                                     cudaStream_t stream, int* launches) {
   if (N == 0) return cudaSuccess;
   ++*launches;
+  // warp per token when the warps fill every SM several times over and a token moves at
+  // most 16 KB; else block per token
+  const bool per_warp = N >= (int64_t)tc::num_sms() * 64 && (int64_t)k * row_bytes <= 16384;
+  if (per_warp) {
+    const unsigned grid = (unsigned)((N + kScatterWarps - 1) / kScatterWarps);
+    const unsigned block = 32 * kScatterWarps;
+    if (xp != nullptr && row_bytes % 16 == 0) {
+      launch_pdl(dispatch_scatter_warp_kernel<uint4>, grid, block, 0, stream, ids, local_rank,
+                 tile_base, offsets, N, k, E, C, slot_row, row_token, drop_mask_out,
+                 (const uint4*)x, (uint4*)xp, row_bytes / 16);
+    } else if (xp != nullptr) {
+      launch_pdl(dispatch_scatter_warp_kernel<uint32_t>, grid, block, 0, stream, ids,
+                 local_rank, tile_base, offsets, N, k, E, C, slot_row, row_token,
+                 drop_mask_out, (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4);
+    } else {
+      launch_pdl(dispatch_scatter_warp_kernel<uint4>, grid, block, 0, stream, ids, local_rank,
+                 tile_base, offsets, N, k, E, C, slot_row, row_token, drop_mask_out, nullptr,
+                 nullptr, 0);
+    }
+    return cudaGetLastError();
+  }
   if (xp != nullptr && row_bytes % 16 == 0) {
-    launch_pdl(dispatch_scatter_kernel<uint4>, (unsigned)N, 128, 0, stream, 
-        ids, local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
-        (const uint4*)x, (uint4*)xp, row_bytes / 16);
+    launch_pdl(dispatch_scatter_kernel<uint4>, (unsigned)N, 128, 0, stream, ids, local_rank,
+               tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
+               (const uint4*)x, (uint4*)xp, row_bytes / 16);
   } else if (xp != nullptr) {
-    launch_pdl(dispatch_scatter_kernel<uint32_t>, (unsigned)N, 128, 0, stream, 
-        ids, local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
-        (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4);
+    launch_pdl(dispatch_scatter_kernel<uint32_t>, (unsigned)N, 128, 0, stream, ids,
+               local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
+               (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4);
   } else {
-    launch_pdl(dispatch_scatter_kernel<uint4>, (unsigned)N, 128, 0, stream, 
-        ids, local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
-        nullptr, nullptr, 0);
+    launch_pdl(dispatch_scatter_kernel<uint4>, (unsigned)N, 128, 0, stream, ids, local_rank,
+               tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out, nullptr,
+               nullptr, 0);
   }
   return cudaGetLastError();
 }

@@ -132,6 +132,11 @@ struct GroupedGemm {
 
 cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* launches,
                                 const char** why);
+namespace tc {
+// SM count of the current device, cached per device (gemm_tc.cu).
+int num_sms();
+}  // namespace tc
+
 // Name of the kernel launch_grouped_gemm launches for g (host only).
 const char* grouped_gemm_kernel_name(const GroupedGemm& g);
 // N width of the tiles of an fp32-store GEMM with n_out columns (the router).

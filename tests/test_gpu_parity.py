@@ -155,7 +155,12 @@ def test_route_reports_bad_modality_flag():
 # permutation (moe_permute): bit-exact
 # ---------------------------------------------------------------------------------------
 @pytest.mark.parametrize("N,E,k,C,dt", [(300, 8, 2, 0, torch.bfloat16), (1000, 64, 6, 70, torch.bfloat16),
-                                       (129, 5, 3, 0, torch.float32), (1, 4, 2, 0, torch.bfloat16)])
+                                       (129, 5, 3, 0, torch.float32), (1, 4, 2, 0, torch.bfloat16),
+                                       # >= 64 tokens per SM with small rows: the
+                                       # warp-per-token scatter
+                                       (9472, 16, 2, 0, torch.bfloat16),
+                                       (12345, 64, 4, 700, torch.bfloat16),
+                                       (10001, 8, 3, 0, torch.float32)])
 def test_permute_bit_exact(N, E, k, C, dt):
     d = 72 if dt == torch.bfloat16 else 68
     z = W.random_logits(N, E, N + E)

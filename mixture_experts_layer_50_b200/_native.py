@@ -330,9 +330,9 @@ def moe_forward_host_batches(cfg, *, x_host: list, W_g, W_gu, W_down, y_host: li
 
 def moe_ffn_kernels(cfg) -> tuple:
     """Names of the kernels the gate/up and the down projections of cfg launch (host only)."""
-    gu = ctypes.create_string_buffer(128)
-    dn = ctypes.create_string_buffer(128)
-    _check(lib.moe_ffn_kernels(ctypes.byref(cfg), gu, dn, 128), "moe_ffn_kernels")
+    gu = ctypes.create_string_buffer(256)
+    dn = ctypes.create_string_buffer(256)
+    _check(lib.moe_ffn_kernels(ctypes.byref(cfg), gu, dn, 256), "moe_ffn_kernels")
     return gu.value.decode(), dn.value.decode()
 
 

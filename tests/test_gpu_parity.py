@@ -251,13 +251,15 @@ def test_expert_ffn(N, d, E, k, F, S, act, clamp, path, monkeypatch):
     assert_close_layer(got[rows], ref[rows])
 
 
-@pytest.mark.parametrize("path", ["1sm", "swap"])
+@pytest.mark.parametrize("path", ["1sm", "swap", "2sm"])
 def test_expert_ffn_group_sizes_around_the_tile_edges(path, monkeypatch):
-    """Groups of 0, 1, 15, 16, 17, 31, 32, 33, 127, 128, 129, 255, 256, 257 rows: the token-in-N
-    kernel rounds a group's last row block up to 16 rows and loads it in 32-row boxes; the
-    1-SM kernel pads to 128-row tiles."""
+    """Groups of 0 ... 513 rows around every tile edge: the token-in-N kernel rounds a group's
+    last row block up to 16 rows and loads it in 32-row boxes; the 1-SM kernel pads to
+    128-row tiles (M = 64 for a last tile of at most 64 rows); the 2-SM kernel to 256-row
+    tiles."""
     monkeypatch.setenv("MOE_B200_GEMM_PATH", path)
-    sizes = [0, 1, 15, 16, 17, 31, 32, 33, 127, 128, 129, 255, 256, 257]
+    sizes = [0, 1, 15, 16, 17, 31, 32, 33, 127, 128, 129, 255, 256, 257, 300, 383, 384, 385,
+             511, 512, 513]
     E, k, d, F = len(sizes), 1, 256, 384
     N = sum(sizes)
     shape = W.LayerShape("t", N=N, d=d, E=E, k=k, F=F, n_shared=1, act=W.SWIGLU, clamp=0.0,

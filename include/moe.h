@@ -173,7 +173,9 @@ MOE_API moe_status moe_combine(const moe_config* cfg, const void* ye, const int3
                        const float* gates, void* y, moe_stream_t stream);
 
 /* The whole layer: route, capacity, permute, expert FFNs (routed + shared), combine.
- * Inputs as above; y [N][d] output; route_out may be NULL or have NULL members. */
+ * Inputs as above; y [N][d] output; route_out may be NULL or have NULL members.  With a
+ * shared expert (bf16) the down GEMM writes the shared expert's rows into y and the combine
+ * adds the kept slots to them in place (y is written by two kernels of the call). */
 MOE_API moe_status moe_forward(const moe_config* cfg, const void* x, const void* W_g,
                        const float* logit_offset, const float* bias,
                        const uint8_t* modality, const void* W_gu, const void* W_down,

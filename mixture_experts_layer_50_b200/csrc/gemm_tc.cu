@@ -250,6 +250,7 @@ struct Args {
   float clamp;
   const float* col_bias;
   void* out;
+  void* out_shared;   // non-null: the shared group's row r goes to row r here, not into out
   int64_t ld_out;
   int* status;
   int k_splits;       // > 1: split K; split s writes rows [s * split_rows, ...) of out
@@ -300,9 +301,10 @@ __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + _
 // accumulator: activation, packing, per-warp staging in shared memory, then coalesced 16-byte
 // stores with row and column masks.  `release` runs right after the last TMEM read.
 template <int BN, int EPI, typename Release>
-__device__ __forceinline__ void epilogue_warp(const Args& p, uint32_t t_row, uint8_t* stg,
-                                              int lane, int n_blk, int64_t out_row0,
-                                              int row_base, int rows_valid, Release&& release) {
+__device__ __forceinline__ void epilogue_warp(const Args& p, void* out, uint32_t t_row,
+                                              uint8_t* stg, int lane, int n_blk,
+                                              int64_t out_row0, int row_base, int rows_valid,
+                                              Release&& release) {
   constexpr int kOutPerTile = (EPI == kEpiSwiglu) ? BN / 2 : BN;
   constexpr int kColsPerChunk = (EPI == kEpiStoreF32) ? 32 : 64;
   constexpr int kChunks = kOutPerTile / kColsPerChunk;
@@ -380,8 +382,8 @@ __device__ __forceinline__ void epilogue_warp(const Args& p, uint32_t t_row, uin
         if constexpr (EPI == kEpiStoreF32) {
           // fp32 rows of n_out = E columns: a 16-byte store only where the row stride and the
           // base keep it 16-byte aligned (E a multiple of 4), else element by element
-          float* o = reinterpret_cast<float*>(p.out) + orow * p.ld_out + col;
-          const bool vec = (p.ld_out & 3) == 0 && (reinterpret_cast<uintptr_t>(p.out) & 15) == 0;
+          float* o = reinterpret_cast<float*>(out) + orow * p.ld_out + col;
+          const bool vec = (p.ld_out & 3) == 0 && (reinterpret_cast<uintptr_t>(out) & 15) == 0;
           if (vec && col + 4 <= p.n_out) {
             *reinterpret_cast<uint4*>(o) = val;
           } else {
@@ -390,7 +392,7 @@ __device__ __forceinline__ void epilogue_warp(const Args& p, uint32_t t_row, uin
             for (int e = 0; e < n; ++e) o[e] = f[e];
           }
         } else {
-          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + orow * p.ld_out + col;
+          __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out) + orow * p.ld_out + col;
           *reinterpret_cast<uint4*>(o) = val;  // n_out % 8 == 0 (checked on the host)
         }
       }
@@ -604,7 +606,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int row_base = m64 ? q * 16 : q * 32;
       const int rows_w = m64 ? min(rows_valid, q * 16 + 16) : rows_valid;
 
-      epilogue_warp<BN, EPI>(p, t_row, stg, lane, n_blk, out_row0, row_base, rows_w, [&] {
+      void* out = (sh && p.out_shared != nullptr) ? p.out_shared : p.out;
+      epilogue_warp<BN, EPI>(p, out, t_row, stg, lane, n_blk, out_row0, row_base, rows_w, [&] {
         // all TMEM reads of this accumulator are done: hand it back to the MMA warp
         tc_fence_before();
         mbar_arrive(&tempty[acc]);
@@ -834,7 +837,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int64_t out_row0 = (int64_t)(sh ? p.shared_out_row0 : p.offsets[g]) + m_blk * BMT;
       const int rows_valid = min(BMT, cnt - m_blk * BMT);
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      epilogue_warp<BN, EPI>(p, t_row, stg, lane, n_blk, out_row0, (int)rank * 128 + q * 32,
+      void* out = (sh && p.out_shared != nullptr) ? p.out_shared : p.out;
+      epilogue_warp<BN, EPI>(p, out, t_row, stg, lane, n_blk, out_row0, (int)rank * 128 + q * 32,
                              rows_valid, [&] {
                                tc_fence_before();
                                __syncwarp();
@@ -1104,7 +1108,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;  // TMEM lanes 32q..32q+31 = weight rows 32q + lane of the operand
     uint8_t* stg = staging + (warp - 2) * kSwapStagingPerWarp;
     __nv_bfloat16* stg_h = reinterpret_cast<__nv_bfloat16*>(stg);
-    __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(p.out);
     // SwiGLU: warp q = 0, 1 holds the gate rows of features f0 + 32q + lane, warp q + 2 their up
     // rows.  Per chunk of 32 group rows the gate warp computes rows 0..15 and the up warp rows
     // 16..31; each passes the other the half it needs through xchg.
@@ -1124,6 +1127,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rows = min(kSwapRows, group_rows(g) - r_blk * kSwapRows);
       const int64_t out_row0 =
           (int64_t)(sh ? p.shared_out_row0 : p.offsets[g]) + (int64_t)r_blk * kSwapRows;
+      __nv_bfloat16* outp = reinterpret_cast<__nv_bfloat16*>(
+          (sh && p.out_shared != nullptr) ? p.out_shared : p.out);
       const int chunks = (rows + 31) / 32;
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256);
       for (int c = 0; c < chunks; ++c) {
@@ -1298,6 +1303,7 @@ Args make_args(const GroupedGemm& g) {
   a.clamp = g.clamp;
   a.col_bias = g.col_bias;
   a.out = g.out;
+  a.out_shared = g.out_shared;
   a.ld_out = g.ld_out;
   a.status = g.status;
   a.k_splits = g.k_splits > 1 ? g.k_splits : 1;

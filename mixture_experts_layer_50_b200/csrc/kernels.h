@@ -77,9 +77,11 @@ cudaError_t launch_zero_padding(const int32_t* counts, int E, int64_t C, void* x
 
 // ---- combine (combine.cu) -------------------------------------------------------------
 // y[t] = sum_j gates[t,j] ye[slot_row[t,j]] (+ ye[shared_row0 + t] when shared_row0 >= 0).
+// shared_row0 >= 0: the shared row of token t is ye[shared_row0 + t]; shared_in_y (bf16):
+// y[t] holds it already (written by the down GEMM) and is updated in place.
 cudaError_t launch_combine(const void* ye, const int32_t* slot_row, const float* gates,
-                           int64_t N, int k, int d, int64_t shared_row0, int is_f32, void* y,
-                           cudaStream_t stream, int* launches);
+                           int64_t N, int k, int d, int64_t shared_row0, int shared_in_y,
+                           int is_f32, void* y, cudaStream_t stream, int* launches);
 
 // ---- fp32 path (simt_f32.cu) ----------------------------------------------------------
 cudaError_t launch_router_f32(const float* x, const float* W_g, const float* logit_offset,
@@ -120,6 +122,8 @@ struct GroupedGemm {
   float clamp;
   const float* col_bias;   // [n_out] fp32 added before the store (fp32 store only)
   void* out;
+  void* out_shared = nullptr;  // non-null: the shared group's row r is written to row r of
+                               // out_shared (same ld_out), not to row shared_out_row0 + r of out
   int64_t ld_out;          // elements
   int64_t rows_out;
   int64_t max_rows_routed; // upper bound of offsets[n_routed] (grid sizing)

@@ -438,11 +438,13 @@ moe::GroupedGemm down_gemm(const moe_config& c, int64_t Nk, const void* h, const
 }
 
 // R: rows of the routed region of xp / h / ye (N k for the compact layout, E C for the
-// padded one); the shared expert's rows follow it.
+// padded one); the shared expert's rows follow it in h, and in ye unless y_shared is given:
+// then (bf16) the down GEMM writes the shared expert's output row t straight into y_shared[t]
+// (the layer output, which stage_combine then completes in place).
 moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
                      const int32_t* offsets, const void* x, const void* W_gu,
                      const void* W_down, void* ye, cudaStream_t st, int* launches,
-                     int64_t R = -1) {
+                     int64_t R = -1, void* y_shared = nullptr) {
   if (c.N == 0) return MOE_OK;
   const int64_t Nk = R >= 0 ? R : c.N * (int64_t)c.k;
   if (c.dtype == MOE_DT_F32) {
@@ -461,18 +463,24 @@ moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
   MOE_CUDA(moe::launch_grouped_gemm(g1, st, launches, &why), why);
   prof_mark(st);
 
-  const moe::GroupedGemm g2 = down_gemm(c, Nk, h, W_down, offsets, ye, status);
+  moe::GroupedGemm g2 = down_gemm(c, Nk, h, W_down, offsets, ye, status);
+  if (y_shared != nullptr && c.n_shared) {
+    g2.out_shared = y_shared;
+    g2.shared_out_row0 = 0;
+  }
   why = "down GEMM launch";
   MOE_CUDA(moe::launch_grouped_gemm(g2, st, launches, &why), why);
   prof_mark(st);
   return MOE_OK;
 }
 
+// shared_in_y: stage_ffn wrote the shared expert's rows into y (bf16 only).
 moe_status stage_combine(const moe_config& c, const void* ye, const int32_t* slot_row,
                          const float* gates, void* y, cudaStream_t st, int* launches,
-                         int64_t R = -1) {
-  const int64_t shared_row0 = c.n_shared ? (R >= 0 ? R : c.N * (int64_t)c.k) : -1;
-  MOE_CUDA(moe::launch_combine(ye, slot_row, gates, c.N, c.k, c.d, shared_row0,
+                         int64_t R = -1, bool shared_in_y = false) {
+  const bool in_y = shared_in_y && c.n_shared && c.dtype == MOE_DT_BF16;
+  const int64_t shared_row0 = (c.n_shared && !in_y) ? (R >= 0 ? R : c.N * (int64_t)c.k) : -1;
+  MOE_CUDA(moe::launch_combine(ye, slot_row, gates, c.N, c.k, c.d, shared_row0, in_y ? 1 : 0,
                                c.dtype == MOE_DT_F32, y, st, launches),
            "combine");
   prof_mark(st);
@@ -520,8 +528,9 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
     if (rerouted != nullptr && c.N > 0)
       MOE_CUDA(cudaMemsetAsync(rerouted, 0, (size_t)c.N * c.k, st), "clear rerouted flags");
   }
-  MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, launches));
-  MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, launches));
+  // fused layer: the shared expert's rows go straight into y (bf16), completed by the combine
+  MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, launches, -1, y));
+  MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, launches, -1, true));
   g_prof.recording = false;
   return MOE_OK;
 }
@@ -785,8 +794,8 @@ moe_status moe_forward_routed(const moe_config* cfg, const void* x, const int32_
   MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, c.capacity, demand, counts, offsets,
                          at<int32_t>(ws, L.slot_row), at<int32_t>(ws, L.row_token), drop, x, xp,
                          st, &launches));
-  MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, &launches));
-  MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, &launches));
+  MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, &launches, -1, y));
+  MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, &launches, -1, true));
   g_last_launches = launches;
   return MOE_OK;
 }
@@ -930,8 +939,8 @@ moe_status moe_forward_padded(const moe_config* cfg, const void* x, const void* 
   MOE_CUDA(moe::launch_zero_padding(counts, c.E, c.capacity, xp, (int)(c.d * el_size(c)),
                                     row_token, st, &launches),
            "zero padding");
-  MOE_TRY(stage_ffn(c, L, ws, xp, offsets_pad, x, W_gu, W_down, ye, st, &launches, R));
-  MOE_TRY(stage_combine(c, ye, slot_row, gates, y, st, &launches, R));
+  MOE_TRY(stage_ffn(c, L, ws, xp, offsets_pad, x, W_gu, W_down, ye, st, &launches, R, y));
+  MOE_TRY(stage_combine(c, ye, slot_row, gates, y, st, &launches, R, true));
   g_last_launches = launches;
   return MOE_OK;
 }

@@ -1385,12 +1385,12 @@ int64_t one_sm_rows(int64_t r) {
   return full + (rem == 0 ? 0 : rem <= 64 ? 64 : BM);
 }
 
-// The 2-SM kernel (256-row tiles, each SM staging half of B) halves the operand bytes that
-// cross from L2 to the SMs per MMA, which is what keeps the 1-SM kernel's tensor pipe from
-// running full (its 128x256 tile needs about 96 B per clock per SM), but it computes more
-// padding rows: a routed group of r rows takes ceil(r / 256) tiles of 256 rows there, against
-// 128-row tiles with an M = 64 last tile on the 1-SM kernel, 96 more rows on average when r
-// is spread evenly modulo 256.  It is taken when that padding is at most a quarter of the
+// The 2-SM kernel (256-row tiles, each SM staging half of B) moves two thirds of the 1-SM
+// kernel's operand bytes from L2 to the SMs per FLOP, and L2-to-SM bandwidth is what keeps
+// the 1-SM kernel's tensor pipe from running full (its 128x256 tile needs about 96 B per
+// clock per SM, the 2-SM tile 64), but it computes more padding rows: a routed group of r
+// rows takes ceil(r / 256) tiles of 256 rows there, against 128-row tiles with an M = 64 last
+// tile on the 1-SM kernel, 96 more rows on average when r is spread evenly modulo 256.  It is taken when that padding is at most a quarter of the
 // rows, estimated from the caller's rows per group.  Measured on one B200: the capacity and
 // Switch layers (padding estimate 1/8 and 3/16) gain 2-6 % per step, the Mixtral-shaped down
 // projection (1/64 to 3/32) gains, and the V3/V4.1-shaped prefill (1/3) loses.  For gate/up

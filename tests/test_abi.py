@@ -211,3 +211,19 @@ def test_ffn_kernel_choice(nat):
     assert buf.value == b"grouped"
     assert nat.lib.moe_ffn_kernels(ctypes.byref(_cfg(nat)), buf, None, 0) == nat.MOE_ERR_INVALID_ARG
     assert nat.lib.moe_ffn_kernels(ctypes.byref(_cfg(nat, k=9)), buf, None, 8) == nat.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("path,kind", [("1sm", "1-SM"), ("1sm128", "1-SM, 128x128 tiles"),
+                                       ("2sm", "2-SM, 256x256 tiles"), ("swap", "token-in-N")])
+def test_ffn_kernel_override(nat, path, kind, monkeypatch):
+    """MOE_B200_GEMM_PATH forces one grouped GEMM for both projections ("1sm" keeps the
+    automatic tile width), and moe_ffn_kernels reports the forced choice (the library reads
+    the variable at every call)."""
+    from mixture_experts_layer_50_b200 import workloads as W
+    monkeypatch.setenv("MOE_B200_GEMM_PATH", path)
+    for name in ("mixtral-n16", "dsv3-n8192", "capacity-cf1"):
+        got = nat.moe_ffn_kernels(nat.config_from_shape(W.PRESETS[name]))
+        assert kind in got[0] and kind in got[1], (path, name, got)
+    monkeypatch.delenv("MOE_B200_GEMM_PATH")
+    got = nat.moe_ffn_kernels(nat.config_from_shape(W.PRESETS["capacity-cf1"]))
+    assert "2-SM" in got[0] and "2-SM" in got[1]

@@ -321,6 +321,62 @@ def test_dense_limit_k_equals_E():
             u = x[t] @ W_gu[e, F:].T
             want[t] += p[t, e] * ((g / (1 + np.exp(-g)) * u) @ W_down[e].T)
     np.testing.assert_allclose(y, want, rtol=1e-10, atol=1e-13)
+    # the oracle's own dense mixture is the same hand sum, and equals the routed layer at k = E
+    dense = O.dense_mixture(x, W_g, W_gu, W_down, E=E)
+    np.testing.assert_allclose(dense, want, rtol=1e-10, atol=1e-13)
+    np.testing.assert_allclose(dense, y, rtol=1e-10, atol=1e-13)
+
+
+def test_dense_mixture_reacts_to_every_term():
+    """Each expert's term, the router and the SwiGLU clamp move ``dense_mixture``: a version
+    that dropped an expert, ignored the logit offset or skipped the clamp would not."""
+    rng = np.random.default_rng(17)
+    N, d, E, F = 7, 5, 4, 3
+    x, W_g, W_gu, W_down = _tiny_layer(rng, N, d, E, F, E)
+    base = O.dense_mixture(x, W_g, W_gu, W_down, E=E)
+    for e in range(E):
+        W_down2 = W_down.copy()
+        W_down2[e] = 0.0
+        p = sp_softmax((x @ W_g.T).astype(np.float32).astype(np.float64), axis=1)
+        g = x @ W_gu[e, :F].T
+        u = x @ W_gu[e, F:].T
+        term = p[:, e:e + 1] * ((g / (1 + np.exp(-g)) * u) @ W_down[e].T)
+        np.testing.assert_allclose(O.dense_mixture(x, W_g, W_gu, W_down2, E=E), base - term,
+                                   rtol=1e-9, atol=1e-12)
+    # a huge offset on expert 2 makes the mixture that expert alone
+    off = np.zeros(E, np.float32)
+    off[2] = 1e3
+    only2 = O.expert_ffn(x, W_gu[2], W_down[2])
+    np.testing.assert_allclose(O.dense_mixture(x, W_g, W_gu, W_down, E=E, logit_offset=off),
+                               only2, rtol=1e-12, atol=1e-12)
+    # the clamp acts on the pre-activations: a tiny clamp bounds every |h| by c * 1
+    big = x * 100
+    clamped = O.dense_mixture(big, W_g, W_gu, W_down, E=E, clamp=0.5)
+    assert not np.allclose(clamped, O.dense_mixture(big, W_g, W_gu, W_down, E=E))
+    bound = 0.5 * 0.5 * np.abs(W_down).sum(axis=2).max()
+    assert np.abs(clamped).max() <= bound + 1e-12
+
+
+def test_forward_equals_dense_evaluation_masked_to_topk():
+    """Brute force: evaluate all E experts on every token, keep the top-k by mask, weight by
+    the renormalised softmax over the kept ones ("Основы MoE", steps 2-4), plus the shared
+    expert with weight 1 ("Le groupe d'experts (MoE)", "Des experts partagés")."""
+    rng = np.random.default_rng(19)
+    N, d, E, F, k = 11, 6, 6, 4, 3
+    x, W_g, W_gu, W_down = _tiny_layer(rng, N, d, E, F, E + 1)
+    y, info = O.forward(x, W_g, W_gu, W_down, k=k, E=E, n_shared=1)
+    z = (x @ W_g.T).astype(np.float32).astype(np.float64)
+    want = np.zeros_like(x)
+    for t in range(N):
+        order = sorted(range(E), key=lambda e: (-z[t, e], e))[:k]
+        w = np.exp(z[t, order] - z[t, order].max())
+        w /= w.sum()
+        outs = [O.expert_ffn(x[t:t + 1], W_gu[e], W_down[e])[0] for e in range(E + 1)]
+        for e in range(E):
+            if e in order:
+                want[t] += w[order.index(e)] * outs[e]
+        want[t] += outs[E]
+    np.testing.assert_allclose(y, want, rtol=1e-10, atol=1e-12)
 
 
 def test_linear_experts_closed_form_with_shared_and_capacity():

@@ -52,6 +52,10 @@ def parse_args():
     p.add_argument("--workload", default="mixtral-n16384", choices=sorted(W.PRESETS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-sweep", action="store_true",
+                   help="skip the secondary sweep of decode and ridge-point layers")
+    p.add_argument("--cpu-sample", type=int, default=256,
+                   help="tokens whose expert math the oracle runs per CPU measurement")
     p.add_argument("--overflow", default="drop", choices=["drop", "reroute"],
                    help="capacity overflow policy: drop, or the slides' 'report' (reroute)")
     p.add_argument("--tokens", type=int, default=None,
@@ -89,6 +93,22 @@ def workload_desc(shape):
             f"{' clamp=' + str(shape.clamp) if shape.clamp > 0 else ''}"
             f"{' cf=' + str(cf) if cf is not None else ''}"
             f"{' zipf-skew' if shape.zipf_skew else ''} {'bf16' if shape.dtype == W.BF16 else 'fp32'}")
+
+
+def l2_note(shape):
+    l2_resident = shape.weight_bytes() + 2 * shape.N * shape.d * (2 if shape.dtype == W.BF16 else 4) < L2_BYTES
+    return l2_resident, ("L2 flushed before every step (256 MB write; the layer's "
+                         f"{shape.weight_bytes() / 1e6:.1f} MB of weights fit in L2)"
+                         if l2_resident else
+                         f"inputs larger than L2 ({shape.weight_bytes() / 1e9:.2f} GB of weights per step)")
+
+
+def bench_config(shape, world, overflow="drop"):
+    """The ``config`` object of the JSON line: the same in both arms."""
+    return {"workload": workload_desc(shape) + (" overflow=reroute" if overflow == "reroute" else ""),
+            "tokens_per_gpu": shape.N, "global_batch": shape.N * world,
+            "l2": l2_note(shape)[1],
+            "parallelism": f"replicas x{world} (no data-path collective)"}
 
 
 def algorithmic_work(shape, counts):
@@ -231,6 +251,113 @@ def make_replica(shape, rank, device="cuda"):
     return t
 
 
+def pick_tensor_peak(peaks, clocks, flops=None, ms=None):
+    """cuBLAS reached bf16_tflops at full clock (burst) and bf16_tflops_sustained once the
+    power cap pulled the clock down: compare against the regime this run's clock shows.  A
+    short run has few clock samples: a launch faster than the sustained peak allows ran at
+    burst clocks, whatever the samples say."""
+    burst = (clocks.get("sm_mhz") or 0) >= 0.95 * (clocks.get("sm_max_mhz") or 1e9)
+    if flops and ms and flops / (ms / 1e3) / 1e12 > peaks["bf16_tflops_sustained"]:
+        burst = True
+    key = "bf16_tflops" if burst else "bf16_tflops_sustained"
+    return key, peaks[key]
+
+
+def layer_roofline(work, ms_step, peaks, tensor_peak):
+    """Whole-layer roofline: time bound = max(F / P, B / BW); the binding roof is the larger."""
+    t_tensor = work["flops_layer"] / (tensor_peak * 1e12)
+    t_hbm = work["bytes_layer"] / (peaks["hbm_gbs"] * 1e9)
+    t_bound = max(t_tensor, t_hbm)
+    return {"flops": work["flops_layer"], "bytes": work["bytes_layer"],
+            "bound": "tensor" if t_tensor >= t_hbm else "hbm",
+            "bound_ms": round(t_bound * 1e3, 4), "frac": round(t_bound * 1e3 / ms_step, 4),
+            "tflops": round(work["flops_layer"] / (ms_step / 1e3) / 1e12, 1),
+            "gbs": round(work["bytes_layer"] / (ms_step / 1e3) / 1e9, 1),
+            "kept_assignments": work["M"], "experts_touched": work["touched"]}
+
+
+def time_graphed(layer, x, y, mod, steps, warmup, world, local, l2_resident):
+    """K replays of the layer captured as one CUDA graph, timed with CUDA events on the
+    launching stream between a barrier + synchronize on both sides.  A layer whose weights
+    and tokens fit in L2 gets L2 flushed before every step (a 256 MB write) and only the
+    replays are timed.  Returns (device ms of all K steps, host enqueue us per step, clocks)."""
+    stream = torch.cuda.current_stream()
+    layer.forward_graphed(x, y, modality=mod)
+    for _ in range(warmup):
+        layer.forward_graphed(x, y, modality=mod)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda") if l2_resident else None
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        if flush is None:
+            ev0.record(stream)
+            h0 = time.perf_counter()
+            for _ in range(steps):
+                layer.forward_graphed(x, y, modality=mod)
+            host_us = (time.perf_counter() - h0) * 1e6 / steps
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            timed_ms = ev0.elapsed_time(ev1)
+        else:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)]
+            h0 = time.perf_counter()
+            for a, b in evs:
+                flush.fill_(1)
+                a.record(stream)
+                layer.forward_graphed(x, y, modality=mod)
+                b.record(stream)
+            host_us = (time.perf_counter() - h0) * 1e6 / steps
+            torch.cuda.synchronize()
+            timed_ms = sum(a.elapsed_time(b) for a, b in evs)
+    barrier(world)
+    return timed_ms, host_us, clk.summary()
+
+
+def route_counts(layer, shape, x, mod):
+    """Kept rows per expert of this batch (untimed), for the algorithmic work."""
+    counts = torch.empty(shape.E, dtype=torch.int32, device="cuda")
+    layer.forward(x, modality=mod, route_out={"counts": counts})
+    assert layer.check_status() == 0
+    return counts.cpu().numpy()
+
+
+# decode-sized and ridge-point layers measured beside the headline (same timing rules)
+SWEEP = ["mixtral-n16", "dsv3-n64", "v41flash-n64", "dsv3-n8192", "v41flash-n16384",
+         "capacity-cf1", "switch-cf1"]
+
+
+def sweep_entry(name, args, world, rank, local, peaks):
+    from mixture_experts_layer_50_b200.layer import MoELayer
+    shape = W.PRESETS[name]
+    t = make_replica(shape, rank)
+    layer = MoELayer.from_workload(shape, t)
+    x, mod = t["x"], t.get("modality")
+    y = torch.empty_like(x)
+    work = algorithmic_work(shape, route_counts(layer, shape, x, mod))
+    l2_resident, _ = l2_note(shape)
+    timed_ms, _, clocks = time_graphed(layer, x, y, mod, args.steps, args.warmup, world, local,
+                                       l2_resident)
+    assert layer.check_status() == 0
+    ms_step = max_over_ranks(timed_ms, world) / args.steps
+    key, tensor_peak = pick_tensor_peak(peaks, clocks)
+    lr = layer_roofline(work, ms_step, peaks, tensor_peak)
+    if lr["bound"] == "tensor":
+        achieved, peak, unit = lr["tflops"], tensor_peak, "TFLOP/s"
+    else:
+        achieved, peak, unit = lr["gbs"], peaks["hbm_gbs"], "GB/s"
+    out = {"workload": workload_desc(shape), "ms_per_step": round(ms_step, 4),
+           "tokens_per_s": round(shape.N * world / (ms_step / 1e3), 1),
+           "bound": lr["bound"], "achieved": achieved, "peak": peak, "unit": unit,
+           "frac": lr["frac"], "peak_key": key if lr["bound"] == "tensor" else "hbm_gbs",
+           "kept_assignments": lr["kept_assignments"], "experts_touched": lr["experts_touched"],
+           "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")}}
+    del layer, t, x, y
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     from mixture_experts_layer_50_b200 import build as _build
     if int(os.environ.get("LOCAL_RANK", "0")) == 0:
@@ -255,52 +382,17 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     names = LAUNCH_NAMES_REROUTE if args.overflow == "reroute" and shape.capacity_factor else LAUNCH_NAMES
 
-    # routing statistics of this batch (untimed), for the algorithmic work
-    counts = torch.empty(shape.E, dtype=torch.int32, device="cuda")
-    layer.forward(x, modality=mod, y=y, route_out={"counts": counts})
-    assert layer.check_status() == 0
-    work = algorithmic_work(shape, counts.cpu().numpy())
-
+    work = algorithmic_work(shape, route_counts(layer, shape, x, mod))
     for _ in range(args.warmup):
         layer.forward(x, modality=mod, y=y)
     torch.cuda.synchronize()
     per_step_launches = nat.moe_last_launch_count()
-    # the step as a CUDA graph: the eight launches captured once, replayed each step
-    layer.forward_graphed(x, y, modality=mod)
-    for _ in range(args.warmup):
-        layer.forward_graphed(x, y, modality=mod)
 
-    # timed region: K replays of the whole layer.  A layer whose weights and tokens fit in
-    # L2 (the fp32 toy) gets L2 flushed before every step (a 256 MB write) and only the
-    # replays themselves are timed; every other layer streams more than L2 per step.
-    l2_resident = shape.weight_bytes() + 2 * x.numel() * x.element_size() < L2_BYTES
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda") if l2_resident else None
-    barrier(world)
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        if flush is None:
-            ev0.record(stream)
-            h0 = time.perf_counter()
-            for _ in range(args.steps):
-                layer.forward_graphed(x, y, modality=mod)
-            host_us = (time.perf_counter() - h0) * 1e6 / args.steps
-            ev1.record(stream)
-            torch.cuda.synchronize()
-            timed_ms = ev0.elapsed_time(ev1)
-        else:
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(args.steps)]
-            h0 = time.perf_counter()
-            for a, b in evs:
-                flush.fill_(1)
-                a.record(stream)
-                layer.forward_graphed(x, y, modality=mod)
-                b.record(stream)
-            host_us = (time.perf_counter() - h0) * 1e6 / args.steps
-            torch.cuda.synchronize()
-            timed_ms = sum(a.elapsed_time(b) for a, b in evs)
-    barrier(world)
+    # timed region: K replays of the whole layer (the eight launches captured once as a
+    # CUDA graph)
+    l2_resident, _ = l2_note(shape)
+    timed_ms, host_us, clocks = time_graphed(layer, x, y, mod, args.steps, args.warmup, world,
+                                             local, l2_resident)
     assert layer.check_status() == 0
 
     # the same K steps launched one kernel at a time, with a CUDA event recorded on the
@@ -345,20 +437,11 @@ def run_ours(args):
     el = x.element_size()
 
     peaks, peak_src = load_peaks()
-    clocks = clk.summary()
-    # cuBLAS reached bf16_tflops at full clock (burst) and bf16_tflops_sustained once the
-    # power cap pulled the clock down: compare against the regime this run's clock shows
-    burst = (clocks.get("sm_mhz") or 0) >= 0.95 * (clocks.get("sm_max_mhz") or 1e9)
     per_launch = {n: launch_ms[i] / max(calls, 1) for i, n in enumerate(names)
                   if i < len(launch_ms)}
     gu_ms = per_launch.get("gemm_gate_up")
     gu_kernel, down_kernel = nat.moe_ffn_kernels(layer.config(shape.N))
-    # a short run has few clock samples: a gate/up launch faster than the sustained peak
-    # allows ran at burst clocks, whatever the samples say
-    if gu_ms and work["flops_gate_up"] / (gu_ms / 1e3) / 1e12 > peaks["bf16_tflops_sustained"]:
-        burst = True
-    tensor_key = "bf16_tflops" if burst else "bf16_tflops_sustained"
-    tensor_peak = peaks[tensor_key]
+    tensor_key, tensor_peak = pick_tensor_peak(peaks, clocks, work["flops_gate_up"], gu_ms)
     ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     intensity = work["flops_gate_up"] / work["bytes_gate_up"]
     roof = None
@@ -377,18 +460,22 @@ def run_ours(args):
         roof["kernel"] = f"gemm_gate_up: {gu_kernel}, {act} epilogue"
         roof["ms_per_launch"] = round(gu_ms, 4)
         roof["peak_source"] = f"{peak_src} ({tensor_key if roof['bound'] == 'tensor' else 'hbm_gbs'})"
-    # whole-layer roofline: time bound = max(F / P, B / BW)
-    t_bound = max(work["flops_layer"] / (tensor_peak * 1e12),
-                  work["bytes_layer"] / (peaks["hbm_gbs"] * 1e9))
-    layer_roof = {"flops": work["flops_layer"], "bytes": work["bytes_layer"],
-                  "bound_ms": round(t_bound * 1e3, 4), "frac": round(t_bound * 1e3 / ms_step, 4),
-                  "tflops": round(work["flops_layer"] / (ms_step / 1e3) / 1e12, 1),
-                  "gbs": round(work["bytes_layer"] / (ms_step / 1e3) / 1e9, 1),
-                  "kept_assignments": work["M"], "experts_touched": work["touched"]}
+    layer_roof = layer_roofline(work, ms_step, peaks, tensor_peak)
+
+    # the headline layer's buffers go before the sweep allocates its own layers
+    del layer, t, x, y, xh, yhs
+    torch.cuda.empty_cache()
+    sweep = None
+    if not args.no_sweep and args.tokens is None and args.experts is None \
+            and args.overflow == "drop":
+        sweep = {}
+        for name in SWEEP:
+            if name != args.workload:
+                sweep[name] = sweep_entry(name, args, world, rank, local, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(shape, t, sample_tokens=384)
+        cpu = cpu_baseline(shape, args.cpu_sample)
 
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -396,14 +483,7 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
         if shape.dtype == W.BF16 else "f32",
         "data": f"synthetic (seeded N(0,{shape.w_std:g}) weights, N(0,1) tokens)",
-        "config": {"workload": workload_desc(shape)
-                   + (" overflow=reroute" if args.overflow == "reroute" else ""),
-                   "tokens_per_gpu": shape.N, "global_batch": shape.N * world,
-                   "l2": ("L2 flushed before every step (256 MB write; the layer's "
-                          f"{shape.weight_bytes() / 1e6:.1f} MB of weights fit in L2)"
-                          if l2_resident else
-                          f"inputs larger than L2 ({shape.weight_bytes() / 1e9:.2f} GB of weights per step)"),
-                   "parallelism": f"replicas x{world} (no data-path collective)"},
+        "config": bench_config(shape, world, args.overflow),
         "roofline": roof, "layer_roofline": layer_roof,
         "launch_ms": {k: round(v, 4) for k, v in per_launch.items()},
         "ffn_kernels": {"gate_up": gu_kernel, "down": down_kernel},
@@ -421,6 +501,7 @@ def run_ours(args):
                   "launch_ms and roofline: the same K steps launched eagerly with CUDA events "
                   "between the kernels on the launching stream",
         "clocks": clocks,
+        "sweep": sweep,
         "cpu_baseline": cpu,
     }
     if rank == 0:
@@ -431,55 +512,132 @@ def run_ours(args):
 
 
 # ------------------------------------------------------------------------------------------
-class _HostExperts:
-    """Per-expert host views of device weights, handed to the oracle as it asks for them."""
+# the CPU oracle timed on this host (the cpu_baseline leg and the reference arm)
+# ------------------------------------------------------------------------------------------
+HOST_F64_BUDGET = 24 << 30      # float64 expert weights kept on the host between measurements
 
-    def __init__(self, t):
-        self.t = t
+
+class _HostExperts:
+    """float64 host copies of the per-expert device weights, made on first use and kept while
+    they fit a host budget.  The time spent making them is counted apart (``fetch_s``) so that
+    it can be taken out of the oracle's own time."""
+
+    def __init__(self, t, cache):
+        self.t, self.cache, self.fetch_s = t, cache, 0.0
 
     def __getitem__(self, e):
-        return self.t[e].float().cpu().numpy()
+        key = (self.t.data_ptr(), e)
+        a = self.cache.get(key)
+        if a is None:
+            t0 = time.perf_counter()
+            a = self.t[e].to(torch.float64).cpu().numpy()     # bf16 -> float64 is exact
+            self.fetch_s += time.perf_counter() - t0
+            if sum(v.nbytes for v in self.cache.values()) + a.nbytes <= HOST_F64_BUDGET:
+                self.cache[key] = a
+        return a
 
 
-def _oracle_inputs(shape, t):
-    x64 = W.bf16_to_f64(t["x"])
-    return dict(x=x64, W_g=W.bf16_to_f64(t["W_g"]), W_gu=_HostExperts(t["W_gu"]),
-                W_down=_HostExperts(t["W_down"]),
-                kw=dict(k=shape.k, E=shape.E, score_fn=shape.score_fn, renorm=shape.renorm,
-                        act=shape.act, clamp=shape.clamp, n_shared=shape.n_shared,
-                        bias=None if "bias" not in t else t["bias"].cpu().numpy(),
-                        modality=None if "modality" not in t else t["modality"].cpu().numpy(),
-                        logit_offset=None if "logit_offset" not in t else t["logit_offset"].cpu().numpy()))
+class OracleTimer:
+    """Times the oracle as it stands on one layer instance: the routing of all N tokens
+    (router projection, scores, top-k, capacity and layout) and the expert math and combine
+    of a seeded token sample, in separate clocks.  The full-layer time per token is
+    extrapolated from the two: t_route / N + t_expert / |sample|."""
+
+    def __init__(self, shape, t):
+        self.shape = shape
+        dev = t["x"].device
+        self.x64 = t["x"].to(torch.float64).cpu().numpy() if dev.type == "cuda" else W.bf16_to_f64(t["x"])
+        self.Wg64 = t["W_g"].to(torch.float64).cpu().numpy()
+        cache = {}
+        self.W_gu, self.W_down = _HostExperts(t["W_gu"], cache), _HostExperts(t["W_down"], cache)
+        self.kw = dict(k=shape.k, E=shape.E, score_fn=shape.score_fn, renorm=shape.renorm,
+                       act=shape.act, clamp=shape.clamp, n_shared=shape.n_shared,
+                       bias=None if "bias" not in t else t["bias"].cpu().numpy(),
+                       modality=None if "modality" not in t else t["modality"].cpu().numpy())
+        self.offset = None if "logit_offset" not in t else t["logit_offset"].cpu().numpy()
+        import oracle as O
+        self.O = O
+        self.C = O.capacity(shape.N, shape.k, shape.E, shape.capacity_factor)
+
+    def prefetch(self, tokens):
+        """Host float64 weights of the experts the sample touches (outside any clock)."""
+        O, kw = self.O, self.kw
+        z = O.router_logits(self.x64[tokens], self.Wg64, self.offset)
+        ids, _ = O.route(z, kw["k"], kw["score_fn"], kw["renorm"], kw["bias"],
+                         None if kw["modality"] is None else kw["modality"][tokens])
+        for e in sorted(set(ids.ravel().tolist())) + list(range(self.shape.E, self.shape.G)):
+            self.W_gu[e], self.W_down[e]
+
+    def measure(self, tokens):
+        O, kw = self.O, self.kw
+        t0 = time.perf_counter()
+        z = O.router_logits(self.x64, self.Wg64, self.offset)
+        ids, _ = O.route(z, kw["k"], kw["score_fn"], kw["renorm"], kw["bias"], kw["modality"])
+        O.dispatch(ids, self.shape.E, self.C)
+        t_route = time.perf_counter() - t0
+        f0 = self.W_gu.fetch_s + self.W_down.fetch_s
+        t1 = time.perf_counter()
+        O.forward(self.x64, None, self.W_gu, self.W_down, logits=z, tokens=tokens, C=self.C, **kw)
+        fetched = self.W_gu.fetch_s + self.W_down.fetch_s - f0
+        t_expert = time.perf_counter() - t1 - fetched
+        return t_route, t_expert
+
+    def sample(self, rng, n):
+        return np.sort(rng.choice(self.shape.N, size=min(n, self.shape.N), replace=False))
 
 
-def _oracle_capacity(shape):
-    import oracle as O
-    return O.capacity(shape.N, shape.k, shape.E, shape.capacity_factor)
-
-
-def _blas_threads():
+def _host_info():
+    cpu_model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    cpu_model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
     try:
         from threadpoolctl import threadpool_info
         n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
-        return max(n) if n else 1
+        blas = max(n) if n else 1
     except Exception:
-        return os.cpu_count()
+        blas = None
+    return {"nproc": len(os.sched_getaffinity(0)), "cpu_model": cpu_model, "blas_threads": blas}
 
 
-def cpu_baseline(shape, t, sample_tokens=64):
-    """The oracle as it stands on this host: full routing, expert math for a token sample."""
-    import oracle as O
-    inp = _oracle_inputs(shape, t)
-    C = _oracle_capacity(shape)
-    rng = np.random.default_rng(0)
-    tokens = np.sort(rng.choice(shape.N, size=min(sample_tokens, shape.N), replace=False))
-    t0 = time.perf_counter()
-    O.forward(inp["x"], inp["W_g"], inp["W_gu"], inp["W_down"], C=C, tokens=tokens, **inp["kw"])
-    dt = time.perf_counter() - t0
-    return {"value": round(len(tokens) / dt, 3), "unit": "tokens/s", "cores": _blas_threads(),
-            "kind": "oracle", "seconds": round(dt, 2),
-            "sample": f"routing of all {shape.N} tokens + expert FFNs and combine of "
-                      f"{len(tokens)} sampled tokens; tokens/s = sampled tokens / wall time"}
+def oracle_runs(shape, t, sample_tokens, steps, warmup, seed):
+    """Per-token full-layer seconds of the oracle over ``steps`` measurements (each on a
+    fresh seeded sample of ``sample_tokens`` tokens) after ``warmup`` untimed ones."""
+    ot = OracleTimer(shape, t)
+    rng = np.random.default_rng(seed)
+    per_token, wall = [], []
+    for s in range(warmup + steps):
+        tokens = ot.sample(rng, sample_tokens)
+        ot.prefetch(tokens)
+        t_route, t_expert = ot.measure(tokens)
+        if s >= warmup:
+            per_token.append(t_route / shape.N + t_expert / len(tokens))
+            wall.append(t_route + t_expert)
+    return per_token, wall, len(tokens)
+
+
+def _oracle_sample_note(shape, n):
+    return (f"per measurement: routing of all {shape.N} tokens (router projection, scores, "
+            f"top-k, capacity, layout) + expert FFNs and combine of {n} seeded sampled tokens, "
+            f"timed apart; value = 1 / (t_route/{shape.N} + t_expert/{n}), the full-layer "
+            "throughput extrapolated from the sample (host float64 weight copies made "
+            "outside the clocks)")
+
+
+def cpu_baseline(shape, sample_tokens):
+    """The oracle as it stands on this host, the same measurement as the reference arm."""
+    t = W.make_inputs(shape, device="cuda" if torch.cuda.is_available() else "cpu")
+    per_token, wall, n = oracle_runs(shape, t, sample_tokens, steps=2, warmup=0, seed=1)
+    info = _host_info()
+    return {"value": round(1.0 / statistics.mean(per_token), 3), "unit": "tokens/s",
+            "cores": info["blas_threads"] or info["nproc"], "kind": "oracle",
+            "seconds": round(sum(wall), 2), "host": info,
+            "sample": "2 measurements; " + _oracle_sample_note(shape, n)}
 
 
 def run_reference(args):
@@ -489,31 +647,21 @@ def run_reference(args):
         return
     shape = workload_shape(args)
     t = W.make_inputs(shape, device="cuda" if torch.cuda.is_available() else "cpu")
-    import oracle as O
-    inp = _oracle_inputs(shape, t)
-    C = _oracle_capacity(shape)
-    per_step = 8
-    rng = np.random.default_rng(1)
-    times, ntok = [], 0
-    for s in range(args.warmup + args.steps):
-        tokens = np.sort(rng.choice(shape.N, size=min(per_step, shape.N), replace=False))
-        t0 = time.perf_counter()
-        O.forward(inp["x"], inp["W_g"], inp["W_gu"], inp["W_down"], C=C, tokens=tokens, **inp["kw"])
-        if s >= args.warmup:
-            times.append(time.perf_counter() - t0)
-            ntok += len(tokens)
-    total = sum(times)
-    value = ntok / total
+    per_token, wall, n = oracle_runs(shape, t, args.cpu_sample, args.steps, args.warmup, seed=1)
+    value = 1.0 / statistics.mean(per_token)
+    info = _host_info()
     out = {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(1e3 * total / args.steps, 2), "higher_is_better": True,
+        "ms_per_step": round(1e3 * shape.N / value, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(shape), "tokens_per_gpu": shape.N},
-        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": _blas_threads(),
-                         "kind": "oracle",
-                         "sample": f"per step: routing of all {shape.N} tokens + expert FFNs of "
-                                   f"{per_step} sampled tokens"},
+        "config": bench_config(shape, world, args.overflow),
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s",
+                         "cores": info["blas_threads"] or info["nproc"], "kind": "oracle",
+                         "seconds": round(sum(wall), 2), "host": info,
+                         "sample": f"{args.steps} measurements after {args.warmup} untimed; "
+                                   + _oracle_sample_note(shape, n)
+                                   + "; ms_per_step = N / value, the extrapolated full layer"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

@@ -282,6 +282,93 @@ MOE_API moe_status moe_forward_padded(const moe_config* cfg, const void* x, cons
                                       const moe_route_out* route_out, void* ws,
                                       moe_stream_t stream);
 
+/* ---- expert parallelism ---------------------------------------------------------------
+ * "Mixture-of-Experts : routage et capacité" slides, "Le problème — Communication", "L'idée —
+ * Communication" and "Support visuel — Communication": the routed experts are spread over
+ * `world` ranks (one process per GPU); each rank routes its own tokens, ships every kept
+ * assignment's row to the rank that owns the expert (dispatch), the owner runs its experts,
+ * and the outputs come back to the token's rank (combine).  Rank o owns the contiguous
+ * experts [moe_ep_first_expert(world, o, E), moe_ep_first_expert(world, o + 1, E)); every
+ * rank holds the router weights and the shared expert.  The result on every rank equals the
+ * single-device layer (moe_forward) over the concatenation of all ranks' tokens, rank 0's
+ * first: capacity serves each expert's assignments in that order.  The calls below are the
+ * per-rank steps; the exchanges between them (an all-gather of per-expert demands and the
+ * row messages the plan lists) belong to the caller's communication library (NCCL). */
+
+/* One run of rows exchanged with one peer for one expert. */
+typedef struct {
+  int32_t peer;    /* the other rank */
+  int32_t expert;  /* global expert id; usable as the message tag */
+  int64_t row;     /* first row in this rank's buffer */
+  int64_t rows;    /* number of rows, > 0 */
+} moe_ep_chunk;
+
+/* First expert owned by `rank` (rank in [0, world]; rank == world gives E), or -1 on a bad
+ * argument.  Experts are split into contiguous runs of floor or ceil(E / world).  Host only. */
+MOE_API int32_t moe_ep_first_expert(int32_t world, int32_t rank, int32_t E);
+
+/* The exchange plan of one rank, from every rank's per-expert demand (host only, no GPU).
+ *   demand_all [world][E] host: assignments per expert of each rank's tokens before capacity
+ *              (moe_route's demand output, all-gathered)
+ *   capacity   C for the whole concatenated batch (<= 0: no limit)
+ * Outputs (host, caller-allocated; any may be NULL):
+ *   cap [E]              how many of this rank's assignments to e it keeps, the first in its
+ *                        token order: C minus the demand of the earlier ranks, clamped to
+ *                        [0, C] (INT32_MAX without a limit); the input of moe_permute_ep
+ *   kept_all [world][E]  kept assignments of every rank per expert
+ *   owned_offsets [E_own + 1]  group offsets of the receive buffer of this rank's experts
+ *   sends [<= E]         this rank's send buffer (moe_permute_ep's xp) as runs: expert e's kept
+ *                        rows go to its owner; listed by increasing expert
+ *   recvs [<= world * E_own]  where the rows of each (expert, source rank) land in the receive
+ *                        buffer: expert-major, then source rank (the concatenated batch's token
+ *                        order); listed by increasing expert, then rank
+ *   n_sends, n_recvs     numbers of runs; rows_kept = this rank's kept rows (send buffer
+ *                        rows), rows_owned = receive buffer rows
+ * Runs with the same peer appear in the same expert order on both sides, so a grouped
+ * send/receive posted in list order matches.  The return trip of the combine uses the same
+ * lists with the roles swapped.  MOE_ERR_INVALID_ARG for a bad rank or negative demand;
+ * MOE_ERR_UNSUPPORTED when world > E or a buffer would exceed 2^30 rows. */
+MOE_API moe_status moe_ep_plan(int32_t world, int32_t rank, int32_t E, int64_t capacity,
+                               const int32_t* demand_all, int32_t* cap, int32_t* kept_all,
+                               int32_t* owned_offsets, moe_ep_chunk* sends, int32_t* n_sends,
+                               moe_ep_chunk* recvs, int32_t* n_recvs, int64_t* rows_kept,
+                               int64_t* rows_owned);
+
+/* Workspace bytes of an expert-parallel rank: cfg is the whole layer (all E experts) with
+ * cfg->N = the most tokens any rank routes; covers moe_route, moe_permute_ep and
+ * moe_ep_expert_ffn.  0 on a bad config or world > E. */
+MOE_API size_t moe_ep_workspace_size(const moe_config* cfg, int32_t world);
+
+/* moe_permute with a per-expert capacity: the assignment (t, j) to expert e is kept iff its
+ * rank among this rank's assignments to e (token order) is below cap[e] (device int32 [E],
+ * from moe_ep_plan).  Outputs as in moe_permute, plus counts [E] (kept per expert) and
+ * drop_mask [N][k] (either may be NULL).  cfg->capacity is not used. */
+MOE_API moe_status moe_permute_ep(const moe_config* cfg, const int32_t* ids, const int32_t* cap,
+                                  const void* x, int32_t* offsets, int32_t* row_token,
+                                  int32_t* slot_row, void* xp, int32_t* counts,
+                                  uint8_t* drop_mask, void* ws, moe_stream_t stream);
+
+/* The owner's expert FFNs (bf16): the received rows xr [rows][d], grouped by owned_offsets
+ * (device int32 [E_own + 1], from moe_ep_plan), through the rank's experts, into ye
+ * [rows][d]; with n_shared == 1 also the shared expert on this rank's own n_tokens tokens
+ * x [n_tokens][d], written into y [n_tokens][d] (moe_ep_combine then adds the routed slots
+ * to it).  cfg is the whole layer exactly as given to moe_ep_workspace_size (cfg->N = the
+ * most tokens any rank routes, which sizes the workspace); n_tokens <= cfg->N.  W_gu
+ * [E_own + S][.][d] and W_down [E_own + S][d][F] hold this rank's experts (shared last).
+ * rows is the host value rows_owned of the plan, at most world * cfg->N * k. */
+MOE_API moe_status moe_ep_expert_ffn(const moe_config* cfg, int32_t world, int32_t rank,
+                                     int64_t n_tokens, int64_t rows, const void* xr,
+                                     const int32_t* owned_offsets, const void* x,
+                                     const void* W_gu, const void* W_down, void* ye, void* y,
+                                     void* ws, moe_stream_t stream);
+
+/* The combine on the token's rank (bf16): ye [rows_kept][d] holds the expert outputs in the
+ * send buffer's row order (the return trip of the plan's runs); with n_shared == 1, y [N][d]
+ * already holds the shared expert's rows (moe_ep_expert_ffn) and the kept slots are added to
+ * them in place, in slot order, one rounding; with n_shared == 0, y = the gate-weighted sum. */
+MOE_API moe_status moe_ep_combine(const moe_config* cfg, const void* ye, const int32_t* slot_row,
+                                  const float* gates, void* y, moe_stream_t stream);
+
 /* moe_forward with x_host and y_host in HOST memory (pinned for full copy speed): copies
  * x to the workspace, runs the layer, copies y back and synchronises the stream.
  * Weights, bias, modality and logit_offset are device pointers as in moe_forward. */
@@ -297,11 +384,14 @@ MOE_API moe_status moe_forward_host(const moe_config* cfg, const void* x_host, c
  * critical loop that must not risk the implicit device synchronisation of cudaMalloc.
  * The pages have no counterpart of this call; it is a deployment convenience.
  * Scratch: a fixed 4 MiB device array inside the library (every GPU that loads the library
- * holds it until the process exits).  The call needs 256 + 4*(2*N*k + 2*ceil(N/32)*E + E + 1)
- * bytes of it, each part rounded up to 256; larger requests return MOE_ERR_UNSUPPORTED
- * (e.g. N = 16384 tokens with k = 8 and E = 256 fits; N = 65536 with k = 8 does not).
- * The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- * with that device current; make that first call before any stream capture.
+ * holds it until the process exits).  The call needs 256 + 4*N*k + 2*(4*ceil(N/32)*E) +
+ * 4*(E + 1) bytes of it, each of the four parts rounded up to 256; larger requests return
+ * MOE_ERR_UNSUPPORTED before anything is enqueued.  Examples: N = 16384, k = 8, E = 256 needs
+ * 1.5 MiB and fits; N = 65536, k = 8, E = 8 needs 2.1 MiB and fits; N = 16384, k = 8,
+ * E = 1024 needs 4.5 MiB (the per-tile histograms dominate) and is refused.
+ * The first call on a device (and again after a device reset, which gives the device a new
+ * context) looks up the array's device address (cudaGetSymbolAddress) with that device
+ * current; make that first call before any stream capture.
  * All calls share the array and it keeps the last call's contents: calls that may overlap
  * on the GPU (other streams, other host threads) race -- order them on one stream.
  *   status: optional device int32; device findings (a modality flag >= n_bias_sets) are

@@ -3,7 +3,8 @@
 The layer runs in ``libmoe_b200.so`` (C ABI in ``include/moe.h``).  This package is the
 thin Python binding: ``moe_route``, ``moe_permute``, ``moe_expert_ffn``, ``moe_combine``,
 ``moe_forward`` and ``moe_forward_host`` keep the C names and take torch CUDA tensors;
-``MoELayer`` bundles a layer's weights and workspace.  Accessing any of them loads the
+``MoELayer`` bundles a layer's weights and workspace; ``EPMoELayer`` is one rank of the
+expert-parallel layer (experts spread over the ranks of a process group).  Accessing any of them loads the
 library and raises ``ImportError`` if it has not been built -- there is no fallback.
 """
 from __future__ import annotations
@@ -18,7 +19,9 @@ _NATIVE_NAMES = {
     "moe_check_status", "moe_last_launch_count", "moe_profile_begin", "moe_profile_end",
     "moe_route_static", "moe_forward_routed", "moe_route_hash", "moe_balance",
     "moe_permute_padded", "moe_forward_padded", "moe_forward_host_batches", "moe_config", "moe_route_out", "make_config",
-    "config_from_shape", "MoeError", "lib", "EXPORTED",
+    "config_from_shape", "MoeError", "lib", "EXPORTED", "moe_ep_first_expert", "moe_ep_plan",
+    "moe_ep_workspace_size", "alloc_ep_workspace", "moe_permute_ep", "moe_ep_expert_ffn",
+    "moe_ep_combine",
 }
 
 
@@ -27,4 +30,6 @@ def __getattr__(name):
         return getattr(importlib.import_module("._native", __name__), name)
     if name == "MoELayer":
         return importlib.import_module(".layer", __name__).MoELayer
+    if name == "EPMoELayer":
+        return importlib.import_module(".ep", __name__).EPMoELayer
     raise AttributeError(name)

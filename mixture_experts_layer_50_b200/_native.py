@@ -78,6 +78,21 @@ lib.moe_route_reroute.argtypes = [_cfgp] + [_vp] * 15
 lib.moe_selftest_wait_timeout.argtypes = [_vp, _i64, _vp]
 lib.moe_forward_reroute.argtypes = [_cfgp] + [_vp] * 12
 lib.moe_ffn_kernels.argtypes = [_cfgp, ctypes.c_char_p, ctypes.c_char_p, ctypes.c_size_t]
+
+
+class moe_ep_chunk(ctypes.Structure):
+    _fields_ = [("peer", ctypes.c_int32), ("expert", ctypes.c_int32), ("row", ctypes.c_int64),
+                ("rows", ctypes.c_int64)]
+
+
+lib.moe_ep_first_expert.argtypes = [_i32, _i32, _i32]
+lib.moe_ep_first_expert.restype = _i32
+lib.moe_ep_plan.argtypes = [_i32, _i32, _i32, _i64] + [_vp] * 10
+lib.moe_ep_workspace_size.argtypes = [_cfgp, _i32]
+lib.moe_ep_workspace_size.restype = _sz
+lib.moe_permute_ep.argtypes = [_cfgp] + [_vp] * 11
+lib.moe_ep_expert_ffn.argtypes = [_cfgp, _i32, _i32, _i64, _i64] + [_vp] * 9
+lib.moe_ep_combine.argtypes = [_cfgp] + [_vp] * 5
 lib.moe_profile_begin.argtypes = [_i32]
 lib.moe_profile_begin.restype = ctypes.c_int
 lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)]
@@ -88,7 +103,8 @@ for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "
            "moe_forward", "moe_forward_host", "moe_check_status", "moe_route_static",
            "moe_forward_routed", "moe_route_hash", "moe_balance", "moe_permute_padded",
            "moe_forward_padded", "moe_forward_host_batches", "moe_route_reroute",
-           "moe_forward_reroute", "moe_selftest_wait_timeout", "moe_ffn_kernels"):
+           "moe_forward_reroute", "moe_selftest_wait_timeout", "moe_ffn_kernels", "moe_ep_plan",
+           "moe_permute_ep", "moe_ep_expert_ffn", "moe_ep_combine"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
@@ -97,7 +113,9 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_rou
             "moe_last_launch_count", "moe_route_static", "moe_forward_routed",
             "moe_route_hash", "moe_balance", "moe_permute_padded", "moe_forward_padded",
             "moe_forward_host_batches", "moe_route_reroute", "moe_forward_reroute",
-            "moe_selftest_wait_timeout", "moe_ffn_kernels")
+            "moe_selftest_wait_timeout", "moe_ffn_kernels", "moe_ep_first_expert",
+            "moe_ep_plan", "moe_ep_workspace_size", "moe_permute_ep", "moe_ep_expert_ffn",
+            "moe_ep_combine")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -363,3 +381,80 @@ def moe_profile_end(max_launches: int = 16):
     if n < 0:
         raise MoeError(MOE_ERR_CUDA, "moe_profile_end")
     return [float(buf[i]) for i in range(min(n, max_launches))], int(calls.value)
+
+
+# ---- expert parallelism --------------------------------------------------------------------
+def moe_ep_first_expert(world: int, rank: int, E: int) -> int:
+    """First expert owned by ``rank`` (``rank == world`` gives E)."""
+    v = int(lib.moe_ep_first_expert(int(world), int(rank), int(E)))
+    if v < 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_ep_first_expert")
+    return v
+
+
+def moe_ep_plan(world: int, rank: int, E: int, capacity: int, demand_all) -> dict:
+    """The exchange plan of one rank (host only).  ``demand_all``: int32 [world][E] (numpy or
+    CPU tensor).  Returns cap [E], kept_all [world][E], owned_offsets [E_own + 1] (numpy
+    int32), sends / recvs as lists of (peer, expert, row, rows), rows_kept, rows_owned."""
+    import numpy as np
+    dem = np.ascontiguousarray(np.asarray(demand_all, dtype=np.int32).reshape(world, E))
+    e_own = moe_ep_first_expert(world, rank + 1, E) - moe_ep_first_expert(world, rank, E)
+    cap = np.zeros(E, np.int32)
+    kept = np.zeros((world, E), np.int32)
+    owned = np.zeros(e_own + 1, np.int32)
+    sends = (moe_ep_chunk * E)()
+    recvs = (moe_ep_chunk * max(1, world * e_own))()
+    ns, nr = _i32(0), _i32(0)
+    rk, ro = _i64(0), _i64(0)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    st = lib.moe_ep_plan(int(world), int(rank), int(E), int(capacity), p(dem), p(cap), p(kept),
+                         p(owned), sends, ctypes.byref(ns), recvs, ctypes.byref(nr),
+                         ctypes.byref(rk), ctypes.byref(ro))
+    _check(st, "moe_ep_plan")
+    as_list = lambda arr, n: [(c.peer, c.expert, c.row, c.rows) for c in arr[:n]]
+    return dict(cap=cap, kept_all=kept, owned_offsets=owned, sends=as_list(sends, ns.value),
+                recvs=as_list(recvs, nr.value), rows_kept=int(rk.value),
+                rows_owned=int(ro.value), first_expert=moe_ep_first_expert(world, rank, E),
+                n_owned=e_own)
+
+
+def moe_ep_workspace_size(cfg: moe_config, world: int) -> int:
+    return int(lib.moe_ep_workspace_size(ctypes.byref(cfg), int(world)))
+
+
+def alloc_ep_workspace(cfg: moe_config, world: int, device="cuda") -> torch.Tensor:
+    size = moe_ep_workspace_size(cfg, world)
+    if size == 0:
+        raise MoeError(MOE_ERR_INVALID_ARG, "moe_ep_workspace_size")
+    ws = torch.empty(size + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    ws = ws[off:off + size]
+    moe_workspace_init(ws)
+    return ws
+
+
+def moe_permute_ep(cfg, *, ids, cap, x, offsets, row_token=None, slot_row, xp, counts=None,
+                   drop_mask=None, ws, stream=None):
+    """Permutation with a per-expert capacity (device int32 [E]) into the send layout."""
+    st = lib.moe_permute_ep(ctypes.byref(cfg), _ptr(ids), _ptr(cap), _ptr(x), _ptr(offsets),
+                            _ptr(row_token), _ptr(slot_row), _ptr(xp), _ptr(counts),
+                            _ptr(drop_mask), _ptr(ws), _stream(stream))
+    _check(st, "moe_permute_ep")
+
+
+def moe_ep_expert_ffn(cfg, world: int, rank: int, n_tokens: int, rows: int, *, xr,
+                      owned_offsets, x=None, W_gu, W_down, ye, y=None, ws, stream=None):
+    """The owner's experts on the received rows (and the shared expert on its own tokens).
+    ``cfg`` is the configuration the workspace was sized with (N = most tokens per rank)."""
+    st = lib.moe_ep_expert_ffn(ctypes.byref(cfg), int(world), int(rank), int(n_tokens),
+                               int(rows), _ptr(xr),
+                               _ptr(owned_offsets), _ptr(x), _ptr(W_gu), _ptr(W_down), _ptr(ye),
+                               _ptr(y), _ptr(ws), _stream(stream))
+    _check(st, "moe_ep_expert_ffn")
+
+
+def moe_ep_combine(cfg, *, ye, slot_row, gates, y, stream=None):
+    """The combine on the token's rank (adds to the shared rows already in y)."""
+    st = lib.moe_ep_combine(ctypes.byref(cfg), _ptr(ye), _ptr(slot_row), _ptr(gates), _ptr(y),
+                            _stream(stream))
+    _check(st, "moe_ep_combine")

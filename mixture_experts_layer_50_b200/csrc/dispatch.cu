@@ -72,7 +72,8 @@ __global__ void __launch_bounds__(32) rank_local_kernel(
 __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
     const int32_t* __restrict__ tile_hist, int n_tiles, int E, int64_t C,
     int32_t* __restrict__ tile_base, int32_t* __restrict__ demand,
-    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* arrive) {
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* arrive,
+    const int32_t* __restrict__ cap_e) {
   pdl_wait();
   __shared__ int32_t part[32][33];  // chunk sums [warp][lane]
   __shared__ int32_t warp_tot[32];
@@ -104,7 +105,10 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
     }
     if (w == 0) {
       demand[e] = total;
-      counts[e] = (C > 0 && total > C) ? (int32_t)C : total;
+      if (cap_e != nullptr)
+        counts[e] = min(total, max(cap_e[e], 0));
+      else
+        counts[e] = (C > 0 && total > C) ? (int32_t)C : total;
       __threadfence();
     }
   }
@@ -153,7 +157,7 @@ __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
     const int32_t* __restrict__ tile_base, const int32_t* __restrict__ offsets, int k, int E,
     int64_t C, int32_t* __restrict__ slot_row, int32_t* __restrict__ row_token,
     uint8_t* __restrict__ drop_mask_out, const V* __restrict__ x, V* __restrict__ xp,
-    int row_vecs) {
+    int row_vecs, const int32_t* __restrict__ cap_e) {
   pdl_wait();
   __shared__ int32_t s_row[32];
   const int64_t t = blockIdx.x;
@@ -167,9 +171,10 @@ __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
     int32_t row = -1;
     if (lr >= 0) {
       const int64_t r = base + lr;
-      if (C <= 0 || r < C) row = off + (int32_t)r;
+      const bool keep = cap_e != nullptr ? r < (int64_t)cap_e[e] : (C <= 0 || r < C);
+      if (keep) row = off + (int32_t)r;
     }
-    slot_row[t * k + j] = row;
+    if (slot_row != nullptr) slot_row[t * k + j] = row;
     if (drop_mask_out != nullptr) drop_mask_out[t * k + j] = row < 0 ? 1 : 0;
     if (row >= 0 && row_token != nullptr) row_token[row] = (int32_t)t;
     s_row[j] = row;
@@ -210,7 +215,7 @@ __global__ void __launch_bounds__(32 * kScatterWarps, 8) dispatch_scatter_warp_k
     const int32_t* __restrict__ tile_base, const int32_t* __restrict__ offsets, int64_t N,
     int k, int E, int64_t C, int32_t* __restrict__ slot_row, int32_t* __restrict__ row_token,
     uint8_t* __restrict__ drop_mask_out, const V* __restrict__ x, V* __restrict__ xp,
-    int row_vecs) {
+    int row_vecs, const int32_t* __restrict__ cap_e) {
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * kScatterWarps + (threadIdx.x >> 5);
@@ -224,9 +229,10 @@ __global__ void __launch_bounds__(32 * kScatterWarps, 8) dispatch_scatter_warp_k
     const int32_t off = offsets[e];
     if (lr >= 0) {
       const int64_t r = base + lr;
-      if (C <= 0 || r < C) row = off + (int32_t)r;
+      const bool keep = cap_e != nullptr ? r < (int64_t)cap_e[e] : (C <= 0 || r < C);
+      if (keep) row = off + (int32_t)r;
     }
-    slot_row[t * k + lane] = row;
+    if (slot_row != nullptr) slot_row[t * k + lane] = row;
     if (drop_mask_out != nullptr) drop_mask_out[t * k + lane] = row < 0 ? 1 : 0;
     if (row >= 0 && row_token != nullptr) row_token[row] = (int32_t)t;
   }
@@ -306,11 +312,11 @@ cudaError_t launch_rank_local(const int32_t* ids, const uint8_t* drop_mask, int6
 cudaError_t launch_dispatch_scan(const int32_t* tile_hist, int64_t N, int E, int64_t C,
                                  int32_t* tile_base, int32_t* demand, int32_t* counts,
                                  int32_t* offsets, int32_t* arrive, cudaStream_t stream,
-                                 int* launches) {
+                                 int* launches, const int32_t* cap_e) {
   const int tiles = (int)((N + kRankTile - 1) / kRankTile);
   ++*launches;
   launch_pdl(dispatch_scan_kernel, (E + 31) / 32, 1024, 0, stream, tile_hist, tiles, E, C, tile_base,
-                                                           demand, counts, offsets, arrive);
+                                                           demand, counts, offsets, arrive, cap_e);
   return cudaGetLastError();
 }
 
@@ -319,7 +325,7 @@ cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_ran
                                     int64_t N, int k, int E, int64_t C, int32_t* slot_row,
                                     int32_t* row_token, uint8_t* drop_mask_out,
                                     const void* x, void* xp, int row_bytes,
-                                    cudaStream_t stream, int* launches) {
+                                    cudaStream_t stream, int* launches, const int32_t* cap_e) {
   if (N == 0) return cudaSuccess;
   ++*launches;
   // warp per token when the warps fill every SM several times over and a token moves at
@@ -331,30 +337,30 @@ cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_ran
     if (xp != nullptr && row_bytes % 16 == 0) {
       launch_pdl(dispatch_scatter_warp_kernel<uint4>, grid, block, 0, stream, ids, local_rank,
                  tile_base, offsets, N, k, E, C, slot_row, row_token, drop_mask_out,
-                 (const uint4*)x, (uint4*)xp, row_bytes / 16);
+                 (const uint4*)x, (uint4*)xp, row_bytes / 16, cap_e);
     } else if (xp != nullptr) {
       launch_pdl(dispatch_scatter_warp_kernel<uint32_t>, grid, block, 0, stream, ids,
                  local_rank, tile_base, offsets, N, k, E, C, slot_row, row_token,
-                 drop_mask_out, (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4);
+                 drop_mask_out, (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4, cap_e);
     } else {
       launch_pdl(dispatch_scatter_warp_kernel<uint4>, grid, block, 0, stream, ids, local_rank,
                  tile_base, offsets, N, k, E, C, slot_row, row_token, drop_mask_out, nullptr,
-                 nullptr, 0);
+                 nullptr, 0, cap_e);
     }
     return cudaGetLastError();
   }
   if (xp != nullptr && row_bytes % 16 == 0) {
     launch_pdl(dispatch_scatter_kernel<uint4>, (unsigned)N, 128, 0, stream, ids, local_rank,
                tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
-               (const uint4*)x, (uint4*)xp, row_bytes / 16);
+               (const uint4*)x, (uint4*)xp, row_bytes / 16, cap_e);
   } else if (xp != nullptr) {
     launch_pdl(dispatch_scatter_kernel<uint32_t>, (unsigned)N, 128, 0, stream, ids,
                local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
-               (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4);
+               (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4, cap_e);
   } else {
     launch_pdl(dispatch_scatter_kernel<uint4>, (unsigned)N, 128, 0, stream, ids, local_rank,
                tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out, nullptr,
-               nullptr, 0);
+               nullptr, 0, cap_e);
   }
   return cudaGetLastError();
 }

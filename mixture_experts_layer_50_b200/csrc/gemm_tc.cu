@@ -97,6 +97,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
+// Wait, after an abort, for copies or MMAs this thread already issued (their barrier phase
+// completes when they land); bounded by the same time limit and poll backstop as mbar_wait,
+// and records nothing: the abort is reported already.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint64_t polls = 0; polls <= kWaitMaxPolls; ++polls)
+    if (mbar_try_wait(bar, parity) || global_timer_ns() - t0 >= kWaitLimitNs) return;
+}
+
 // ---- TMA -----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1) {
@@ -522,9 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < STAGES && i < armed; ++i) {
           stage = (stage + STAGES - 1) % STAGES;
           if (stage == STAGES - 1) phase ^= 1;
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(&full[stage], phase) && global_timer_ns() - t0 < kWaitLimitNs) {
-          }
+          mbar_drain(&full[stage], phase);
         }
       }
     }
@@ -576,9 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) {
         // wait for the MMAs already issued before TMEM is released
         mma_commit(drain);
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
+        mbar_drain(drain, 0);
       }
     }
   } else {
@@ -766,9 +771,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int i = 0; i < STAGES && i < armed; ++i) {
           stage = (stage + STAGES - 1) % STAGES;
           if (stage == STAGES - 1) phase ^= 1;
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(&full[stage], phase) && global_timer_ns() - t0 < kWaitLimitNs) {
-          }
+          mbar_drain(&full[stage], phase);
         }
       }
     }
@@ -813,9 +816,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         mma_commit_pair_local(drain);
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
+        mbar_drain(drain, 0);
       }
     }
   } else {
@@ -1048,9 +1049,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < STAGES && i < armed; ++i) {
           stage = (stage + STAGES - 1) % STAGES;
           if (stage == STAGES - 1) phase ^= 1;
-          const uint64_t t0 = global_timer_ns();
-          while (!mbar_try_wait(&full[stage], phase) && global_timer_ns() - t0 < kWaitLimitNs) {
-          }
+          mbar_drain(&full[stage], phase);
         }
       }
     }
@@ -1098,9 +1097,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) {
         mma_commit(drain);
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(drain, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
+        mbar_drain(drain, 0);
       }
     }
   } else {

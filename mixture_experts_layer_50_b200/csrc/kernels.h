@@ -41,20 +41,23 @@ cudaError_t launch_route_hash(const int32_t* token_ids, int64_t N, int E, int k,
 cudaError_t launch_rank_local(const int32_t* ids, const uint8_t* drop_mask, int64_t N, int k,
                               int E, int32_t* local_rank, int32_t* tile_hist, int* status,
                               cudaStream_t stream, int* launches);
-// Pass 2: scan over tiles and experts: tile_base, demand, counts (capped at C when C > 0)
-// and offsets (exclusive scan of counts, E + 1 entries).
+// Pass 2: scan over tiles and experts: tile_base, demand, counts (capped at C when C > 0,
+// or at cap_e[e] per expert when cap_e is not null) and offsets (exclusive scan of counts,
+// E + 1 entries).
 cudaError_t launch_dispatch_scan(const int32_t* tile_hist, int64_t N, int E, int64_t C,
                                  int32_t* tile_base, int32_t* demand, int32_t* counts,
                                  int32_t* offsets, int32_t* arrive, cudaStream_t stream,
-                                 int* launches);
-// Pass 3: capacity decision, slot rows, row -> token map, drop mask, and (when xp is not
-// null) the gather of x rows into the per-expert layout.
+                                 int* launches, const int32_t* cap_e = nullptr);
+// Pass 3: capacity decision (rank < C, or rank < cap_e[e] when cap_e is not null), slot
+// rows (when slot_row is not null), row -> token map, drop mask, and (when xp is not null)
+// the gather of x rows into the per-expert layout.
 cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_rank,
                                     const int32_t* tile_base, const int32_t* offsets,
                                     int64_t N, int k, int E, int64_t C, int32_t* slot_row,
                                     int32_t* row_token, uint8_t* drop_mask_out,
                                     const void* x, void* xp, int row_bytes,
-                                    cudaStream_t stream, int* launches);
+                                    cudaStream_t stream, int* launches,
+                                    const int32_t* cap_e = nullptr);
 
 // ---- balancing statistics (balance.cu) ------------------------------------------------
 // f [E] share of assignments, P [E] mean router probability, aux = E sum f P, set_load

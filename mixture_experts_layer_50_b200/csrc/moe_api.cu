@@ -128,6 +128,16 @@ Ws layout(const moe_config& c) {
   return w;
 }
 
+// The workspace of an expert-parallel rank: the layout of the same layer over world * N
+// tokens, so that the owner's grouped GEMMs can take every row the ranks may send it (each
+// token sends at most one row per expert, so at most world * N * k rows arrive).
+moe_config ep_ws_config(const moe_config& c, int32_t world) {
+  moe_config w = c;
+  w.N = c.N * world;
+  w.capacity = 0;
+  return w;
+}
+
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
@@ -304,7 +314,7 @@ moe_status stage_dispatch(const moe_config& c, const Ws& L, void* ws, const int3
                           const uint8_t* drop_in, int64_t C, int32_t* demand, int32_t* counts,
                           int32_t* offsets, int32_t* slot_row, int32_t* row_token,
                           uint8_t* drop_out, const void* x, void* xp, cudaStream_t st,
-                          int* launches) {
+                          int* launches, const int32_t* cap_e = nullptr) {
   int* status = at<int>(ws, L.status);
   MOE_CUDA(moe::launch_rank_local(ids, drop_in, c.N, c.k, c.E, at<int32_t>(ws, L.local_rank),
                                   at<int32_t>(ws, L.tile_hist), status, st, launches),
@@ -312,13 +322,13 @@ moe_status stage_dispatch(const moe_config& c, const Ws& L, void* ws, const int3
   prof_mark(st);
   MOE_CUDA(moe::launch_dispatch_scan(at<int32_t>(ws, L.tile_hist), c.N, c.E, C,
                                      at<int32_t>(ws, L.tile_base), demand, counts, offsets,
-                                     arrive_counter(ws, L), st, launches),
+                                     arrive_counter(ws, L), st, launches, cap_e),
            "scan pass");
   prof_mark(st);
   MOE_CUDA(moe::launch_dispatch_scatter(ids, at<int32_t>(ws, L.local_rank),
                                         at<int32_t>(ws, L.tile_base), offsets, c.N, c.k, c.E, C,
                                         slot_row, row_token, drop_out, x, xp,
-                                        (int)(c.d * el_size(c)), st, launches),
+                                        (int)(c.d * el_size(c)), st, launches, cap_e),
            "scatter pass");
   prof_mark(st);
   return MOE_OK;
@@ -945,6 +955,104 @@ moe_status moe_forward_padded(const moe_config* cfg, const void* x, const void* 
   return MOE_OK;
 }
 
+// ---- expert parallelism ("Le problème — Communication", "L'idée — Communication") ----------
+size_t moe_ep_workspace_size(const moe_config* cfg, int32_t world) {
+  if (world < 1 || check_cfg(cfg) != MOE_OK || world > cfg->E) return 0;
+  const moe_config w = ep_ws_config(*cfg, world);
+  if (check_cfg(&w) != MOE_OK) return 0;
+  return layout(w).total;
+}
+
+moe_status moe_permute_ep(const moe_config* cfg, const int32_t* ids, const int32_t* cap,
+                          const void* x, int32_t* offsets, int32_t* row_token, int32_t* slot_row,
+                          void* xp, int32_t* counts, uint8_t* drop_mask, void* ws,
+                          moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  if (ids == nullptr || cap == nullptr || offsets == nullptr || slot_row == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "ids, cap, offsets and slot_row are required");
+  MOE_TRY(need(x, "x"));
+  MOE_TRY(need(xp, "xp"));
+  const moe_config& c = *cfg;
+  const Ws L = layout(c);
+  int launches = 0;
+  MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, 0, at<int32_t>(ws, L.demand),
+                         counts != nullptr ? counts : at<int32_t>(ws, L.counts), offsets,
+                         slot_row, row_token,
+                         drop_mask != nullptr ? drop_mask : at<uint8_t>(ws, L.drop_mask), x, xp,
+                         (cudaStream_t)stream, &launches, cap));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_ep_expert_ffn(const moe_config* cfg, int32_t world, int32_t rank,
+                             int64_t n_tokens, int64_t rows, const void* xr,
+                             const int32_t* offsets, const void* x, const void* W_gu,
+                             const void* W_down, void* ye, void* y, void* ws,
+                             moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  if (world < 1 || rank < 0 || rank >= world)
+    return fail(MOE_ERR_INVALID_ARG, "rank must be in [0, world)");
+  if (world > cfg->E) return fail(MOE_ERR_UNSUPPORTED, "more ranks than experts");
+  if (cfg->dtype != MOE_DT_BF16)
+    return fail(MOE_ERR_UNSUPPORTED, "the expert-parallel FFN is bf16 only");
+  if (n_tokens < 0 || n_tokens > cfg->N)
+    return fail(MOE_ERR_INVALID_ARG, "n_tokens must be in [0, cfg->N]");
+  if (rows < 0 || rows > cfg->N * (int64_t)world * cfg->k)
+    return fail(MOE_ERR_INVALID_ARG, "rows must be in [0, world * N * k]");
+  if (offsets == nullptr) return fail(MOE_ERR_INVALID_ARG, "offsets is NULL");
+  if (rows > 0) {
+    MOE_TRY(need(xr, "xr"));
+    MOE_TRY(need(ye, "ye"));
+  }
+  if (cfg->n_shared && n_tokens > 0) {
+    MOE_TRY(need(x, "x"));
+    MOE_TRY(need(y, "y"));
+  }
+  MOE_TRY(need(W_gu, "W_gu"));
+  MOE_TRY(need(W_down, "W_down"));
+  const int32_t e0 = moe_ep_first_expert(world, rank, cfg->E);
+  const int32_t e1 = moe_ep_first_expert(world, rank + 1, cfg->E);
+  moe_config c = *cfg;  // the owned experts as the layer's routed experts, this call's tokens
+  c.E = e1 - e0;
+  c.N = n_tokens;
+  c.capacity = 0;
+  if (c.N == 0) {
+    // no tokens of its own (no shared rows), but the owner may still have received rows;
+    // N only sizes the shared group and the rows-per-expert estimate of the kernel choice
+    c.n_shared = 0;
+    c.N = std::max<int64_t>(1, (rows + c.k - 1) / c.k);
+  }
+  const Ws L = layout(ep_ws_config(*cfg, world));
+  int launches = 0;
+  if (rows == 0 && c.n_shared == 0) return MOE_OK;
+  // routed groups: the received rows [offsets[i], offsets[i+1]) of owned expert e0 + i; the
+  // shared expert runs on this rank's own tokens and writes its rows into y
+  MOE_TRY(stage_ffn(c, L, ws, rows > 0 ? xr : x, offsets, x, W_gu, W_down, rows > 0 ? ye : y,
+                    (cudaStream_t)stream, &launches, rows, c.n_shared ? y : nullptr));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_ep_combine(const moe_config* cfg, const void* ye, const int32_t* slot_row,
+                          const float* gates, void* y, moe_stream_t stream) {
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  if (cfg->dtype != MOE_DT_BF16) return fail(MOE_ERR_UNSUPPORTED, "the expert-parallel combine is bf16 only");
+  MOE_TRY(need(ye, "ye"));
+  MOE_TRY(need(y, "y"));
+  if (slot_row == nullptr || gates == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "slot_row and gates are required");
+  int launches = 0;
+  MOE_TRY(stage_combine(*cfg, ye, slot_row, gates, y, (cudaStream_t)stream, &launches, -1,
+                        cfg->n_shared != 0));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
 moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const void* W_g,
                             const float* logit_offset, const float* bias,
                             const uint8_t* modality, const void* W_gu, const void* W_down,
@@ -1057,17 +1165,40 @@ __device__ __align__(256) unsigned char g_route_scratch[kStaticScratchBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+void* g_scratch_ctx[kMaxDevices] = {};  // the context the address was looked up in
 
-// Device address of g_route_scratch on the current device (looked up once per device).
+// The current driver context (cuCtxGetCurrent through the runtime's entry-point lookup, so
+// the library does not link libcuda); nullptr if it cannot be read.
+void* current_context() {
+  using Fn = int (*)(void**);
+  static Fn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<Fn>(p);
+  });
+  void* ctx = nullptr;
+  if (fn == nullptr || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
+// Device address of g_route_scratch on the current device: looked up once per device and
+// context (a device reset or another context on the device loads the module anew, at a new
+// address, so the lookup is repeated then).
 moe_status static_scratch(void** out) {
   int dev = 0;
   MOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device ordinal >= 64");
+  void* ctx = current_context();
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (g_scratch_addr[dev] == nullptr || ctx == nullptr || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     MOE_CUDA(cudaGetSymbolAddress(&p, g_route_scratch), "cudaGetSymbolAddress(route scratch)");
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = current_context();
   }
   *out = g_scratch_addr[dev];
   return MOE_OK;
@@ -1096,12 +1227,11 @@ moe_status moe_route_static(const moe_config* cfg, const float* logits, const fl
     off = align_up(off + bytes, 256);
     return o;
   };
-  // o_arrive: the scan's ticket counter; zero when the module loads, and every scan leaves
-  // it at zero
+  // o_arrive: the scan's ticket counter, set to zero by every call before its scan (so an
+  // earlier overlapping call that raced on it cannot leave it wrong for later ones)
   const size_t o_arrive = take(256);
   const size_t o_rank = take(Nk * 4), o_hist = take(tiles * c.E * 4),
-               o_base = take(tiles * c.E * 4), o_offs = take(((size_t)c.E + 1) * 4),
-               o_slot = take(Nk * 4);
+               o_base = take(tiles * c.E * 4), o_offs = take(((size_t)c.E + 1) * 4);
   if (off > kStaticScratchBytes) {
     char buf[160];
     snprintf(buf, sizeof(buf), "moe_route_static needs %zu bytes of scratch; its static array holds %zu",
@@ -1112,6 +1242,8 @@ moe_status moe_route_static(const moe_config* cfg, const float* logits, const fl
   MOE_TRY(static_scratch(&scratch));
   cudaStream_t st = (cudaStream_t)stream;
   int launches = 0;
+  MOE_CUDA(cudaMemsetAsync(at<int32_t>(scratch, o_arrive), 0, sizeof(int32_t), st),
+           "clear the scan ticket");
   MOE_TRY(stage_route(c, finished_logits(logits), bias, modality, ids, gates, status, st,
                       &launches));
   MOE_CUDA(moe::launch_rank_local(ids, nullptr, c.N, c.k, c.E, at<int32_t>(scratch, o_rank),
@@ -1125,8 +1257,8 @@ moe_status moe_route_static(const moe_config* cfg, const float* logits, const fl
   MOE_CUDA(moe::launch_dispatch_scatter(ids, at<int32_t>(scratch, o_rank),
                                         at<int32_t>(scratch, o_base),
                                         at<int32_t>(scratch, o_offs), c.N, c.k, c.E,
-                                        c.capacity, at<int32_t>(scratch, o_slot), nullptr,
-                                        drop_mask, nullptr, nullptr, 0, st, &launches),
+                                        c.capacity, nullptr, nullptr, drop_mask, nullptr,
+                                        nullptr, 0, st, &launches),
            "scatter pass");
   g_last_launches = launches;
   return MOE_OK;

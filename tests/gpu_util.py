@@ -76,14 +76,62 @@ def assert_close_layer(got, ref, bf16=True):
         assert err <= 1e-4, err
 
 
-def fragile_tokens(logits_o, logits_g, k, score_fn, bias=None, modality=None):
-    """Tokens whose top-k set could change under the observed logit discrepancy."""
+def _key_gaps(logits_o, logits_g, score_fn, bias, modality):
     eps = 8 * float(np.abs(logits_g.astype(np.float64) - logits_o.astype(np.float64)).max()) + 1e-6
     keys = O.selection_keys(logits_o, score_fn, bias, modality).astype(np.float64)
     if score_fn == O.SIGMOID:
         eps = eps * 0.25 + 1e-6          # |d sigma / dz| <= 1/4
     srt = -np.sort(-keys, axis=1)
-    if k >= keys.shape[1]:
-        return np.zeros(keys.shape[0], bool)
-    gap = srt[:, k - 1] - srt[:, k]
-    return gap <= 2 * eps
+    return srt[:, :-1] - srt[:, 1:], eps
+
+
+def fragile_tokens(logits_o, logits_g, k, score_fn, bias=None, modality=None):
+    """Tokens whose top-k set could change under the observed logit discrepancy: the k-th
+    and (k+1)-th largest keys lie within twice the largest possible key error."""
+    if k >= logits_o.shape[1]:
+        return np.zeros(logits_o.shape[0], bool)
+    gaps, eps = _key_gaps(logits_o, logits_g, score_fn, bias, modality)
+    return gaps[:, k - 1] <= 2 * eps
+
+
+def order_fragile_tokens(logits_o, logits_g, k, score_fn, bias=None, modality=None):
+    """Tokens whose slot order (descending key) could change: two of the k largest keys lie
+    within twice the largest possible key error."""
+    if k < 2:
+        return np.zeros(logits_o.shape[0], bool)
+    gaps, eps = _key_gaps(logits_o, logits_g, score_fn, bias, modality)
+    return (gaps[:, :k - 1] <= 2 * eps).any(axis=1)
+
+
+def explain_routing_differences(route_g, info, logits_o, logits_g, k, score_fn, bias=None,
+                                modality=None, capacity=0):
+    """Checks that every token routed differently from independently computed logits is
+    explained by the logit discrepancy, and returns the mask of tokens routed alike.
+
+    * a token whose expert *set* differs must be fragile (its k-th and (k+1)-th keys within
+      the key error);
+    * a token with the same set in another slot order must be order-fragile;
+    * a token with the same ids but another drop mask is a capacity knock-on: an expert that
+      a token leaves (and the one it joins instead) sees every later token's rank move by
+      one, which moves its keep/drop boundary by one token, so there are at most two such
+      tokens per expert exchanged (none without a capacity).  Ranks count demand, not kept
+      rows, so knock-ons do not chain.
+    """
+    ids_g, ids_o = np.asarray(route_g["ids"]), np.asarray(info["ids"])
+    same_ids = (ids_g == ids_o).all(1)
+    same_set = (np.sort(ids_g, 1) == np.sort(ids_o, 1)).all(1)
+    same_drop = (np.asarray(route_g["drop_mask"]) == np.asarray(info["drop_mask"])).all(1)
+    frag = fragile_tokens(logits_o, logits_g, k, score_fn, bias, modality)
+    ofrag = order_fragile_tokens(logits_o, logits_g, k, score_fn, bias, modality)
+    set_changed = ~same_set
+    assert frag[set_changed].all(), np.nonzero(set_changed & ~frag)[0][:10]
+    assert ofrag[same_set & ~same_ids].all(), np.nonzero(same_set & ~same_ids & ~ofrag)[0][:10]
+    knock_on = same_ids & ~same_drop
+    # experts a changed token left (each such move also adds one expert it joined)
+    moves = sum(len(set(ids_o[t].tolist()) - set(ids_g[t].tolist()))
+                for t in np.nonzero(set_changed)[0])
+    allowed = 2 * moves if capacity > 0 else 0
+    assert int(knock_on.sum()) <= allowed, (int(knock_on.sum()), moves)
+    return same_ids & same_drop, dict(set_changed=int(set_changed.sum()),
+                                      order_changed=int((same_set & ~same_ids).sum()),
+                                      knock_on=int(knock_on.sum()), fragile=int(frag.sum()))

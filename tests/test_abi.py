@@ -227,3 +227,30 @@ def test_ffn_kernel_override(nat, path, kind, monkeypatch):
     monkeypatch.delenv("MOE_B200_GEMM_PATH")
     got = nat.moe_ffn_kernels(nat.config_from_shape(W.PRESETS["capacity-cf1"]))
     assert "2-SM" in got[0] and "2-SM" in got[1]
+
+
+def test_expert_parallel_entry_points_validate_on_host(nat):
+    """The expert-parallel calls reject bad arguments before touching the GPU."""
+    fake = ctypes.c_void_p(0x100000)
+    lib = nat.lib
+    c = _cfg(nat)
+    assert nat.moe_ep_workspace_size(c, 1) >= nat.moe_workspace_size(c)
+    assert nat.moe_ep_workspace_size(c, 2) > nat.moe_workspace_size(c)
+    assert nat.moe_ep_workspace_size(c, c.E + 1) == 0          # more ranks than experts
+    assert nat.moe_ep_workspace_size(c, 0) == 0
+    # moe_permute_ep: the per-expert capacity is required
+    assert lib.moe_permute_ep(ctypes.byref(c), fake, None, fake, fake, None, fake, fake, None,
+                              None, fake, None) == nat.MOE_ERR_INVALID_ARG
+    # moe_ep_expert_ffn: rank range, token count, row bound, offsets
+    args = lambda world, rank, n, rows, off: (ctypes.byref(c), world, rank, n, rows, fake, off,
+                                              fake, fake, fake, fake, fake, fake, None)
+    assert lib.moe_ep_expert_ffn(*args(2, 2, 1, 1, fake)) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_expert_ffn(*args(2, 0, c.N + 1, 1, fake)) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_expert_ffn(*args(2, 0, 1, 2 * c.N * c.k + 1, fake)) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_expert_ffn(*args(2, 0, 1, 1, None)) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_expert_ffn(*args(c.E + 1, 0, 1, 1, fake)) == nat.MOE_ERR_UNSUPPORTED
+    f32 = nat.make_config(c.N, 64, c.E, c.k, 64, dtype=nat.F32)
+    assert lib.moe_ep_expert_ffn(ctypes.byref(f32), 1, 0, 1, 1, fake, fake, fake, fake, fake,
+                                 fake, fake, fake, None) == nat.MOE_ERR_UNSUPPORTED
+    assert lib.moe_ep_combine(ctypes.byref(c), fake, None, fake, fake, None) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_combine(ctypes.byref(f32), fake, fake, fake, fake, None) == nat.MOE_ERR_UNSUPPORTED

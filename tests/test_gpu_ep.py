@@ -1,0 +1,178 @@
+"""Expert-parallel layer on one GPU: the library's kernels on the per-rank layouts.
+
+"Mixture-of-Experts : routage et capacité" slides, "L'idée — Communication".  A run here has one
+GPU, so several ranks are emulated in one process: each emulated rank has its own layer object
+(its experts, its workspace) and the row exchange is ``loopback_exchange`` (plain copies between
+the ranks' buffers, in the plan's runs).  No kernel waits on another rank.  The result must equal
+the single-device layer over the concatenated batch: bit for bit against the fused call given
+the same routing, and within the bf16 bar against the oracle.
+"""
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from gpu_util import assert_close_layer, check_status, f64, host
+from mixture_experts_layer_50_b200 import _native as nat
+from mixture_experts_layer_50_b200 import workloads as W
+from mixture_experts_layer_50_b200.ep import EPMoELayer, loopback_exchange
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _needs_cuda(cuda_dev):
+    yield
+
+
+def _layers(shape, t, world, max_tokens, cf):
+    return [EPMoELayer.from_full_weights(
+        W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], k=shape.k, E=shape.E, world=world,
+        rank=r, n_shared=shape.n_shared, score_fn=shape.score_fn, renorm=shape.renorm,
+        act=shape.act, clamp=shape.clamp, bias=t.get("bias"), logit_offset=t.get("logit_offset"),
+        capacity_factor=cf, max_tokens=max_tokens) for r in range(world)]
+
+
+def emulate(layers, xs, mods):
+    """Every phase of the layer for all emulated ranks, the exchanges by loopback copies."""
+    world = len(layers)
+    dem = [L.route(x, m) for L, x, m in zip(layers, xs, mods)]
+    gathered = torch.stack(dem).cpu()
+    plans = [L.set_plan(gathered) for L in layers]
+    sends = [L.permute(x) for L, x in zip(layers, xs)]
+    recv = [L.new_recv_buffer() for L in layers]
+    loopback_exchange(sends, recv, [p["sends"] for p in plans], [p["recvs"] for p in plans])
+    ys = [torch.empty_like(x) for x in xs]
+    ye = [L.run_experts(r, x, y) for L, r, x, y in zip(layers, recv, xs, ys)]
+    back = [L.new_return_buffer() for L in layers]
+    loopback_exchange(ye, back, [p["recvs"] for p in plans], [p["sends"] for p in plans])
+    for L, b, y in zip(layers, back, ys):
+        L.combine(b, y)
+        check_status(L.ws)
+    return ys, plans
+
+
+def _split(N, world, seed, empty_rank=None):
+    rng = np.random.default_rng(seed)
+    cuts = np.sort(rng.integers(N // 8, N - N // 8, world - 1)) if world > 1 else np.zeros(0, int)
+    sizes = np.diff(np.r_[0, cuts, N]).astype(int)
+    if empty_rank is not None and world > 1:
+        other = (empty_rank + 1) % world
+        sizes[other] += sizes[empty_rank]
+        sizes[empty_rank] = 0
+    return sizes
+
+
+CASES = [
+    # preset, N, d, E, F, k, cf
+    ("capacity-cf1", 600, 256, 16, 256, 2, 1),
+    ("dsv3-n64", 500, 256, 24, 128, 4, None),
+    ("v41flash-n64", 700, 512, 30, 256, 3, 1.25),
+    ("mixtral-n16", 400, 256, 8, 384, 2, None),
+    ("switch-cf1", 512, 128, 12, 128, 1, 1),
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_one_rank_equals_the_fused_layer_bit_for_bit(case):
+    """world = 1: route, plan, permute, a local exchange, the experts and the combine give
+    moe_forward's output bits (and moe_forward_padded's, with a capacity)."""
+    name, N, d, E, F, k, cf = case
+    shape = W.PRESETS[name].replace(N=N, d=d, E=E, F=F, k=k)
+    t = W.make_inputs(shape, device="cuda")
+    C = O.capacity(N, k, E, cf)
+    (L,) = _layers(shape, t, 1, N, cf)
+    (y_ep,), _ = emulate([L], [t["x"]], [t.get("modality")])
+    cfg = nat.config_from_shape(shape, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    y = torch.empty_like(t["x"])
+    kw = dict(x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y,
+              logit_offset=t.get("logit_offset"), bias=t.get("bias"), modality=t.get("modality"),
+              ws=ws)
+    nat.moe_forward(cfg, **kw)
+    check_status(ws)
+    assert torch.equal(y_ep, y)
+    if C > 0:
+        nat.moe_forward_padded(cfg, **kw)
+        check_status(ws)
+        assert torch.equal(y_ep, y)
+
+
+@pytest.mark.parametrize("world", [2, 3, 4])
+@pytest.mark.parametrize("case", CASES)
+def test_emulated_ranks_equal_the_single_device_layer(world, case, monkeypatch):
+    """Several emulated ranks (one without tokens in some cases): every rank's output equals,
+    bit for bit, the fused layer over the concatenated batch given the same routing
+    (moe_forward_routed: the ranks' own ids and gates, capacity in the concatenated token
+    order), and the oracle within the bf16 bar; the drop masks equal the oracle's."""
+    monkeypatch.setenv("MOE_B200_GEMM_PATH", "1sm")       # one GEMM kernel on both sides
+    name, N, d, E, F, k, cf = case
+    shape = W.PRESETS[name].replace(N=N, d=d, E=E, F=F, k=k)
+    if world > E:
+        pytest.skip("more ranks than experts")
+    t = W.make_inputs(shape, device="cuda")
+    sizes = _split(N, world, seed=world * 31 + E, empty_rank=1 if world == 3 else None)
+    starts = np.r_[0, np.cumsum(sizes)]
+    xs = [t["x"][starts[r]:starts[r + 1]] for r in range(world)]
+    mod = t.get("modality")
+    mods = [None if mod is None else mod[starts[r]:starts[r + 1]] for r in range(world)]
+    layers = _layers(shape, t, world, int(sizes.max()) if sizes.max() > 0 else 1, cf)
+    ys, plans = emulate(layers, xs, mods)
+    y_ep = torch.cat(ys)
+    ids = torch.cat([L.ids[:L.N] for L in layers])
+    gates = torch.cat([L.gates[:L.N] for L in layers])
+    drop = torch.cat([L.drop_mask[:L.N] for L in layers])
+    C = O.capacity(N, k, E, cf)
+    assert all(p["capacity"] == C for p in plans)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    y = torch.empty_like(t["x"])
+    ro = dict(drop_mask=torch.empty((N, k), dtype=torch.uint8, device="cuda"))
+    nat.moe_forward_routed(cfg, x=t["x"], ids=ids, gates=gates, W_gu=t["W_gu"],
+                           W_down=t["W_down"], y=y, route_out=ro, ws=ws)
+    check_status(ws)
+    assert torch.equal(drop, ro["drop_mask"])
+    assert torch.equal(y_ep, y)
+    # the oracle on the same routing (the ranks' ids and gates), capacity in token order
+    ref, info = O.forward(f64(t["x"]), None, f64(t["W_gu"]), f64(t["W_down"]), k=k, E=E,
+                          n_shared=shape.n_shared, act=shape.act, clamp=shape.clamp,
+                          ids=host(ids), gates=host(gates).astype(np.float64), C=C)
+    np.testing.assert_array_equal(host(drop), info["drop_mask"])
+    assert_close_layer(host(y_ep), ref)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_forward_over_a_one_rank_nccl_group():
+    """EPMoELayer.forward itself (NCCL all-gather of the demands, the row exchange) on a
+    one-rank NCCL group equals moe_forward bit for bit."""
+    import torch.distributed as dist
+    shape = W.PRESETS["v41flash-n64"].replace(N=300, d=256, E=16, F=128, k=4)
+    t = W.make_inputs(shape, device="cuda")
+    store = dist.TCPStore("127.0.0.1", _free_port(), 1, True,
+                          timeout=datetime.timedelta(seconds=60))
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        (L,) = _layers(shape, t, 1, shape.N, 1.25)
+        y_ep = L.forward(t["x"], modality=t["modality"])
+        assert L.check_status() == 0
+    finally:
+        dist.destroy_process_group()
+    C = O.capacity(shape.N, shape.k, shape.E, 1.25)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    y = torch.empty_like(t["x"])
+    nat.moe_forward(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y,
+                    bias=t["bias"], modality=t["modality"], ws=ws)
+    check_status(ws)
+    assert torch.equal(y_ep, y)

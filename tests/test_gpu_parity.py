@@ -13,7 +13,7 @@ import torch
 
 import oracle as O
 from gpu_util import (assert_close_layer, assert_route_equal, check_status, dev, err_stats,
-                      f64, fragile_tokens, gpu_route, host)
+                      explain_routing_differences, f64, fragile_tokens, gpu_route, host)
 from golden.reader import load
 from mixture_experts_layer_50_b200 import _native as nat
 from mixture_experts_layer_50_b200 import workloads as W
@@ -365,7 +365,40 @@ def test_forward_toy_fp32_page_config():
     assert launches == 8
 
 
-def _forward_case(name, N=None, sample=None, tol_rows=None):
+def tile_edge_tokens(route, N, n_shared, tile_rows=(128, 256)):
+    """Tokens that sit at the edges of the grouped GEMMs' M tiles: for every expert with kept
+    rows, the first and last row of its first tile and of its last tile (for 128- and
+    256-row tiles), and for the shared expert (all N tokens in token order) the tokens at
+    the same edges of its tiles."""
+    off = np.asarray(route["offsets"], np.int64)
+    row_token = np.asarray(route["row_token"], np.int64)
+    toks = []
+    for e in range(off.size - 1):
+        r0, r1 = int(off[e]), int(off[e + 1])
+        if r1 == r0:
+            continue
+        cnt = r1 - r0
+        for tr in tile_rows:
+            last_base = (cnt - 1) // tr * tr
+            for r in (0, min(tr, cnt) - 1, last_base, cnt - 1):
+                toks.append(row_token[r0 + r])
+    if n_shared:
+        for tr in tile_rows:
+            last_base = (N - 1) // tr * tr
+            toks += [0, min(tr, N) - 1, last_base, N - 1]
+    return np.unique(np.asarray(toks, np.int64))
+
+
+def full_range_sample(route, N, n_shared, seed=0, n_random=96):
+    """Tile-edge tokens plus a seeded uniform draw over the whole token range, the last
+    tokens (the last arrivals, the first to be dropped under a capacity) included."""
+    rng = np.random.default_rng(seed)
+    extra = rng.integers(0, N, n_random) if N > 0 else np.zeros(0, np.int64)
+    tail = np.arange(max(0, N - 8), N)
+    return np.unique(np.r_[tile_edge_tokens(route, N, n_shared), extra, tail]).astype(np.int64)
+
+
+def _forward_case(name, N=None, sample=None, full_range=False):
     shape = W.PRESETS[name]
     if N is not None:
         shape = shape.replace(N=N)
@@ -378,19 +411,22 @@ def _forward_case(name, N=None, sample=None, tol_rows=None):
     z_o = O.router_logits(x64, f64(t["W_g"]), off)
     zerr = np.abs(ro["logits"].astype(np.float64) - z_o).max()
     assert zerr <= 1e-3 * np.abs(z_o).max(), zerr
-    tokens = np.arange(shape.N) if sample is None else sample
     kw = _oracle_kwargs(shape, t, C)
+    kw_no_off = {k: v for k, v in kw.items() if k != "logit_offset"}
+    if full_range:
+        # routing of every token first (cheap), then the rows at every tile edge of the
+        # oracle's own layout and a draw over the whole token range
+        ids_o, _ = O.route(z_o, shape.k, shape.score_fn, shape.renorm, kw["bias"], kw["modality"])
+        sample = full_range_sample(O.dispatch(ids_o, shape.E, C), shape.N, shape.n_shared,
+                                   seed=shape.seed)
+    tokens = np.arange(shape.N) if sample is None else np.asarray(sample, np.int64)
     ref, info = O.forward(x64, f64(t["W_g"]), _LazyF64(t["W_gu"]), _LazyF64(t["W_down"]),
-                          tokens=tokens, logits=z_o, **{k: v for k, v in kw.items()
-                                                        if k != "logit_offset"})
+                          tokens=tokens, logits=z_o, **kw_no_off)
     # Routing from the GPU's logits may differ from routing on float64 logits only where the
-    # top-k decision sits within the logit discrepancy ("fragile" tokens); with a capacity, a
-    # flip can move the keep/drop boundary of the two experts involved.
-    frag = fragile_tokens(z_o, ro["logits"], shape.k, shape.score_fn, kw["bias"], kw["modality"])
-    same_tok = (ro["ids"] == info["ids"]).all(1) & (ro["drop_mask"] == info["drop_mask"]).all(1)
+    # logit discrepancy can explain it (fragile tokens and their capacity knock-ons)
+    same_tok, why = explain_routing_differences(ro, info, z_o, ro["logits"], shape.k,
+                                                shape.score_fn, kw["bias"], kw["modality"], C)
     n_diff = int((~same_tok).sum())
-    assert n_diff <= 3 * int(frag.sum()), (n_diff, int(frag.sum()))
-    assert n_diff <= max(2, shape.N // 200), n_diff
     if n_diff == 0:
         np.testing.assert_array_equal(ro["counts"], info["counts"])
         np.testing.assert_array_equal(ro["offsets"], info["offsets"])
@@ -398,7 +434,9 @@ def _forward_case(name, N=None, sample=None, tol_rows=None):
     assert keep.mean() > 0.9
     mx, rms = err_stats(host(y)[tokens][keep], ref[keep])
     print(f"PARITY {name} N={shape.N}: logit err {zerr:.2e}, routing differs on {n_diff} "
-          f"tokens ({int(frag.sum())} fragile), output max err {mx:.2e} x max|ref|, rms {rms:.2e}")
+          f"tokens ({why}), {int(keep.sum())} sampled rows compared, token range "
+          f"{int(tokens.min()) if tokens.size else -1}..{int(tokens.max()) if tokens.size else -1}, "
+          f"output max err {mx:.2e} x max|ref|, rms {rms:.2e}")
     assert_close_layer(host(y)[tokens][keep], ref[keep])
     assert launches == 8
     return ro
@@ -411,7 +449,8 @@ class _LazyF64:
         self.t = t
 
     def __getitem__(self, e):
-        return f64(self.t[e])
+        # bf16 -> float64 is exact; widening on the device makes the copy the only host cost
+        return self.t[e].to(torch.float64).cpu().numpy()
 
 
 def test_forward_small_shapes_all_tokens():
@@ -435,15 +474,15 @@ def test_forward_capacity_configs_reduced():
         _forward_case(name, N=2048, sample=np.r_[0:64, 2000:2048])
 
 
-SAMPLE = np.r_[0:6, 1000:1004, 8185:8192]
-
-
-@pytest.mark.parametrize("name", ["mixtral-n16384", "dsv3-n8192", "v41flash-n16384",
-                                  "capacity-cf1", "switch-cf1.25"])
+@pytest.mark.parametrize("name", ["mixtral-n256", "mixtral-n16384", "dsv3-n8192",
+                                  "v41flash-n16384", "capacity-cf1", "capacity-cf1.25",
+                                  "capacity-cfinf", "switch-cf1", "switch-cf1.25",
+                                  "switch-cfinf"])
 def test_forward_full_size_sampled(name):
-    shape = W.PRESETS[name]
-    sample = SAMPLE[SAMPLE < shape.N]
-    _forward_case(name, sample=sample)
+    """Each preset layer at its stated token count: rows at the edges of every expert's first
+    and last M tile (128- and 256-row tiles), the shared expert's tile edges, the last tokens
+    and a uniform draw over the whole token range, against the oracle."""
+    _forward_case(name, full_range=True)
 
 
 def test_forward_zero_tokens_is_a_no_op():
@@ -664,7 +703,7 @@ def test_forward_random_configurations_wide(seed):
     assert rel.max() <= 1e-5, (shape, rel.max())
     got = host(y)[rows].astype(np.float64)
     if shape.dtype == W.F32:
-        assert np.abs(got - ref).max() <= 1e-4 * max(1.0, np.abs(ref).max()), shape
+        assert np.abs(got - ref).max() <= 1e-4, (shape, np.abs(got - ref).max())
     else:
         assert_close_layer(got, ref)
 

@@ -35,11 +35,20 @@ from mixture_experts_layer_50_b200 import workloads as W  # noqa: E402
 METRIC = "MoE-layer fwd tokens/s and % of bf16 tensor (prefill) or HBM (decode) roofline"
 LAUNCH_NAMES = ["router_gemm", "route_topk", "rank_local", "dispatch_scan", "scatter_gather",
                 "gemm_gate_up", "gemm_down", "combine"]
+# with top-k fused with the rank pass (opt-in, MOE_B200_FUSED_TOPK_RANK=1)
+LAUNCH_NAMES_FUSED = ["router_gemm", "route_topk_rank", "dispatch_scan", "scatter_gather",
+                      "gemm_gate_up", "gemm_down", "combine"]
 # with the "report" overflow policy: the capacity pass, the offers and the final layout
 LAUNCH_NAMES_REROUTE = ["router_gemm", "route_topk", "rank_local", "dispatch_scan",
                         "capacity_pass", "reroute_offer", "rank_offers", "scan_offers",
                         "reroute_accept", "rank_final", "scan_final", "scatter_gather",
                         "gemm_gate_up", "gemm_down", "combine"]
+# a small batch (N <= 256, N k <= 2048) runs the three dispatch passes as one launch
+LAUNCH_NAMES_SMALL = ["router_gemm", "route_topk", "dispatch_small", "gemm_gate_up",
+                      "gemm_down", "combine"]
+LAUNCH_NAMES_REROUTE_SMALL = ["router_gemm", "route_topk", "capacity_pass", "reroute_offer",
+                              "rank_offers", "scan_offers", "reroute_accept", "dispatch_final",
+                              "gemm_gate_up", "gemm_down", "combine"]
 L2_BYTES = 128 << 20          # B200 L2: 126 MB
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -141,6 +150,7 @@ class ClockSampler:
 
     def __init__(self, index):
         self.samples, self.reasons, self.ok = [], set(), False
+        self.power = []
         self.max_mhz = None
         try:
             import pynvml
@@ -157,6 +167,7 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.power.append(self.nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0)
                 get = getattr(self.nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
                     self.nv.nvmlDeviceGetCurrentClocksThrottleReasons
                 r = get(self.h)
@@ -183,7 +194,8 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
                     "samples": len(self.samples)}
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples),
+                "power_w": round(statistics.median(self.power), 1) if self.power else None}
 
 
 def read_traffic(kernel, workload):
@@ -352,7 +364,7 @@ def sweep_entry(name, args, world, rank, local, peaks):
            "bound": lr["bound"], "achieved": achieved, "peak": peak, "unit": unit,
            "frac": lr["frac"], "peak_key": key if lr["bound"] == "tensor" else "hbm_gbs",
            "kept_assignments": lr["kept_assignments"], "experts_touched": lr["experts_touched"],
-           "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")}}
+           "clocks": {k: clocks.get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons", "power_w")}}
     del layer, t, x, y
     torch.cuda.empty_cache()
     return out
@@ -380,13 +392,15 @@ def run_ours(args):
     x, mod = t["x"], t.get("modality")
     y = torch.empty_like(x)
     stream = torch.cuda.current_stream()
-    names = LAUNCH_NAMES_REROUTE if args.overflow == "reroute" and shape.capacity_factor else LAUNCH_NAMES
-
     work = algorithmic_work(shape, route_counts(layer, shape, x, mod))
     for _ in range(args.warmup):
         layer.forward(x, modality=mod, y=y)
     torch.cuda.synchronize()
     per_step_launches = nat.moe_last_launch_count()
+    names = {8: LAUNCH_NAMES, 7: LAUNCH_NAMES_FUSED, 6: LAUNCH_NAMES_SMALL,
+             15: LAUNCH_NAMES_REROUTE,
+             11: LAUNCH_NAMES_REROUTE_SMALL}.get(per_step_launches,
+                                                 [f"launch_{i}" for i in range(per_step_launches)])
 
     # timed region: K replays of the whole layer (the eight launches captured once as a
     # CUDA graph)
@@ -497,7 +511,8 @@ def run_ours(args):
         "gpu_launches": per_step_launches * args.steps,
         "host_enqueue_us_per_step": round(host_us, 1),
         "eager_profiled_ms_per_step": round(eager_ms, 4),
-        "timing": "timed region: K replays of the layer captured as one CUDA graph (8 kernels); "
+        "timing": f"timed region: K replays of the layer captured as one CUDA graph "
+                  f"({per_step_launches} kernels); "
                   "launch_ms and roofline: the same K steps launched eagerly with CUDA events "
                   "between the kernels on the launching stream",
         "clocks": clocks,

@@ -426,6 +426,32 @@ MOE_API moe_status moe_forward_host_batches(const moe_config* cfg, int32_t n_bat
  * outside the range. */
 MOE_API moe_status moe_selftest_wait_timeout(void* ws, int64_t limit_ns, moe_stream_t stream);
 
+/* Debugging aid (the pages have no counterpart): checks a dispatch layout's invariants on
+ * the host -- ids in range and distinct within a token; offsets[0] = 0 and offsets[e+1] -
+ * offsets[e] = counts[e] <= capacity (if > 0) and <= demand[e] (if demand is given); a slot
+ * is dropped iff its slot_row is -1; every kept slot's row lies in its expert's group, rows
+ * are used once and row_token maps them back (if given); kept + dropped = N k; each expert's
+ * rows follow token order and it keeps no token after one it dropped (the capacity rule of
+ * "Mixture-of-Experts : routage et capacité", "L'idée — Capacité").  All arrays in HOST memory
+ * (row_token [offsets[E]] may be NULL, demand may be NULL).  Returns MOE_OK, or
+ * MOE_ERR_INVALID_INPUT with the first broken invariant written to msg (msg_len bytes).
+ * With the environment variable MOE_B200_DEBUG=1 the fused forward calls run this check on
+ * their own layout after the dispatch passes (synchronising the stream: eager calls only). */
+MOE_API moe_status moe_check_dispatch_host(int64_t N, int32_t k, int32_t E, int64_t capacity,
+                                           const int32_t* ids, const uint8_t* drop_mask,
+                                           const int32_t* counts, const int32_t* demand,
+                                           const int32_t* offsets, const int32_t* slot_row,
+                                           const int32_t* row_token, char* msg,
+                                           size_t msg_len);
+
+/* The same check on DEVICE arrays (copied to the host; synchronises `stream`): cfg->N, k, E
+ * and capacity give the shapes and the rule.  The broken invariant is in moe_last_error(). */
+MOE_API moe_status moe_check_dispatch(const moe_config* cfg, const int32_t* ids,
+                                      const uint8_t* drop_mask, const int32_t* counts,
+                                      const int32_t* demand, const int32_t* offsets,
+                                      const int32_t* slot_row, const int32_t* row_token,
+                                      moe_stream_t stream);
+
 /* Synchronise `stream`, read and clear the workspace status word.  Returns MOE_OK or the
  * first device-detected error (MOE_ERR_INVALID_INPUT, MOE_ERR_TIMEOUT) since the last
  * check; MOE_ERR_CUDA if the stream reports an asynchronous CUDA error. */

@@ -93,6 +93,8 @@ lib.moe_ep_workspace_size.restype = _sz
 lib.moe_permute_ep.argtypes = [_cfgp] + [_vp] * 11
 lib.moe_ep_expert_ffn.argtypes = [_cfgp, _i32, _i32, _i64, _i64] + [_vp] * 9
 lib.moe_ep_combine.argtypes = [_cfgp] + [_vp] * 5
+lib.moe_check_dispatch_host.argtypes = [_i64, _i32, _i32, _i64] + [_vp] * 8 + [_sz]
+lib.moe_check_dispatch.argtypes = [_cfgp] + [_vp] * 8
 lib.moe_profile_begin.argtypes = [_i32]
 lib.moe_profile_begin.restype = ctypes.c_int
 lib.moe_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), _i32, ctypes.POINTER(_i32)]
@@ -104,7 +106,8 @@ for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "
            "moe_forward_routed", "moe_route_hash", "moe_balance", "moe_permute_padded",
            "moe_forward_padded", "moe_forward_host_batches", "moe_route_reroute",
            "moe_forward_reroute", "moe_selftest_wait_timeout", "moe_ffn_kernels", "moe_ep_plan",
-           "moe_permute_ep", "moe_ep_expert_ffn", "moe_ep_combine"):
+           "moe_permute_ep", "moe_ep_expert_ffn", "moe_ep_combine", "moe_check_dispatch_host",
+           "moe_check_dispatch"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
@@ -115,7 +118,7 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_rou
             "moe_forward_host_batches", "moe_route_reroute", "moe_forward_reroute",
             "moe_selftest_wait_timeout", "moe_ffn_kernels", "moe_ep_first_expert",
             "moe_ep_plan", "moe_ep_workspace_size", "moe_permute_ep", "moe_ep_expert_ffn",
-            "moe_ep_combine")
+            "moe_ep_combine", "moe_check_dispatch_host", "moe_check_dispatch")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -458,3 +461,26 @@ def moe_ep_combine(cfg, *, ye, slot_row, gates, y, stream=None):
     st = lib.moe_ep_combine(ctypes.byref(cfg), _ptr(ye), _ptr(slot_row), _ptr(gates), _ptr(y),
                             _stream(stream))
     _check(st, "moe_ep_combine")
+
+
+# ---- debugging aid -------------------------------------------------------------------------
+def moe_check_dispatch_host(N, k, E, capacity, *, ids, drop_mask, counts, offsets, slot_row,
+                            demand=None, row_token=None):
+    """Invariants of a dispatch layout, on host (numpy) arrays.  Returns (status, message)."""
+    import numpy as np
+    a = lambda v, dt: None if v is None else np.ascontiguousarray(np.asarray(v, dtype=dt))
+    arrs = [a(ids, np.int32), a(drop_mask, np.uint8), a(counts, np.int32), a(demand, np.int32),
+            a(offsets, np.int32), a(slot_row, np.int32), a(row_token, np.int32)]
+    p = [None if v is None else v.ctypes.data_as(ctypes.c_void_p) for v in arrs]
+    msg = ctypes.create_string_buffer(256)
+    st = lib.moe_check_dispatch_host(int(N), int(k), int(E), int(capacity), *p, msg, 256)
+    return int(st), msg.value.decode()
+
+
+def moe_check_dispatch(cfg, *, ids, drop_mask, counts, offsets, slot_row, demand=None,
+                       row_token=None, stream=None):
+    """The same check on device tensors (synchronises); raises MoeError on a broken one."""
+    st = lib.moe_check_dispatch(ctypes.byref(cfg), _ptr(ids), _ptr(drop_mask), _ptr(counts),
+                                _ptr(demand), _ptr(offsets), _ptr(slot_row), _ptr(row_token),
+                                _stream(stream))
+    _check(st, "moe_check_dispatch")

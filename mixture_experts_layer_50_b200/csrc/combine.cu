@@ -9,6 +9,8 @@
 // In the fused layer the down GEMM writes the shared expert's rows straight into y; the
 // combine then reads y[t] as the shared row, adds the kept slots to it in place, and leaves a
 // token with no kept slot as the GEMM wrote it.
+#include <cstdlib>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -78,6 +80,58 @@ __global__ void __launch_bounds__(128) combine_bf16_kernel(
   }
 }
 
+// The same sums with one warp per token and kCombineWarps tokens per block: a token's
+// slots and gates sit in lanes 0..k-1 and are broadcast with shuffles, a token with no kept
+// slot costs one ballot.  Used where tokens are many and rows small (8x fewer blocks than
+// the block-per-token kernel); the summation order is the same, so the bits are.
+constexpr int kCombineWarps = 8;
+
+template <int KMAX>
+__global__ void __launch_bounds__(32 * kCombineWarps) combine_bf16_warp_kernel(
+    const uint4* __restrict__ ye, const int32_t* __restrict__ slot_row,
+    const float* __restrict__ gates, int64_t N, int k, int vecs, int64_t shared_row0,
+    int shared_in_y, uint4* __restrict__ y) {
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+  if (t >= N) return;  // warp-uniform
+  int32_t my_row = -1;
+  float my_g = 0.f;
+  if (lane < k) {
+    my_row = slot_row[t * k + lane];
+    my_g = gates[t * k + lane];
+  }
+  const unsigned kept = __ballot_sync(0xffffffffu, my_row >= 0);
+  if (shared_in_y && kept == 0u) return;  // y[t] is the shared row already
+  int32_t rj[KMAX];
+  float gj[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    rj[j] = __shfl_sync(0xffffffffu, my_row, j);
+    gj[j] = __shfl_sync(0xffffffffu, my_g, j);
+  }
+  const uint4* shp = shared_in_y ? y + t * vecs
+                                 : (shared_row0 >= 0 ? ye + (shared_row0 + t) * vecs : nullptr);
+  for (int v = lane; v < vecs; v += 32) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    uint4 rows[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (j < k && rj[j] >= 0) rows[j] = ye[(int64_t)rj[j] * vecs + v];
+    uint4 sh = make_uint4(0u, 0u, 0u, 0u);
+    if (shp != nullptr) sh = shp[v];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+      if (j < k && rj[j] >= 0) accum_bf16x8(acc, rows[j], gj[j]);
+    if (shp != nullptr) accum_bf16x8(acc, sh, 1.0f);
+    uint4 o;
+    __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) po[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+    y[t * vecs + v] = o;
+  }
+}
+
 __global__ void __launch_bounds__(128) combine_f32_kernel(
     const float4* __restrict__ ye, const int32_t* __restrict__ slot_row,
     const float* __restrict__ gates, int k, int vecs, int64_t shared_row0,
@@ -115,6 +169,12 @@ __global__ void __launch_bounds__(128) combine_f32_kernel(
   }
 }
 
+// MOE_B200_COMBINE_WARP=0 keeps the block-per-token kernel everywhere (A/B measurements).
+bool combine_warp_enabled() {
+  const char* v = std::getenv("MOE_B200_COMBINE_WARP");
+  return !(v != nullptr && v[0] == '0');
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const void* ye, const int32_t* slot_row, const float* gates,
@@ -128,6 +188,23 @@ cudaError_t launch_combine(const void* ye, const int32_t* slot_row, const float*
   } else {
     const uint4* src = (const uint4*)ye;
     uint4* dst = (uint4*)y;
+    // warp per token when the warps fill every SM several times over and a token reads at
+    // most 8 KB of expert rows; else block per token.  Measured: the capacity and Switch
+    // layers (8 and 4 KB per token) 19.7 -> 16.4 and 16.6 -> 14.2 us; the Mixtral-shaped
+    // prefill (16 KB per token) 72.5 -> 77.4 us, so it keeps a block per token.
+    const int row_bytes = d * 2;
+    if (k <= 8 && N >= (int64_t)tc::num_sms() * 64 && (int64_t)k * row_bytes <= 8192 &&
+        combine_warp_enabled()) {
+      const unsigned wblocks = (unsigned)((N + kCombineWarps - 1) / kCombineWarps);
+      const unsigned th = 32 * kCombineWarps;
+      if (k <= 2)
+        launch_pdl(combine_bf16_warp_kernel<2>, wblocks, th, 0, stream, src, slot_row, gates, N, k, d / 8, shared_row0, shared_in_y, dst);
+      else if (k <= 4)
+        launch_pdl(combine_bf16_warp_kernel<4>, wblocks, th, 0, stream, src, slot_row, gates, N, k, d / 8, shared_row0, shared_in_y, dst);
+      else
+        launch_pdl(combine_bf16_warp_kernel<8>, wblocks, th, 0, stream, src, slot_row, gates, N, k, d / 8, shared_row0, shared_in_y, dst);
+      return cudaGetLastError();
+    }
     const unsigned blocks = (unsigned)N;
     if (k <= 2)
       launch_pdl(combine_bf16_kernel<2>, blocks, 128, 0, stream, src, slot_row, gates, k, d / 8, shared_row0, shared_in_y, dst);

@@ -36,6 +36,33 @@ __device__ __forceinline__ float warp_sum(float v) {
 // Token-tile size of the dispatch kernels (tokens ranked by one warp in order).
 constexpr int kRankTile = 32;
 
+// One warp ranks the assignments of `ntok` consecutive tokens in token order, continuing the
+// per-expert counters cnt[] (shared memory): sid[t * k + j] is the expert of slot j of token
+// t, or -1 for none.  rank(t, e) = the number of earlier tokens that chose e.  An expert listed
+// twice by one token keeps its first slot only.  out(t, j, r) receives each slot's rank (-1 for
+// none); returns true (in every lane) if some token listed an expert twice.
+template <typename Out>
+__device__ __forceinline__ bool warp_rank_walk(const int32_t* sid, int ntok, int k,
+                                               int32_t* cnt, int lane, Out&& out) {
+  bool bad = false;
+  for (int t = 0; t < ntok; ++t) {
+    int v = lane < k ? sid[t * k + lane] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, v);
+    if (v >= 0 && (__ffs(peers) - 1) != lane) {
+      bad = true;
+      v = -1;
+    }
+    int r = -1;
+    if (v >= 0) {
+      r = cnt[v];
+      cnt[v] = r + 1;
+    }
+    if (lane < k) out(t, lane, r);
+    __syncwarp();
+  }
+  return __any_sync(0xffffffffu, bad);
+}
+
 // Programmatic dependent launch.  Every kernel of the library is launched with programmatic
 // stream serialisation (launch_pdl), so the GPU may schedule it while its predecessor on the
 // stream is still running; pdl_wait() returns once that predecessor has completed and its

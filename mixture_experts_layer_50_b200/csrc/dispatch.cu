@@ -15,6 +15,9 @@
 //      over the experts (offsets);
 //   3. one block (or one warp) per token: rank = tile_base + local rank, keep iff rank < C,
 //      row = offsets[e] + rank; the token's x row is copied to each kept row (the gather).
+#include <algorithm>
+#include <cstdlib>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -44,22 +47,8 @@ __global__ void __launch_bounds__(32) rank_local_kernel(
     sid[i] = v;
   }
   __syncwarp();
-  for (int t = 0; t < ntok; ++t) {
-    int v = lane < k ? sid[t * k + lane] : -1;
-    // an expert listed twice by one token: keep the first slot only
-    const unsigned peers = __match_any_sync(0xffffffffu, v);
-    if (v >= 0 && (__ffs(peers) - 1) != lane) {
-      bad = true;
-      v = -1;
-    }
-    int r = -1;
-    if (v >= 0) {
-      r = cnt[v];
-      cnt[v] = r + 1;
-    }
-    if (lane < k) local_rank[(t0 + t) * k + lane] = r;
-    __syncwarp();
-  }
+  bad |= warp_rank_walk(sid, ntok, k, cnt, lane,
+                        [&](int t, int j, int r) { local_rank[(t0 + t) * k + j] = r; });
   if (bad) report_status(status, kStatusInvalidInput);
   for (int e = lane; e < E; e += 32) tile_hist[(int64_t)blockIdx.x * E + e] = cnt[e];
 }
@@ -259,6 +248,115 @@ __global__ void __launch_bounds__(32 * kScatterWarps, 8) dispatch_scatter_warp_k
   }
 }
 
+// The three passes in one launch for a small batch (decode): every block ranks all N*k
+// assignments itself (warp 0 walks the tokens in order, as a rank-pass warp walks its tile),
+// scans the capped counts over the experts and resolves every slot's row, so that no block
+// waits for another; block 0 writes the routing outputs and each block gathers its share of
+// the kept rows (slots b, b + gridDim.x, ...).  The results are those of the three passes.
+template <typename V>
+__global__ void __launch_bounds__(kSmallDispatchThreads) dispatch_small_kernel(
+    const int32_t* __restrict__ ids, const uint8_t* __restrict__ drop_in, int N, int k, int E,
+    int64_t C, const int32_t* __restrict__ cap_e, int32_t* __restrict__ demand,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ slot_row,
+    int32_t* __restrict__ row_token, uint8_t* __restrict__ drop_mask_out,
+    const V* __restrict__ x, V* __restrict__ xp, int row_vecs, int* status) {
+  pdl_wait();
+  extern __shared__ int32_t sm[];
+  int32_t* cnt = sm;                 // [E]
+  int32_t* offs = cnt + E;           // [E + 1]
+  int32_t* s_id = offs + E + 1;      // [N * k]
+  int32_t* s_rank = s_id + N * k;    // [N * k], then the slot's row
+  __shared__ int32_t warp_tot[32];
+  __shared__ int s_bad;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int nk = N * k;
+  const bool writer = blockIdx.x == 0;
+  if (tid == 0) s_bad = 0;
+  for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+  for (int i = tid; i < nk; i += blockDim.x) {
+    int v = ids[i];
+    if (v < 0 || v >= E) {
+      s_bad = 1;
+      v = -1;
+    } else if (drop_in != nullptr && drop_in[i]) {
+      v = -1;
+    }
+    s_id[i] = v;
+  }
+  __syncthreads();
+  if (w == 0) {
+    const bool bad = warp_rank_walk(s_id, N, k, cnt, lane,
+                                    [&](int t, int j, int r) { s_rank[t * k + j] = r; });
+    if (bad && lane == 0) s_bad = 1;
+  }
+  __syncthreads();
+  // capped counts and their exclusive scan over the experts (E <= blockDim.x)
+  const int e_me = tid;
+  const int32_t dem = e_me < E ? cnt[e_me] : 0;
+  int32_t kept = dem;
+  if (e_me < E) {
+    if (cap_e != nullptr) kept = min(dem, max(cap_e[e_me], 0));
+    else if (C > 0 && dem > C) kept = (int32_t)C;
+  }
+  int32_t incl = kept;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) warp_tot[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    int32_t v = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t u = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += u;
+    }
+    warp_tot[lane] = v;
+  }
+  __syncthreads();
+  const int32_t excl = incl - kept + (w > 0 ? warp_tot[w - 1] : 0);
+  if (e_me < E) {
+    offs[e_me] = excl;
+    if (writer) {
+      demand[e_me] = dem;
+      counts[e_me] = kept;
+      offsets[e_me] = excl;
+    }
+    if (e_me == E - 1) {
+      offs[E] = excl + kept;
+      if (writer) offsets[E] = excl + kept;
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < nk; i += blockDim.x) {
+    const int r = s_rank[i];
+    const int e = s_id[i];
+    int32_t row = -1;
+    if (r >= 0) {
+      const bool keep = cap_e != nullptr ? r < cap_e[e] : (C <= 0 || r < C);
+      if (keep) row = offs[e] + r;
+    }
+    s_rank[i] = row;
+    if (writer) {
+      if (slot_row != nullptr) slot_row[i] = row;
+      if (drop_mask_out != nullptr) drop_mask_out[i] = row < 0 ? 1 : 0;
+      if (row >= 0 && row_token != nullptr) row_token[row] = i / k;
+    }
+  }
+  if (writer && tid == 0 && s_bad) report_status(status, kStatusInvalidInput);
+  if (xp == nullptr) return;
+  __syncthreads();
+  for (int i = blockIdx.x; i < nk; i += gridDim.x) {
+    const int32_t row = s_rank[i];
+    if (row < 0) continue;
+    const V* src = x + (int64_t)(i / k) * row_vecs;
+    V* dst = xp + (int64_t)row * row_vecs;
+    for (int v = tid; v < row_vecs; v += blockDim.x) dst[v] = src[v];
+  }
+}
+
 __global__ void pad_offsets_kernel(int E, int64_t C, int32_t* __restrict__ offsets_pad) {
   pdl_wait();
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
@@ -278,6 +376,35 @@ __global__ void __launch_bounds__(128) zero_padding_kernel(
 }
 
 }  // namespace
+
+bool use_small_dispatch(int64_t N, int k, int E) {
+  if (N <= 0 || N > kSmallDispatchMaxTokens || N * k > kSmallDispatchMaxSlots) return false;
+  const char* v = std::getenv("MOE_B200_SMALL_DISPATCH");
+  (void)E;
+  return !(v != nullptr && v[0] == '0');
+}
+
+cudaError_t launch_dispatch_small(const int32_t* ids, const uint8_t* drop_in, int64_t N, int k,
+                                  int E, int64_t C, const int32_t* cap_e, int32_t* demand,
+                                  int32_t* counts, int32_t* offsets, int32_t* slot_row,
+                                  int32_t* row_token, uint8_t* drop_mask_out, const void* x,
+                                  void* xp, int row_bytes, int* status, cudaStream_t stream,
+                                  int* launches) {
+  ++*launches;
+  const int nk = (int)(N * k);
+  const size_t smem = sizeof(int32_t) * ((size_t)E + (size_t)E + 1 + 2 * (size_t)nk);
+  const int grid = xp != nullptr ? std::max(1, std::min(nk, tc::num_sms())) : 1;
+  if (xp != nullptr && row_bytes % 16 == 0) {
+    launch_pdl(dispatch_small_kernel<uint4>, grid, kSmallDispatchThreads, smem, stream, ids,
+               drop_in, (int)N, k, E, C, cap_e, demand, counts, offsets, slot_row, row_token,
+               drop_mask_out, (const uint4*)x, (uint4*)xp, row_bytes / 16, status);
+  } else {
+    launch_pdl(dispatch_small_kernel<uint32_t>, grid, kSmallDispatchThreads, smem, stream, ids,
+               drop_in, (int)N, k, E, C, cap_e, demand, counts, offsets, slot_row, row_token,
+               drop_mask_out, (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4, status);
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pad_offsets(int E, int64_t C, int32_t* offsets_pad, cudaStream_t stream,
                                int* launches) {

@@ -265,6 +265,8 @@ struct Args {
   int k_splits;       // > 1: split K; split s writes rows [s * split_rows, ...) of out
   int64_t split_rows;
   int m64_tails;      // 1-SM kernel: a tile with at most 64 valid rows issues M = 64 MMAs
+  int half_tails;     // 2-SM kernel: a tile with at most 128 valid rows issues M = 128 MMAs
+  int band;           // > 0: M blocks of a large group run in bands of this many (decode_tile)
 };
 
 template <int BN, int STAGES>
@@ -282,9 +284,12 @@ struct Layout {
 // Tile -> (group, M block, N block).  Tiles are numbered group by group; inside a group the
 // operand with the smaller total panel is kept resident in L2 while the other streams: if the
 // group's A rows outnumber its B rows, M blocks are outer and N blocks inner, else the reverse.
+// band > 0 (a group whose A panel outgrows L2): the group's M blocks run in bands of `band`;
+// inside a band, N blocks outer and the band's M blocks inner, so the band's A rows stay in
+// L2 while the weights stream once per band.
 template <int BMT, int BN>
 __device__ __forceinline__ void decode_tile(int tile, const int* s_start, int G, int nt,
-                                            int& g, int& m_blk, int& n_blk) {
+                                            int& g, int& m_blk, int& n_blk, int band = 0) {
   int lo = 0, hi = G;  // largest g with s_start[g] <= tile
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -293,7 +298,14 @@ __device__ __forceinline__ void decode_tile(int tile, const int* s_start, int G,
   g = lo;
   const int r = tile - s_start[g];
   const int mt = (s_start[g + 1] - s_start[g]) / nt;
-  if (mt * BMT > nt * BN) {
+  if (band > 0 && mt > band && mt * BMT <= nt * BN) {
+    const int per_band = band * nt;
+    const int b = r / per_band;
+    const int rr = r - b * per_band;
+    const int mb = min(band, mt - b * band);
+    n_blk = rr / mb;
+    m_blk = b * band + (rr - n_blk * mb);
+  } else if (mt * BMT > nt * BN) {
     m_blk = r / nt;
     n_blk = r - m_blk * nt;
   } else {
@@ -309,16 +321,20 @@ __device__ __forceinline__ float silu_f(float a) { return __fdividef(a, 1.0f + _
 // One epilogue warp drains its 32 TMEM lanes (rows row_base + lane of the output tile) of an
 // accumulator: activation, packing, per-warp staging in shared memory, then coalesced 16-byte
 // stores with row and column masks.  `release` runs right after the last TMEM read.
+// `chunks` (default: the whole tile) chunks of output columns are drained, starting at TMEM
+// column 0 of the accumulator and at output column n_blk * kOutPerTile + col_extra.
 template <int BN, int EPI, typename Release>
 __device__ __forceinline__ void epilogue_warp(const Args& p, void* out, uint32_t t_row,
                                               uint8_t* stg, int lane, int n_blk,
                                               int64_t out_row0, int row_base, int rows_valid,
-                                              Release&& release) {
+                                              Release&& release, int chunks = -1,
+                                              int col_extra = 0) {
   constexpr int kOutPerTile = (EPI == kEpiSwiglu) ? BN / 2 : BN;
   constexpr int kColsPerChunk = (EPI == kEpiStoreF32) ? 32 : 64;
   constexpr int kChunks = kOutPerTile / kColsPerChunk;
+  const int n_chunks = chunks < 0 ? kChunks : chunks;
 #pragma unroll 1
-  for (int c = 0; c < kChunks; ++c) {
+  for (int c = 0; c < n_chunks; ++c) {
     uint32_t packed[32];
     if constexpr (EPI == kEpiSwiglu) {
       float gv[32], uv[32];
@@ -369,7 +385,7 @@ __device__ __forceinline__ void epilogue_warp(const Args& p, void* out, uint32_t
         }
       }
     }
-    if (c == kChunks - 1) release();
+    if (c == n_chunks - 1) release();
     // stage this thread's 128-byte row piece (row stride 144 B: conflict-free)
     uint4* my = reinterpret_cast<uint4*>(stg + lane * 144);
 #pragma unroll
@@ -378,7 +394,7 @@ __device__ __forceinline__ void epilogue_warp(const Args& p, void* out, uint32_t
     __syncwarp();
     // coalesced copy-out: 4 rows x 128 bytes per instruction
     constexpr int kElPerPiece = (EPI == kEpiStoreF32) ? 4 : 8;
-    const int col_base = n_blk * kOutPerTile + c * kColsPerChunk;
+    const int col_base = n_blk * kOutPerTile + col_extra + c * kColsPerChunk;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int rr = i * 4 + (lane >> 3);
@@ -497,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         int g, m_blk, n_blk;
-        decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk);
+        decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
         const int kb0 = (tile % ks_n) * kper, kb1 = min(nk, kb0 + kper);
         const bool sh = g >= p.n_routed;
         const int a_row = (sh ? p.shared_a_row0 : p.offsets[g]) + m_blk * BM;
@@ -549,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         int g, m_blk, n_blk;
-        decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk);
+        decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
         const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
         const uint32_t idesc = (p.m64_tails && cnt - m_blk * BM <= 64) ? kIdesc64 : kIdesc;
         if (!mbar_wait(&tempty[acc], aph ^ 1, s_abort, p.status)) {
@@ -593,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       int g, m_blk, n_blk;
-      decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk);
+      decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       // warp-uniform decision: tcgen05.ld below needs all 32 lanes
@@ -657,6 +673,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   pdl_wait();
   constexpr int BN = 256;   // MMA N
   constexpr int BMT = 256;  // tile rows (128 per CTA)
+  // half tiles for group tails: an elementwise epilogue only (SwiGLU pairs columns c and
+  // c + 128, which a half tile's accumulator keeps in different warps' lanes)
+  constexpr bool kHalfTiles = EPI != kEpiSwiglu;
   using L = Layout2<STAGES>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -736,9 +755,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       int armed = 0;
       bool ok = true;
+      // a half tile (at most 128 valid rows) gives each CTA 64 rows: CTA 1's start at 64
       auto a_row_of = [&](int g, int m_blk) {
         const bool sh = g >= p.n_routed;
-        return (sh ? p.shared_a_row0 : p.offsets[g]) + m_blk * BMT + (int)rank * 128;
+        const int cnt = sh ? p.shared_rows : p.offsets[g + 1] - p.offsets[g];
+        const bool half = kHalfTiles && p.half_tails && cnt - m_blk * BMT <= BMT / 2;
+        return (sh ? p.shared_a_row0 : p.offsets[g]) + m_blk * BMT + (int)rank * (half ? 64 : 128);
       };
       auto b_row_of = [&](int n_blk) {
         if (EPI == kEpiSwiglu) return rank == 0 ? n_blk * 128 : p.up_row0 + n_blk * 128;
@@ -746,7 +768,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       };
       for (int tile = pair; ok && tile < total; tile += npairs) {
         int g, m_blk, n_blk;
-        decode_tile<BMT, BN>(tile, s_start, G, nt, g, m_blk, n_blk);
+        decode_tile<BMT, BN>(tile, s_start, G, nt, g, m_blk, n_blk, p.band);
         const CUtensorMap* mA = g >= p.n_routed ? &tmAs : &tmA;
         const int a_row = a_row_of(g, m_blk);
         const int b_row = b_row_of(n_blk);
@@ -780,6 +802,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0 && rank == 0) {
       constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
                                   ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BMT >> 4) << 24);
+      // M = 128 across the pair (64 rows per CTA): the same descriptor with the M field halved
+      constexpr uint32_t kIdescHalf = (kIdesc & ~(0x1Fu << 24)) | ((uint32_t)(128 >> 4) << 24);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
@@ -787,6 +811,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int tile = pair; ok && tile < total; tile += npairs, ++it) {
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
+        int g, m_blk, n_blk;
+        decode_tile<BMT, BN>(tile, s_start, G, nt, g, m_blk, n_blk, p.band);
+        const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
+        const uint32_t idesc =
+            (kHalfTiles && p.half_tails && cnt - m_blk * BMT <= BMT / 2) ? kIdescHalf : kIdesc;
         if (!mbar_wait(&tempty[acc], aph ^ 1, s_abort, p.status)) {
           ok = false;
           break;
@@ -803,7 +832,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t b0 = smem_u32(sB + stage * L::kStageB);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            mma_bf16_pair(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), kIdesc,
+            mma_bf16_pair(d_tmem, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), idesc,
                           (kb | kk) != 0 ? 1u : 0u);
           }
           mma_commit_pair_both(&empty[stage]);
@@ -827,7 +856,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int it = 0;
     for (int tile = pair; tile < total; tile += npairs, ++it) {
       int g, m_blk, n_blk;
-      decode_tile<BMT, BN>(tile, s_start, G, nt, g, m_blk, n_blk);
+      decode_tile<BMT, BN>(tile, s_start, G, nt, g, m_blk, n_blk, p.band);
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       const bool ready = mbar_wait(&tfull[acc], aph, s_abort, p.status);
@@ -838,13 +867,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int64_t out_row0 = (int64_t)(sh ? p.shared_out_row0 : p.offsets[g]) + m_blk * BMT;
       const int rows_valid = min(BMT, cnt - m_blk * BMT);
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      // a half tile's accumulator (M = 128 across the pair) holds CTA r's 64 rows twice over
+      // the lanes: lane m has row 64 r + m for output columns 0..127, lane 64 + m the same row
+      // for columns 128..255, both at TMEM columns 0..127.  Warp q drains lanes 32 q .. + 31:
+      // rows 64 r + 32 (q & 1) + lane, output columns 128 (q >> 1) .. + 127 (two chunks).
+      const bool half = kHalfTiles && p.half_tails && rows_valid <= BMT / 2;
+      const int row_base = half ? (int)rank * 64 + (q & 1) * 32 : (int)rank * 128 + q * 32;
       void* out = (sh && p.out_shared != nullptr) ? p.out_shared : p.out;
-      epilogue_warp<BN, EPI>(p, out, t_row, stg, lane, n_blk, out_row0, (int)rank * 128 + q * 32,
-                             rows_valid, [&] {
+      epilogue_warp<BN, EPI>(p, out, t_row, stg, lane, n_blk, out_row0, row_base, rows_valid, [&] {
                                tc_fence_before();
                                __syncwarp();
                                if (lane == 0) mbar_arrive_cluster(tempty_first + 8u * (uint32_t)acc);
-                             });
+                             },
+                             half ? 2 : -1, half ? (q >> 1) * 128 : 0);
     }
   }
 
@@ -1286,6 +1321,12 @@ cudaError_t allow_max_smem(Kernel kern, bool (&done)[kMaxDev]) {
   return e;
 }
 
+// 2-SM kernel: half-height tiles for group tails (MOE_B200_2SM_HALF_TAILS=0 turns them off).
+bool half_tails_enabled() {
+  const char* v = std::getenv("MOE_B200_2SM_HALF_TAILS");
+  return !(v != nullptr && std::strcmp(v, "0") == 0);
+}
+
 Args make_args(const GroupedGemm& g) {
   Args a;
   a.offsets = g.offsets;
@@ -1307,7 +1348,22 @@ Args make_args(const GroupedGemm& g) {
   a.split_rows = g.split_rows;
   const char* m64 = std::getenv("MOE_B200_M64_TAILS");
   a.m64_tails = (m64 != nullptr && std::strcmp(m64, "0") == 0) ? 0 : 1;
+  a.half_tails = half_tails_enabled() ? 1 : 0;
+  a.band = 0;
   return a;
+}
+
+// Bands of M blocks for groups whose A panel outgrows L2 (MOE_B200_BAND: unset or 0 = off,
+// 1 = bands of about a third of L2 of A rows, n > 1 = bands of n M blocks).  Only groups
+// that run N blocks outer (their B panel at least as large as their A panel) are banded.
+int band_for(const GroupedGemm& g, int bmt) {
+  const char* v = std::getenv("MOE_B200_BAND");
+  if (v == nullptr) return 0;
+  const int n = std::atoi(v);
+  if (n <= 0) return 0;
+  if (n > 1) return n;
+  const int64_t tile_bytes = (int64_t)bmt * g.K * 2;
+  return (int)std::max<int64_t>(1, l2_bytes() / 3 / tile_bytes);
 }
 
 template <int BN, int EPI, int STAGES>
@@ -1318,7 +1374,9 @@ cudaError_t launch_t(const GroupedGemm& g, const CUtensorMap& mA, const CUtensor
   static bool done[kMaxDev] = {};
   const cudaError_t e = allow_max_smem(kern, done);
   if (e != cudaSuccess) return e;
-  launch_pdl(kern, grid, kThreads, smem, stream, mA, mAs, mB, make_args(g));
+  Args a = make_args(g);
+  a.band = band_for(g, BM);
+  launch_pdl(kern, grid, kThreads, smem, stream, mA, mAs, mB, a);
   return cudaGetLastError();
 }
 
@@ -1330,7 +1388,9 @@ cudaError_t launch_2sm(const GroupedGemm& g, const CUtensorMap& mA, const CUtens
   static bool done[kMaxDev] = {};
   const cudaError_t e = allow_max_smem(kern, done);
   if (e != cudaSuccess) return e;
-  launch_pdl(kern, 2 * pairs, kThreads, smem, stream, mA, mAs, mB, make_args(g));
+  Args a = make_args(g);
+  a.band = band_for(g, 256);
+  launch_pdl(kern, 2 * pairs, kThreads, smem, stream, mA, mAs, mB, a);
   return cudaGetLastError();
 }
 
@@ -1403,6 +1463,10 @@ bool use_two_sm(const GroupedGemm& g) {
   const int64_t routed = g.n_routed > 0 ? avg_group_rows(g) * g.n_routed : 0;
   const int64_t shared = g.has_shared ? g.shared_rows : 0;
   if (routed + shared <= 0) return false;
+  // a group's last tile pads to 256 rows against 128 (64 with an M = 64 tile) on the 1-SM
+  // kernel: on average 96 more rows per group.  (Half tiles, where the 2-SM kernel runs an
+  // elementwise epilogue, cut that to 32, but at the ridge-point layers the 1-SM kernel still
+  // won with them -- V4.1-shaped prefill 9.47 vs 9.71-9.86 ms -- so the estimate keeps 96.)
   int64_t extra = 96LL * g.n_routed;
   if (shared > 0) extra += (shared + 255) / 256 * 256 - one_sm_rows(shared);
   if (4 * extra > routed + shared) return false;

@@ -18,6 +18,17 @@ cudaError_t launch_route_topk(const float* logits, int n_parts, int64_t part_str
                               int* status, cudaStream_t stream, int* launches,
                               int k_extra = 0, int32_t* cand = nullptr,
                               float* cand_val = nullptr);
+// Top-k and the dispatch's rank pass in one launch (kRankTile tokens per block): ids, gates,
+// and the local ranks and tile histograms launch_rank_local would write (no drop mask).
+// Opt-in: MOE_B200_FUSED_TOPK_RANK=1.
+constexpr int kFusedTopkRankMaxE = 384;
+bool fused_topk_rank_enabled();
+cudaError_t launch_route_topk_rank(const float* logits, int n_parts, int64_t part_stride,
+                                   const float* offset, float* logits_out, int64_t N, int E,
+                                   int k, int score_fn, int renorm, const float* bias,
+                                   int n_bias_sets, const uint8_t* modality, int32_t* ids,
+                                   float* gates, int* status, int32_t* local_rank,
+                                   int32_t* tile_hist, cudaStream_t stream, int* launches);
 // Overflow policy "report": offers of the dropped slots to the next-best candidates, and the
 // decision on them (csrc/reroute.cu).
 cudaError_t launch_reroute_offer(const int32_t* ids, const uint8_t* drop1, const int32_t* cand,
@@ -58,6 +69,19 @@ cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_ran
                                     const void* x, void* xp, int row_bytes,
                                     cudaStream_t stream, int* launches,
                                     const int32_t* cap_e = nullptr);
+
+// The three passes in one launch for a small batch (N <= kSmallDispatchMaxTokens and
+// N * k <= kSmallDispatchMaxSlots): the same outputs, plus the device status for bad ids.
+constexpr int kSmallDispatchThreads = 1024;   // >= E (at most 1024)
+constexpr int kSmallDispatchMaxTokens = 256;
+constexpr int kSmallDispatchMaxSlots = 2048;
+bool use_small_dispatch(int64_t N, int k, int E);   // MOE_B200_SMALL_DISPATCH=0: never
+cudaError_t launch_dispatch_small(const int32_t* ids, const uint8_t* drop_in, int64_t N, int k,
+                                  int E, int64_t C, const int32_t* cap_e, int32_t* demand,
+                                  int32_t* counts, int32_t* offsets, int32_t* slot_row,
+                                  int32_t* row_token, uint8_t* drop_mask_out, const void* x,
+                                  void* xp, int row_bytes, int* status, cudaStream_t stream,
+                                  int* launches);
 
 // ---- balancing statistics (balance.cu) ------------------------------------------------
 // f [E] share of assignments, P [E] mean router probability, aux = E sum f P, set_load

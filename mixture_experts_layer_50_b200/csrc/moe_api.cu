@@ -239,6 +239,13 @@ LogitSrc finished_logits(const float* z) { return LogitSrc{z, 1, 0, nullptr, nul
 
 int router_splits(const moe_config& c) {
   if (c.dtype != MOE_DT_BF16 || c.N == 0) return 1;
+  if (const char* v = std::getenv("MOE_B200_ROUTER_SPLITS")) {
+    // a fixed slice count (A/B measurements): at most kMaxLogitSplits, no empty slice
+    const int nk = (c.d + 63) / 64;
+    const int want = std::max(1, std::min({std::atoi(v), kMaxLogitSplits, nk}));
+    const int per = (nk + want - 1) / want;
+    return (nk + per - 1) / per;
+  }
   const int bn = moe::router_tile_n(c.E);
   const int64_t tiles = ((c.N + 127) / 128) * ((c.E + bn - 1) / bn);
   const int nk = (c.d + 63) / 64;
@@ -309,17 +316,51 @@ moe_status stage_route(const moe_config& c, const LogitSrc& z, const float* bias
   return MOE_OK;
 }
 
-// Ranks, capacity, offsets, slot rows; gathers x into xp when xp != nullptr.
+// A batch that takes the three dispatch passes (not a small one) runs top-k and the rank
+// pass as one launch (route_topk_rank); stage_dispatch then skips its rank pass.
+// (E <= kFusedTopkRankMaxE: with 1024 threads a block, more keys per lane would spill.)
+bool fuse_topk_rank(const moe_config& c) {
+  return c.N > 0 && c.E <= moe::kFusedTopkRankMaxE && moe::fused_topk_rank_enabled() &&
+         !moe::use_small_dispatch(c.N, c.k, c.E);
+}
+
+moe_status stage_route_rank(const moe_config& c, const Ws& L, void* ws, const LogitSrc& z,
+                            const float* bias, const uint8_t* modality, int32_t* ids,
+                            float* gates, int* status, cudaStream_t st, int* launches) {
+  MOE_CUDA(moe::launch_route_topk_rank(z.src, z.n_parts, z.part_stride, z.offset, z.final_out,
+                                       c.N, c.E, c.k, c.score_fn, c.renorm, bias, c.n_bias_sets,
+                                       modality, ids, gates, status,
+                                       at<int32_t>(ws, L.local_rank),
+                                       at<int32_t>(ws, L.tile_hist), st, launches),
+           "top-k routing with the rank pass");
+  prof_mark(st);
+  return MOE_OK;
+}
+
+// Ranks, capacity, offsets, slot rows; gathers x into xp when xp != nullptr.  ranked: the rank
+// pass already ran (stage_route_rank) and only the scan and scatter passes remain.
 moe_status stage_dispatch(const moe_config& c, const Ws& L, void* ws, const int32_t* ids,
                           const uint8_t* drop_in, int64_t C, int32_t* demand, int32_t* counts,
                           int32_t* offsets, int32_t* slot_row, int32_t* row_token,
                           uint8_t* drop_out, const void* x, void* xp, cudaStream_t st,
-                          int* launches, const int32_t* cap_e = nullptr) {
+                          int* launches, const int32_t* cap_e = nullptr,
+                          bool ranked = false) {
   int* status = at<int>(ws, L.status);
-  MOE_CUDA(moe::launch_rank_local(ids, drop_in, c.N, c.k, c.E, at<int32_t>(ws, L.local_rank),
-                                  at<int32_t>(ws, L.tile_hist), status, st, launches),
-           "rank pass");
-  prof_mark(st);
+  if (!ranked && moe::use_small_dispatch(c.N, c.k, c.E)) {
+    // a small batch: the three passes in one launch, with the same outputs
+    MOE_CUDA(moe::launch_dispatch_small(ids, drop_in, c.N, c.k, c.E, C, cap_e, demand, counts,
+                                        offsets, slot_row, row_token, drop_out, x, xp,
+                                        (int)(c.d * el_size(c)), status, st, launches),
+             "dispatch (small batch)");
+    prof_mark(st);
+    return MOE_OK;
+  }
+  if (!ranked) {
+    MOE_CUDA(moe::launch_rank_local(ids, drop_in, c.N, c.k, c.E, at<int32_t>(ws, L.local_rank),
+                                    at<int32_t>(ws, L.tile_hist), status, st, launches),
+             "rank pass");
+    prof_mark(st);
+  }
   MOE_CUDA(moe::launch_dispatch_scan(at<int32_t>(ws, L.tile_hist), c.N, c.E, C,
                                      at<int32_t>(ws, L.tile_base), demand, counts, offsets,
                                      arrive_counter(ws, L), st, launches, cap_e),
@@ -497,6 +538,48 @@ moe_status stage_combine(const moe_config& c, const void* ye, const int32_t* slo
   return MOE_OK;
 }
 
+// MOE_B200_DEBUG=1: the fused forward calls check their dispatch layout on the host after the
+// dispatch passes (moe_check_dispatch_host).  Synchronises the stream: for eager calls only,
+// never inside a stream capture.
+bool debug_checks() {
+  const char* v = std::getenv("MOE_B200_DEBUG");
+  return v != nullptr && v[0] == '1';
+}
+
+moe_status check_dispatch_device(const moe_config& c, const int32_t* ids, const uint8_t* drop,
+                                 const int32_t* counts, const int32_t* demand,
+                                 const int32_t* offsets, const int32_t* slot_row,
+                                 const int32_t* row_token, int64_t capacity, cudaStream_t st) {
+  const size_t nk = (size_t)c.N * c.k, E = (size_t)c.E;
+  std::vector<int32_t> h_ids(nk), h_cnt(E), h_dem(E), h_off(E + 1), h_slot(nk);
+  std::vector<uint8_t> h_drop(nk);
+  MOE_CUDA(cudaStreamSynchronize(st), "debug check: synchronise");
+  auto get = [&](void* dst, const void* src, size_t bytes) {
+    return bytes == 0 ? cudaSuccess : cudaMemcpy(dst, src, bytes, cudaMemcpyDeviceToHost);
+  };
+  MOE_CUDA(get(h_ids.data(), ids, nk * 4), "debug check: copy ids");
+  MOE_CUDA(get(h_drop.data(), drop, nk), "debug check: copy drop mask");
+  MOE_CUDA(get(h_cnt.data(), counts, E * 4), "debug check: copy counts");
+  if (demand != nullptr) MOE_CUDA(get(h_dem.data(), demand, E * 4), "debug check: copy demand");
+  MOE_CUDA(get(h_off.data(), offsets, (E + 1) * 4), "debug check: copy offsets");
+  MOE_CUDA(get(h_slot.data(), slot_row, nk * 4), "debug check: copy slot rows");
+  std::vector<int32_t> h_rt;
+  if (row_token != nullptr && h_off[E] >= 0 && (size_t)h_off[E] <= nk) {
+    h_rt.resize((size_t)h_off[E]);
+    MOE_CUDA(get(h_rt.data(), row_token, h_rt.size() * 4), "debug check: copy row map");
+  }
+  char msg[200];
+  const moe_status s = moe_check_dispatch_host(
+      c.N, c.k, c.E, capacity, h_ids.data(), h_drop.data(), h_cnt.data(),
+      demand != nullptr ? h_dem.data() : nullptr, h_off.data(), h_slot.data(),
+      h_rt.empty() ? nullptr : h_rt.data(), msg, sizeof(msg));
+  if (s != MOE_OK) {
+    std::string m = std::string("dispatch layout check: ") + msg;
+    return fail(s, m.c_str());
+  }
+  return MOE_OK;
+}
+
 moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
                         const float* logit_offset, const float* bias, const uint8_t* modality,
                         const void* W_gu, const void* W_down, void* y,
@@ -518,6 +601,7 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
   int32_t* offsets = pick(ro ? ro->offsets : (int32_t*)nullptr, L.offsets);
   void* xp = at<char>(ws, L.xp);
   void* ye = at<char>(ws, L.ye);
+  int32_t* row_token = at<int32_t>(ws, L.row_token);
   prof_call_begin(st);
   LogitSrc zsrc;
   MOE_TRY(stage_logits(c, L, ws, x, W_g, logit_offset, logits, status, st, launches, &zsrc));
@@ -528,16 +612,24 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
     MOE_TRY(stage_route_reroute(c, L, ws, zsrc, bias, modality, ids, gates, demand, drop,
                                 rerouted, st, launches));
     MOE_TRY(stage_dispatch(c, L, ws, ids, drop, 0, at<int32_t>(ws, L.rr_scratch), counts,
-                           offsets, at<int32_t>(ws, L.slot_row), at<int32_t>(ws, L.row_token),
-                           drop, x, xp, st, launches));
+                           offsets, at<int32_t>(ws, L.slot_row), row_token, drop, x, xp, st,
+                           launches));
   } else {
-    MOE_TRY(stage_route(c, zsrc, bias, modality, ids, gates, status, st, launches));
+    const bool fused = fuse_topk_rank(c);
+    if (fused)
+      MOE_TRY(stage_route_rank(c, L, ws, zsrc, bias, modality, ids, gates, status, st, launches));
+    else
+      MOE_TRY(stage_route(c, zsrc, bias, modality, ids, gates, status, st, launches));
     MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, c.capacity, demand, counts, offsets,
-                           at<int32_t>(ws, L.slot_row), at<int32_t>(ws, L.row_token), drop, x,
-                           xp, st, launches));
+                           at<int32_t>(ws, L.slot_row), row_token, drop, x, xp, st,
+                           launches, nullptr, fused));
     if (rerouted != nullptr && c.N > 0)
       MOE_CUDA(cudaMemsetAsync(rerouted, 0, (size_t)c.N * c.k, st), "clear rerouted flags");
   }
+  if (debug_checks())
+    MOE_TRY(check_dispatch_device(c, ids, drop, counts, (reroute && c.capacity > 0) ? nullptr : demand,
+                                  offsets, at<int32_t>(ws, L.slot_row),
+                                  at<int32_t>(ws, L.row_token), c.capacity, st));
   // fused layer: the shared expert's rows go straight into y (bf16), completed by the combine
   MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, launches, -1, y));
   MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, launches, -1, true));
@@ -593,13 +685,17 @@ moe_status moe_route(const moe_config* cfg, const float* logits, const void* x,
   }
   int32_t* ids_p = ids != nullptr ? ids : at<int32_t>(ws, L.ids);
   float* gates_p = gates != nullptr ? gates : at<float>(ws, L.gates);
-  MOE_TRY(stage_route(c, z, bias, modality, ids_p, gates_p, status, st, &launches));
+  const bool fused = fuse_topk_rank(c);
+  if (fused)
+    MOE_TRY(stage_route_rank(c, L, ws, z, bias, modality, ids_p, gates_p, status, st, &launches));
+  else
+    MOE_TRY(stage_route(c, z, bias, modality, ids_p, gates_p, status, st, &launches));
   MOE_TRY(stage_dispatch(c, L, ws, ids_p, nullptr, c.capacity,
                          demand != nullptr ? demand : at<int32_t>(ws, L.demand),
                          counts != nullptr ? counts : at<int32_t>(ws, L.counts),
                          at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.slot_row), nullptr,
                          drop_mask != nullptr ? drop_mask : at<uint8_t>(ws, L.drop_mask),
-                         nullptr, nullptr, st, &launches));
+                         nullptr, nullptr, st, &launches, nullptr, fused));
   g_last_launches = launches;
   return MOE_OK;
 }
@@ -1289,6 +1385,19 @@ moe_status moe_check_status(void* ws, moe_stream_t stream) {
   if (host == MOE_ERR_TIMEOUT) return fail(MOE_ERR_TIMEOUT, "a bounded device wait ran out");
   if (host != 0) return fail(MOE_ERR_CUDA, "unknown device status");
   return MOE_OK;
+}
+
+moe_status moe_check_dispatch(const moe_config* cfg, const int32_t* ids,
+                              const uint8_t* drop_mask, const int32_t* counts,
+                              const int32_t* demand, const int32_t* offsets,
+                              const int32_t* slot_row, const int32_t* row_token,
+                              moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg));
+  if (ids == nullptr || drop_mask == nullptr || counts == nullptr || offsets == nullptr ||
+      slot_row == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "ids, drop_mask, counts, offsets and slot_row are required");
+  return check_dispatch_device(*cfg, ids, drop_mask, counts, demand, offsets, slot_row,
+                               row_token, cfg->capacity, (cudaStream_t)stream);
 }
 
 moe_status moe_profile_begin(int32_t max_calls) {

@@ -13,6 +13,8 @@
 // range reduction and a Taylor polynomial out of correctly rounded float32 operations
 // (explicit _rn intrinsics, never contracted into FMAs), so that sigmoid keys -- and the
 // experts they select -- are reproducible bit for bit on any IEEE float32 machine.
+#include <cstdlib>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -52,17 +54,22 @@ __device__ __forceinline__ bool beats(float ka, int ea, float kb, int eb) {
   return ka > kb || (ka == kb && ea < eb);
 }
 
+// The selection of one token by one warp: scores, keys, `rounds` rounds of arg-max and the
+// gates.  Lane r returns the r-th selection (e = -1 past `rounds`), its score and, for r < k,
+// its gate.  Every lane of the warp must call it.
+struct TokenSel {
+  int e;
+  float sc;
+  float g;
+};
+
 template <int J>  // keys per lane: E <= 32 * J
-__global__ void __launch_bounds__(256) route_topk_kernel(
+__device__ __forceinline__ TokenSel select_token(
     const float* __restrict__ logits, int n_parts, int64_t part_stride,
-    const float* __restrict__ offset, float* __restrict__ logits_out, int64_t N, int E, int k,
+    const float* __restrict__ offset, float* __restrict__ logits_out, int64_t t, int E, int k,
     int score_fn, int renorm, const float* __restrict__ bias, int n_bias_sets,
-    const uint8_t* __restrict__ modality, int32_t* __restrict__ ids, float* __restrict__ gates,
-    int* status, int k_extra, int32_t* __restrict__ cand, float* __restrict__ cand_val) {
-  pdl_wait();
+    const uint8_t* __restrict__ modality, int* status, int rounds) {
   const int lane = threadIdx.x & 31;
-  const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (t >= N) return;
   const float* z = logits + t * E;
   const float* b = nullptr;
   if (bias != nullptr) {
@@ -101,9 +108,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
     }
   }
 
-  // k rounds of warp arg-max (k + k_extra when the next-best candidates are asked for, at
-  // most E).  Lane r keeps the r-th selection.
-  const int rounds = cand != nullptr ? min(E, k + k_extra) : k;
+  // `rounds` rounds of warp arg-max (k, or more when the next-best candidates are asked for;
+  // at most E).  Lane r keeps the r-th selection.
   uint32_t taken = 0;
   int my_e = -1;
   float my_sc = 0.0f;
@@ -163,17 +169,76 @@ __global__ void __launch_bounds__(256) route_topk_kernel(
       g = my_sc;
     }
   }
-  if (mine) {
-    ids[t * k + lane] = my_e;
-    gates[t * k + lane] = g;
+  return TokenSel{my_e, my_sc, g};
+}
+
+template <int J>
+__global__ void __launch_bounds__(256) route_topk_kernel(
+    const float* __restrict__ logits, int n_parts, int64_t part_stride,
+    const float* __restrict__ offset, float* __restrict__ logits_out, int64_t N, int E, int k,
+    int score_fn, int renorm, const float* __restrict__ bias, int n_bias_sets,
+    const uint8_t* __restrict__ modality, int32_t* __restrict__ ids, float* __restrict__ gates,
+    int* status, int k_extra, int32_t* __restrict__ cand, float* __restrict__ cand_val) {
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= N) return;
+  const int rounds = cand != nullptr ? min(E, k + k_extra) : k;
+  const TokenSel s = select_token<J>(logits, n_parts, part_stride, offset, logits_out, t, E, k,
+                                     score_fn, renorm, bias, n_bias_sets, modality, status,
+                                     rounds);
+  if (lane < k) {
+    ids[t * k + lane] = s.e;
+    gates[t * k + lane] = s.g;
   }
   if (cand != nullptr) {
     // candidates k .. k + k_extra - 1 (-1 past E), and per selection the value the gates are
     // computed from: the unbiased score (renorm) or the raw gate (no renorm)
-    if (lane >= k && lane < k + k_extra) cand[t * k_extra + (lane - k)] = lane < rounds ? my_e : -1;
+    if (lane >= k && lane < k + k_extra) cand[t * k_extra + (lane - k)] = lane < rounds ? s.e : -1;
     if (lane < k + k_extra)
-      cand_val[t * (k + k_extra) + lane] = lane < rounds ? (renorm ? my_sc : g) : 0.0f;
+      cand_val[t * (k + k_extra) + lane] = lane < rounds ? (renorm ? s.sc : s.g) : 0.0f;
   }
+}
+
+// Top-k and the dispatch's rank pass in one launch: block b selects the experts of the
+// kRankTile tokens of tile b (one warp per token, the selection above), then its first warp
+// ranks the tile's assignments in token order and writes the tile's per-expert histogram --
+// the rank pass's outputs for that tile.
+template <int J>
+__global__ void __launch_bounds__(32 * kRankTile) route_topk_rank_kernel(
+    const float* __restrict__ logits, int n_parts, int64_t part_stride,
+    const float* __restrict__ offset, float* __restrict__ logits_out, int64_t N, int E, int k,
+    int score_fn, int renorm, const float* __restrict__ bias, int n_bias_sets,
+    const uint8_t* __restrict__ modality, int32_t* __restrict__ ids, float* __restrict__ gates,
+    int* status, int32_t* __restrict__ local_rank, int32_t* __restrict__ tile_hist) {
+  pdl_wait();
+  extern __shared__ int32_t sm[];
+  int32_t* cnt = sm;       // [E]
+  int32_t* sid = sm + E;   // [kRankTile * k]
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t t0 = (int64_t)blockIdx.x * kRankTile;
+  const int ntok = (int)min((int64_t)kRankTile, N - t0);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  if (w < ntok) {
+    const int64_t t = t0 + w;
+    const TokenSel s = select_token<J>(logits, n_parts, part_stride, offset, logits_out, t, E,
+                                       k, score_fn, renorm, bias, n_bias_sets, modality, status,
+                                       k);
+    if (lane < k) {
+      ids[t * k + lane] = s.e;
+      gates[t * k + lane] = s.g;
+      sid[w * k + lane] = s.e;
+    }
+  }
+  __syncthreads();
+  if (w == 0) {
+    const bool bad = warp_rank_walk(sid, ntok, k, cnt, lane, [&](int t, int j, int r) {
+      local_rank[(t0 + t) * k + j] = r;
+    });
+    if (bad && lane == 0) report_status(status, kStatusInvalidInput);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) tile_hist[(int64_t)blockIdx.x * E + e] = cnt[e];
 }
 
 template <int J>
@@ -187,6 +252,20 @@ cudaError_t launch_j(const float* logits, int n_parts, int64_t part_stride, cons
   launch_pdl(route_topk_kernel<J>, (unsigned)blocks, threads, 0, stream, 
       logits, n_parts, part_stride, offset, logits_out, N, E, k, score_fn, renorm, bias,
       n_bias_sets, modality, ids, gates, status, k_extra, cand, cand_val);
+  return cudaGetLastError();
+}
+
+template <int J>
+cudaError_t launch_rank_j(const float* logits, int n_parts, int64_t part_stride,
+                          const float* offset, float* logits_out, int64_t N, int E, int k,
+                          int score_fn, int renorm, const float* bias, int n_bias_sets,
+                          const uint8_t* modality, int32_t* ids, float* gates, int* status,
+                          int32_t* local_rank, int32_t* tile_hist, cudaStream_t stream) {
+  const int64_t tiles = (N + kRankTile - 1) / kRankTile;
+  const size_t smem = sizeof(int32_t) * ((size_t)E + (size_t)kRankTile * k);
+  launch_pdl(route_topk_rank_kernel<J>, (unsigned)tiles, 32 * kRankTile, smem, stream, logits,
+             n_parts, part_stride, offset, logits_out, N, E, k, score_fn, renorm, bias,
+             n_bias_sets, modality, ids, gates, status, local_rank, tile_hist);
   return cudaGetLastError();
 }
 
@@ -252,6 +331,35 @@ __global__ void __launch_bounds__(256) hash_topk_kernel(const int32_t* __restric
 }
 
 }  // namespace
+
+// Opt-in (MOE_B200_FUSED_TOPK_RANK=1): the fusion saves a launch but its 1024-thread blocks
+// ran the top-k slower than the 256-thread top-k kernel, and the capacity and Switch layers
+// measured 0.7-1.2 % slower per step with it (0.3104 vs 0.3081 ms, 0.2708 vs 0.2675 ms).
+bool fused_topk_rank_enabled() {
+  const char* v = std::getenv("MOE_B200_FUSED_TOPK_RANK");
+  return v != nullptr && v[0] == '1';
+}
+
+cudaError_t launch_route_topk_rank(const float* logits, int n_parts, int64_t part_stride,
+                                   const float* offset, float* logits_out, int64_t N, int E,
+                                   int k, int score_fn, int renorm, const float* bias,
+                                   int n_bias_sets, const uint8_t* modality, int32_t* ids,
+                                   float* gates, int* status, int32_t* local_rank,
+                                   int32_t* tile_hist, cudaStream_t stream, int* launches) {
+  if (N == 0) return cudaSuccess;
+  ++*launches;
+  const int J = (E + 31) / 32;
+#define MOE_ROUTE_RANK_CASE(JJ) \
+  if (J <= JJ)                  \
+    return launch_rank_j<JJ>(logits, n_parts, part_stride, offset, logits_out, N, E, k, score_fn, renorm, bias, n_bias_sets, modality, ids, gates, status, local_rank, tile_hist, stream);
+  MOE_ROUTE_RANK_CASE(1)
+  MOE_ROUTE_RANK_CASE(2)
+  MOE_ROUTE_RANK_CASE(4)
+  MOE_ROUTE_RANK_CASE(8)
+  MOE_ROUTE_RANK_CASE(12)  // E <= kFusedTopkRankMaxE = 384
+#undef MOE_ROUTE_RANK_CASE
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_route_hash(const int32_t* token_ids, int64_t N, int E, int k, int32_t* ids,
                               float* gates, cudaStream_t stream, int* launches) {

@@ -24,6 +24,19 @@ def f64(t):
     return W.bf16_to_f64(t)
 
 
+def small_dispatch(N, k):
+    """Whether the library takes its one-launch dispatch for a batch of N tokens (the rule of
+    moe::use_small_dispatch: N <= 256 and N * k <= 2048)."""
+    return 0 < N <= 256 and N * k <= 2048
+
+
+def forward_launches(N, k, E=8):
+    """Kernel launches of one bf16 moe_forward: router GEMM, top-k, the rank, scan and
+    scatter passes (one launch for all three in a small batch), gate/up and down GEMMs,
+    combine."""
+    return 6 if small_dispatch(N, k) else 8
+
+
 def check_status(ws):
     st = nat.moe_check_status(ws)
     assert st == 0, f"device status {nat.STATUS_NAMES.get(st, st)}"

@@ -332,3 +332,114 @@ def test_layer_with_reroute_policy_device_and_host_buffers():
     layer.forward_host_batches([xh, xh], yh)
     assert torch.equal(yh[0], y_ref.cpu()) and torch.equal(yh[1], y_ref.cpu())
     assert layer.check_status() == 0
+
+
+@pytest.mark.parametrize("N,E,k,cf,sf,nb", [(1, 8, 2, None, 0, 0), (16, 8, 2, 1, 0, 0),
+                                            (64, 256, 8, None, 1, 1), (64, 384, 6, 1.25, 1, 2),
+                                            (200, 64, 2, 1, 0, 0), (256, 1024, 8, 2, 1, 1)])
+def test_small_batch_dispatch_equals_the_three_passes(N, E, k, cf, sf, nb, monkeypatch):
+    """A small batch takes the one-launch dispatch; it must give the three passes' results bit
+    for bit (routing outputs, layout, layer output)."""
+    shape = W.LayerShape("small", N=N, d=256, E=E, k=k, F=128, n_shared=1, score_fn=sf,
+                         n_bias_sets=nb, capacity_factor=cf, w_std=0.05, seed=N + E)
+    t = W.make_inputs(shape, device="cuda")
+    C = O.capacity(N, k, E, cf)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_SMALL_DISPATCH", flag)
+        ws = nat.alloc_workspace(cfg)
+        ro = _route_out(N, E, k)
+        y = torch.empty_like(t["x"])
+        nat.moe_forward(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y,
+                        bias=t.get("bias"), modality=t.get("modality"), route_out=ro, ws=ws)
+        check_status(ws)
+        outs.append((y, ro, nat.moe_last_launch_count()))
+    (y1, r1, l1), (y0, r0, l0) = outs
+    assert (l1, l0) == (6, 8)
+    assert torch.equal(y1, y0)
+    for name in r1:
+        assert torch.equal(r1[name], r0[name]), name
+
+
+def test_small_batch_dispatch_reports_bad_ids_like_the_three_passes(monkeypatch):
+    """Forced routing with an id out of range and an id repeated within a token: both dispatch
+    forms drop them and report MOE_ERR_INVALID_INPUT, with the same layout otherwise."""
+    N, E, k = 12, 6, 3
+    shape = W.LayerShape("bad", N=N, d=128, E=E, k=k, F=64, w_std=0.05, seed=5)
+    t = W.make_inputs(shape, device="cuda")
+    ids = np.tile(np.array([0, 1, 2], np.int32), (N, 1))
+    ids[3] = [4, 4, 5]          # repeated within the token
+    ids[7] = [1, 9, 2]          # out of range
+    gates = np.full((N, k), 1.0 / k, np.float32)
+    cfg = nat.config_from_shape(shape, capacity=4)
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_SMALL_DISPATCH", flag)
+        ws = nat.alloc_workspace(cfg)
+        ro = {n: v for n, v in _route_out(N, E, k).items() if n in ("counts", "demand",
+                                                                    "drop_mask", "offsets")}
+        y = torch.empty_like(t["x"])
+        nat.moe_forward_routed(cfg, x=t["x"], ids=dev(ids), gates=dev(gates), W_gu=t["W_gu"],
+                               W_down=t["W_down"], y=y, route_out=ro, ws=ws)
+        assert nat.moe_check_status(ws) == nat.MOE_ERR_INVALID_INPUT
+        outs.append((y, ro))
+    (y1, r1), (y0, r0) = outs
+    assert torch.equal(y1, y0)
+    for name in r1:
+        assert torch.equal(r1[name], r0[name]), name
+
+
+@pytest.mark.parametrize("N,E,k,cf,sf,nb", [(3000, 384, 6, None, 1, 2), (4097, 64, 2, 1, 0, 0),
+                                            (1000, 300, 32, 0.5, 1, 1), (300, 8, 1, 1.25, 0, 0)])
+def test_topk_fused_with_the_rank_pass_equals_separate_launches(N, E, k, cf, sf, nb, monkeypatch):
+    """Top-k fused with the rank pass (opt-in, MOE_B200_FUSED_TOPK_RANK=1): the outputs must
+    be those of the separate launches, bit for bit."""
+    shape = W.LayerShape("fused", N=N, d=128, E=E, k=k, F=64, n_shared=1, score_fn=sf,
+                         renorm=1, n_bias_sets=nb, capacity_factor=cf, w_std=0.05, seed=N + k)
+    t = W.make_inputs(shape, device="cuda")
+    C = O.capacity(N, k, E, cf)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_FUSED_TOPK_RANK", flag)
+        ws = nat.alloc_workspace(cfg)
+        ro = _route_out(N, E, k)
+        y = torch.empty_like(t["x"])
+        nat.moe_forward(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y,
+                        bias=t.get("bias"), modality=t.get("modality"), route_out=ro, ws=ws)
+        check_status(ws)
+        outs.append((y, ro, nat.moe_last_launch_count()))
+    (y1, r1, l1), (y0, r0, l0) = outs
+    assert (l1, l0) == (7, 8)
+    assert torch.equal(y1, y0)
+    for name in r1:
+        assert torch.equal(r1[name], r0[name]), name
+
+
+@pytest.mark.parametrize("N,E,k,cf,reroute", [(16, 8, 2, None, False), (3000, 64, 2, 1, False),
+                                              (700, 384, 6, 1.25, False), (900, 16, 2, 1, True)])
+def test_debug_mode_checks_the_layout_of_every_call(N, E, k, cf, reroute, monkeypatch):
+    """MOE_B200_DEBUG=1: the fused calls check their dispatch layout on the host (it holds),
+    and moe_check_dispatch on the device outputs agrees."""
+    monkeypatch.setenv("MOE_B200_DEBUG", "1")
+    shape = W.LayerShape("dbg", N=N, d=128, E=E, k=k, F=64, n_shared=1, capacity_factor=cf,
+                         w_std=0.05, seed=N)
+    t = W.make_inputs(shape, device="cuda")
+    C = O.capacity(N, k, E, cf)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    ro = _route_out(N, E, k)
+    y = torch.empty_like(t["x"])
+    fwd = nat.moe_forward_reroute if reroute else nat.moe_forward
+    fwd(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y, route_out=ro,
+        ws=ws)
+    check_status(ws)
+    if not reroute:
+        slot = torch.empty((N, k), dtype=torch.int32, device="cuda")
+        xp = torch.empty((N * k, shape.d), dtype=torch.bfloat16, device="cuda")
+        off = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+        nat.moe_permute(cfg, ids=ro["ids"], drop_mask=ro["drop_mask"], x=t["x"], offsets=off,
+                        slot_row=slot, xp=xp, ws=ws)
+        nat.moe_check_dispatch(cfg, ids=ro["ids"], drop_mask=ro["drop_mask"], counts=ro["counts"],
+                               demand=ro["demand"], offsets=off, slot_row=slot)

@@ -269,8 +269,11 @@ struct Args {
   int band;           // > 0: M blocks of a large group run in bands of this many (decode_tile)
 };
 
-template <int BN, int STAGES>
+// AM: A rows a stage holds (128; 64 for a batch whose groups all fit 64 rows, which leaves
+// room for more stages of weights).
+template <int BN, int STAGES, int AM = BM>
 struct Layout {
+  static constexpr int kStageA = AM * BK * 2;
   static constexpr int kStageB = BN * BK * 2;
   static constexpr int kOffB = STAGES * kStageA;
   static constexpr int kOffStaging = kOffB + STAGES * kStageB;
@@ -426,13 +429,15 @@ __device__ __forceinline__ void epilogue_warp(const Args& p, void* out, uint32_t
   }
 }
 
-template <int BN, int EPI, int STAGES>
+template <int BN, int EPI, int STAGES, int AM = BM>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmAs,
                         const __grid_constant__ CUtensorMap tmB, const Args p) {
   pdl_wait();
-  using L = Layout<BN, STAGES>;
+  using L = Layout<BN, STAGES, AM>;
+  // AM = 64: every tile has at most 64 rows (the host guarantees it) and runs M = 64 MMAs
+  constexpr bool kAll64 = AM < BM;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -523,8 +528,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          mbar_expect_tx(&full[stage], kStageA + L::kStageB);
-          tma_load_2d(sA + stage * kStageA, mA, &full[stage], kb * BK, a_row);
+          mbar_expect_tx(&full[stage], L::kStageA + L::kStageB);
+          tma_load_2d(sA + stage * L::kStageA, mA, &full[stage], kb * BK, a_row);
           uint8_t* b_dst = sB + stage * L::kStageB;
           if (EPI == kEpiSwiglu) {
             tma_load_3d(b_dst, &tmB, &full[stage], kb * BK, n_blk * (BN / 2), g);
@@ -567,7 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int g, m_blk, n_blk;
         decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
         const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
-        const uint32_t idesc = (p.m64_tails && cnt - m_blk * BM <= 64) ? kIdesc64 : kIdesc;
+        const uint32_t idesc =
+            (kAll64 || (p.m64_tails && cnt - m_blk * BM <= 64)) ? kIdesc64 : kIdesc;
         if (!mbar_wait(&tempty[acc], aph ^ 1, s_abort, p.status)) {
           ok = false;
           break;
@@ -581,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * kStageA);
+          const uint32_t a0 = smem_u32(sA + stage * L::kStageA);
           const uint32_t b0 = smem_u32(sB + stage * L::kStageB);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
@@ -623,7 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rows_valid = min(BM, cnt - m_blk * BM);
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       // an M = 64 accumulator holds rows 16q .. 16q + 15 in lanes 32q .. 32q + 15
-      const bool m64 = p.m64_tails && rows_valid <= 64;
+      const bool m64 = kAll64 || (p.m64_tails && rows_valid <= 64);
       const int row_base = m64 ? q * 16 : q * 32;
       const int rows_w = m64 ? min(rows_valid, q * 16 + 16) : rows_valid;
 
@@ -1366,11 +1372,11 @@ int band_for(const GroupedGemm& g, int bmt) {
   return (int)std::max<int64_t>(1, l2_bytes() / 3 / tile_bytes);
 }
 
-template <int BN, int EPI, int STAGES>
+template <int BN, int EPI, int STAGES, int AM = BM>
 cudaError_t launch_t(const GroupedGemm& g, const CUtensorMap& mA, const CUtensorMap& mAs,
                      const CUtensorMap& mB, cudaStream_t stream, int grid) {
-  auto kern = grouped_gemm_kernel<BN, EPI, STAGES>;
-  const size_t smem = Layout<BN, STAGES>::bytes(g.n_routed + g.has_shared);
+  auto kern = grouped_gemm_kernel<BN, EPI, STAGES, AM>;
+  const size_t smem = Layout<BN, STAGES, AM>::bytes(g.n_routed + g.has_shared);
   static bool done[kMaxDev] = {};
   const cudaError_t e = allow_max_smem(kern, done);
   if (e != cudaSuccess) return e;
@@ -1494,6 +1500,17 @@ int pick_bn_1sm(const GroupedGemm& g) {
   return tail_eff(128) > tail_eff(256) + 0.02 ? 128 : 256;
 }
 
+// 64-row A stages: every group (and the shared group) has at most 64 rows, so each tile runs
+// M = 64 MMAs and a stage needs only 64 A rows; the freed shared memory holds more stages of
+// weights (decode: more weight bytes in flight per SM).  MOE_B200_DECODE_A64=0 turns it off.
+bool use_a64(const GroupedGemm& g) {
+  if (g.epilogue == kEpiStoreF32 || g.k_splits > 1 || use_swap(g) || use_two_sm(g)) return false;
+  if (g.n_routed > 0 && (g.max_group_rows <= 0 || g.max_group_rows > 64)) return false;
+  if (g.has_shared && g.shared_rows > 64) return false;
+  const char* v = std::getenv("MOE_B200_DECODE_A64");
+  return !(v != nullptr && v[0] == '0');
+}
+
 }  // namespace tc
 
 cudaError_t launch_wait_selftest(int* status, uint64_t limit_ns, int* out, cudaStream_t stream,
@@ -1537,6 +1554,9 @@ const char* grouped_gemm_kernel_name(const GroupedGemm& g) {
     }
   }
   if (use_two_sm(g)) return "grouped_gemm_2sm_kernel (2-SM, 256x256 tiles)";
+  if (use_a64(g))
+    return pick_bn_1sm(g) == 128 ? "grouped_gemm_kernel (1-SM, 128x128 tiles, 64-row A stages)"
+                                 : "grouped_gemm_kernel (1-SM, 128x256 tiles, 64-row A stages)";
   return pick_bn_1sm(g) == 128 ? "grouped_gemm_kernel (1-SM, 128x128 tiles)"
                                : "grouped_gemm_kernel (1-SM, 128x256 tiles)";
 }
@@ -1579,12 +1599,14 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
     BN = two_sm ? 256 : pick_bn_1sm(g);
   }
   const int box_b = two_sm ? 128 : (g.epilogue == kEpiSwiglu) ? BN / 2 : BN;
+  const bool a64 = use_a64(g);
+  const int box_a = a64 ? 64 : BM;
   CUtensorMap mA, mAs, mB;
   const void* a_ptr = g.a != nullptr ? g.a : g.a_shared;
   const int64_t a_rows = g.a != nullptr ? g.rows_a : g.rows_a_shared;
-  if (!make_map(&mA, a_ptr, g.K, std::max<int64_t>(a_rows, 1), 0, BM) ||
+  if (!make_map(&mA, a_ptr, g.K, std::max<int64_t>(a_rows, 1), 0, box_a) ||
       !make_map(&mAs, g.a_shared != nullptr ? g.a_shared : a_ptr, g.K,
-                std::max<int64_t>(g.a_shared != nullptr ? g.rows_a_shared : a_rows, 1), 0, BM) ||
+                std::max<int64_t>(g.a_shared != nullptr ? g.rows_a_shared : a_rows, 1), 0, box_a) ||
       !make_map(&mB, g.b, g.K, g.rows_b, g.groups_b, box_b)) {
     *why = "cuTensorMapEncodeTiled failed (pointer alignment, strides or driver entry point)";
     return cudaErrorInvalidValue;
@@ -1607,6 +1629,21 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
       case kEpiSwiglu: return launch_2sm<kEpiSwiglu, 6>(g, mA, mAs, mB, stream, pairs);
       case kEpiRelu: return launch_2sm<kEpiRelu, 6>(g, mA, mAs, mB, stream, pairs);
       default: return launch_2sm<kEpiStoreBf16, 6>(g, mA, mAs, mB, stream, pairs);
+    }
+  }
+  if (a64) {
+    // 64-row A stages: 8 stages of 24 KB (128-wide tiles) or 5 of 40 KB (256-wide)
+    if (BN == 128) {
+      switch (g.epilogue) {
+        case kEpiSwiglu: return launch_t<128, kEpiSwiglu, 8, 64>(g, mA, mAs, mB, stream, grid);
+        case kEpiRelu: return launch_t<128, kEpiRelu, 8, 64>(g, mA, mAs, mB, stream, grid);
+        default: return launch_t<128, kEpiStoreBf16, 8, 64>(g, mA, mAs, mB, stream, grid);
+      }
+    }
+    switch (g.epilogue) {
+      case kEpiSwiglu: return launch_t<256, kEpiSwiglu, 5, 64>(g, mA, mAs, mB, stream, grid);
+      case kEpiRelu: return launch_t<256, kEpiRelu, 5, 64>(g, mA, mAs, mB, stream, grid);
+      default: return launch_t<256, kEpiStoreBf16, 5, 64>(g, mA, mAs, mB, stream, grid);
     }
   }
   if (BN == 128 && g.epilogue != kEpiStoreF32) {

@@ -159,6 +159,8 @@ struct GroupedGemm {
   int* status;
   int k_splits = 1;        // > 1 (fp32 store only): K split in slices, slice s written at
   int64_t split_rows = 0;  // out rows [s * split_rows, ...): partial sums, col_bias ignored
+  int64_t max_group_rows = -1;  // > 0: no routed group has more rows (lets a batch whose
+                                // groups all fit 64 rows use 64-row A stages)
 };
 
 cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* launches,

@@ -239,13 +239,6 @@ LogitSrc finished_logits(const float* z) { return LogitSrc{z, 1, 0, nullptr, nul
 
 int router_splits(const moe_config& c) {
   if (c.dtype != MOE_DT_BF16 || c.N == 0) return 1;
-  if (const char* v = std::getenv("MOE_B200_ROUTER_SPLITS")) {
-    // a fixed slice count (A/B measurements): at most kMaxLogitSplits, no empty slice
-    const int nk = (c.d + 63) / 64;
-    const int want = std::max(1, std::min({std::atoi(v), kMaxLogitSplits, nk}));
-    const int per = (nk + want - 1) / want;
-    return (nk + per - 1) / per;
-  }
   const int bn = moe::router_tile_n(c.E);
   const int64_t tiles = ((c.N + 127) / 128) * ((c.E + bn - 1) / bn);
   const int nk = (c.d + 63) / 64;
@@ -495,9 +488,12 @@ moe::GroupedGemm down_gemm(const moe_config& c, int64_t Nk, const void* h, const
 moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
                      const int32_t* offsets, const void* x, const void* W_gu,
                      const void* W_down, void* ye, cudaStream_t st, int* launches,
-                     int64_t R = -1, void* y_shared = nullptr) {
+                     int64_t R = -1, void* y_shared = nullptr, int64_t group_rows_max = -1) {
   if (c.N == 0) return MOE_OK;
   const int64_t Nk = R >= 0 ? R : c.N * (int64_t)c.k;
+  // the most rows a routed group can have: N in the layer's own compact layout (a token
+  // picks an expert at most once); otherwise what the caller states, or the whole region
+  const int64_t grp_max = group_rows_max > 0 ? group_rows_max : Nk;
   if (c.dtype == MOE_DT_F32) {
     MOE_CUDA(moe::launch_ffn_f32((const float*)xp, (const float*)x, offsets, c.N, Nk, c.d, c.E,
                                  c.F, c.n_shared, c.act, c.clamp, (const float*)W_gu,
@@ -509,12 +505,14 @@ moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
   }
   int* status = at<int>(ws, L.status);
   void* h = at<char>(ws, L.h);
-  const moe::GroupedGemm g1 = gate_up_gemm(c, Nk, xp, x, W_gu, offsets, h, status);
+  moe::GroupedGemm g1 = gate_up_gemm(c, Nk, xp, x, W_gu, offsets, h, status);
+  g1.max_group_rows = grp_max;
   const char* why = "gate/up GEMM launch";
   MOE_CUDA(moe::launch_grouped_gemm(g1, st, launches, &why), why);
   prof_mark(st);
 
   moe::GroupedGemm g2 = down_gemm(c, Nk, h, W_down, offsets, ye, status);
+  g2.max_group_rows = grp_max;
   if (y_shared != nullptr && c.n_shared) {
     g2.out_shared = y_shared;
     g2.shared_out_row0 = 0;
@@ -631,7 +629,7 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
                                   offsets, at<int32_t>(ws, L.slot_row),
                                   at<int32_t>(ws, L.row_token), c.capacity, st));
   // fused layer: the shared expert's rows go straight into y (bf16), completed by the combine
-  MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, launches, -1, y));
+  MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, launches, -1, y, c.N));
   MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, launches, -1, true));
   g_prof.recording = false;
   return MOE_OK;
@@ -797,10 +795,12 @@ moe_status moe_ffn_kernels(const moe_config* cfg, char* gate_up, char* down, siz
   const char* dn = "ffn_down_f32_kernel (SIMT fp32)";
   if (c.dtype == MOE_DT_BF16) {
     const int64_t Nk = c.N * (int64_t)c.k;
-    gu = moe::grouped_gemm_kernel_name(
-        gate_up_gemm(c, Nk, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr));
-    dn = moe::grouped_gemm_kernel_name(
-        down_gemm(c, Nk, nullptr, nullptr, nullptr, nullptr, nullptr));
+    // the choice of the fused forward calls, whose groups have at most N rows
+    moe::GroupedGemm g1 = gate_up_gemm(c, Nk, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+    moe::GroupedGemm g2 = down_gemm(c, Nk, nullptr, nullptr, nullptr, nullptr, nullptr);
+    g1.max_group_rows = g2.max_group_rows = c.N;
+    gu = moe::grouped_gemm_kernel_name(g1);
+    dn = moe::grouped_gemm_kernel_name(g2);
   }
   if (c.N == 0) gu = dn = "none";
   for (auto [buf, name] : {std::pair<char*, const char*>{gate_up, gu}, {down, dn}}) {
@@ -900,7 +900,7 @@ moe_status moe_forward_routed(const moe_config* cfg, const void* x, const int32_
   MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, c.capacity, demand, counts, offsets,
                          at<int32_t>(ws, L.slot_row), at<int32_t>(ws, L.row_token), drop, x, xp,
                          st, &launches));
-  MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, &launches, -1, y));
+  MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, &launches, -1, y, c.N));
   MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, &launches, -1, true));
   g_last_launches = launches;
   return MOE_OK;
@@ -1045,7 +1045,8 @@ moe_status moe_forward_padded(const moe_config* cfg, const void* x, const void* 
   MOE_CUDA(moe::launch_zero_padding(counts, c.E, c.capacity, xp, (int)(c.d * el_size(c)),
                                     row_token, st, &launches),
            "zero padding");
-  MOE_TRY(stage_ffn(c, L, ws, xp, offsets_pad, x, W_gu, W_down, ye, st, &launches, R, y));
+  MOE_TRY(stage_ffn(c, L, ws, xp, offsets_pad, x, W_gu, W_down, ye, st, &launches, R, y,
+                    c.capacity));
   MOE_TRY(stage_combine(c, ye, slot_row, gates, y, st, &launches, R, true));
   g_last_launches = launches;
   return MOE_OK;

@@ -443,3 +443,34 @@ def test_debug_mode_checks_the_layout_of_every_call(N, E, k, cf, reroute, monkey
                         slot_row=slot, xp=xp, ws=ws)
         nat.moe_check_dispatch(cfg, ids=ro["ids"], drop_mask=ro["drop_mask"], counts=ro["counts"],
                                demand=ro["demand"], offsets=off, slot_row=slot)
+
+
+@pytest.mark.parametrize("N,d,E,k,F,S,cf,act", [(16, 256, 8, 2, 384, 0, None, W.SWIGLU),
+                                                (64, 512, 48, 6, 256, 1, None, W.SWIGLU),
+                                                (37, 136, 6, 3, 200, 1, 1.25, W.SWIGLU),
+                                                (1, 128, 4, 2, 128, 1, None, W.SWIGLU),
+                                                (50, 192, 8, 2, 320, 0, 1, W.RELU)])
+def test_decode_batch_64_row_stages_equal_full_stages(N, d, E, k, F, S, cf, act, monkeypatch):
+    """A batch of at most 64 tokens runs the 1-SM GEMMs with 64-row A stages (every group fits
+    64 rows); the layer output, compact and padded, must be the bits of the 128-row stages."""
+    shape = W.LayerShape("a64", N=N, d=d, E=E, k=k, F=F, n_shared=S, act=act,
+                         capacity_factor=cf, w_std=0.05, seed=N + d)
+    t = W.make_inputs(shape, device="cuda")
+    C = O.capacity(N, k, E, cf)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    names = []
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MOE_B200_DECODE_A64", flag)
+        names.append(nat.moe_ffn_kernels(cfg))
+        ws = nat.alloc_workspace(cfg)
+        ys = []
+        for fwd in ([nat.moe_forward] + ([nat.moe_forward_padded] if C > 0 else [])):
+            y = torch.empty_like(t["x"])
+            fwd(cfg, x=t["x"], W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], y=y, ws=ws)
+            check_status(ws)
+            ys.append(y)
+        outs.append(ys)
+    assert all("64-row A stages" in n for n in names[0]) and not any("64-row" in n for n in names[1])
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)

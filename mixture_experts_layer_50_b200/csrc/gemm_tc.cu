@@ -436,8 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tmB, const Args p) {
   pdl_wait();
   using L = Layout<BN, STAGES, AM>;
-  // AM = 64: every tile has at most 64 rows (the host guarantees it) and runs M = 64 MMAs
+  // AM = 64: groups are cut into 64-row tiles, each running M = 64 MMAs
   constexpr bool kAll64 = AM < BM;
+  constexpr int TM = AM;  // rows of an output tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -467,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int local = 0;
     for (int g = g0; g < g1; ++g) {
       const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
-      local += ((cnt + BM - 1) / BM) * nt;
+      local += ((cnt + TM - 1) / TM) * nt;
     }
     int incl = local;
 #pragma unroll
@@ -479,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = g0; g < g1; ++g) {
       s_start[g] = run;
       const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
-      run += ((cnt + BM - 1) / BM) * nt;
+      run += ((cnt + TM - 1) / TM) * nt;
     }
     if (lane == 31) s_start[G] = incl;
     if (lane == 0) {
@@ -518,10 +519,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         int g, m_blk, n_blk;
-        decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
+        decode_tile<TM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
         const int kb0 = (tile % ks_n) * kper, kb1 = min(nk, kb0 + kper);
         const bool sh = g >= p.n_routed;
-        const int a_row = (sh ? p.shared_a_row0 : p.offsets[g]) + m_blk * BM;
+        const int a_row = (sh ? p.shared_a_row0 : p.offsets[g]) + m_blk * TM;
         const CUtensorMap* mA = sh ? &tmAs : &tmA;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, p.status)) {
@@ -570,10 +571,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         int g, m_blk, n_blk;
-        decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
+        decode_tile<TM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
         const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
         const uint32_t idesc =
-            (kAll64 || (p.m64_tails && cnt - m_blk * BM <= 64)) ? kIdesc64 : kIdesc;
+            (kAll64 || (p.m64_tails && cnt - m_blk * TM <= 64)) ? kIdesc64 : kIdesc;
         if (!mbar_wait(&tempty[acc], aph ^ 1, s_abort, p.status)) {
           ok = false;
           break;
@@ -615,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       int g, m_blk, n_blk;
-      decode_tile<BM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
+      decode_tile<TM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       // warp-uniform decision: tcgen05.ld below needs all 32 lanes
@@ -624,9 +625,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool sh = g >= p.n_routed;
       const int cnt = sh ? p.shared_rows : p.offsets[g + 1] - p.offsets[g];
-      const int64_t out_row0 = (int64_t)(sh ? p.shared_out_row0 : p.offsets[g]) + m_blk * BM +
+      const int64_t out_row0 = (int64_t)(sh ? p.shared_out_row0 : p.offsets[g]) + m_blk * TM +
                                (int64_t)(tile % ks_n) * p.split_rows;
-      const int rows_valid = min(BM, cnt - m_blk * BM);
+      const int rows_valid = min(TM, cnt - m_blk * TM);
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       // an M = 64 accumulator holds rows 16q .. 16q + 15 in lanes 32q .. 32q + 15
       const bool m64 = kAll64 || (p.m64_tails && rows_valid <= 64);
@@ -1500,15 +1501,22 @@ int pick_bn_1sm(const GroupedGemm& g) {
   return tail_eff(128) > tail_eff(256) + 0.02 ? 128 : 256;
 }
 
-// 64-row A stages: every group (and the shared group) has at most 64 rows, so each tile runs
-// M = 64 MMAs and a stage needs only 64 A rows; the freed shared memory holds more stages of
-// weights (decode: more weight bytes in flight per SM).  MOE_B200_DECODE_A64=0 turns it off.
+// 64-row tiles: groups are cut into 64-row output tiles, each running M = 64 MMAs, so a stage
+// holds 64 A rows and the freed shared memory holds more stages of weights (more weight bytes
+// in flight per SM).  Taken when every group fits one such tile (the caller's bound on a
+// routed group, and the shared group): decode-sized batches.  With larger groups it lost
+// badly (Mixtral-shaped, 256 tokens, about 64 rows per expert: 0.503 -> 0.587 ms per step;
+// 4096 tokens: 2.36 -> 3.09 ms): the weights of a group are then read by two M tiles and the
+// M = 64 MMAs halve the rows per instruction.
+// MOE_B200_DECODE_A64=0 turns it off; =2 forces it on any group sizes (tests).
 bool use_a64(const GroupedGemm& g) {
   if (g.epilogue == kEpiStoreF32 || g.k_splits > 1 || use_swap(g) || use_two_sm(g)) return false;
-  if (g.n_routed > 0 && (g.max_group_rows <= 0 || g.max_group_rows > 64)) return false;
-  if (g.has_shared && g.shared_rows > 64) return false;
   const char* v = std::getenv("MOE_B200_DECODE_A64");
-  return !(v != nullptr && v[0] == '0');
+  if (v != nullptr && v[0] == '0') return false;
+  if (v != nullptr && v[0] == '2') return true;
+  if (g.has_shared && g.shared_rows > 64) return false;
+  if (g.n_routed > 0 && (g.max_group_rows <= 0 || g.max_group_rows > 64)) return false;
+  return true;
 }
 
 }  // namespace tc
@@ -1555,8 +1563,8 @@ const char* grouped_gemm_kernel_name(const GroupedGemm& g) {
   }
   if (use_two_sm(g)) return "grouped_gemm_2sm_kernel (2-SM, 256x256 tiles)";
   if (use_a64(g))
-    return pick_bn_1sm(g) == 128 ? "grouped_gemm_kernel (1-SM, 128x128 tiles, 64-row A stages)"
-                                 : "grouped_gemm_kernel (1-SM, 128x256 tiles, 64-row A stages)";
+    return pick_bn_1sm(g) == 128 ? "grouped_gemm_kernel (1-SM, 64x128 tiles)"
+                                 : "grouped_gemm_kernel (1-SM, 64x256 tiles)";
   return pick_bn_1sm(g) == 128 ? "grouped_gemm_kernel (1-SM, 128x128 tiles)"
                                : "grouped_gemm_kernel (1-SM, 128x256 tiles)";
 }
@@ -1614,9 +1622,10 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
   // grid: at most one CTA per SM, no more than an upper bound of the tile count
   const int out_per_tile = (g.epilogue == kEpiSwiglu) ? BN / 2 : BN;
   const int64_t nt = (g.n_out + out_per_tile - 1) / out_per_tile;
+  const int tm = a64 ? 64 : BM;  // rows of an output tile
   int64_t mtiles = 0;
-  if (g.n_routed > 0) mtiles += (g.max_rows_routed + BM - 1) / BM + g.n_routed;
-  if (g.has_shared) mtiles += (g.shared_rows + BM - 1) / BM;
+  if (g.n_routed > 0) mtiles += (g.max_rows_routed + tm - 1) / tm + g.n_routed;
+  if (g.has_shared) mtiles += (g.shared_rows + tm - 1) / tm;
   const int64_t bound = mtiles * nt * std::max(1, g.k_splits);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(num_sms(), bound));
   ++*launches;

@@ -73,8 +73,8 @@ cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_ran
 // The three passes in one launch for a small batch (N <= kSmallDispatchMaxTokens and
 // N * k <= kSmallDispatchMaxSlots): the same outputs, plus the device status for bad ids.
 constexpr int kSmallDispatchThreads = 1024;   // >= E (at most 1024)
-constexpr int kSmallDispatchMaxTokens = 256;
-constexpr int kSmallDispatchMaxSlots = 2048;
+constexpr int kSmallDispatchMaxTokens = 64;
+constexpr int kSmallDispatchMaxSlots = 1024;
 bool use_small_dispatch(int64_t N, int k, int E);   // MOE_B200_SMALL_DISPATCH=0: never
 cudaError_t launch_dispatch_small(const int32_t* ids, const uint8_t* drop_in, int64_t N, int k,
                                   int E, int64_t C, const int32_t* cap_e, int32_t* demand,

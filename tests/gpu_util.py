@@ -26,15 +26,16 @@ def f64(t):
 
 def small_dispatch(N, k):
     """Whether the library takes its one-launch dispatch for a batch of N tokens (the rule of
-    moe::use_small_dispatch: N <= 256 and N * k <= 2048)."""
-    return 0 < N <= 256 and N * k <= 2048
+    moe::use_small_dispatch: N <= 64 and N * k <= 1024)."""
+    return 0 < N <= 64 and N * k <= 1024
 
 
-def forward_launches(N, k, E=8):
-    """Kernel launches of one bf16 moe_forward: router GEMM, top-k, the rank, scan and
-    scatter passes (one launch for all three in a small batch), gate/up and down GEMMs,
-    combine."""
-    return 6 if small_dispatch(N, k) else 8
+def forward_launches(N, k, E=8, S=0, bf16=True):
+    """Kernel launches of one moe_forward: router GEMM, top-k, the rank, scan and scatter
+    passes (one launch for all three in a small batch), gate/up and down GEMMs, combine; with
+    a shared expert (bf16) its own gate/up and down GEMMs on the side stream."""
+    n = 6 if small_dispatch(N, k) else 8
+    return n + (2 if S and bf16 and N > 0 and k <= 2 else 0)
 
 
 def check_status(ws):

@@ -188,13 +188,15 @@ def test_ffn_kernel_choice(nat):
     from mixture_experts_layer_50_b200 import workloads as W
     one_256, one_128 = "1-SM, 128x256 tiles", "1-SM, 128x128 tiles"
     two = "2-SM, 256x256 tiles"
+    # decode-sized batches (every group within 64 rows): 64-row tiles
+    d64_256, d64_128 = "1-SM, 64x256 tiles", "1-SM, 64x128 tiles"
     want = {
-        "mixtral-n16": (one_128, one_256), "mixtral-n256": (one_128, one_256),
+        "mixtral-n16": (d64_128, d64_256), "mixtral-n256": (one_128, one_256),
         # gate/up: 235 MB weight panels per expert stay on the 1-SM kernel
         "mixtral-n4096": (one_256, two), "mixtral-n16384": (one_256, two),
         # ~256 rows per expert: 256-row tiles would pad a third more rows
-        "dsv3-n64": (one_256, one_256), "dsv3-n8192": (one_256, one_256),
-        "v41flash-n64": (one_256, one_256), "v41flash-n16384": (one_256, one_256),
+        "dsv3-n64": (d64_256, d64_256), "dsv3-n8192": (one_256, one_256),
+        "v41flash-n64": (d64_256, d64_256), "v41flash-n16384": (one_256, one_256),
         # the shared expert's 16384 rows dominate; 11.5 MB panels
         "capacity-cf1": (two, two), "capacity-cfinf": (two, two),
         "switch-cf1": (two, two), "switch-cfinf": (two, two),
@@ -213,7 +215,7 @@ def test_ffn_kernel_choice(nat):
     assert nat.lib.moe_ffn_kernels(ctypes.byref(_cfg(nat, k=9)), buf, None, 8) == nat.MOE_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("path,kind", [("1sm", "1-SM"), ("1sm128", "1-SM, 128x128 tiles"),
+@pytest.mark.parametrize("path,kind", [("1sm", "1-SM"), ("1sm128", "x128 tiles"),
                                        ("2sm", "2-SM, 256x256 tiles"), ("swap", "token-in-N")])
 def test_ffn_kernel_override(nat, path, kind, monkeypatch):
     """MOE_B200_GEMM_PATH forces one grouped GEMM for both projections ("1sm" keeps the

@@ -217,12 +217,13 @@ FFN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["1sm", "1sm128", "2sm", "swap"])
+@pytest.mark.parametrize("path", ["1sm", "1sm128", "2sm", "swap", "1sm64"])
 @pytest.mark.parametrize("N,d,E,k,F,S,act,clamp", FFN_CASES)
 def test_expert_ffn(N, d, E, k, F, S, act, clamp, path, monkeypatch):
-    # every grouped-GEMM variant (1-SM 128x256 and 128x128 tiles, 2-SM 256x256, and the
-    # token-in-N kernel with weights in M) on every case
-    monkeypatch.setenv("MOE_B200_GEMM_PATH", path)
+    # every grouped-GEMM variant (1-SM 128x256 and 128x128 tiles, 2-SM 256x256, the
+    # token-in-N kernel with weights in M, and the 1-SM kernel forced to 64-row tiles) on
+    # every case
+    _set_path(path, monkeypatch)
     shape = W.LayerShape("t", N=N, d=d, E=E, k=k, F=F, n_shared=S, act=act, clamp=clamp,
                          w_std=0.08, seed=N + d)
     t = W.make_inputs(shape, device="cuda")
@@ -252,13 +253,25 @@ def test_expert_ffn(N, d, E, k, F, S, act, clamp, path, monkeypatch):
     assert_close_layer(got[rows], ref[rows])
 
 
-@pytest.mark.parametrize("path", ["1sm", "swap", "2sm"])
+def _set_path(path, monkeypatch):
+    """MOE_B200_GEMM_PATH for one kernel variant; "1sm64" is the 1-SM kernel forced to
+    64-row tiles (MOE_B200_DECODE_A64=2), which the layer otherwise takes for small groups."""
+    if path == "1sm64":
+        monkeypatch.setenv("MOE_B200_GEMM_PATH", "1sm")
+        monkeypatch.setenv("MOE_B200_DECODE_A64", "2")
+    else:
+        monkeypatch.setenv("MOE_B200_GEMM_PATH", path)
+        monkeypatch.setenv("MOE_B200_DECODE_A64", "0")
+
+
+@pytest.mark.parametrize("path", ["1sm", "swap", "2sm", "1sm64"])
 def test_expert_ffn_group_sizes_around_the_tile_edges(path, monkeypatch):
     """Groups of 0 ... 513 rows around every tile edge: the token-in-N kernel rounds a group's
     last row block up to 16 rows and loads it in 32-row boxes; the 1-SM kernel pads to
-    128-row tiles (M = 64 for a last tile of at most 64 rows); the 2-SM kernel to 256-row
-    tiles."""
-    monkeypatch.setenv("MOE_B200_GEMM_PATH", path)
+    128-row tiles (M = 64 for a last tile of at most 64 rows), or cuts groups into 64-row
+    tiles; the 2-SM kernel pads to 256-row tiles (128 with a half tile for the down
+    projection)."""
+    _set_path(path, monkeypatch)
     sizes = [0, 1, 15, 16, 17, 31, 32, 33, 127, 128, 129, 255, 256, 257, 300, 383, 384, 385,
              511, 512, 513]
     E, k, d, F = len(sizes), 1, 256, 384
@@ -363,7 +376,7 @@ def test_forward_toy_fp32_page_config():
     assert_close_layer(host(y)[same], ref[same], bf16=False)
     # per-expert load fractions (bincount / N) sum to k
     assert ro["demand"].sum() / shape.N == pytest.approx(2.0)
-    assert launches == forward_launches(shape.N, shape.k, shape.E)
+    assert launches == forward_launches(shape.N, shape.k, shape.E, shape.n_shared, shape.dtype == W.BF16)
 
 
 def tile_edge_tokens(route, N, n_shared, tile_rows=(128, 256)):
@@ -439,7 +452,7 @@ def _forward_case(name, N=None, sample=None, full_range=False):
           f"{int(tokens.min()) if tokens.size else -1}..{int(tokens.max()) if tokens.size else -1}, "
           f"output max err {mx:.2e} x max|ref|, rms {rms:.2e}")
     assert_close_layer(host(y)[tokens][keep], ref[keep])
-    assert launches == forward_launches(shape.N, shape.k, shape.E)
+    assert launches == forward_launches(shape.N, shape.k, shape.E, shape.n_shared, shape.dtype == W.BF16)
     return ro
 
 
@@ -642,7 +655,7 @@ def test_forward_random_configurations(seed):
     rel = np.abs(ro["gates"] - info["gates"]) / np.maximum(np.abs(info["gates"]), 1e-30)
     assert rel.max() <= 1e-5, (shape, rel.max())
     assert_close_layer(host(y), ref)
-    assert launches == forward_launches(shape.N, shape.k, shape.E)
+    assert launches == forward_launches(shape.N, shape.k, shape.E, shape.n_shared, shape.dtype == W.BF16)
 
 
 def _random_shape_wide(seed):
@@ -724,7 +737,7 @@ def test_forward_largest_expert_count_and_k(sf, nb, cf):
     for name in ("ids", "drop_mask", "counts", "demand", "offsets"):
         np.testing.assert_array_equal(ro[name], info[name], err_msg=name)
     assert_close_layer(host(y), ref)
-    assert launches == forward_launches(shape.N, shape.k, shape.E)
+    assert launches == forward_launches(shape.N, shape.k, shape.E, shape.n_shared, shape.dtype == W.BF16)
 
 
 @pytest.mark.parametrize("seed", range(12))

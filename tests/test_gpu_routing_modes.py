@@ -336,7 +336,7 @@ def test_layer_with_reroute_policy_device_and_host_buffers():
 
 @pytest.mark.parametrize("N,E,k,cf,sf,nb", [(1, 8, 2, None, 0, 0), (16, 8, 2, 1, 0, 0),
                                             (64, 256, 8, None, 1, 1), (64, 384, 6, 1.25, 1, 2),
-                                            (200, 64, 2, 1, 0, 0), (256, 1024, 8, 2, 1, 1)])
+                                            (48, 64, 2, 1, 0, 0), (64, 1024, 8, 2, 1, 1)])
 def test_small_batch_dispatch_equals_the_three_passes(N, E, k, cf, sf, nb, monkeypatch):
     """A small batch takes the one-launch dispatch; it must give the three passes' results bit
     for bit (routing outputs, layout, layer output)."""
@@ -356,7 +356,8 @@ def test_small_batch_dispatch_equals_the_three_passes(N, E, k, cf, sf, nb, monke
         check_status(ws)
         outs.append((y, ro, nat.moe_last_launch_count()))
     (y1, r1, l1), (y0, r0, l0) = outs
-    assert (l1, l0) == (6, 8)
+    side = 2 if k <= 2 else 0   # the shared expert's two GEMMs on the side stream
+    assert (l1, l0) == (6 + side, 8 + side)
     assert torch.equal(y1, y0)
     for name in r1:
         assert torch.equal(r1[name], r0[name]), name
@@ -411,7 +412,8 @@ def test_topk_fused_with_the_rank_pass_equals_separate_launches(N, E, k, cf, sf,
         check_status(ws)
         outs.append((y, ro, nat.moe_last_launch_count()))
     (y1, r1, l1), (y0, r0, l0) = outs
-    assert (l1, l0) == (7, 8)
+    side = 2 if k <= 2 else 0   # the shared expert's two GEMMs on the side stream
+    assert (l1, l0) == (7 + side, 8 + side)
     assert torch.equal(y1, y0)
     for name in r1:
         assert torch.equal(r1[name], r0[name]), name
@@ -451,8 +453,9 @@ def test_debug_mode_checks_the_layout_of_every_call(N, E, k, cf, reroute, monkey
                                                 (1, 128, 4, 2, 128, 1, None, W.SWIGLU),
                                                 (50, 192, 8, 2, 320, 0, 1, W.RELU)])
 def test_decode_batch_64_row_stages_equal_full_stages(N, d, E, k, F, S, cf, act, monkeypatch):
-    """A batch of at most 64 tokens runs the 1-SM GEMMs with 64-row A stages (every group fits
-    64 rows); the layer output, compact and padded, must be the bits of the 128-row stages."""
+    """A batch of at most 64 tokens runs the 1-SM GEMMs with 64-row tiles (every group fits
+    one); the layer output, compact and padded, must be the bits of the 128-row tiles (whose
+    tiles of at most 64 rows run the same M = 64 MMAs)."""
     shape = W.LayerShape("a64", N=N, d=d, E=E, k=k, F=F, n_shared=S, act=act,
                          capacity_factor=cf, w_std=0.05, seed=N + d)
     t = W.make_inputs(shape, device="cuda")
@@ -471,6 +474,33 @@ def test_decode_batch_64_row_stages_equal_full_stages(N, d, E, k, F, S, cf, act,
             check_status(ws)
             ys.append(y)
         outs.append(ys)
-    assert all("64-row A stages" in n for n in names[0]) and not any("64-row" in n for n in names[1])
+    assert all("1-SM, 64x" in n for n in names[0]) and not any("64x" in n for n in names[1])
     for a, b in zip(*outs):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name,N,k", [("capacity-cf1", 3000, 2), ("dsv3-n64", 64, 2),
+                                      ("v41flash-n64", 300, 1), ("switch-cf1", 777, 1)])
+def test_shared_expert_on_the_side_stream_gives_the_same_bits(name, N, k, monkeypatch):
+    """The shared expert's GEMMs on the library's side stream (concurrent with the routing
+    chain) give the bits of the shared group inside the routed GEMM launches, eagerly and
+    replayed from a CUDA graph that captured the fork and the join."""
+    shape = W.PRESETS[name].replace(N=N, d=256, F=256, k=k)
+    t = W.make_inputs(shape, device="cuda")
+    from mixture_experts_layer_50_b200 import MoELayer
+    ys = []
+    for flag in ("0", "1"):
+        monkeypatch.setenv("MOE_B200_SHARED_STREAM", flag)
+        layer = MoELayer.from_workload(shape, t)
+        y = layer.forward(t["x"], modality=t.get("modality")).clone()
+        assert layer.check_status() == 0
+        launches = nat.moe_last_launch_count()
+        yg = torch.empty_like(y)
+        for _ in range(2):
+            layer.forward_graphed(t["x"], yg, modality=t.get("modality"))
+        torch.cuda.synchronize()
+        assert torch.equal(yg, y)
+        ys.append((y, launches))
+    (y0, l0), (y1, l1) = ys
+    assert l1 == l0 + 2
+    assert torch.equal(y0, y1)

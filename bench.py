@@ -49,6 +49,9 @@ LAUNCH_NAMES_SMALL = ["router_gemm", "route_topk", "dispatch_small", "gemm_gate_
 LAUNCH_NAMES_REROUTE_SMALL = ["router_gemm", "route_topk", "capacity_pass", "reroute_offer",
                               "rank_offers", "scan_offers", "reroute_accept", "dispatch_final",
                               "gemm_gate_up", "gemm_down", "combine"]
+# fp32 layers: SIMT router, and the two SIMT FFN kernels timed as one stage
+LAUNCH_NAMES_F32 = ["router_gemm", "route_topk", "rank_local", "dispatch_scan",
+                    "scatter_gather", "ffn_up_down_f32", "combine"]
 L2_BYTES = 128 << 20          # B200 L2: 126 MB
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -421,8 +424,9 @@ def run_ours(args):
     launch_ms, calls = nat.moe_profile_end(16)
     # the profiled calls run every launch on the launching stream (the shared expert inside
     # the routed GEMMs), in this order
-    names = {8: LAUNCH_NAMES, 7: LAUNCH_NAMES_FUSED, 6: LAUNCH_NAMES_SMALL,
-             15: LAUNCH_NAMES_REROUTE,
+    names = {8: LAUNCH_NAMES,
+             7: LAUNCH_NAMES_FUSED if shape.dtype == W.BF16 else LAUNCH_NAMES_F32,
+             6: LAUNCH_NAMES_SMALL, 15: LAUNCH_NAMES_REROUTE,
              11: LAUNCH_NAMES_REROUTE_SMALL}.get(len(launch_ms),
                                                  [f"launch_{i}" for i in range(len(launch_ms))])
     eager_ms = max_over_ranks(p0.elapsed_time(p1), world) / args.steps

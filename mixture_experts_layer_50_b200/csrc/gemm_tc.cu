@@ -24,6 +24,9 @@
 //               columns beyond n_out.
 // Tiles are numbered group by group, N-block outer and M-block inner, so the CTAs working
 // at the same time share B panels (weights) and A panels (tokens) through L2.
+// Tall tiles (AM = 256, BN = 256): a tile is 256 rows, two M = 128 MMAs per k-step on one
+// B stage, their accumulators in TMEM columns [0, 256) and [256, 512); half the shared-memory
+// operand bytes per MMA of the 128-row tile, and each stage holds twice the MMA time.
 // Every wait is bounded (globaltimer); on expiry the kernel records MOE_ERR_TIMEOUT in
 // the status word, lets the other roles stop, drains what it issued and frees TMEM.
 #include <cuda.h>
@@ -45,7 +48,7 @@ constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 bf16 = one 128-byte swizzle row
 constexpr int kThreads = 192;
 constexpr int kStageA = BM * BK * 2;   // 16 KB
-constexpr int kStagingPerWarp = 32 * 144;
+constexpr int kStagingPerWarp = 32 * 128;   // 32 rows of 128 B, 16-byte pieces XOR-swizzled
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -270,7 +273,7 @@ struct Args {
 };
 
 // AM: A rows a stage holds (128; 64 for a batch whose groups all fit 64 rows, which leaves
-// room for more stages of weights).
+// room for more stages of weights; 256 for tall tiles).
 template <int BN, int STAGES, int AM = BM>
 struct Layout {
   static constexpr int kStageA = AM * BK * 2;
@@ -389,11 +392,14 @@ __device__ __forceinline__ void epilogue_warp(const Args& p, void* out, uint32_t
       }
     }
     if (c == n_chunks - 1) release();
-    // stage this thread's 128-byte row piece (row stride 144 B: conflict-free)
-    uint4* my = reinterpret_cast<uint4*>(stg + lane * 144);
+    // stage this thread's 128-byte row piece: piece i of row r at 16 * (i ^ (r & 7)), so the
+    // eight threads of each quarter-warp access hit eight different bank groups, in the
+    // row-wise writes here and in the piece-wise reads below
+    uint8_t* my = stg + lane * 128;
 #pragma unroll
     for (int i = 0; i < 8; ++i)
-      my[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+      *reinterpret_cast<uint4*>(my + 16 * (i ^ (lane & 7))) =
+          make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
     __syncwarp();
     // coalesced copy-out: 4 rows x 128 bytes per instruction
     constexpr int kElPerPiece = (EPI == kEpiStoreF32) ? 4 : 8;
@@ -405,7 +411,7 @@ __device__ __forceinline__ void epilogue_warp(const Args& p, void* out, uint32_t
       const int row_in_tile = row_base + rr;
       const int col = col_base + pc * kElPerPiece;
       if (row_in_tile < rows_valid && col < p.n_out) {
-        const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 144 + pc * 16);
+        const uint4 val = *reinterpret_cast<const uint4*>(stg + rr * 128 + 16 * (pc ^ (rr & 7)));
         const int64_t orow = out_row0 + row_in_tile;
         if constexpr (EPI == kEpiStoreF32) {
           // fp32 rows of n_out = E columns: a 16-byte store only where the row stride and the
@@ -438,6 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   using L = Layout<BN, STAGES, AM>;
   // AM = 64: groups are cut into 64-row tiles, each running M = 64 MMAs
   constexpr bool kAll64 = AM < BM;
+  // AM = 256: tall tiles, one accumulator in two halves of BN columns (rows 0-127, 128-255)
+  constexpr bool kTall = AM > BM;
+  static_assert(!kTall || (AM == 2 * BM && 2 * BN <= 512), "tall tiles: 256 rows, 2 BN <= 512");
   constexpr int TM = AM;  // rows of an output tile
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -514,6 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================= TMA producer =================
     if (lane == 0) {
       int stage = 0;
+
       uint32_t phase = 0;
       int armed = 0;  // stages armed so far (for the drain on abort)
       bool ok = true;
@@ -524,13 +534,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool sh = g >= p.n_routed;
         const int a_row = (sh ? p.shared_a_row0 : p.offsets[g]) + m_blk * TM;
         const CUtensorMap* mA = sh ? &tmAs : &tmA;
+        // tall tiles: the second 128-row A box only when the tile has rows past 128
+        bool a_hi = false;
+        if constexpr (kTall) {
+          const int cnt = sh ? p.shared_rows : p.offsets[g + 1] - p.offsets[g];
+          a_hi = cnt - m_blk * TM > BM;
+        }
+        constexpr int kBoxA = kTall ? BM * BK * 2 : L::kStageA;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, s_abort, p.status)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(&full[stage], L::kStageA + L::kStageB);
+          mbar_expect_tx(&full[stage], (a_hi ? 2 : 1) * kBoxA + L::kStageB);
           tma_load_2d(sA + stage * L::kStageA, mA, &full[stage], kb * BK, a_row);
+          if (a_hi)
+            tma_load_2d(sA + stage * L::kStageA + kBoxA, mA, &full[stage], kb * BK, a_row + BM);
           uint8_t* b_dst = sB + stage * L::kStageB;
           if (EPI == kEpiSwiglu) {
             tma_load_3d(b_dst, &tmB, &full[stage], kb * BK, n_blk * (BN / 2), g);
@@ -568,11 +587,101 @@ __global__ void __launch_bounds__(kThreads, 1)
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t aph = (it >> 1) & 1;
         int g, m_blk, n_blk;
         decode_tile<TM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
         const int cnt = g < p.n_routed ? p.offsets[g + 1] - p.offsets[g] : p.shared_rows;
+        if constexpr (kTall) {
+          // One accumulator in two halves.  The epilogue hands back half 0 (tempty[0]) and
+          // then half 1 (tempty[1]) of the previous tile; this tile starts its half-0 MMAs
+          // as soon as half 0 is free and defers the half-1 MMAs of up to STAGES - 1 stages
+          // (their stages stay held) until half 1 is free.  Both barriers are waited once
+          // per tile, so their phases stay in step with the tile count.
+          const uint32_t ph = (uint32_t)(it & 1);
+          const int rows = cnt - m_blk * TM;
+          const bool two = rows > BM;
+          const uint32_t id0 = (p.m64_tails && rows <= 64) ? kIdesc64 : kIdesc;
+          const uint32_t id1 = (p.m64_tails && rows - BM <= 64) ? kIdesc64 : kIdesc;
+          if (!mbar_wait(&tempty[0], ph ^ 1, s_abort, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int kb0 = (tile % ks_n) * kper, kb1 = min(nk, kb0 + kper);
+          bool h1 = false;              // half 1 of the accumulator is free
+          int pend = 0, pend_stage = 0, pend_kb = 0;  // deferred half-1 k-blocks
+          auto half1 = [&](int st, int kb) {
+            const uint32_t a1 = smem_u32(sA + st * L::kStageA + BM * BK * 2);
+            const uint32_t b1 = smem_u32(sB + st * L::kStageB);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              mma_bf16(tmem_base + (uint32_t)BN, sw128_desc(a1 + kk * 32),
+                       sw128_desc(b1 + kk * 32), id1, (kb > kb0 || kk > 0) ? 1u : 0u);
+          };
+          auto flush = [&]() {
+            int st = pend_stage;
+            for (int i = 0; i < pend; ++i) {
+              half1(st, pend_kb + i);
+              mma_commit(&empty[st]);
+              st = st + 1 == STAGES ? 0 : st + 1;
+            }
+            pend = 0;
+          };
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait(&full[stage], phase, s_abort, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a0 = smem_u32(sA + stage * L::kStageA);
+            const uint32_t b0 = smem_u32(sB + stage * L::kStageB);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              mma_bf16(tmem_base, sw128_desc(a0 + kk * 32), sw128_desc(b0 + kk * 32), id0,
+                       (kb > kb0 || kk > 0) ? 1u : 0u);
+            bool commit = true;
+            if (two) {
+              if (!h1) h1 = mbar_try_wait(&tempty[1], ph ^ 1);
+              if (!h1 && pend < STAGES - 1) {
+                if (pend == 0) {
+                  pend_stage = stage;
+                  pend_kb = kb;
+                }
+                ++pend;
+                commit = false;
+              } else {
+                if (!h1) {
+                  if (!mbar_wait(&tempty[1], ph ^ 1, s_abort, p.status)) {
+                    ok = false;
+                    break;
+                  }
+                  h1 = true;
+                }
+                tc_fence_after();
+                flush();
+                half1(stage, kb);
+              }
+            }
+            if (commit) mma_commit(&empty[stage]);
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+          if (!ok) break;
+          if (!h1) {
+            // a one-half tile, or a K loop shorter than the deferral: wait for half 1 here
+            if (!mbar_wait(&tempty[1], ph ^ 1, s_abort, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            flush();
+          }
+          mma_commit(&tfull[0]);
+          continue;
+        }
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
         const uint32_t idesc =
             (kAll64 || (p.m64_tails && cnt - m_blk * TM <= 64)) ? kIdesc64 : kIdesc;
         if (!mbar_wait(&tempty[acc], aph ^ 1, s_abort, p.status)) {
@@ -617,8 +726,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       int g, m_blk, n_blk;
       decode_tile<TM, BN>(tile / ks_n, s_start, G, nt, g, m_blk, n_blk, p.band);
-      const int acc = it & 1;
-      const uint32_t aph = (it >> 1) & 1;
+      const int acc = kTall ? 0 : it & 1;
+      const uint32_t aph = kTall ? (uint32_t)(it & 1) : (uint32_t)((it >> 1) & 1);
       // warp-uniform decision: tcgen05.ld below needs all 32 lanes
       const bool ready = mbar_wait(&tfull[acc], aph, s_abort, p.status);
       if (!__all_sync(0xffffffffu, ready)) break;
@@ -628,13 +737,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t out_row0 = (int64_t)(sh ? p.shared_out_row0 : p.offsets[g]) + m_blk * TM +
                                (int64_t)(tile % ks_n) * p.split_rows;
       const int rows_valid = min(TM, cnt - m_blk * TM);
+      void* out = (sh && p.out_shared != nullptr) ? p.out_shared : p.out;
+      if constexpr (kTall) {
+        // half h: rows 128 h .. 128 h + 127 of the tile, TMEM columns [BN h, BN h + BN);
+        // each half is handed back to the MMA warp as soon as it is read
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          const int rows_h = min(BM, rows_valid - h * BM);
+          if (rows_h <= 0) {
+            tc_fence_before();
+            mbar_arrive(&tempty[h]);
+            continue;
+          }
+          const uint32_t t_row =
+              tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * BN);
+          const bool m64 = p.m64_tails && rows_h <= 64;
+          const int row_base = m64 ? q * 16 : q * 32;
+          const int rows_w = m64 ? min(rows_h, q * 16 + 16) : rows_h;
+          epilogue_warp<BN, EPI>(p, out, t_row, stg, lane, n_blk, out_row0 + h * BM, row_base,
+                                 rows_w, [&] {
+                                   tc_fence_before();
+                                   mbar_arrive(&tempty[h]);
+                                 });
+        }
+        continue;
+      }
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       // an M = 64 accumulator holds rows 16q .. 16q + 15 in lanes 32q .. 32q + 15
       const bool m64 = kAll64 || (p.m64_tails && rows_valid <= 64);
       const int row_base = m64 ? q * 16 : q * 32;
       const int rows_w = m64 ? min(rows_valid, q * 16 + 16) : rows_valid;
 
-      void* out = (sh && p.out_shared != nullptr) ? p.out_shared : p.out;
       epilogue_warp<BN, EPI>(p, out, t_row, stg, lane, n_blk, out_row0, row_base, rows_w, [&] {
         // all TMEM reads of this accumulator are done: hand it back to the MMA warp
         tc_fence_before();
@@ -1382,7 +1515,7 @@ cudaError_t launch_t(const GroupedGemm& g, const CUtensorMap& mA, const CUtensor
   const cudaError_t e = allow_max_smem(kern, done);
   if (e != cudaSuccess) return e;
   Args a = make_args(g);
-  a.band = band_for(g, BM);
+  a.band = band_for(g, AM > BM ? AM : BM);
   launch_pdl(kern, grid, kThreads, smem, stream, mA, mAs, mB, a);
   return cudaGetLastError();
 }
@@ -1464,7 +1597,7 @@ int64_t one_sm_rows(int64_t r) {
 bool use_two_sm(const GroupedGemm& g) {
   if (g.epilogue == kEpiStoreF32 || g.k_splits > 1) return false;
   if (const char* env = path_override()) {
-    if (std::strncmp(env, "1sm", 3) == 0) return false;
+    if (std::strncmp(env, "1sm", 3) == 0 || std::strcmp(env, "tall") == 0) return false;
     if (std::strcmp(env, "2sm") == 0) return true;
   }
   const int64_t routed = g.n_routed > 0 ? avg_group_rows(g) * g.n_routed : 0;
@@ -1479,6 +1612,20 @@ bool use_two_sm(const GroupedGemm& g) {
   if (4 * extra > routed + shared) return false;
   if (g.epilogue == kEpiStoreBf16) return true;
   return (int64_t)g.rows_b * g.K * 2 <= l2_bytes() / 4;
+}
+
+// Tall tiles (1-SM kernel, 256x256), on request only (MOE_B200_GEMM_PATH=tall): two M = 128
+// MMAs per k-step share one B stage, so a stage of 64 KB feeds 1024 MMA cycles where a 48 KB
+// stage of the 128x256 tile feeds 512, and the operands cross from shared memory at 64 B per
+// clock instead of 96.  A tile with at most 128 rows issues only the first MMA (and loads
+// only the first A box), so groups pad exactly as on the 128-row tiles.  Measured slower or
+// level everywhere: the V3/V4.1-shaped prefill gate/up 4.53 -> 5.91 ms and 5.85 -> 7.86 ms
+// (its many short groups get 3 stages of weights in flight instead of 4), the Mixtral-shaped
+// 16384-token step 9.45 ms either way (9.66 with tall gate/up and the 2-SM down).
+bool use_tall(const GroupedGemm& g) {
+  if (g.epilogue == kEpiStoreF32 || g.k_splits > 1) return false;
+  const char* env = path_override();
+  return env != nullptr && std::strcmp(env, "tall") == 0;
 }
 
 // N width of the 1-SM kernel's tiles.  256 keeps the tensor pipe busiest; when nearly every
@@ -1510,7 +1657,9 @@ int pick_bn_1sm(const GroupedGemm& g) {
 // M = 64 MMAs halve the rows per instruction.
 // MOE_B200_DECODE_A64=0 turns it off; =2 forces it on any group sizes (tests).
 bool use_a64(const GroupedGemm& g) {
-  if (g.epilogue == kEpiStoreF32 || g.k_splits > 1 || use_swap(g) || use_two_sm(g)) return false;
+  if (g.epilogue == kEpiStoreF32 || g.k_splits > 1 || use_swap(g) || use_two_sm(g) ||
+      use_tall(g))
+    return false;
   const char* v = std::getenv("MOE_B200_DECODE_A64");
   if (v != nullptr && v[0] == '0') return false;
   if (v != nullptr && v[0] == '2') return true;
@@ -1562,6 +1711,7 @@ const char* grouped_gemm_kernel_name(const GroupedGemm& g) {
     }
   }
   if (use_two_sm(g)) return "grouped_gemm_2sm_kernel (2-SM, 256x256 tiles)";
+  if (use_tall(g)) return "grouped_gemm_kernel (1-SM, 256x256 tiles)";
   if (use_a64(g))
     return pick_bn_1sm(g) == 128 ? "grouped_gemm_kernel (1-SM, 64x128 tiles)"
                                  : "grouped_gemm_kernel (1-SM, 64x256 tiles)";
@@ -1601,10 +1751,11 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
   }
   int BN;
   const bool two_sm = use_two_sm(g);
+  const bool tall = !two_sm && use_tall(g);
   if (g.epilogue == kEpiStoreF32) {
     BN = router_tile_n(g.n_out);
   } else {
-    BN = two_sm ? 256 : pick_bn_1sm(g);
+    BN = (two_sm || tall) ? 256 : pick_bn_1sm(g);
   }
   const int box_b = two_sm ? 128 : (g.epilogue == kEpiSwiglu) ? BN / 2 : BN;
   const bool a64 = use_a64(g);
@@ -1622,7 +1773,7 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
   // grid: at most one CTA per SM, no more than an upper bound of the tile count
   const int out_per_tile = (g.epilogue == kEpiSwiglu) ? BN / 2 : BN;
   const int64_t nt = (g.n_out + out_per_tile - 1) / out_per_tile;
-  const int tm = a64 ? 64 : BM;  // rows of an output tile
+  const int tm = a64 ? 64 : tall ? 256 : BM;  // rows of an output tile
   int64_t mtiles = 0;
   if (g.n_routed > 0) mtiles += (g.max_rows_routed + tm - 1) / tm + g.n_routed;
   if (g.has_shared) mtiles += (g.shared_rows + tm - 1) / tm;
@@ -1638,6 +1789,14 @@ cudaError_t launch_grouped_gemm(const GroupedGemm& g, cudaStream_t stream, int* 
       case kEpiSwiglu: return launch_2sm<kEpiSwiglu, 6>(g, mA, mAs, mB, stream, pairs);
       case kEpiRelu: return launch_2sm<kEpiRelu, 6>(g, mA, mAs, mB, stream, pairs);
       default: return launch_2sm<kEpiStoreBf16, 6>(g, mA, mAs, mB, stream, pairs);
+    }
+  }
+  if (tall) {
+    // 256-row tiles: 3 stages of 64 KB
+    switch (g.epilogue) {
+      case kEpiSwiglu: return launch_t<256, kEpiSwiglu, 3, 256>(g, mA, mAs, mB, stream, grid);
+      case kEpiRelu: return launch_t<256, kEpiRelu, 3, 256>(g, mA, mAs, mB, stream, grid);
+      default: return launch_t<256, kEpiStoreBf16, 3, 256>(g, mA, mAs, mB, stream, grid);
     }
   }
   if (a64) {

@@ -216,7 +216,8 @@ def test_ffn_kernel_choice(nat):
 
 
 @pytest.mark.parametrize("path,kind", [("1sm", "1-SM"), ("1sm128", "x128 tiles"),
-                                       ("2sm", "2-SM, 256x256 tiles"), ("swap", "token-in-N")])
+                                       ("2sm", "2-SM, 256x256 tiles"), ("swap", "token-in-N"),
+                                       ("tall", "1-SM, 256x256 tiles")])
 def test_ffn_kernel_override(nat, path, kind, monkeypatch):
     """MOE_B200_GEMM_PATH forces one grouped GEMM for both projections ("1sm" keeps the
     automatic tile width), and moe_ffn_kernels reports the forced choice (the library reads

@@ -217,12 +217,12 @@ FFN_CASES = [
 ]
 
 
-@pytest.mark.parametrize("path", ["1sm", "1sm128", "2sm", "swap", "1sm64"])
+@pytest.mark.parametrize("path", ["1sm", "1sm128", "2sm", "swap", "1sm64", "tall"])
 @pytest.mark.parametrize("N,d,E,k,F,S,act,clamp", FFN_CASES)
 def test_expert_ffn(N, d, E, k, F, S, act, clamp, path, monkeypatch):
     # every grouped-GEMM variant (1-SM 128x256 and 128x128 tiles, 2-SM 256x256, the
-    # token-in-N kernel with weights in M, and the 1-SM kernel forced to 64-row tiles) on
-    # every case
+    # token-in-N kernel with weights in M, the 1-SM kernel forced to 64-row tiles, and its
+    # 256-row tall tiles) on every case
     _set_path(path, monkeypatch)
     shape = W.LayerShape("t", N=N, d=d, E=E, k=k, F=F, n_shared=S, act=act, clamp=clamp,
                          w_std=0.08, seed=N + d)
@@ -264,13 +264,13 @@ def _set_path(path, monkeypatch):
         monkeypatch.setenv("MOE_B200_DECODE_A64", "0")
 
 
-@pytest.mark.parametrize("path", ["1sm", "swap", "2sm", "1sm64"])
+@pytest.mark.parametrize("path", ["1sm", "swap", "2sm", "1sm64", "tall"])
 def test_expert_ffn_group_sizes_around_the_tile_edges(path, monkeypatch):
     """Groups of 0 ... 513 rows around every tile edge: the token-in-N kernel rounds a group's
     last row block up to 16 rows and loads it in 32-row boxes; the 1-SM kernel pads to
     128-row tiles (M = 64 for a last tile of at most 64 rows), or cuts groups into 64-row
-    tiles; the 2-SM kernel pads to 256-row tiles (128 with a half tile for the down
-    projection)."""
+    tiles, or 256-row tall tiles whose second half is skipped or runs M = 64; the 2-SM kernel
+    pads to 256-row tiles (128 with a half tile for the down projection)."""
     _set_path(path, monkeypatch)
     sizes = [0, 1, 15, 16, 17, 31, 32, 33, 127, 128, 129, 255, 256, 257, 300, 383, 384, 385,
              511, 512, 513]
@@ -480,6 +480,15 @@ def test_forward_large_groups_take_the_2sm_kernel(monkeypatch):
     _forward_case("mixtral-n4096", sample=np.r_[0:8, 4090:4096])
     monkeypatch.setenv("MOE_B200_GEMM_PATH", "1sm")
     _forward_case("mixtral-n4096", sample=np.r_[0:8, 4090:4096])
+
+
+def test_forward_tall_tiles(monkeypatch):
+    """The 1-SM kernel's 256-row tiles on whole layers: a ridge-shaped layer (about 256 rows
+    per expert, skewed, most groups ending in a half or an M = 64 tile) and a Mixtral-shaped
+    one (1024-row groups), sampled over the whole token range."""
+    monkeypatch.setenv("MOE_B200_GEMM_PATH", "tall")
+    _forward_case("dsv3-n8192", N=2048, full_range=True)
+    _forward_case("mixtral-n4096", full_range=True)
 
 
 def test_forward_capacity_configs_reduced():

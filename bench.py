@@ -119,7 +119,7 @@ def bench_config(shape, world, overflow="drop"):
     """The ``config`` object of the JSON line: the same in both arms."""
     return {"workload": workload_desc(shape) + (" overflow=reroute" if overflow == "reroute" else ""),
             "tokens_per_gpu": shape.N, "global_batch": shape.N * world,
-            "l2": l2_note(shape)[1],
+            "seed": shape.seed, "l2": l2_note(shape)[1],
             "parallelism": f"replicas x{world} (no data-path collective)"}
 
 

@@ -2,6 +2,7 @@
 // layout, and the order of launches on the caller's stream.  No entry point allocates
 // device memory; none synchronises except moe_check_status and moe_forward_host.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -16,6 +17,16 @@
 #include "../../include/moe.h"
 #include "common.cuh"
 #include "kernels.h"
+
+// NVTX range over the host-side span of an API call or of a stage of the fused forward:
+// visible on a profiler's timeline and usable to filter kernels (ncu --nvtx --nvtx-include
+// "moe_forward/"); a no-op when no tool is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 namespace {
 
@@ -680,9 +691,13 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
     MOE_CUDA(cudaEventRecord(side->fork, st), "fork the side stream");
   }
   LogitSrc zsrc;
-  MOE_TRY(stage_logits(c, L, ws, x, W_g, logit_offset, logits, status, st, launches, &zsrc));
+  {
+    NvtxRange r("moe.router");
+    MOE_TRY(stage_logits(c, L, ws, x, W_g, logit_offset, logits, status, st, launches, &zsrc));
+  }
   if (side != nullptr) {
     // launched after the router, so the router's CTAs are placed first
+    NvtxRange r("moe.shared_expert");
     MOE_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0), "fork the side stream");
     MOE_TRY(stage_shared_ffn(c, L, ws, x, W_gu, W_down, y, side->s, launches));
     MOE_CUDA(cudaEventRecord(side->join, side->s), "join the side stream");
@@ -691,12 +706,14 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
     // final slots after the overflow policy; the capacity is already met, so the dispatch
     // below only lays the kept slots out (its demand output is scratch: demand keeps the
     // router's first-pass demand)
+    NvtxRange r("moe.route_dispatch");
     MOE_TRY(stage_route_reroute(c, L, ws, zsrc, bias, modality, ids, gates, demand, drop,
                                 rerouted, st, launches));
     MOE_TRY(stage_dispatch(c, L, ws, ids, drop, 0, at<int32_t>(ws, L.rr_scratch), counts,
                            offsets, at<int32_t>(ws, L.slot_row), row_token, drop, x, xp, st,
                            launches));
   } else {
+    NvtxRange r("moe.route_dispatch");
     const bool fused = fuse_topk_rank(c);
     if (fused)
       MOE_TRY(stage_route_rank(c, L, ws, zsrc, bias, modality, ids, gates, status, st, launches));
@@ -713,10 +730,16 @@ moe_status forward_impl(const moe_config* cfg, const void* x, const void* W_g,
                                   offsets, at<int32_t>(ws, L.slot_row),
                                   at<int32_t>(ws, L.row_token), c.capacity, st));
   // fused layer: the shared expert's rows go straight into y (bf16), completed by the combine
-  MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, launches, -1, y, c.N,
-                    side != nullptr));
+  {
+    NvtxRange r("moe.expert_ffn");
+    MOE_TRY(stage_ffn(c, L, ws, xp, offsets, x, W_gu, W_down, ye, st, launches, -1, y, c.N,
+                      side != nullptr));
+  }
   if (side != nullptr) MOE_CUDA(cudaStreamWaitEvent(st, side->join, 0), "join the side stream");
-  MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, launches, -1, true));
+  {
+    NvtxRange r("moe.combine");
+    MOE_TRY(stage_combine(c, ye, at<int32_t>(ws, L.slot_row), gates, y, st, launches, -1, true));
+  }
   g_prof.recording = false;
   return MOE_OK;
 }
@@ -749,6 +772,7 @@ moe_status moe_route(const moe_config* cfg, const float* logits, const void* x,
                      const uint8_t* modality, int32_t* ids, float* gates, int32_t* counts,
                      int32_t* demand, uint8_t* drop_mask, float* logits_out, void* ws,
                      moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_route");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -790,6 +814,7 @@ moe_status moe_route_reroute(const moe_config* cfg, const float* logits, const v
                              int32_t* counts, int32_t* demand, uint8_t* drop_mask,
                              uint8_t* rerouted, float* logits_out, void* ws,
                              moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_route_reroute");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -836,6 +861,7 @@ moe_status moe_route_reroute(const moe_config* cfg, const float* logits, const v
 moe_status moe_permute(const moe_config* cfg, const int32_t* ids, const uint8_t* drop_mask,
                        const void* x, int32_t* offsets, int32_t* row_token,
                        int32_t* slot_row, void* xp, void* ws, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_permute");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -856,6 +882,7 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* ids, const uint8_t*
 moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const int32_t* offsets,
                           const void* x, const void* W_gu, const void* W_down, void* ye,
                           void* ws, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_expert_ffn");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -900,6 +927,7 @@ moe_status moe_ffn_kernels(const moe_config* cfg, char* gate_up, char* down, siz
 
 moe_status moe_combine(const moe_config* cfg, const void* ye, const int32_t* slot_row,
                        const float* gates, void* y, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_combine");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(need(ye, "ye"));
@@ -917,6 +945,7 @@ moe_status moe_forward_reroute(const moe_config* cfg, const void* x, const void*
                                const uint8_t* modality, const void* W_gu, const void* W_down,
                                void* y, const moe_route_out* route_out, uint8_t* rerouted,
                                void* ws, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_forward_reroute");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -942,6 +971,7 @@ moe_status moe_forward(const moe_config* cfg, const void* x, const void* W_g,
                        const uint8_t* modality, const void* W_gu, const void* W_down,
                        void* y, const moe_route_out* route_out, void* ws,
                        moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_forward");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -964,6 +994,7 @@ moe_status moe_forward_routed(const moe_config* cfg, const void* x, const int32_
                               const float* gates, const void* W_gu, const void* W_down,
                               void* y, const moe_route_out* route_out, void* ws,
                               moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_forward_routed");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -995,6 +1026,7 @@ moe_status moe_forward_routed(const moe_config* cfg, const void* x, const int32_
 moe_status moe_route_hash(const moe_config* cfg, const int32_t* token_ids, int32_t* ids,
                           float* gates, int32_t* counts, int32_t* demand, uint8_t* drop_mask,
                           void* ws, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_route_hash");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -1020,6 +1052,7 @@ moe_status moe_balance(const moe_config* cfg, const float* logits, const int32_t
                        const uint8_t* modality, float* f, float* P, float* aux,
                        int32_t* set_load, float* bias, float gamma, void* ws,
                        moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_balance");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -1043,6 +1076,7 @@ moe_status moe_permute_padded(const moe_config* cfg, const int32_t* ids,
                               const uint8_t* drop_mask, const void* x, int32_t* offsets_pad,
                               int32_t* counts, int32_t* row_token_pad, int32_t* slot_row,
                               void* xp_pad, void* ws, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_permute_padded");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -1083,6 +1117,7 @@ moe_status moe_forward_padded(const moe_config* cfg, const void* x, const void* 
                               const uint8_t* modality, const void* W_gu, const void* W_down,
                               void* y, const moe_route_out* ro, void* ws,
                               moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_forward_padded");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -1150,6 +1185,7 @@ moe_status moe_permute_ep(const moe_config* cfg, const int32_t* ids, const int32
                           const void* x, int32_t* offsets, int32_t* row_token, int32_t* slot_row,
                           void* xp, int32_t* counts, uint8_t* drop_mask, void* ws,
                           moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_permute_ep");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -1174,6 +1210,7 @@ moe_status moe_ep_expert_ffn(const moe_config* cfg, int32_t world, int32_t rank,
                              const int32_t* offsets, const void* x, const void* W_gu,
                              const void* W_down, void* ye, void* y, void* ws,
                              moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_ep_expert_ffn");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -1222,6 +1259,7 @@ moe_status moe_ep_expert_ffn(const moe_config* cfg, int32_t world, int32_t rank,
 
 moe_status moe_ep_combine(const moe_config* cfg, const void* ye, const int32_t* slot_row,
                           const float* gates, void* y, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_ep_combine");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   if (cfg->dtype != MOE_DT_BF16) return fail(MOE_ERR_UNSUPPORTED, "the expert-parallel combine is bf16 only");
@@ -1240,6 +1278,7 @@ moe_status moe_forward_host(const moe_config* cfg, const void* x_host, const voi
                             const float* logit_offset, const float* bias,
                             const uint8_t* modality, const void* W_gu, const void* W_down,
                             void* y_host, void* ws, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_forward_host");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -1273,6 +1312,7 @@ moe_status moe_forward_host_batches(const moe_config* cfg, int32_t n_batches,
                                     const uint8_t* const* modality, const void* W_gu,
                                     const void* W_down, void* const* y_host, void* ws,
                                     moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_forward_host_batches");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_ws(cfg, ws));
@@ -1395,6 +1435,7 @@ moe_status moe_route_static(const moe_config* cfg, const float* logits, const fl
                             const uint8_t* modality, int32_t* ids, float* gates,
                             int32_t* counts, int32_t* demand, uint8_t* drop_mask,
                             int32_t* status, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_route_static");
   g_last_launches = 0;
   MOE_TRY(check_cfg(cfg));
   MOE_TRY(check_bias(cfg, bias, modality));

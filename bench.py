@@ -139,8 +139,11 @@ def algorithmic_work(shape, counts):
     b_layer = w_gu + w_down + E * d * el + 2 * N * d * el
     # gate/up launch: its weights, its activation rows in, its hidden rows out
     b_gate_up = w_gu + rows * d * el + rows * F * el
+    # the down launch: its weights, the hidden rows in, the expert outputs out
+    b_down = w_down + rows * F * el + rows * d * el
     return dict(M=M, touched=touched, flops_layer=f_gate_up + f_down + f_router,
-                bytes_layer=b_layer, flops_gate_up=f_gate_up, bytes_gate_up=b_gate_up)
+                bytes_layer=b_layer, flops_gate_up=f_gate_up, bytes_gate_up=b_gate_up,
+                flops_down=f_down, bytes_down=b_down)
 
 
 class ClockSampler:
@@ -339,8 +342,30 @@ def route_counts(layer, shape, x, mod):
 
 
 # decode-sized and ridge-point layers measured beside the headline (same timing rules)
-SWEEP = ["mixtral-n16", "dsv3-n64", "v41flash-n64", "dsv3-n8192", "v41flash-n16384",
-         "capacity-cf1", "switch-cf1"]
+# lightest first: a layer timed right after a ~1 kW one inherits the power-cap governor's
+# low clock for a second or so (see settle_power)
+SWEEP = ["capacity-cf1", "switch-cf1", "mixtral-n16", "dsv3-n64", "v41flash-n64", "dsv3-n8192",
+         "v41flash-n16384"]
+
+
+def settle_power(index, limit_s=3.0):
+    """Wait (at most limit_s, idle) until the board's power reading falls below half its
+    limit.  NVML reports a moving average, and while it stays high after a heavy layer the
+    power-cap governor holds the clock down: a short layer timed then would measure that
+    layer's leftover state, not its own.  Returns the seconds waited."""
+    t0 = time.perf_counter()
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(index)
+        lim = pynvml.nvmlDeviceGetEnforcedPowerLimit(h) / 1000.0
+        while time.perf_counter() - t0 < limit_s:
+            if pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0 < 0.5 * lim:
+                break
+            time.sleep(0.1)
+    except Exception:  # no NVML: nothing to wait for
+        pass
+    return time.perf_counter() - t0
 
 
 def sweep_entry(name, args, world, rank, local, peaks):
@@ -352,6 +377,8 @@ def sweep_entry(name, args, world, rank, local, peaks):
     y = torch.empty_like(x)
     work = algorithmic_work(shape, route_counts(layer, shape, x, mod))
     l2_resident, _ = l2_note(shape)
+    torch.cuda.synchronize()
+    waited = settle_power(local)
     timed_ms, _, clocks = time_graphed(layer, x, y, mod, args.steps, args.warmup, world, local,
                                        l2_resident)
     assert layer.check_status() == 0
@@ -367,7 +394,8 @@ def sweep_entry(name, args, world, rank, local, peaks):
            "bound": lr["bound"], "achieved": achieved, "peak": peak, "unit": unit,
            "frac": lr["frac"], "peak_key": key if lr["bound"] == "tensor" else "hbm_gbs",
            "kept_assignments": lr["kept_assignments"], "experts_touched": lr["experts_touched"],
-           "clocks": {k: clocks.get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons", "power_w")}}
+           "clocks": {k: clocks.get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons", "power_w")},
+           "settle_s": round(waited, 2)}
     del layer, t, x, y
     torch.cuda.empty_cache()
     return out
@@ -462,6 +490,13 @@ def run_ours(args):
                   if i < len(launch_ms)}
     gu_ms = per_launch.get("gemm_gate_up")
     gu_kernel, down_kernel = nat.moe_ffn_kernels(layer.config(shape.N))
+    roof_name = "gemm_gate_up"
+    if gu_ms is None and "ffn_up_down_f32" in per_launch:
+        # fp32 layers: the two SIMT FFN kernels are timed as one stage; its work is both
+        gu_ms = per_launch["ffn_up_down_f32"]
+        work = dict(work, flops_gate_up=work["flops_gate_up"] + work["flops_down"],
+                    bytes_gate_up=work["bytes_gate_up"] + work["bytes_down"])
+        roof_name = "ffn_up_down_f32"
     tensor_key, tensor_peak = pick_tensor_peak(peaks, clocks, work["flops_gate_up"], gu_ms)
     ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     intensity = work["flops_gate_up"] / work["bytes_gate_up"]
@@ -476,9 +511,10 @@ def run_ours(args):
             peak = peaks["hbm_gbs"]
             roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s"}
         roof["frac"] = round(ach / peak, 4)
-        roof["traffic"] = read_traffic("gemm_gate_up", args.workload)
+        roof["traffic"] = read_traffic(roof_name, args.workload)
         act = "SwiGLU" if shape.act == W.SWIGLU else "ReLU"
-        roof["kernel"] = f"gemm_gate_up: {gu_kernel}, {act} epilogue"
+        roof["kernel"] = (f"gemm_gate_up: {gu_kernel}, {act} epilogue" if roof_name == "gemm_gate_up"
+                          else f"ffn_up_down_f32: {gu_kernel} + {down_kernel} (one stage)")
         roof["ms_per_launch"] = round(gu_ms, 4)
         roof["peak_source"] = f"{peak_src} ({tensor_key if roof['bound'] == 'tensor' else 'hbm_gbs'})"
     layer_roof = layer_roofline(work, ms_step, peaks, tensor_peak)

@@ -102,3 +102,45 @@ def test_algorithmic_work_of_the_roofline():
     rows = int(counts.sum()) + 64
     assert w["flops_gate_up"] == 2 * rows * 7168 * 2 * 2048
     assert w["bytes_layer"] == 2 * ((w["touched"] + 1) * 3 * 7168 * 2048 + 256 * 7168 + 2 * 64 * 7168)
+
+
+def test_settle_power_waits_for_the_power_reading_with_a_fake_nvml(monkeypatch):
+    """The sweep's settle step reads NVML only (no setting is changed): it waits while the
+    board's power reading is at or above half its limit, returns once it falls below, gives up
+    after its time limit, and returns at once when NVML is unavailable."""
+    import sys
+    import types
+    import bench
+
+    class FakeNvml(types.ModuleType):
+        def __init__(self, readings_mw, limit_mw=1_000_000):
+            super().__init__("pynvml")
+            self.readings = list(readings_mw)
+            self.limit = limit_mw
+            self.calls = 0
+
+        def nvmlInit(self):
+            pass
+
+        def nvmlDeviceGetHandleByIndex(self, i):
+            return i
+
+        def nvmlDeviceGetEnforcedPowerLimit(self, h):
+            return self.limit
+
+        def nvmlDeviceGetPowerUsage(self, h):
+            self.calls += 1
+            return self.readings[min(self.calls - 1, len(self.readings) - 1)]
+
+    monkeypatch.setattr(bench.time, "sleep", lambda s: None)
+    fake = FakeNvml([900_000, 700_000, 600_000, 400_000])    # 900 W ... 400 W, limit 1 kW
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    bench.settle_power(0, limit_s=5.0)
+    assert fake.calls == 4                                   # stopped at the first reading < 500 W
+    fake = FakeNvml([900_000])                                # never settles
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    waited = bench.settle_power(0, limit_s=0.05)
+    assert 0.05 <= waited < 1.0 and fake.calls > 1
+    broken = types.ModuleType("pynvml")                       # no NVML entry points
+    monkeypatch.setitem(sys.modules, "pynvml", broken)
+    assert bench.settle_power(0) < 0.5

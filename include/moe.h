@@ -369,6 +369,36 @@ MOE_API moe_status moe_ep_expert_ffn(const moe_config* cfg, int32_t world, int32
 MOE_API moe_status moe_ep_combine(const moe_config* cfg, const void* ye, const int32_t* slot_row,
                                   const float* gates, void* y, moe_stream_t stream);
 
+/* The exchange of the plan's row runs over peer memory ("Support visuel — Communication"):
+ * one launch writes rows of src [src_rows][row_bytes] (this device) straight into other
+ * buffers -- another process's allocation mapped with moe_ipc_open (on a multi-GPU node,
+ * reached over NVLink), or a local buffer.
+ *   dst_base [n_bufs]  device array of destination buffer addresses (uint64)
+ *   dst_rows [n_bufs]  device array of their sizes in rows (int64): bounds of every write
+ *   runs [n_runs][4]   device int32: (src_row, dst_buf, dst_row, rows) per run, rows > 0
+ *   run_start [n_runs + 1]  device int32 prefix of the runs' rows; total_rows = its last entry
+ *   row_bytes          a multiple of 16; every buffer 16-byte aligned
+ *   ws                 NULL, or a workspace whose status word records out-of-range runs
+ *                      (those are skipped; MOE_ERR_INVALID_INPUT from moe_check_status)
+ * The caller orders it against the destinations' own work: a stream-ordered barrier before
+ * (the destination is done with the buffer's previous contents) and after (its next kernels
+ * see the rows).  MOE_ERR_INVALID_ARG on a bad size or a null pointer. */
+MOE_API moe_status moe_ep_copy_runs(const void* src, int64_t src_rows,
+                                    const uint64_t* dst_base, const int64_t* dst_rows,
+                                    int32_t n_bufs, const int32_t* runs,
+                                    const int32_t* run_start, int32_t n_runs, int64_t total_rows,
+                                    int64_t row_bytes, void* ws, moe_stream_t stream);
+
+/* CUDA IPC for moe_ep_copy_runs' destinations.  moe_ipc_handle: the 64-byte handle of the
+ * allocation containing the device pointer ptr, and ptr's byte offset inside it (a caching
+ * allocator hands out pointers inside larger allocations).  moe_ipc_open: map another
+ * process's handle into this one (peer access enabled as needed); *base is the allocation's
+ * base, to which the owner's offset is added.  moe_ipc_close: unmap it.  A handle cannot be
+ * opened in the process that made it.  MOE_ERR_CUDA on a driver refusal. */
+MOE_API moe_status moe_ipc_handle(const void* ptr, void* handle, int64_t* offset);
+MOE_API moe_status moe_ipc_open(const void* handle, void** base);
+MOE_API moe_status moe_ipc_close(void* base);
+
 /* moe_forward with x_host and y_host in HOST memory (pinned for full copy speed): copies
  * x to the workspace, runs the layer, copies y back and synchronises the stream.
  * Weights, bias, modality and logit_offset are device pointers as in moe_forward. */

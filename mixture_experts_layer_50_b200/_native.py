@@ -93,6 +93,10 @@ lib.moe_ep_workspace_size.restype = _sz
 lib.moe_permute_ep.argtypes = [_cfgp] + [_vp] * 11
 lib.moe_ep_expert_ffn.argtypes = [_cfgp, _i32, _i32, _i64, _i64] + [_vp] * 9
 lib.moe_ep_combine.argtypes = [_cfgp] + [_vp] * 5
+lib.moe_ep_copy_runs.argtypes = [_vp, _i64, _vp, _vp, _i32, _vp, _vp, _i32, _i64, _i64, _vp, _vp]
+lib.moe_ipc_handle.argtypes = [_vp, _vp, ctypes.POINTER(_i64)]
+lib.moe_ipc_open.argtypes = [_vp, ctypes.POINTER(_vp)]
+lib.moe_ipc_close.argtypes = [_vp]
 lib.moe_check_dispatch_host.argtypes = [_i64, _i32, _i32, _i64] + [_vp] * 8 + [_sz]
 lib.moe_check_dispatch.argtypes = [_cfgp] + [_vp] * 8
 lib.moe_profile_begin.argtypes = [_i32]
@@ -107,7 +111,8 @@ for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "
            "moe_forward_padded", "moe_forward_host_batches", "moe_route_reroute",
            "moe_forward_reroute", "moe_selftest_wait_timeout", "moe_ffn_kernels", "moe_ep_plan",
            "moe_permute_ep", "moe_ep_expert_ffn", "moe_ep_combine", "moe_check_dispatch_host",
-           "moe_check_dispatch"):
+           "moe_check_dispatch", "moe_ep_copy_runs", "moe_ipc_handle", "moe_ipc_open",
+           "moe_ipc_close"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
@@ -118,7 +123,8 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_rou
             "moe_forward_host_batches", "moe_route_reroute", "moe_forward_reroute",
             "moe_selftest_wait_timeout", "moe_ffn_kernels", "moe_ep_first_expert",
             "moe_ep_plan", "moe_ep_workspace_size", "moe_permute_ep", "moe_ep_expert_ffn",
-            "moe_ep_combine", "moe_check_dispatch_host", "moe_check_dispatch")
+            "moe_ep_combine", "moe_check_dispatch_host", "moe_check_dispatch",
+            "moe_ep_copy_runs", "moe_ipc_handle", "moe_ipc_open", "moe_ipc_close")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -461,6 +467,48 @@ def moe_ep_combine(cfg, *, ye, slot_row, gates, y, stream=None):
     st = lib.moe_ep_combine(ctypes.byref(cfg), _ptr(ye), _ptr(slot_row), _ptr(gates), _ptr(y),
                             _stream(stream))
     _check(st, "moe_ep_combine")
+
+
+def moe_ep_copy_runs(src, *, dst_base, dst_rows, runs, ws=None, stream=None):
+    """Copy row runs of ``src`` [rows][d] into the buffers ``dst_base`` (device int64 tensor
+    of addresses, as from ``ipc_open`` or ``tensor.data_ptr()``) of sizes ``dst_rows`` (device
+    int64 tensor, rows): ``runs`` is a list of (src_row, dst_buf, dst_row, rows)."""
+    runs = [tuple(int(v) for v in r) for r in runs if int(r[3]) > 0]
+    if not runs:
+        return
+    dev = src.device
+    run_t = torch.tensor(runs, dtype=torch.int32).to(dev, non_blocking=True)
+    start = [0]
+    for r in runs:
+        start.append(start[-1] + r[3])
+    start_t = torch.tensor(start, dtype=torch.int32).to(dev, non_blocking=True)
+    row_bytes = src.shape[1] * src.element_size()
+    st = lib.moe_ep_copy_runs(_ptr(src), src.shape[0], _ptr(dst_base), _ptr(dst_rows),
+                              dst_base.numel(), _ptr(run_t), _ptr(start_t), len(runs),
+                              start[-1], row_bytes, _ptr(ws), _stream(stream))
+    _check(st, "moe_ep_copy_runs")
+
+
+def ipc_handle(t: torch.Tensor):
+    """(64-byte CUDA IPC handle of the allocation holding ``t``, ``t``'s byte offset in it)."""
+    h = ctypes.create_string_buffer(64)
+    off = _i64(0)
+    _check(lib.moe_ipc_handle(_ptr(t), h, ctypes.byref(off)), "moe_ipc_handle")
+    return bytes(h.raw), int(off.value)
+
+
+def ipc_open(handle: bytes) -> int:
+    """Map another process's allocation; returns its base address in this process."""
+    if len(handle) != 64:
+        raise ValueError("a CUDA IPC handle is 64 bytes")
+    base = _vp()
+    _check(lib.moe_ipc_open(ctypes.create_string_buffer(handle, 64), ctypes.byref(base)),
+           "moe_ipc_open")
+    return int(base.value)
+
+
+def ipc_close(base: int) -> None:
+    _check(lib.moe_ipc_close(_vp(base)), "moe_ipc_close")
 
 
 # ---- debugging aid -------------------------------------------------------------------------

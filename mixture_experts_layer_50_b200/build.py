@@ -17,7 +17,7 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmoe_b200.so")
 SOURCES = ["moe_api.cu", "route.cu", "dispatch.cu", "combine.cu", "gemm_tc.cu", "simt_f32.cu",
-           "reroute.cu", "balance.cu", "ep_plan.cu", "layout_check.cu"]
+           "reroute.cu", "balance.cu", "ep_plan.cu", "ep_p2p.cu", "layout_check.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 
 NVCC_FLAGS = [

@@ -83,6 +83,18 @@ cudaError_t launch_dispatch_small(const int32_t* ids, const uint8_t* drop_in, in
                                   void* xp, int row_bytes, int* status, cudaStream_t stream,
                                   int* launches);
 
+// ---- expert-parallel rows over peer memory (ep_p2p.cu) ---------------------------------
+// Copy row runs (runs [n_runs][4] int32: src_row, dst_buf, dst_row, rows; run_start
+// [n_runs + 1] the prefix of their rows) from src [src_rows][row_bytes] to the buffers
+// dst_base[dst_buf] ([dst_rows[dst_buf]][row_bytes]); out-of-range runs are skipped and
+// reported (status, when not null).  row_bytes % 16 == 0, buffers 16-byte aligned.
+cudaError_t launch_copy_runs(const void* src, int64_t src_rows, const unsigned long long* dst_base,
+                             const int64_t* dst_rows, int n_bufs, const int32_t* runs,
+                             const int32_t* run_start, int n_runs, int64_t total_rows,
+                             int row_bytes, int* status, cudaStream_t stream, int* launches);
+// Base of the device allocation containing ptr.
+cudaError_t allocation_base(const void* ptr, void** base);
+
 // ---- balancing statistics (balance.cu) ------------------------------------------------
 // f [E] share of assignments, P [E] mean router probability, aux = E sum f P, set_load
 // [n_sets][E] assignments per modality set; when bias != nullptr, bias += gamma * sign(mean

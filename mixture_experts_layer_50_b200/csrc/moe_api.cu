@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdio>
+#include <climits>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -1271,6 +1272,59 @@ moe_status moe_ep_combine(const moe_config* cfg, const void* ye, const int32_t* 
   MOE_TRY(stage_combine(*cfg, ye, slot_row, gates, y, (cudaStream_t)stream, &launches, -1,
                         cfg->n_shared != 0));
   g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_ep_copy_runs(const void* src, int64_t src_rows, const uint64_t* dst_base,
+                            const int64_t* dst_rows, int32_t n_bufs, const int32_t* runs,
+                            const int32_t* run_start, int32_t n_runs, int64_t total_rows,
+                            int64_t row_bytes, void* ws, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_ep_copy_runs");
+  g_last_launches = 0;
+  if (src_rows < 0 || n_bufs < 0 || n_runs < 0 || total_rows < 0 || row_bytes <= 0 ||
+      row_bytes % 16 != 0 || row_bytes > (int64_t)INT32_MAX)
+    return fail(MOE_ERR_INVALID_ARG, "moe_ep_copy_runs: bad sizes (row_bytes a multiple of 16)");
+  if (n_runs == 0 || total_rows == 0) return MOE_OK;
+  if (src == nullptr || dst_base == nullptr || dst_rows == nullptr || runs == nullptr ||
+      run_start == nullptr || n_bufs == 0)
+    return fail(MOE_ERR_INVALID_ARG, "moe_ep_copy_runs: null pointer");
+  if ((reinterpret_cast<uintptr_t>(src) & 15) != 0)
+    return fail(MOE_ERR_INVALID_ARG, "moe_ep_copy_runs: src not 16-byte aligned");
+  int launches = 0;
+  MOE_CUDA(moe::launch_copy_runs(src, src_rows, (const unsigned long long*)dst_base, dst_rows,
+                                 n_bufs, runs, run_start, n_runs, total_rows, (int)row_bytes,
+                                 ws != nullptr ? (int*)ws : nullptr, (cudaStream_t)stream,
+                                 &launches),
+           "copy runs");
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_ipc_handle(const void* ptr, void* handle, int64_t* offset) {
+  if (ptr == nullptr || handle == nullptr || offset == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "moe_ipc_handle: null pointer");
+  void* base = nullptr;
+  MOE_CUDA(moe::allocation_base(ptr, &base), "moe_ipc_handle: allocation of the pointer");
+  cudaIpcMemHandle_t h;
+  MOE_CUDA(cudaIpcGetMemHandle(&h, base), "cudaIpcGetMemHandle");
+  static_assert(sizeof(h) == 64, "CUDA IPC handles are 64 bytes");
+  std::memcpy(handle, &h, sizeof(h));
+  *offset = (int64_t)((const char*)ptr - (const char*)base);
+  return MOE_OK;
+}
+
+moe_status moe_ipc_open(const void* handle, void** base) {
+  if (handle == nullptr || base == nullptr)
+    return fail(MOE_ERR_INVALID_ARG, "moe_ipc_open: null pointer");
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof(h));
+  MOE_CUDA(cudaIpcOpenMemHandle(base, h, cudaIpcMemLazyEnablePeerAccess), "cudaIpcOpenMemHandle");
+  return MOE_OK;
+}
+
+moe_status moe_ipc_close(void* base) {
+  if (base == nullptr) return fail(MOE_ERR_INVALID_ARG, "moe_ipc_close: null pointer");
+  MOE_CUDA(cudaIpcCloseMemHandle(base), "cudaIpcCloseMemHandle");
   return MOE_OK;
 }
 

@@ -13,7 +13,9 @@ the experts ``[first(r), first(r+1))`` and a copy of the shared expert.  A forwa
 3. ``moe_ep_plan`` (host, C): the capacity share of this rank per expert, every rank's kept
    counts, the row runs to send and where received runs land;
 4. ``moe_permute_ep``: this rank's kept rows in the send layout (expert-major);
-5. dispatch: one grouped point-to-point exchange of the row runs (NCCL on GPUs);
+5. dispatch: one grouped point-to-point exchange of the row runs (NCCL on GPUs), or with
+   ``transport="p2p"`` one launch that writes the runs straight into the owners' receive
+   buffers over peer memory (CUDA IPC mappings; NVLink on a multi-GPU node);
 6. ``moe_ep_expert_ffn``: the owned experts on the received rows (tcgen05 grouped GEMMs), and
    the shared expert on the rank's own tokens, written straight into y;
 7. combine trip: the same runs back to their source ranks;
@@ -93,6 +95,97 @@ def loopback_exchange(send_bufs: Sequence[torch.Tensor], recv_bufs: Sequence[tor
         raise RuntimeError(f"receive runs without a sender: {sorted(pending)}")
 
 
+def all_plans(world: int, E: int, capacity: int, demand_all) -> list:
+    """Every rank's plan from the all-gathered demands (each rank can compute the others')."""
+    return [nat.moe_ep_plan(world, r, E, capacity, demand_all) for r in range(world)]
+
+
+def peer_runs(rank: int, plans: Sequence[dict], direction: str) -> list:
+    """This rank's runs for ``moe_ep_copy_runs`` as (src_row, dst_rank, dst_row, rows):
+    ``"dispatch"``: each run of its send buffer lands where its owner receives (rank, expert);
+    ``"return"``: each run of its receive buffer (expert outputs) goes back to the row of the
+    source's send run (rank, expert), i.e. into the source's return buffer."""
+    mine, theirs = ("sends", "recvs") if direction == "dispatch" else ("recvs", "sends")
+    out = []
+    for peer, e, row, rows in plans[rank][mine]:
+        dst = {(p, ex): (r, n) for p, ex, r, n in plans[peer][theirs]}
+        if (rank, e) not in dst or dst[(rank, e)][1] != rows:
+            raise RuntimeError(f"rank {rank} -> {peer} expert {e}: no matching run of {rows} rows")
+        out.append((row, peer, dst[(rank, e)][0], rows))
+    return out
+
+
+class PeerTransport:
+    """The rows of an expert-parallel layer moved by ``moe_ep_copy_runs`` into the peers'
+    buffers (their allocations mapped with CUDA IPC) instead of NCCL messages.  The receive
+    buffer (every rank's rows for this rank's experts: at most world * max_tokens * k) and the
+    return buffer (this rank's kept rows) are one allocation made once; its handle is
+    exchanged once.  ``barrier`` (default: a one-element all-reduce on the stream for NCCL
+    groups, else a synchronise and a host barrier) follows each copy launch: after it every
+    rank's rows have landed, and since every rank reaches it only after its earlier reads of
+    both buffers, the next copies cannot overwrite rows still in use."""
+
+    def __init__(self, layer: "EPMoELayer", group=None, barrier=None):
+        import torch.distributed as dist
+        self.layer, self.group = layer, group
+        dev = layer.xp.device
+        self.rows_recv = max(1, layer.world * layer.max_tokens * layer.k)
+        self.rows_ret = max(1, layer.max_tokens * layer.k)
+        self.buf = torch.empty((self.rows_recv + self.rows_ret, layer.d), dtype=torch.bfloat16,
+                               device=dev)
+        self.recv, self.ret = self.buf[:self.rows_recv], self.buf[self.rows_recv:]
+        handle, offset = nat.ipc_handle(self.buf)
+        gathered = [None] * layer.world
+        dist.all_gather_object(gathered, (handle, offset, self.rows_recv, self.rows_ret),
+                               group=group)
+        self.mapped = []
+        row_bytes = layer.d * 2
+        recv_base, ret_base, recv_rows, ret_rows = [], [], [], []
+        for r, (h, off, nr, nt) in enumerate(gathered):
+            if r == layer.rank:
+                base = self.buf.data_ptr()
+            else:
+                mapped = nat.ipc_open(h)
+                self.mapped.append(mapped)
+                base = mapped + off
+            recv_base.append(base)
+            ret_base.append(base + nr * row_bytes)
+            recv_rows.append(nr)
+            ret_rows.append(nt)
+        i64 = dict(dtype=torch.int64, device=dev)
+        self.recv_base, self.recv_rows = torch.tensor(recv_base, **i64), torch.tensor(recv_rows, **i64)
+        self.ret_base, self.ret_rows = torch.tensor(ret_base, **i64), torch.tensor(ret_rows, **i64)
+        if barrier is None:
+            if dist.get_backend(group) == "nccl":
+                flag = torch.zeros(1, dtype=torch.int32, device=dev)
+                barrier = lambda: dist.all_reduce(flag, group=group)
+            else:
+                def barrier():
+                    torch.cuda.current_stream(dev).synchronize()
+                    dist.barrier(group=group)
+        self.barrier = barrier
+
+    def dispatch(self, xp: torch.Tensor, plans: Sequence[dict]) -> torch.Tensor:
+        L = self.layer
+        nat.moe_ep_copy_runs(xp, dst_base=self.recv_base, dst_rows=self.recv_rows,
+                             runs=peer_runs(L.rank, plans, "dispatch"), ws=L.ws)
+        self.barrier()
+        return self.recv[:max(1, plans[L.rank]["rows_owned"])]
+
+    def give_back(self, ye: torch.Tensor, plans: Sequence[dict]) -> torch.Tensor:
+        L = self.layer
+        nat.moe_ep_copy_runs(ye, dst_base=self.ret_base, dst_rows=self.ret_rows,
+                             runs=peer_runs(L.rank, plans, "return"), ws=L.ws)
+        self.barrier()
+        return self.ret[:max(1, plans[L.rank]["rows_kept"])]
+
+    def close(self):
+        torch.cuda.synchronize(self.buf.device)
+        for m in self.mapped:
+            nat.ipc_close(m)
+        self.mapped = []
+
+
 class EPMoELayer:
     """One rank of an expert-parallel MoE layer (bf16).
 
@@ -101,11 +194,15 @@ class EPMoELayer:
     batch: C = ceil(T k / E * cf) with T the tokens of all ranks.  ``forward`` runs the whole
     layer with torch.distributed (``group``); the phase methods (``route``, ``set_plan``,
     ``permute``, ``run_experts``, ``combine``) let a caller drive the exchanges itself.
+    ``transport``: ``"nccl"`` (grouped point-to-point messages) or ``"p2p"`` (``PeerTransport``:
+    the rows written straight into the peers' buffers); a p2p layer is built collectively, by
+    every rank of the group, and released with ``close``.
     """
 
     def __init__(self, *, W_g, W_gu, W_down, k, world: int, rank: int, n_shared=0,
                  score_fn=nat.SOFTMAX, renorm=1, act=nat.SWIGLU, clamp=0.0, bias=None,
-                 logit_offset=None, capacity_factor=None, max_tokens: int, group=None):
+                 logit_offset=None, capacity_factor=None, max_tokens: int, group=None,
+                 transport: str = "nccl", barrier=None):
         if W_gu.dtype != torch.bfloat16:
             raise ValueError("the expert-parallel layer is bf16")
         self.E, self.d = W_g.shape
@@ -138,7 +235,11 @@ class EPMoELayer:
         self.cap = torch.empty(self.E, **i32)
         self.owned_offsets = torch.empty(self.n_owned + 1, **i32)
         self.plan = None
+        self.plans = None
         self.N = 0
+        if transport not in ("nccl", "p2p"):
+            raise ValueError(f"transport must be 'nccl' or 'p2p', not {transport!r}")
+        self.transport = PeerTransport(self, group, barrier) if transport == "p2p" else None
 
     @classmethod
     def from_full_weights(cls, *, W_g, W_gu, W_down, k, E, world, rank, n_shared=0, **kw):
@@ -175,7 +276,8 @@ class EPMoELayer:
                        dtype=np.int64).reshape(self.world, self.E + 1)
         T = int(g[:, self.E].sum())
         C = nat.moe_capacity(T, self.k, self.E, self.capacity_factor)
-        self.plan = nat.moe_ep_plan(self.world, self.rank, self.E, C, g[:, :self.E])
+        self.plans = all_plans(self.world, self.E, C, g[:, :self.E])
+        self.plan = self.plans[self.rank]
         self.plan["capacity"] = C
         self.cap.copy_(torch.from_numpy(self.plan["cap"]), non_blocking=False)
         self.owned_offsets.copy_(torch.from_numpy(self.plan["owned_offsets"]), non_blocking=False)
@@ -220,10 +322,19 @@ class EPMoELayer:
         if y is None:
             y = torch.empty_like(x)
         demand = self.route(x, modality)
-        gathered = torch.empty(self.world * (self.E + 1), dtype=torch.int32, device=demand.device)
-        dist.all_gather_into_tensor(gathered, demand, group=self.group)
+        if dist.get_backend(self.group) == "nccl":
+            gathered = torch.empty(self.world * (self.E + 1), dtype=torch.int32,
+                                   device=demand.device)
+            dist.all_gather_into_tensor(gathered, demand, group=self.group)
+        else:  # a CPU backend (gloo) moves host tensors
+            gathered = torch.empty(self.world * (self.E + 1), dtype=torch.int32)
+            dist.all_gather_into_tensor(gathered, demand.cpu(), group=self.group)
         plan = self.set_plan(gathered)
         xp = self.permute(x)
+        if self.transport is not None:
+            xr = self.transport.dispatch(xp, self.plans)
+            ye = self.run_experts(xr, x, y)
+            return self.combine(self.transport.give_back(ye, self.plans), y)
         xr = self.new_recv_buffer()
         exchange_rows(xp, xr, plan["sends"], plan["recvs"], self.rank, self.group)
         ye = self.run_experts(xr, x, y)
@@ -231,8 +342,14 @@ class EPMoELayer:
         exchange_rows(ye, ye_back, plan["recvs"], plan["sends"], self.rank, self.group)
         return self.combine(ye_back, y)
 
+    def close(self):
+        """Unmap the peers' buffers (p2p transport)."""
+        if self.transport is not None:
+            self.transport.close()
+
     def check_status(self) -> int:
         return nat.moe_check_status(self.ws)
 
 
-__all__ = ["EPMoELayer", "shard_experts", "exchange_rows", "loopback_exchange"]
+__all__ = ["EPMoELayer", "PeerTransport", "shard_experts", "exchange_rows", "loopback_exchange",
+           "all_plans", "peer_runs"]

@@ -135,3 +135,39 @@ def test_plan_rejects_bad_arguments():
     with pytest.raises(nat.MoeError):
         nat.moe_ep_plan(2, 0, 4, 0, np.array([[1, -1, 0, 0], [0, 0, 0, 0]], np.int32))
     assert nat.lib.moe_ep_first_expert(0, 0, 4) == -1
+
+
+@pytest.mark.parametrize("seed,world,N,E,k,cf", [
+    (0, 2, 300, 8, 2, 1), (1, 3, 500, 7, 2, 1.25), (2, 4, 257, 16, 4, None), (5, 8, 64, 64, 8, 2)])
+def test_peer_runs_move_the_rows_the_message_exchange_moves(seed, world, N, E, k, cf):
+    """The peer-memory transport's runs (each rank writes its rows straight into the peers'
+    buffers): applied to tagged rows, in both directions, they leave every buffer exactly as
+    the message exchange (``loopback_exchange``) does."""
+    import torch
+    from mixture_experts_layer_50_b200.ep import all_plans, loopback_exchange, peer_runs
+    ids, C, sizes, starts, demand = _case(seed, world, N, E, k, cf)
+    plans = all_plans(world, E, C, demand)
+    rows = lambda n: max(1, n)
+    sends = [torch.arange(rows(p["rows_kept"]) * 2, dtype=torch.float64).reshape(-1, 2) + 1000 * r
+             for r, p in enumerate(plans)]
+    # dispatch: send buffers -> owners' receive buffers
+    want = [torch.full((rows(p["rows_owned"]), 2), -1.0, dtype=torch.float64) for p in plans]
+    loopback_exchange(sends, want, [p["sends"] for p in plans], [p["recvs"] for p in plans])
+    got = [torch.full_like(w, -1.0) for w in want]
+    for r in range(world):
+        for src_row, dst, dst_row, n in peer_runs(r, plans, "dispatch"):
+            got[dst][dst_row:dst_row + n] = sends[r][src_row:src_row + n]
+    for g, w in zip(got, want):
+        assert torch.equal(g, w)
+    # return: receive buffers (the expert outputs) -> the sources' return buffers
+    outs = [w + 0.5 for w in want]
+    want_back = [torch.full_like(s, -1.0) for s in sends]
+    loopback_exchange(outs, want_back, [p["recvs"] for p in plans], [p["sends"] for p in plans])
+    got_back = [torch.full_like(s, -1.0) for s in sends]
+    for r in range(world):
+        for src_row, dst, dst_row, n in peer_runs(r, plans, "return"):
+            got_back[dst][dst_row:dst_row + n] = outs[r][src_row:src_row + n]
+    for g, w in zip(got_back, want_back):
+        assert torch.equal(g, w)
+    kept = sum(p["rows_kept"] for p in plans)
+    assert sum(n for r in range(world) for *_, n in peer_runs(r, plans, "dispatch")) == kept

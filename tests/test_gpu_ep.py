@@ -176,3 +176,143 @@ def test_forward_over_a_one_rank_nccl_group():
                     bias=t["bias"], modality=t["modality"], ws=ws)
     check_status(ws)
     assert torch.equal(y_ep, y)
+
+
+# ---- the peer-memory transport (moe_ep_copy_runs, CUDA IPC) --------------------------------
+@pytest.mark.parametrize("world", [2, 4])
+def test_copy_runs_moves_the_rows_the_message_exchange_moves(world):
+    """moe_ep_copy_runs with a table of destination buffers (local here, one per emulated
+    rank) leaves every receive and return buffer bit for bit as the message exchange does;
+    a run that points past its buffer is skipped and reported."""
+    from mixture_experts_layer_50_b200.ep import all_plans, loopback_exchange, peer_runs
+    N, d, E, k = 500, 264, 12, 3
+    rng = np.random.default_rng(world)
+    z = rng.normal(0, 1, (N, E)).astype(np.float32)
+    z[:, 0] += 1.0
+    ids, _ = O.route(z, k)
+    C = O.capacity(N, k, E, 1.25)
+    sizes = _split(N, world, seed=world)
+    starts = np.r_[0, np.cumsum(sizes)]
+    demand = np.stack([np.bincount(ids[starts[r]:starts[r + 1]].ravel(), minlength=E)
+                       for r in range(world)]).astype(np.int32)
+    plans = all_plans(world, E, C, demand)
+    bf = dict(dtype=torch.bfloat16, device="cuda")
+    sends = [torch.randn(max(1, p["rows_kept"]), d, device="cuda").to(torch.bfloat16)
+             for p in plans]
+    want = [torch.zeros(max(1, p["rows_owned"]), d, **bf) for p in plans]
+    loopback_exchange(sends, want, [p["sends"] for p in plans], [p["recvs"] for p in plans])
+    got = [torch.zeros_like(w) for w in want]
+    base = torch.tensor([g.data_ptr() for g in got], dtype=torch.int64, device="cuda")
+    rows = torch.tensor([g.shape[0] for g in got], dtype=torch.int64, device="cuda")
+    ws = nat.alloc_workspace(nat.make_config(16, d, E, k, 64))
+    for r in range(world):
+        nat.moe_ep_copy_runs(sends[r], dst_base=base, dst_rows=rows,
+                             runs=peer_runs(r, plans, "dispatch"), ws=ws)
+    check_status(ws)
+    for g, w in zip(got, want):
+        assert torch.equal(g, w)
+    outs = [w.float().mul(0.5).to(torch.bfloat16) for w in want]
+    want_back = [torch.zeros_like(s) for s in sends]
+    loopback_exchange(outs, want_back, [p["recvs"] for p in plans], [p["sends"] for p in plans])
+    got_back = [torch.zeros_like(s) for s in sends]
+    base_b = torch.tensor([g.data_ptr() for g in got_back], dtype=torch.int64, device="cuda")
+    rows_b = torch.tensor([g.shape[0] for g in got_back], dtype=torch.int64, device="cuda")
+    for r in range(world):
+        nat.moe_ep_copy_runs(outs[r], dst_base=base_b, dst_rows=rows_b,
+                             runs=peer_runs(r, plans, "return"), ws=ws)
+    check_status(ws)
+    for g, w in zip(got_back, want_back):
+        assert torch.equal(g, w)
+    # out of range: a destination row past the buffer, a buffer index past the table
+    before = [g.clone() for g in got]
+    nat.moe_ep_copy_runs(sends[0], dst_base=base, dst_rows=rows,
+                         runs=[(0, 0, int(rows[0]) - 1, 2), (0, world, 0, 1)], ws=ws)
+    assert nat.moe_check_status(ws) == nat.MOE_ERR_INVALID_INPUT
+    assert torch.equal(got[0][:-1], before[0][:-1])      # only the in-range row was written
+    assert torch.equal(got[0][-1], sends[0][0])
+
+
+def _p2p_worker(rank, world, port, case, out_dir):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port),
+                      MOE_B200_GEMM_PATH="1sm")             # one GEMM kernel on both sides
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        torch.cuda.set_device(0)
+        from mixture_experts_layer_50_b200.ep import EPMoELayer
+        name, N, d, E, F, k, cf, sizes = case
+        shape = W.PRESETS[name].replace(N=N, d=d, E=E, F=F, k=k)
+        t = W.make_inputs(shape, device="cuda")             # the same seed on every rank
+        starts = np.r_[0, np.cumsum(sizes)]
+        x = t["x"][starts[rank]:starts[rank + 1]].contiguous()
+        mod = t.get("modality")
+        mod = None if mod is None else mod[starts[rank]:starts[rank + 1]].contiguous()
+        layer = EPMoELayer.from_full_weights(
+            W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], k=k, E=E, world=world, rank=rank,
+            n_shared=shape.n_shared, score_fn=shape.score_fn, renorm=shape.renorm,
+            act=shape.act, clamp=shape.clamp, bias=t.get("bias"),
+            logit_offset=t.get("logit_offset"), capacity_factor=cf,
+            max_tokens=int(max(sizes)), transport="p2p")
+        ys = []
+        for _ in range(2):                                    # the buffers are reused
+            ys.append(layer.forward(x, modality=mod).clone())
+        torch.cuda.synchronize()
+        assert layer.check_status() == 0
+        n = x.shape[0]
+        torch.save(dict(y=[v.cpu() for v in ys], ids=layer.ids[:n].cpu(),
+                        gates=layer.gates[:n].cpu(), drop=layer.drop_mask[:n].cpu()),
+                   os.path.join(out_dir, f"rank{rank}.pt"))
+        dist.barrier()
+        layer.close()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("case", [
+    ("capacity-cf1", 600, 256, 16, 256, 2, 1, (350, 250)),
+    ("v41flash-n64", 700, 512, 30, 256, 3, 1.25, (200, 0, 500)),
+])
+def test_peer_transport_between_processes_equals_the_single_device_layer(case, tmp_path,
+                                                                        monkeypatch):
+    """Ranks as separate processes sharing the GPU: each maps the others' buffers with CUDA
+    IPC and writes its rows into them with moe_ep_copy_runs (no message passing for the rows;
+    host barriers between the phases, no kernel waiting on another).  Every rank's output, on
+    two consecutive calls, equals bit for bit the fused layer over the concatenated batch given
+    the ranks' routing, and the drop masks equal the oracle's for it."""
+    import torch.multiprocessing as tmp
+    name, N, d, E, F, k, cf, sizes = case
+    world = len(sizes)
+    ctx = tmp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_p2p_worker, args=(r, world, port, case, str(tmp_path)))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=600)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = [torch.load(tmp_path / f"rank{r}.pt") for r in range(world)]
+    monkeypatch.setenv("MOE_B200_GEMM_PATH", "1sm")
+    shape = W.PRESETS[name].replace(N=N, d=d, E=E, F=F, k=k)
+    t = W.make_inputs(shape, device="cuda")
+    ids = torch.cat([r["ids"] for r in res]).cuda()
+    gates = torch.cat([r["gates"] for r in res]).cuda()
+    drop = torch.cat([r["drop"] for r in res])
+    C = O.capacity(N, k, E, cf)
+    cfg = nat.config_from_shape(shape, capacity=C)
+    ws = nat.alloc_workspace(cfg)
+    y = torch.empty_like(t["x"])
+    ro = dict(drop_mask=torch.empty((N, k), dtype=torch.uint8, device="cuda"))
+    nat.moe_forward_routed(cfg, x=t["x"], ids=ids, gates=gates, W_gu=t["W_gu"],
+                           W_down=t["W_down"], y=y, route_out=ro, ws=ws)
+    check_status(ws)
+    assert torch.equal(drop, ro["drop_mask"].cpu())
+    np.testing.assert_array_equal(drop.numpy(), O.dispatch(host(ids), E, C)["drop_mask"])
+    for call in range(2):
+        y_ep = torch.cat([r["y"][call] for r in res]).cuda()
+        assert torch.equal(y_ep, y), call

@@ -348,6 +348,22 @@ MOE_API moe_status moe_permute_ep(const moe_config* cfg, const int32_t* ids, con
                                   int32_t* slot_row, void* xp, int32_t* counts,
                                   uint8_t* drop_mask, void* ws, moe_stream_t stream);
 
+/* moe_permute_ep with the kept rows written straight into their destinations instead of a
+ * send buffer: the dispatch passes and the transfer in one pass over the rows (peer-memory
+ * expert parallelism).  Expert e's kept rows, in their layout order, go to rows dst_row0[e],
+ * dst_row0[e] + 1, ... of the buffer at dst_base[e] (device uint64 [E]: the receive buffer of
+ * e's owner -- another process's allocation mapped with moe_ipc_open, or a local buffer),
+ * which holds dst_rows[e] rows (device int64 [E]; a row past it is skipped and reported as
+ * MOE_ERR_INVALID_INPUT by moe_check_status).  Other outputs as in moe_permute_ep (no
+ * row_token).  bf16 only; d * 2 a multiple of 16.  The caller orders it against the
+ * destinations' work as for moe_ep_copy_runs. */
+MOE_API moe_status moe_permute_ep_p2p(const moe_config* cfg, const int32_t* ids,
+                                      const int32_t* cap, const void* x, int32_t* offsets,
+                                      int32_t* slot_row, const uint64_t* dst_base,
+                                      const int32_t* dst_row0, const int64_t* dst_rows,
+                                      int32_t* counts, uint8_t* drop_mask, void* ws,
+                                      moe_stream_t stream);
+
 /* The owner's expert FFNs (bf16): the received rows xr [rows][d], grouped by owned_offsets
  * (device int32 [E_own + 1], from moe_ep_plan), through the rank's experts, into ye
  * [rows][d]; with n_shared == 1 also the shared expert on this rank's own n_tokens tokens

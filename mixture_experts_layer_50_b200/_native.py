@@ -94,6 +94,7 @@ lib.moe_permute_ep.argtypes = [_cfgp] + [_vp] * 11
 lib.moe_ep_expert_ffn.argtypes = [_cfgp, _i32, _i32, _i64, _i64] + [_vp] * 9
 lib.moe_ep_combine.argtypes = [_cfgp] + [_vp] * 5
 lib.moe_ep_copy_runs.argtypes = [_vp, _i64, _vp, _vp, _i32, _vp, _vp, _i32, _i64, _i64, _vp, _vp]
+lib.moe_permute_ep_p2p.argtypes = [_cfgp] + [_vp] * 12
 lib.moe_ipc_handle.argtypes = [_vp, _vp, ctypes.POINTER(_i64)]
 lib.moe_ipc_open.argtypes = [_vp, ctypes.POINTER(_vp)]
 lib.moe_ipc_close.argtypes = [_vp]
@@ -112,7 +113,7 @@ for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "
            "moe_forward_reroute", "moe_selftest_wait_timeout", "moe_ffn_kernels", "moe_ep_plan",
            "moe_permute_ep", "moe_ep_expert_ffn", "moe_ep_combine", "moe_check_dispatch_host",
            "moe_check_dispatch", "moe_ep_copy_runs", "moe_ipc_handle", "moe_ipc_open",
-           "moe_ipc_close"):
+           "moe_ipc_close", "moe_permute_ep_p2p"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
@@ -124,7 +125,8 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_rou
             "moe_selftest_wait_timeout", "moe_ffn_kernels", "moe_ep_first_expert",
             "moe_ep_plan", "moe_ep_workspace_size", "moe_permute_ep", "moe_ep_expert_ffn",
             "moe_ep_combine", "moe_check_dispatch_host", "moe_check_dispatch",
-            "moe_ep_copy_runs", "moe_ipc_handle", "moe_ipc_open", "moe_ipc_close")
+            "moe_ep_copy_runs", "moe_ipc_handle", "moe_ipc_open", "moe_ipc_close",
+            "moe_permute_ep_p2p")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -487,6 +489,16 @@ def moe_ep_copy_runs(src, *, dst_base, dst_rows, runs, ws=None, stream=None):
                               dst_base.numel(), _ptr(run_t), _ptr(start_t), len(runs),
                               start[-1], row_bytes, _ptr(ws), _stream(stream))
     _check(st, "moe_ep_copy_runs")
+
+
+def moe_permute_ep_p2p(cfg, *, ids, cap, x, offsets, slot_row, dst_base, dst_row0, dst_rows,
+                       counts=None, drop_mask=None, ws, stream=None):
+    """moe_permute_ep with expert e's kept rows written into rows dst_row0[e]... of the
+    buffer at dst_base[e] (device int64 [E] addresses, int32 [E] first rows, int64 [E] sizes)."""
+    st = lib.moe_permute_ep_p2p(ctypes.byref(cfg), _ptr(ids), _ptr(cap), _ptr(x), _ptr(offsets),
+                                _ptr(slot_row), _ptr(dst_base), _ptr(dst_row0), _ptr(dst_rows),
+                                _ptr(counts), _ptr(drop_mask), _ptr(ws), _stream(stream))
+    _check(st, "moe_permute_ep_p2p")
 
 
 def ipc_handle(t: torch.Tensor):

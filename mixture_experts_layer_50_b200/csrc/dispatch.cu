@@ -24,6 +24,25 @@
 namespace moe {
 namespace {
 
+// Where the gather writes the kept row `row` (compact per-expert layout, `off` = its
+// expert's first row): into xp, or with kRemote straight into the destination of its expert
+// e -- row rem.row0[e] + (row - off) of the buffer at rem.base[e] (another device's receive
+// buffer reached through peer memory, or a local one); null (reported) past that buffer.
+template <bool kRemote, typename V>
+__device__ __forceinline__ V* gather_dst(V* xp, const RemoteRows& rem, int e, int32_t row,
+                                         int32_t off, int row_vecs) {
+  if constexpr (kRemote) {
+    const int64_t d = (int64_t)rem.row0[e] + (row - off);
+    if (d < 0 || d >= rem.rows[e]) {
+      if (rem.status != nullptr) report_status(rem.status, kStatusInvalidInput);
+      return nullptr;
+    }
+    return reinterpret_cast<V*>(rem.base[e]) + d * row_vecs;
+  } else {
+    return xp + (int64_t)row * row_vecs;
+  }
+}
+
 __global__ void __launch_bounds__(32) rank_local_kernel(
     const int32_t* __restrict__ ids, const uint8_t* __restrict__ drop_mask, int64_t N, int k,
     int E, int32_t* __restrict__ local_rank, int32_t* __restrict__ tile_hist, int* status) {
@@ -140,15 +159,16 @@ __global__ void __launch_bounds__(1024) dispatch_scan_kernel(
 // rank and expert together, then the expert's tile base and offset together: a local rank
 // >= 0 implies a valid expert, set by the rank pass), then the block copies the token's row
 // to each kept slot, two vectors in flight per thread.
-template <typename V>
+template <typename V, bool kRemote>
 __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
     const int32_t* __restrict__ ids, const int32_t* __restrict__ local_rank,
     const int32_t* __restrict__ tile_base, const int32_t* __restrict__ offsets, int k, int E,
     int64_t C, int32_t* __restrict__ slot_row, int32_t* __restrict__ row_token,
     uint8_t* __restrict__ drop_mask_out, const V* __restrict__ x, V* __restrict__ xp,
-    int row_vecs, const int32_t* __restrict__ cap_e) {
+    int row_vecs, const int32_t* __restrict__ cap_e, RemoteRows rem) {
   pdl_wait();
   __shared__ int32_t s_row[32];
+  __shared__ V* s_dst[32];
   const int64_t t = blockIdx.x;
   if (threadIdx.x < k) {
     const int j = threadIdx.x;
@@ -167,8 +187,9 @@ __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
     if (drop_mask_out != nullptr) drop_mask_out[t * k + j] = row < 0 ? 1 : 0;
     if (row >= 0 && row_token != nullptr) row_token[row] = (int32_t)t;
     s_row[j] = row;
+    s_dst[j] = row < 0 ? nullptr : gather_dst<kRemote>(xp, rem, e, row, off, row_vecs);
   }
-  if (xp == nullptr) return;
+  if (!kRemote && xp == nullptr) return;
   __syncthreads();
   // a token whose slots were all dropped is not read at all
   bool any = false;
@@ -182,9 +203,8 @@ __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
     V b{};
     if (two) b = src[v + step];
     for (int j = 0; j < k; ++j) {
-      const int32_t row = s_row[j];
-      if (row < 0) continue;
-      V* dst = xp + (int64_t)row * row_vecs;
+      V* dst = s_dst[j];
+      if (dst == nullptr) continue;
       dst[v] = a;
       if (two) dst[v + step] = b;
     }
@@ -198,18 +218,19 @@ __global__ void __launch_bounds__(128) dispatch_scatter_kernel(
 constexpr int kScatterWarps = 8;
 constexpr int kScatterUnroll = 4;
 
-template <typename V>
+template <typename V, bool kRemote>
 __global__ void __launch_bounds__(32 * kScatterWarps, 8) dispatch_scatter_warp_kernel(
     const int32_t* __restrict__ ids, const int32_t* __restrict__ local_rank,
     const int32_t* __restrict__ tile_base, const int32_t* __restrict__ offsets, int64_t N,
     int k, int E, int64_t C, int32_t* __restrict__ slot_row, int32_t* __restrict__ row_token,
     uint8_t* __restrict__ drop_mask_out, const V* __restrict__ x, V* __restrict__ xp,
-    int row_vecs, const int32_t* __restrict__ cap_e) {
+    int row_vecs, const int32_t* __restrict__ cap_e, RemoteRows rem) {
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * kScatterWarps + (threadIdx.x >> 5);
   if (t >= N) return;  // warp-uniform
   int32_t row = -1;
+  V* my_dst = nullptr;
   if (lane < k) {
     const int lr = local_rank[t * k + lane];
     const int e_raw = ids[t * k + lane];
@@ -224,8 +245,9 @@ __global__ void __launch_bounds__(32 * kScatterWarps, 8) dispatch_scatter_warp_k
     if (slot_row != nullptr) slot_row[t * k + lane] = row;
     if (drop_mask_out != nullptr) drop_mask_out[t * k + lane] = row < 0 ? 1 : 0;
     if (row >= 0 && row_token != nullptr) row_token[row] = (int32_t)t;
+    if (row >= 0) my_dst = gather_dst<kRemote>(xp, rem, e, row, off, row_vecs);
   }
-  if (xp == nullptr) return;
+  if (!kRemote && xp == nullptr) return;
   if (__ballot_sync(0xffffffffu, row >= 0) == 0u) return;
   const V* src = x + t * row_vecs;
   for (int v0 = 0; v0 < row_vecs; v0 += 32 * kScatterUnroll) {
@@ -236,9 +258,9 @@ __global__ void __launch_bounds__(32 * kScatterWarps, 8) dispatch_scatter_warp_k
       if (v < row_vecs) val[u] = src[v];
     }
     for (int j = 0; j < k; ++j) {
-      const int32_t r = __shfl_sync(0xffffffffu, row, j);
-      if (r < 0) continue;
-      V* dst = xp + (int64_t)r * row_vecs;
+      V* dst = reinterpret_cast<V*>(
+          __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_dst), j));
+      if (dst == nullptr) continue;
 #pragma unroll
       for (int u = 0; u < kScatterUnroll; ++u) {
         const int v = v0 + u * 32 + lane;
@@ -253,13 +275,13 @@ __global__ void __launch_bounds__(32 * kScatterWarps, 8) dispatch_scatter_warp_k
 // scans the capped counts over the experts and resolves every slot's row, so that no block
 // waits for another; block 0 writes the routing outputs and each block gathers its share of
 // the kept rows (slots b, b + gridDim.x, ...).  The results are those of the three passes.
-template <typename V>
+template <typename V, bool kRemote>
 __global__ void __launch_bounds__(kSmallDispatchThreads) dispatch_small_kernel(
     const int32_t* __restrict__ ids, const uint8_t* __restrict__ drop_in, int N, int k, int E,
     int64_t C, const int32_t* __restrict__ cap_e, int32_t* __restrict__ demand,
     int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ slot_row,
     int32_t* __restrict__ row_token, uint8_t* __restrict__ drop_mask_out,
-    const V* __restrict__ x, V* __restrict__ xp, int row_vecs, int* status) {
+    const V* __restrict__ x, V* __restrict__ xp, int row_vecs, int* status, RemoteRows rem) {
   pdl_wait();
   extern __shared__ int32_t sm[];
   int32_t* cnt = sm;                 // [E]
@@ -346,13 +368,14 @@ __global__ void __launch_bounds__(kSmallDispatchThreads) dispatch_small_kernel(
     }
   }
   if (writer && tid == 0 && s_bad) report_status(status, kStatusInvalidInput);
-  if (xp == nullptr) return;
+  if (!kRemote && xp == nullptr) return;
   __syncthreads();
   for (int i = blockIdx.x; i < nk; i += gridDim.x) {
     const int32_t row = s_rank[i];
     if (row < 0) continue;
     const V* src = x + (int64_t)(i / k) * row_vecs;
-    V* dst = xp + (int64_t)row * row_vecs;
+    V* dst = gather_dst<kRemote>(xp, rem, s_id[i], row, offs[s_id[i]], row_vecs);
+    if (dst == nullptr) continue;
     for (int v = tid; v < row_vecs; v += blockDim.x) dst[v] = src[v];
   }
 }
@@ -389,19 +412,29 @@ cudaError_t launch_dispatch_small(const int32_t* ids, const uint8_t* drop_in, in
                                   int32_t* counts, int32_t* offsets, int32_t* slot_row,
                                   int32_t* row_token, uint8_t* drop_mask_out, const void* x,
                                   void* xp, int row_bytes, int* status, cudaStream_t stream,
-                                  int* launches) {
+                                  int* launches, const RemoteRows* rem) {
+  if (rem != nullptr && row_bytes % 16 != 0) return cudaErrorInvalidValue;
   ++*launches;
   const int nk = (int)(N * k);
   const size_t smem = sizeof(int32_t) * ((size_t)E + (size_t)E + 1 + 2 * (size_t)nk);
-  const int grid = xp != nullptr ? std::max(1, std::min(nk, tc::num_sms())) : 1;
-  if (xp != nullptr && row_bytes % 16 == 0) {
-    launch_pdl(dispatch_small_kernel<uint4>, grid, kSmallDispatchThreads, smem, stream, ids,
-               drop_in, (int)N, k, E, C, cap_e, demand, counts, offsets, slot_row, row_token,
-               drop_mask_out, (const uint4*)x, (uint4*)xp, row_bytes / 16, status);
+  const bool gather = xp != nullptr || rem != nullptr;
+  const int grid = gather ? std::max(1, std::min(nk, tc::num_sms())) : 1;
+  const RemoteRows none{};
+  if (rem != nullptr) {
+    launch_pdl(dispatch_small_kernel<uint4, true>, grid, kSmallDispatchThreads, smem, stream,
+               ids, drop_in, (int)N, k, E, C, cap_e, demand, counts, offsets, slot_row,
+               row_token, drop_mask_out, (const uint4*)x, (uint4*)nullptr, row_bytes / 16,
+               status, *rem);
+  } else if (xp != nullptr && row_bytes % 16 == 0) {
+    launch_pdl(dispatch_small_kernel<uint4, false>, grid, kSmallDispatchThreads, smem, stream,
+               ids, drop_in, (int)N, k, E, C, cap_e, demand, counts, offsets, slot_row,
+               row_token, drop_mask_out, (const uint4*)x, (uint4*)xp, row_bytes / 16, status,
+               none);
   } else {
-    launch_pdl(dispatch_small_kernel<uint32_t>, grid, kSmallDispatchThreads, smem, stream, ids,
-               drop_in, (int)N, k, E, C, cap_e, demand, counts, offsets, slot_row, row_token,
-               drop_mask_out, (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4, status);
+    launch_pdl(dispatch_small_kernel<uint32_t, false>, grid, kSmallDispatchThreads, smem,
+               stream, ids, drop_in, (int)N, k, E, C, cap_e, demand, counts, offsets, slot_row,
+               row_token, drop_mask_out, (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4,
+               status, none);
   }
   return cudaGetLastError();
 }
@@ -452,42 +485,53 @@ cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_ran
                                     int64_t N, int k, int E, int64_t C, int32_t* slot_row,
                                     int32_t* row_token, uint8_t* drop_mask_out,
                                     const void* x, void* xp, int row_bytes,
-                                    cudaStream_t stream, int* launches, const int32_t* cap_e) {
+                                    cudaStream_t stream, int* launches, const int32_t* cap_e,
+                                    const RemoteRows* rem) {
   if (N == 0) return cudaSuccess;
+  if (rem != nullptr && row_bytes % 16 != 0) return cudaErrorInvalidValue;
   ++*launches;
+  const RemoteRows none{};
   // warp per token when the warps fill every SM several times over and a token moves at
   // most 16 KB; else block per token
   const bool per_warp = N >= (int64_t)tc::num_sms() * 64 && (int64_t)k * row_bytes <= 16384;
   if (per_warp) {
     const unsigned grid = (unsigned)((N + kScatterWarps - 1) / kScatterWarps);
     const unsigned block = 32 * kScatterWarps;
-    if (xp != nullptr && row_bytes % 16 == 0) {
-      launch_pdl(dispatch_scatter_warp_kernel<uint4>, grid, block, 0, stream, ids, local_rank,
-                 tile_base, offsets, N, k, E, C, slot_row, row_token, drop_mask_out,
-                 (const uint4*)x, (uint4*)xp, row_bytes / 16, cap_e);
-    } else if (xp != nullptr) {
-      launch_pdl(dispatch_scatter_warp_kernel<uint32_t>, grid, block, 0, stream, ids,
+    if (rem != nullptr) {
+      launch_pdl(dispatch_scatter_warp_kernel<uint4, true>, grid, block, 0, stream, ids,
                  local_rank, tile_base, offsets, N, k, E, C, slot_row, row_token,
-                 drop_mask_out, (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4, cap_e);
+                 drop_mask_out, (const uint4*)x, (uint4*)nullptr, row_bytes / 16, cap_e, *rem);
+    } else if (xp != nullptr && row_bytes % 16 == 0) {
+      launch_pdl(dispatch_scatter_warp_kernel<uint4, false>, grid, block, 0, stream, ids,
+                 local_rank, tile_base, offsets, N, k, E, C, slot_row, row_token,
+                 drop_mask_out, (const uint4*)x, (uint4*)xp, row_bytes / 16, cap_e, none);
+    } else if (xp != nullptr) {
+      launch_pdl(dispatch_scatter_warp_kernel<uint32_t, false>, grid, block, 0, stream, ids,
+                 local_rank, tile_base, offsets, N, k, E, C, slot_row, row_token,
+                 drop_mask_out, (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4, cap_e, none);
     } else {
-      launch_pdl(dispatch_scatter_warp_kernel<uint4>, grid, block, 0, stream, ids, local_rank,
-                 tile_base, offsets, N, k, E, C, slot_row, row_token, drop_mask_out, nullptr,
-                 nullptr, 0, cap_e);
+      launch_pdl(dispatch_scatter_warp_kernel<uint4, false>, grid, block, 0, stream, ids,
+                 local_rank, tile_base, offsets, N, k, E, C, slot_row, row_token,
+                 drop_mask_out, nullptr, nullptr, 0, cap_e, none);
     }
     return cudaGetLastError();
   }
-  if (xp != nullptr && row_bytes % 16 == 0) {
-    launch_pdl(dispatch_scatter_kernel<uint4>, (unsigned)N, 128, 0, stream, ids, local_rank,
-               tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
-               (const uint4*)x, (uint4*)xp, row_bytes / 16, cap_e);
-  } else if (xp != nullptr) {
-    launch_pdl(dispatch_scatter_kernel<uint32_t>, (unsigned)N, 128, 0, stream, ids,
+  if (rem != nullptr) {
+    launch_pdl(dispatch_scatter_kernel<uint4, true>, (unsigned)N, 128, 0, stream, ids,
                local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
-               (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4, cap_e);
+               (const uint4*)x, (uint4*)nullptr, row_bytes / 16, cap_e, *rem);
+  } else if (xp != nullptr && row_bytes % 16 == 0) {
+    launch_pdl(dispatch_scatter_kernel<uint4, false>, (unsigned)N, 128, 0, stream, ids,
+               local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
+               (const uint4*)x, (uint4*)xp, row_bytes / 16, cap_e, none);
+  } else if (xp != nullptr) {
+    launch_pdl(dispatch_scatter_kernel<uint32_t, false>, (unsigned)N, 128, 0, stream, ids,
+               local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
+               (const uint32_t*)x, (uint32_t*)xp, row_bytes / 4, cap_e, none);
   } else {
-    launch_pdl(dispatch_scatter_kernel<uint4>, (unsigned)N, 128, 0, stream, ids, local_rank,
-               tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out, nullptr,
-               nullptr, 0, cap_e);
+    launch_pdl(dispatch_scatter_kernel<uint4, false>, (unsigned)N, 128, 0, stream, ids,
+               local_rank, tile_base, offsets, k, E, C, slot_row, row_token, drop_mask_out,
+               nullptr, nullptr, 0, cap_e, none);
   }
   return cudaGetLastError();
 }

@@ -59,16 +59,28 @@ cudaError_t launch_dispatch_scan(const int32_t* tile_hist, int64_t N, int E, int
                                  int32_t* tile_base, int32_t* demand, int32_t* counts,
                                  int32_t* offsets, int32_t* arrive, cudaStream_t stream,
                                  int* launches, const int32_t* cap_e = nullptr);
+// Per-expert destinations of the gathered rows (expert parallelism over peer memory): the
+// kept rows of expert e go to rows row0[e], row0[e] + 1, ... (in their layout order) of the
+// buffer at base[e] -- another device's receive buffer, or a local one.  Device arrays [E].
+struct RemoteRows {
+  const unsigned long long* base;
+  const int32_t* row0;
+  const int64_t* rows;   // [E]: rows of the buffer at base[e]; a row past it is skipped
+  int* status;           // where a skipped row is reported (invalid input), or null
+};
+
 // Pass 3: capacity decision (rank < C, or rank < cap_e[e] when cap_e is not null), slot
 // rows (when slot_row is not null), row -> token map, drop mask, and (when xp is not null)
-// the gather of x rows into the per-expert layout.
+// the gather of x rows into the per-expert layout -- or, with rem, into each expert's
+// destination instead (row_bytes % 16 == 0).
 cudaError_t launch_dispatch_scatter(const int32_t* ids, const int32_t* local_rank,
                                     const int32_t* tile_base, const int32_t* offsets,
                                     int64_t N, int k, int E, int64_t C, int32_t* slot_row,
                                     int32_t* row_token, uint8_t* drop_mask_out,
                                     const void* x, void* xp, int row_bytes,
                                     cudaStream_t stream, int* launches,
-                                    const int32_t* cap_e = nullptr);
+                                    const int32_t* cap_e = nullptr,
+                                    const RemoteRows* rem = nullptr);
 
 // The three passes in one launch for a small batch (N <= kSmallDispatchMaxTokens and
 // N * k <= kSmallDispatchMaxSlots): the same outputs, plus the device status for bad ids.
@@ -81,7 +93,7 @@ cudaError_t launch_dispatch_small(const int32_t* ids, const uint8_t* drop_in, in
                                   int32_t* counts, int32_t* offsets, int32_t* slot_row,
                                   int32_t* row_token, uint8_t* drop_mask_out, const void* x,
                                   void* xp, int row_bytes, int* status, cudaStream_t stream,
-                                  int* launches);
+                                  int* launches, const RemoteRows* rem = nullptr);
 
 // ---- expert-parallel rows over peer memory (ep_p2p.cu) ---------------------------------
 // Copy row runs (runs [n_runs][4] int32: src_row, dst_buf, dst_row, rows; run_start

@@ -349,13 +349,13 @@ moe_status stage_dispatch(const moe_config& c, const Ws& L, void* ws, const int3
                           int32_t* offsets, int32_t* slot_row, int32_t* row_token,
                           uint8_t* drop_out, const void* x, void* xp, cudaStream_t st,
                           int* launches, const int32_t* cap_e = nullptr,
-                          bool ranked = false) {
+                          bool ranked = false, const moe::RemoteRows* rem = nullptr) {
   int* status = at<int>(ws, L.status);
   if (!ranked && moe::use_small_dispatch(c.N, c.k, c.E)) {
     // a small batch: the three passes in one launch, with the same outputs
     MOE_CUDA(moe::launch_dispatch_small(ids, drop_in, c.N, c.k, c.E, C, cap_e, demand, counts,
                                         offsets, slot_row, row_token, drop_out, x, xp,
-                                        (int)(c.d * el_size(c)), status, st, launches),
+                                        (int)(c.d * el_size(c)), status, st, launches, rem),
              "dispatch (small batch)");
     prof_mark(st);
     return MOE_OK;
@@ -374,7 +374,7 @@ moe_status stage_dispatch(const moe_config& c, const Ws& L, void* ws, const int3
   MOE_CUDA(moe::launch_dispatch_scatter(ids, at<int32_t>(ws, L.local_rank),
                                         at<int32_t>(ws, L.tile_base), offsets, c.N, c.k, c.E, C,
                                         slot_row, row_token, drop_out, x, xp,
-                                        (int)(c.d * el_size(c)), st, launches, cap_e),
+                                        (int)(c.d * el_size(c)), st, launches, cap_e, rem),
            "scatter pass");
   prof_mark(st);
   return MOE_OK;
@@ -1202,6 +1202,36 @@ moe_status moe_permute_ep(const moe_config* cfg, const int32_t* ids, const int32
                          slot_row, row_token,
                          drop_mask != nullptr ? drop_mask : at<uint8_t>(ws, L.drop_mask), x, xp,
                          (cudaStream_t)stream, &launches, cap));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_permute_ep_p2p(const moe_config* cfg, const int32_t* ids, const int32_t* cap,
+                              const void* x, int32_t* offsets, int32_t* slot_row,
+                              const uint64_t* dst_base, const int32_t* dst_row0,
+                              const int64_t* dst_rows, int32_t* counts, uint8_t* drop_mask,
+                              void* ws, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_permute_ep_p2p");
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  if (ids == nullptr || cap == nullptr || offsets == nullptr || slot_row == nullptr ||
+      dst_base == nullptr || dst_row0 == nullptr || dst_rows == nullptr)
+    return fail(MOE_ERR_INVALID_ARG,
+                "ids, cap, offsets, slot_row, dst_base, dst_row0 and dst_rows are required");
+  MOE_TRY(need(x, "x"));
+  const moe_config& c = *cfg;
+  if (c.dtype != MOE_DT_BF16 || (c.d * el_size(c)) % 16 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_permute_ep_p2p: bf16 rows of a multiple of 16 bytes");
+  const Ws L = layout(c);
+  const moe::RemoteRows rem{(const unsigned long long*)dst_base, dst_row0, dst_rows,
+                            at<int>(ws, L.status)};
+  int launches = 0;
+  MOE_TRY(stage_dispatch(c, L, ws, ids, nullptr, 0, at<int32_t>(ws, L.demand),
+                         counts != nullptr ? counts : at<int32_t>(ws, L.counts), offsets,
+                         slot_row, nullptr,
+                         drop_mask != nullptr ? drop_mask : at<uint8_t>(ws, L.drop_mask), x,
+                         nullptr, (cudaStream_t)stream, &launches, cap, false, &rem));
   g_last_launches = launches;
   return MOE_OK;
 }

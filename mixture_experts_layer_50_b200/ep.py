@@ -14,8 +14,9 @@ the experts ``[first(r), first(r+1))`` and a copy of the shared expert.  A forwa
    counts, the row runs to send and where received runs land;
 4. ``moe_permute_ep``: this rank's kept rows in the send layout (expert-major);
 5. dispatch: one grouped point-to-point exchange of the row runs (NCCL on GPUs), or with
-   ``transport="p2p"`` one launch that writes the runs straight into the owners' receive
-   buffers over peer memory (CUDA IPC mappings; NVLink on a multi-GPU node);
+   ``transport="p2p"`` the dispatch passes of step 4 write the kept rows straight into the
+   owners' receive buffers over peer memory (CUDA IPC mappings; NVLink on a multi-GPU node)
+   and the return trip is one copy launch;
 6. ``moe_ep_expert_ffn``: the owned experts on the received rows (tcgen05 grouped GEMMs), and
    the shared expert on the rank's own tokens, written straight into y;
 7. combine trip: the same runs back to their source ranks;
@@ -153,6 +154,7 @@ class PeerTransport:
             recv_rows.append(nr)
             ret_rows.append(nt)
         i64 = dict(dtype=torch.int64, device=dev)
+        self._recv_base_host, self._recv_rows_host = recv_base, recv_rows
         self.recv_base, self.recv_rows = torch.tensor(recv_base, **i64), torch.tensor(recv_rows, **i64)
         self.ret_base, self.ret_rows = torch.tensor(ret_base, **i64), torch.tensor(ret_rows, **i64)
         if barrier is None:
@@ -165,7 +167,40 @@ class PeerTransport:
                     dist.barrier(group=group)
         self.barrier = barrier
 
+    def expert_destinations(self, plans: Sequence[dict]):
+        """Per expert e: the receive buffer of e's owner, the row where this rank's kept rows
+        of e start in it, and its size (host lists of E entries)."""
+        L = self.layer
+        E, rank = L.E, L.rank
+        base, row0, rows = [self._recv_base_host[rank]] * E, [0] * E, [0] * E
+        for peer, e, _, n in plans[rank]["sends"]:
+            dst = {(p, ex): r for p, ex, r, _ in plans[peer]["recvs"]}
+            base[e], row0[e], rows[e] = (self._recv_base_host[peer], dst[(rank, e)],
+                                         self._recv_rows_host[peer])
+        return base, row0, rows
+
+    def dispatch_fused(self, x: torch.Tensor, plans: Sequence[dict]) -> torch.Tensor:
+        """The dispatch passes with the kept rows written straight into their owners'
+        receive buffers (moe_permute_ep_p2p), then the barrier; returns this rank's received
+        rows."""
+        L = self.layer
+        N = L.N
+        if N > 0:
+            dev = x.device
+            base, row0, rows = self.expert_destinations(plans)
+            nat.moe_permute_ep_p2p(
+                L.config(N), ids=L.ids[:N], cap=L.cap, x=x, offsets=L.offsets,
+                slot_row=L.slot_row[:N],
+                dst_base=torch.tensor(base, dtype=torch.int64).to(dev, non_blocking=True),
+                dst_row0=torch.tensor(row0, dtype=torch.int32).to(dev, non_blocking=True),
+                dst_rows=torch.tensor(rows, dtype=torch.int64).to(dev, non_blocking=True),
+                counts=L.counts, drop_mask=L.drop_mask[:N], ws=L.ws)
+        self.barrier()
+        return self.recv[:max(1, plans[L.rank]["rows_owned"])]
+
     def dispatch(self, xp: torch.Tensor, plans: Sequence[dict]) -> torch.Tensor:
+        """The rows of a send buffer (moe_permute_ep's layout) copied into the owners' receive
+        buffers (moe_ep_copy_runs), then the barrier."""
         L = self.layer
         nat.moe_ep_copy_runs(xp, dst_base=self.recv_base, dst_rows=self.recv_rows,
                              runs=peer_runs(L.rank, plans, "dispatch"), ws=L.ws)
@@ -330,11 +365,12 @@ class EPMoELayer:
             gathered = torch.empty(self.world * (self.E + 1), dtype=torch.int32)
             dist.all_gather_into_tensor(gathered, demand.cpu(), group=self.group)
         plan = self.set_plan(gathered)
-        xp = self.permute(x)
         if self.transport is not None:
-            xr = self.transport.dispatch(xp, self.plans)
+            # the dispatch passes write the kept rows straight into the owners' buffers
+            xr = self.transport.dispatch_fused(x, self.plans)
             ye = self.run_experts(xr, x, y)
             return self.combine(self.transport.give_back(ye, self.plans), y)
+        xp = self.permute(x)
         xr = self.new_recv_buffer()
         exchange_rows(xp, xr, plan["sends"], plan["recvs"], self.rank, self.group)
         ye = self.run_experts(xr, x, y)

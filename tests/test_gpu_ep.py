@@ -316,3 +316,71 @@ def test_peer_transport_between_processes_equals_the_single_device_layer(case, t
     for call in range(2):
         y_ep = torch.cat([r["y"][call] for r in res]).cuda()
         assert torch.equal(y_ep, y), call
+
+
+@pytest.mark.parametrize("world,case", [(2, CASES[0]), (3, CASES[2]), (4, CASES[1])])
+def test_dispatch_passes_writing_into_the_owners_buffers(world, case):
+    """moe_permute_ep_p2p: the dispatch passes write each kept row straight into its owner's
+    receive buffer (per-expert destinations from every rank's plan; local buffers here, one per
+    emulated rank).  Receive buffers, slot rows, counts and drop masks equal moe_permute_ep
+    followed by the message exchange, bit for bit; a destination too small is reported."""
+    from mixture_experts_layer_50_b200.ep import all_plans
+    name, N, d, E, F, k, cf = case
+    shape = W.PRESETS[name].replace(N=N, d=d, E=E, F=F, k=k)
+    t = W.make_inputs(shape, device="cuda")
+    sizes = _split(N, world, seed=world * 7 + E)
+    starts = np.r_[0, np.cumsum(sizes)]
+    xs = [t["x"][starts[r]:starts[r + 1]] for r in range(world)]
+    mod = t.get("modality")
+    mods = [None if mod is None else mod[starts[r]:starts[r + 1]] for r in range(world)]
+    layers = _layers(shape, t, world, int(sizes.max()), cf)
+    dem = [L.route(x, m) for L, x, m in zip(layers, xs, mods)]
+    gathered = torch.stack(dem).cpu()
+    plans = [L.set_plan(gathered) for L in layers]
+    # the reference: send buffers and the message exchange
+    sends = [L.permute(x) for L, x in zip(layers, xs)]
+    want = [L.new_recv_buffer().zero_() for L in layers]
+    loopback_exchange(sends, want, [p["sends"] for p in plans], [p["recvs"] for p in plans])
+    ref = [dict(slot=L.slot_row[:L.N].clone(), counts=L.counts.clone(),
+                drop=L.drop_mask[:L.N].clone()) for L in layers]
+    # the dispatch passes writing into the owners' buffers
+    got = [torch.zeros_like(w) for w in want]
+    addr = [g.data_ptr() for g in got]
+    nrows = [g.shape[0] for g in got]
+    for r, L in enumerate(layers):
+        base, row0, rows = [addr[r]] * E, [0] * E, [0] * E
+        for peer, e, _, n in plans[r]["sends"]:
+            dst = {(p_, ex): rr for p_, ex, rr, _ in plans[peer]["recvs"]}
+            base[e], row0[e], rows[e] = addr[peer], dst[(r, e)], nrows[peer]
+        if L.N == 0:
+            continue
+        L.slot_row.fill_(-7)
+        nat.moe_permute_ep_p2p(
+            L.config(L.N), ids=L.ids[:L.N], cap=L.cap, x=xs[r], offsets=L.offsets,
+            slot_row=L.slot_row[:L.N],
+            dst_base=torch.tensor(base, dtype=torch.int64, device="cuda"),
+            dst_row0=torch.tensor(row0, dtype=torch.int32, device="cuda"),
+            dst_rows=torch.tensor(rows, dtype=torch.int64, device="cuda"),
+            counts=L.counts, drop_mask=L.drop_mask[:L.N], ws=L.ws)
+        check_status(L.ws)
+        assert torch.equal(L.slot_row[:L.N], ref[r]["slot"])
+        assert torch.equal(L.counts, ref[r]["counts"])
+        assert torch.equal(L.drop_mask[:L.N], ref[r]["drop"])
+    for g, w in zip(got, want):
+        assert torch.equal(g, w)
+    # a destination one row too small: that row is skipped and reported
+    r = next(i for i, L in enumerate(layers) if plans[i]["sends"])
+    L = layers[r]
+    peer, e, _, n = plans[r]["sends"][-1]
+    dst = {(p_, ex): rr for p_, ex, rr, _ in plans[peer]["recvs"]}
+    base, row0, rows = [addr[r]] * E, [0] * E, [0] * E
+    for pp, ee, _, nn in plans[r]["sends"]:
+        dd = {(p_, ex): rr for p_, ex, rr, _ in plans[pp]["recvs"]}
+        base[ee], row0[ee], rows[ee] = addr[pp], dd[(r, ee)], nrows[pp]
+    rows[e] = dst[(r, e)] + n - 1
+    nat.moe_permute_ep_p2p(
+        L.config(L.N), ids=L.ids[:L.N], cap=L.cap, x=xs[r], offsets=L.offsets,
+        slot_row=L.slot_row[:L.N], dst_base=torch.tensor(base, dtype=torch.int64, device="cuda"),
+        dst_row0=torch.tensor(row0, dtype=torch.int32, device="cuda"),
+        dst_rows=torch.tensor(rows, dtype=torch.int64, device="cuda"), ws=L.ws)
+    assert nat.moe_check_status(L.ws) == nat.MOE_ERR_INVALID_INPUT

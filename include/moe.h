@@ -385,6 +385,24 @@ MOE_API moe_status moe_ep_expert_ffn(const moe_config* cfg, int32_t world, int32
 MOE_API moe_status moe_ep_combine(const moe_config* cfg, const void* ye, const int32_t* slot_row,
                                   const float* gates, void* y, moe_stream_t stream);
 
+/* moe_ep_combine with the return trip folded in ("Support visuel — Communication": the
+ * expert's output travels back to the token's device): each kept slot's expert output is read
+ * where its owner wrote it, instead of from a local ye.  Slot (t, j), kept for expert
+ * e = ids[t][j] at row r = slot_row[t][j] of this rank's send layout (offsets [E + 1] from
+ * moe_permute_ep / moe_permute_ep_p2p), reads row src_row0[e] + (r - offsets[e]) of the buffer
+ * at src_base[e] (device uint64 [E]: the output buffer of e's owner, another process's
+ * allocation mapped with moe_ipc_open, or a local buffer), which holds src_rows[e] rows (device
+ * int64 [E]).  A slot whose expert or row falls outside these bounds contributes nothing and
+ * is reported as MOE_ERR_INVALID_INPUT by moe_check_status.  The sums, their order and the
+ * rounding are those of moe_ep_combine, so the bits are too.  bf16 only; d * 2 a multiple of
+ * 16.  The caller orders it after the owners' expert FFNs (a stream-ordered barrier) and
+ * keeps the owners from overwriting their outputs until every rank's combine is done. */
+MOE_API moe_status moe_ep_combine_p2p(const moe_config* cfg, const int32_t* ids,
+                                      const int32_t* slot_row, const float* gates,
+                                      const int32_t* offsets, const uint64_t* src_base,
+                                      const int32_t* src_row0, const int64_t* src_rows, void* y,
+                                      void* ws, moe_stream_t stream);
+
 /* The exchange of the plan's row runs over peer memory ("Support visuel — Communication"):
  * one launch writes rows of src [src_rows][row_bytes] (this device) straight into other
  * buffers -- another process's allocation mapped with moe_ipc_open (on a multi-GPU node,

@@ -21,7 +21,8 @@ _NATIVE_NAMES = {
     "moe_permute_padded", "moe_forward_padded", "moe_forward_host_batches", "moe_config", "moe_route_out", "make_config",
     "config_from_shape", "MoeError", "lib", "EXPORTED", "moe_ep_first_expert", "moe_ep_plan",
     "moe_ep_workspace_size", "alloc_ep_workspace", "moe_permute_ep", "moe_ep_expert_ffn",
-    "moe_ep_combine",
+    "moe_ep_combine", "moe_ep_copy_runs", "moe_permute_ep_p2p", "moe_ep_combine_p2p",
+    "ipc_handle", "ipc_open", "ipc_close",
 }
 
 

@@ -95,6 +95,7 @@ lib.moe_ep_expert_ffn.argtypes = [_cfgp, _i32, _i32, _i64, _i64] + [_vp] * 9
 lib.moe_ep_combine.argtypes = [_cfgp] + [_vp] * 5
 lib.moe_ep_copy_runs.argtypes = [_vp, _i64, _vp, _vp, _i32, _vp, _vp, _i32, _i64, _i64, _vp, _vp]
 lib.moe_permute_ep_p2p.argtypes = [_cfgp] + [_vp] * 12
+lib.moe_ep_combine_p2p.argtypes = [_cfgp] + [_vp] * 10
 lib.moe_ipc_handle.argtypes = [_vp, _vp, ctypes.POINTER(_i64)]
 lib.moe_ipc_open.argtypes = [_vp, ctypes.POINTER(_vp)]
 lib.moe_ipc_close.argtypes = [_vp]
@@ -113,7 +114,7 @@ for _f in ("moe_workspace_init", "moe_route", "moe_permute", "moe_expert_ffn", "
            "moe_forward_reroute", "moe_selftest_wait_timeout", "moe_ffn_kernels", "moe_ep_plan",
            "moe_permute_ep", "moe_ep_expert_ffn", "moe_ep_combine", "moe_check_dispatch_host",
            "moe_check_dispatch", "moe_ep_copy_runs", "moe_ipc_handle", "moe_ipc_open",
-           "moe_ipc_close", "moe_permute_ep_p2p"):
+           "moe_ipc_close", "moe_permute_ep_p2p", "moe_ep_combine_p2p"):
     getattr(lib, _f).restype = ctypes.c_int
 
 EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_route",
@@ -126,7 +127,7 @@ EXPORTED = ("moe_workspace_size", "moe_workspace_init", "moe_capacity", "moe_rou
             "moe_ep_plan", "moe_ep_workspace_size", "moe_permute_ep", "moe_ep_expert_ffn",
             "moe_ep_combine", "moe_check_dispatch_host", "moe_check_dispatch",
             "moe_ep_copy_runs", "moe_ipc_handle", "moe_ipc_open", "moe_ipc_close",
-            "moe_permute_ep_p2p")
+            "moe_permute_ep_p2p", "moe_ep_combine_p2p")
 
 
 def make_config(N, d, E, k, F, n_shared=0, n_bias_sets=0, score_fn=SOFTMAX, renorm=1,
@@ -499,6 +500,17 @@ def moe_permute_ep_p2p(cfg, *, ids, cap, x, offsets, slot_row, dst_base, dst_row
                                 _ptr(slot_row), _ptr(dst_base), _ptr(dst_row0), _ptr(dst_rows),
                                 _ptr(counts), _ptr(drop_mask), _ptr(ws), _stream(stream))
     _check(st, "moe_permute_ep_p2p")
+
+
+def moe_ep_combine_p2p(cfg, *, ids, slot_row, gates, offsets, src_base, src_row0, src_rows, y,
+                       ws, stream=None):
+    """moe_ep_combine reading slot (t, j)'s expert output (expert e = ids[t, j], send-layout
+    row r) at row src_row0[e] + r - offsets[e] of the buffer at src_base[e] (device int64 [E]
+    addresses, int32 [E] first rows, int64 [E] sizes)."""
+    st = lib.moe_ep_combine_p2p(ctypes.byref(cfg), _ptr(ids), _ptr(slot_row), _ptr(gates),
+                                _ptr(offsets), _ptr(src_base), _ptr(src_row0), _ptr(src_rows),
+                                _ptr(y), _ptr(ws), _stream(stream))
+    _check(st, "moe_ep_combine_p2p")
 
 
 def ipc_handle(t: torch.Tensor):

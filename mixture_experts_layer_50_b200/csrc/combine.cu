@@ -9,6 +9,11 @@
 // In the fused layer the down GEMM writes the shared expert's rows straight into y; the
 // combine then reads y[t] as the shared row, adds the kept slots to it in place, and leaves a
 // token with no kept slot as the GEMM wrote it.
+//
+// Expert parallelism over peer memory ("Support visuel — Communication"): the remote variants
+// read each kept slot's expert output where its owner wrote it -- row row0[e] + (r - offsets[e])
+// of the owner's output buffer, e = ids[t, j], r the slot's row in the send layout -- so the
+// return trip of the rows and the combine are one pass.
 #include <cstdlib>
 
 #include "common.cuh"
@@ -27,22 +32,61 @@ __device__ __forceinline__ void accum_bf16x8(float (&acc)[8], const uint4& v, fl
   }
 }
 
+// The first 16-byte vector of slot (t, j)'s expert output row, or null when the slot was
+// dropped (r < 0) or, for the remote variant, its expert or row falls outside the tables
+// (reported in rem.status; the slot then contributes nothing).
+template <bool kRemote>
+__device__ __forceinline__ const uint4* slot_src(const uint4* ye, const RemoteSrc& rem,
+                                                 int64_t slot, int32_t r, int vecs) {
+  if (r < 0) return nullptr;
+  if constexpr (!kRemote) {
+    return ye + (int64_t)r * vecs;
+  } else {
+    const int32_t e = rem.ids[slot];
+    if (e >= 0 && e < rem.E) {
+      const int64_t lo = rem.offsets[e], hi = rem.offsets[e + 1];
+      const int64_t row = (int64_t)rem.row0[e] + (r - lo);
+      if (r >= lo && r < hi && row >= 0 && row < rem.rows[e])
+        return reinterpret_cast<const uint4*>(rem.base[e]) + row * vecs;
+    }
+    if (rem.status != nullptr) report_status(rem.status, kStatusInvalidInput);
+    return nullptr;
+  }
+}
+
+// Local rows come through the read-only path (they were written by an earlier kernel and
+// this one does not write them); remote rows are read at L2, bypassing L1.
+template <bool kRemote>
+__device__ __forceinline__ uint4 load_row_vec(const uint4* p) {
+  if constexpr (kRemote) return __ldcg(p);
+  else return __ldg(p);
+}
+
 // KMAX >= k bounds the slots so that the k row loads of a vector are issued together
 // before the sums (KMAX = 0: any k, one load after the other).  Either way the sum runs in
 // slot order and then adds the shared row, so every KMAX gives the same bits.  The shared row
 // is ye[shared_row0 + t] (shared_row0 >= 0), y[t] itself (shared_in_y), or absent.
-template <int KMAX>
+template <int KMAX, bool kRemote>
 __global__ void __launch_bounds__(128) combine_bf16_kernel(
     const uint4* __restrict__ ye, const int32_t* __restrict__ slot_row,
     const float* __restrict__ gates, int k, int vecs, int64_t shared_row0, int shared_in_y,
-    uint4* __restrict__ y) {
+    RemoteSrc rem, uint4* __restrict__ y) {
   pdl_wait();
-  __shared__ int32_t s_row[33];
+  __shared__ int32_t s_row[33];        // local: the slot's row of ye, -1 when dropped
+  __shared__ const uint4* s_src[33];   // remote: the slot's row address, null when dropped
   __shared__ float s_g[33];
   const int64_t t = blockIdx.x;
   if (threadIdx.x < k) {
-    s_row[threadIdx.x] = slot_row[t * k + threadIdx.x];
-    s_g[threadIdx.x] = gates[t * k + threadIdx.x];
+    const int64_t slot = t * k + threadIdx.x;
+    const int32_t r = slot_row[slot];
+    if constexpr (kRemote) {
+      const uint4* p = slot_src<true>(ye, rem, slot, r, vecs);
+      s_src[threadIdx.x] = p;
+      s_row[threadIdx.x] = p != nullptr ? 0 : -1;
+    } else {
+      s_row[threadIdx.x] = r;
+    }
+    s_g[threadIdx.x] = gates[slot];
   }
   __syncthreads();
   if (shared_in_y) {
@@ -50,6 +94,9 @@ __global__ void __launch_bounds__(128) combine_bf16_kernel(
     for (int j = 0; j < k; ++j) any |= s_row[j] >= 0;
     if (!any) return;  // y[t] is the shared row already
   }
+  auto row_vec = [&](int j, int v) {
+    return load_row_vec<kRemote>(kRemote ? s_src[j] + v : ye + (int64_t)s_row[j] * vecs + v);
+  };
   const uint4* shp = shared_in_y ? y + t * vecs
                                  : (shared_row0 >= 0 ? ye + (shared_row0 + t) * vecs : nullptr);
   for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
@@ -58,7 +105,7 @@ __global__ void __launch_bounds__(128) combine_bf16_kernel(
       uint4 rows[KMAX];
 #pragma unroll
       for (int j = 0; j < KMAX; ++j)
-        if (j < k && s_row[j] >= 0) rows[j] = ye[(int64_t)s_row[j] * vecs + v];
+        if (j < k && s_row[j] >= 0) rows[j] = row_vec(j, v);
       uint4 sh = make_uint4(0u, 0u, 0u, 0u);
       if (shp != nullptr) sh = shp[v];
 #pragma unroll
@@ -66,10 +113,8 @@ __global__ void __launch_bounds__(128) combine_bf16_kernel(
         if (j < k && s_row[j] >= 0) accum_bf16x8(acc, rows[j], s_g[j]);
       if (shp != nullptr) accum_bf16x8(acc, sh, 1.0f);
     } else {
-      for (int j = 0; j < k; ++j) {
-        const int32_t r = s_row[j];
-        if (r >= 0) accum_bf16x8(acc, ye[(int64_t)r * vecs + v], s_g[j]);
-      }
+      for (int j = 0; j < k; ++j)
+        if (s_row[j] >= 0) accum_bf16x8(acc, row_vec(j, v), s_g[j]);
       if (shp != nullptr) accum_bf16x8(acc, shp[v], 1.0f);
     }
     uint4 o;
@@ -86,28 +131,41 @@ __global__ void __launch_bounds__(128) combine_bf16_kernel(
 // the block-per-token kernel); the summation order is the same, so the bits are.
 constexpr int kCombineWarps = 8;
 
-template <int KMAX>
+template <int KMAX, bool kRemote>
 __global__ void __launch_bounds__(32 * kCombineWarps) combine_bf16_warp_kernel(
     const uint4* __restrict__ ye, const int32_t* __restrict__ slot_row,
     const float* __restrict__ gates, int64_t N, int k, int vecs, int64_t shared_row0,
-    int shared_in_y, uint4* __restrict__ y) {
+    int shared_in_y, RemoteSrc rem, uint4* __restrict__ y) {
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
   if (t >= N) return;  // warp-uniform
+  // lane j < k holds slot j: its row index (local) or its row's address (remote; the 64-bit
+  // broadcast is kept out of the local variant, where the extra registers cost occupancy)
   int32_t my_row = -1;
+  const uint4* my_src = nullptr;
   float my_g = 0.f;
   if (lane < k) {
-    my_row = slot_row[t * k + lane];
-    my_g = gates[t * k + lane];
+    const int64_t slot = t * k + lane;
+    my_row = slot_row[slot];
+    if constexpr (kRemote) my_src = slot_src<true>(ye, rem, slot, my_row, vecs);
+    my_g = gates[slot];
   }
-  const unsigned kept = __ballot_sync(0xffffffffu, my_row >= 0);
+  const unsigned kept = __ballot_sync(0xffffffffu, kRemote ? my_src != nullptr : my_row >= 0);
   if (shared_in_y && kept == 0u) return;  // y[t] is the shared row already
   int32_t rj[KMAX];
+  const uint4* pj[KMAX];
   float gj[KMAX];
 #pragma unroll
   for (int j = 0; j < KMAX; ++j) {
-    rj[j] = __shfl_sync(0xffffffffu, my_row, j);
+    if constexpr (kRemote) {
+      pj[j] = reinterpret_cast<const uint4*>(
+          __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_src), j));
+      rj[j] = pj[j] != nullptr ? 0 : -1;
+    } else {
+      rj[j] = __shfl_sync(0xffffffffu, my_row, j);
+      pj[j] = nullptr;
+    }
     gj[j] = __shfl_sync(0xffffffffu, my_g, j);
   }
   const uint4* shp = shared_in_y ? y + t * vecs
@@ -117,7 +175,8 @@ __global__ void __launch_bounds__(32 * kCombineWarps) combine_bf16_warp_kernel(
     uint4 rows[KMAX];
 #pragma unroll
     for (int j = 0; j < KMAX; ++j)
-      if (j < k && rj[j] >= 0) rows[j] = ye[(int64_t)rj[j] * vecs + v];
+      if (j < k && rj[j] >= 0)
+        rows[j] = load_row_vec<kRemote>(kRemote ? pj[j] + v : ye + (int64_t)rj[j] * vecs + v);
     uint4 sh = make_uint4(0u, 0u, 0u, 0u);
     if (shp != nullptr) sh = shp[v];
 #pragma unroll
@@ -177,43 +236,58 @@ bool combine_warp_enabled() {
 
 }  // namespace
 
+namespace {
+
+template <bool kRemote>
+void launch_combine_bf16(const uint4* src, const int32_t* slot_row, const float* gates,
+                         int64_t N, int k, int d, int64_t shared_row0, int shared_in_y,
+                         const RemoteSrc& rem, uint4* dst, cudaStream_t stream) {
+  // warp per token when the warps fill every SM several times over and a token reads at
+  // most 8 KB of expert rows; else block per token.  Measured: the capacity and Switch
+  // layers (8 and 4 KB per token) 19.7 -> 16.4 and 16.6 -> 14.2 us; the Mixtral-shaped
+  // prefill (16 KB per token) 72.5 -> 77.4 us, so it keeps a block per token.
+  const int row_bytes = d * 2;
+  const int vecs = d / 8;
+  if (k <= 8 && N >= (int64_t)tc::num_sms() * 64 && (int64_t)k * row_bytes <= 8192 &&
+      combine_warp_enabled()) {
+    const unsigned wblocks = (unsigned)((N + kCombineWarps - 1) / kCombineWarps);
+    const unsigned th = 32 * kCombineWarps;
+    if (k <= 2)
+      launch_pdl(combine_bf16_warp_kernel<2, kRemote>, wblocks, th, 0, stream, src, slot_row, gates, N, k, vecs, shared_row0, shared_in_y, rem, dst);
+    else if (k <= 4)
+      launch_pdl(combine_bf16_warp_kernel<4, kRemote>, wblocks, th, 0, stream, src, slot_row, gates, N, k, vecs, shared_row0, shared_in_y, rem, dst);
+    else
+      launch_pdl(combine_bf16_warp_kernel<8, kRemote>, wblocks, th, 0, stream, src, slot_row, gates, N, k, vecs, shared_row0, shared_in_y, rem, dst);
+    return;
+  }
+  const unsigned blocks = (unsigned)N;
+  if (k <= 2)
+    launch_pdl(combine_bf16_kernel<2, kRemote>, blocks, 128, 0, stream, src, slot_row, gates, k, vecs, shared_row0, shared_in_y, rem, dst);
+  else if (k <= 4)
+    launch_pdl(combine_bf16_kernel<4, kRemote>, blocks, 128, 0, stream, src, slot_row, gates, k, vecs, shared_row0, shared_in_y, rem, dst);
+  else if (k <= 8)
+    launch_pdl(combine_bf16_kernel<8, kRemote>, blocks, 128, 0, stream, src, slot_row, gates, k, vecs, shared_row0, shared_in_y, rem, dst);
+  else
+    launch_pdl(combine_bf16_kernel<0, kRemote>, blocks, 128, 0, stream, src, slot_row, gates, k, vecs, shared_row0, shared_in_y, rem, dst);
+}
+
+}  // namespace
+
 cudaError_t launch_combine(const void* ye, const int32_t* slot_row, const float* gates,
                            int64_t N, int k, int d, int64_t shared_row0, int shared_in_y,
-                           int is_f32, void* y, cudaStream_t stream, int* launches) {
+                           int is_f32, void* y, cudaStream_t stream, int* launches,
+                           const RemoteSrc* rem) {
   if (N == 0) return cudaSuccess;
   ++*launches;
   if (is_f32) {
     launch_pdl(combine_f32_kernel, (unsigned)N, 128, 0, stream, (const float4*)ye, slot_row, gates, k,
                                                         d / 4, shared_row0, (float4*)y);
+  } else if (rem != nullptr) {
+    launch_combine_bf16<true>((const uint4*)ye, slot_row, gates, N, k, d, shared_row0,
+                              shared_in_y, *rem, (uint4*)y, stream);
   } else {
-    const uint4* src = (const uint4*)ye;
-    uint4* dst = (uint4*)y;
-    // warp per token when the warps fill every SM several times over and a token reads at
-    // most 8 KB of expert rows; else block per token.  Measured: the capacity and Switch
-    // layers (8 and 4 KB per token) 19.7 -> 16.4 and 16.6 -> 14.2 us; the Mixtral-shaped
-    // prefill (16 KB per token) 72.5 -> 77.4 us, so it keeps a block per token.
-    const int row_bytes = d * 2;
-    if (k <= 8 && N >= (int64_t)tc::num_sms() * 64 && (int64_t)k * row_bytes <= 8192 &&
-        combine_warp_enabled()) {
-      const unsigned wblocks = (unsigned)((N + kCombineWarps - 1) / kCombineWarps);
-      const unsigned th = 32 * kCombineWarps;
-      if (k <= 2)
-        launch_pdl(combine_bf16_warp_kernel<2>, wblocks, th, 0, stream, src, slot_row, gates, N, k, d / 8, shared_row0, shared_in_y, dst);
-      else if (k <= 4)
-        launch_pdl(combine_bf16_warp_kernel<4>, wblocks, th, 0, stream, src, slot_row, gates, N, k, d / 8, shared_row0, shared_in_y, dst);
-      else
-        launch_pdl(combine_bf16_warp_kernel<8>, wblocks, th, 0, stream, src, slot_row, gates, N, k, d / 8, shared_row0, shared_in_y, dst);
-      return cudaGetLastError();
-    }
-    const unsigned blocks = (unsigned)N;
-    if (k <= 2)
-      launch_pdl(combine_bf16_kernel<2>, blocks, 128, 0, stream, src, slot_row, gates, k, d / 8, shared_row0, shared_in_y, dst);
-    else if (k <= 4)
-      launch_pdl(combine_bf16_kernel<4>, blocks, 128, 0, stream, src, slot_row, gates, k, d / 8, shared_row0, shared_in_y, dst);
-    else if (k <= 8)
-      launch_pdl(combine_bf16_kernel<8>, blocks, 128, 0, stream, src, slot_row, gates, k, d / 8, shared_row0, shared_in_y, dst);
-    else
-      launch_pdl(combine_bf16_kernel<0>, blocks, 128, 0, stream, src, slot_row, gates, k, d / 8, shared_row0, shared_in_y, dst);
+    launch_combine_bf16<false>((const uint4*)ye, slot_row, gates, N, k, d, shared_row0,
+                               shared_in_y, RemoteSrc{}, (uint4*)y, stream);
   }
   return cudaGetLastError();
 }

@@ -130,9 +130,22 @@ cudaError_t launch_zero_padding(const int32_t* counts, int E, int64_t C, void* x
 // y[t] = sum_j gates[t,j] ye[slot_row[t,j]] (+ ye[shared_row0 + t] when shared_row0 >= 0).
 // shared_row0 >= 0: the shared row of token t is ye[shared_row0 + t]; shared_in_y (bf16):
 // y[t] holds it already (written by the down GEMM) and is updated in place.
+// rem (bf16 only): slot (t, j) kept for expert e = ids[t, j] at send-layout row r reads row
+// row0[e] + (r - offsets[e]) of the buffer at base[e] (rows[e] rows; offsets [E + 1]) instead
+// of ye[r]; a slot outside those bounds contributes nothing and is reported in status.
+struct RemoteSrc {
+  const unsigned long long* base;
+  const int32_t* row0;
+  const int64_t* rows;
+  const int32_t* offsets;
+  const int32_t* ids;
+  int E;
+  int* status;
+};
 cudaError_t launch_combine(const void* ye, const int32_t* slot_row, const float* gates,
                            int64_t N, int k, int d, int64_t shared_row0, int shared_in_y,
-                           int is_f32, void* y, cudaStream_t stream, int* launches);
+                           int is_f32, void* y, cudaStream_t stream, int* launches,
+                           const RemoteSrc* rem = nullptr);
 
 // ---- fp32 path (simt_f32.cu) ----------------------------------------------------------
 cudaError_t launch_router_f32(const float* x, const float* W_g, const float* logit_offset,

@@ -541,11 +541,12 @@ moe_status stage_ffn(const moe_config& c, const Ws& L, void* ws, const void* xp,
 // shared_in_y: stage_ffn wrote the shared expert's rows into y (bf16 only).
 moe_status stage_combine(const moe_config& c, const void* ye, const int32_t* slot_row,
                          const float* gates, void* y, cudaStream_t st, int* launches,
-                         int64_t R = -1, bool shared_in_y = false) {
+                         int64_t R = -1, bool shared_in_y = false,
+                         const moe::RemoteSrc* rem = nullptr) {
   const bool in_y = shared_in_y && c.n_shared && c.dtype == MOE_DT_BF16;
   const int64_t shared_row0 = (c.n_shared && !in_y) ? (R >= 0 ? R : c.N * (int64_t)c.k) : -1;
   MOE_CUDA(moe::launch_combine(ye, slot_row, gates, c.N, c.k, c.d, shared_row0, in_y ? 1 : 0,
-                               c.dtype == MOE_DT_F32, y, st, launches),
+                               c.dtype == MOE_DT_F32, y, st, launches, rem),
            "combine");
   prof_mark(st);
   return MOE_OK;
@@ -1301,6 +1302,33 @@ moe_status moe_ep_combine(const moe_config* cfg, const void* ye, const int32_t* 
   int launches = 0;
   MOE_TRY(stage_combine(*cfg, ye, slot_row, gates, y, (cudaStream_t)stream, &launches, -1,
                         cfg->n_shared != 0));
+  g_last_launches = launches;
+  return MOE_OK;
+}
+
+moe_status moe_ep_combine_p2p(const moe_config* cfg, const int32_t* ids,
+                              const int32_t* slot_row, const float* gates,
+                              const int32_t* offsets, const uint64_t* src_base,
+                              const int32_t* src_row0, const int64_t* src_rows, void* y,
+                              void* ws, moe_stream_t stream) {
+  NvtxRange nvtx_range("moe_ep_combine_p2p");
+  g_last_launches = 0;
+  MOE_TRY(check_cfg(cfg));
+  MOE_TRY(check_ws(cfg, ws));
+  if (ids == nullptr || slot_row == nullptr || gates == nullptr || offsets == nullptr ||
+      src_base == nullptr || src_row0 == nullptr || src_rows == nullptr)
+    return fail(MOE_ERR_INVALID_ARG,
+                "ids, slot_row, gates, offsets, src_base, src_row0 and src_rows are required");
+  MOE_TRY(need(y, "y"));
+  const moe_config& c = *cfg;
+  if (c.dtype != MOE_DT_BF16 || (c.d * el_size(c)) % 16 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "moe_ep_combine_p2p: bf16 rows of a multiple of 16 bytes");
+  const Ws L = layout(c);
+  const moe::RemoteSrc rem{(const unsigned long long*)src_base, src_row0, src_rows, offsets, ids,
+                           c.E, at<int>(ws, L.status)};
+  int launches = 0;
+  MOE_TRY(stage_combine(c, nullptr, slot_row, gates, y, (cudaStream_t)stream, &launches, -1,
+                        c.n_shared != 0, &rem));
   g_last_launches = launches;
   return MOE_OK;
 }

@@ -15,11 +15,11 @@ the experts ``[first(r), first(r+1))`` and a copy of the shared expert.  A forwa
 4. ``moe_permute_ep``: this rank's kept rows in the send layout (expert-major);
 5. dispatch: one grouped point-to-point exchange of the row runs (NCCL on GPUs), or with
    ``transport="p2p"`` the dispatch passes of step 4 write the kept rows straight into the
-   owners' receive buffers over peer memory (CUDA IPC mappings; NVLink on a multi-GPU node)
-   and the return trip is one copy launch;
+   owners' receive buffers over peer memory (CUDA IPC mappings; NVLink on a multi-GPU node);
 6. ``moe_ep_expert_ffn``: the owned experts on the received rows (tcgen05 grouped GEMMs), and
    the shared expert on the rank's own tokens, written straight into y;
-7. combine trip: the same runs back to their source ranks;
+7. combine trip: the same runs back to their source ranks (NCCL), or with ``"p2p"`` nothing:
+   step 8 reads the outputs where the owners wrote them (``moe_ep_combine_p2p``);
 8. ``moe_ep_combine``: the gate-weighted sum onto y.
 
 The result on every rank equals the single-device layer over the concatenation of all ranks'
@@ -117,46 +117,46 @@ def peer_runs(rank: int, plans: Sequence[dict], direction: str) -> list:
 
 
 class PeerTransport:
-    """The rows of an expert-parallel layer moved by ``moe_ep_copy_runs`` into the peers'
-    buffers (their allocations mapped with CUDA IPC) instead of NCCL messages.  The receive
-    buffer (every rank's rows for this rank's experts: at most world * max_tokens * k) and the
-    return buffer (this rank's kept rows) are one allocation made once; its handle is
-    exchanged once.  ``barrier`` (default: a one-element all-reduce on the stream for NCCL
-    groups, else a synchronise and a host barrier) follows each copy launch: after it every
-    rank's rows have landed, and since every rank reaches it only after its earlier reads of
-    both buffers, the next copies cannot overwrite rows still in use."""
+    """The rows of an expert-parallel layer moved through peer memory (the peers' allocations
+    mapped with CUDA IPC) instead of NCCL messages.  One allocation, made once, holds the
+    receive buffer (every rank's rows for this rank's experts: at most world * max_tokens * k
+    rows) and, row for row beside it, the output buffer of this rank's experts; its handle is
+    exchanged once.  A forward takes two barriers (``barrier``; default: a one-element
+    all-reduce on the stream for NCCL groups, else a synchronise and a host barrier):
+
+    1. ``dispatch_fused``: the dispatch passes write each kept row into its owner's receive
+       buffer, then the barrier;
+    2. the owner's experts write their outputs into its output buffer, then the barrier;
+    3. ``combine``: each rank's combine reads its slots' outputs from the owners' output
+       buffers (the return trip and the combine in one pass).
+
+    An owner rewrites its receive buffer only after barrier 2 (its experts have read it) and
+    its output buffer only after the next forward's barrier 1, which every rank reaches after
+    its combine, so no row is overwritten while still in use."""
 
     def __init__(self, layer: "EPMoELayer", group=None, barrier=None):
         import torch.distributed as dist
         self.layer, self.group = layer, group
         dev = layer.xp.device
-        self.rows_recv = max(1, layer.world * layer.max_tokens * layer.k)
-        self.rows_ret = max(1, layer.max_tokens * layer.k)
-        self.buf = torch.empty((self.rows_recv + self.rows_ret, layer.d), dtype=torch.bfloat16,
-                               device=dev)
-        self.recv, self.ret = self.buf[:self.rows_recv], self.buf[self.rows_recv:]
+        self.rows = max(1, layer.world * layer.max_tokens * layer.k)
+        self.buf = torch.empty((2 * self.rows, layer.d), dtype=torch.bfloat16, device=dev)
+        self.recv, self.out = self.buf[:self.rows], self.buf[self.rows:]
         handle, offset = nat.ipc_handle(self.buf)
         gathered = [None] * layer.world
-        dist.all_gather_object(gathered, (handle, offset, self.rows_recv, self.rows_ret),
-                               group=group)
+        dist.all_gather_object(gathered, (handle, offset, self.rows), group=group)
         self.mapped = []
         row_bytes = layer.d * 2
-        recv_base, ret_base, recv_rows, ret_rows = [], [], [], []
-        for r, (h, off, nr, nt) in enumerate(gathered):
+        self._recv_base, self._out_base, self._rows = [], [], []
+        for r, (h, off, n) in enumerate(gathered):
             if r == layer.rank:
                 base = self.buf.data_ptr()
             else:
                 mapped = nat.ipc_open(h)
                 self.mapped.append(mapped)
                 base = mapped + off
-            recv_base.append(base)
-            ret_base.append(base + nr * row_bytes)
-            recv_rows.append(nr)
-            ret_rows.append(nt)
-        i64 = dict(dtype=torch.int64, device=dev)
-        self._recv_base_host, self._recv_rows_host = recv_base, recv_rows
-        self.recv_base, self.recv_rows = torch.tensor(recv_base, **i64), torch.tensor(recv_rows, **i64)
-        self.ret_base, self.ret_rows = torch.tensor(ret_base, **i64), torch.tensor(ret_rows, **i64)
+            self._recv_base.append(base)
+            self._out_base.append(base + n * row_bytes)
+            self._rows.append(n)
         if barrier is None:
             if dist.get_backend(group) == "nccl":
                 flag = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -166,18 +166,27 @@ class PeerTransport:
                     torch.cuda.current_stream(dev).synchronize()
                     dist.barrier(group=group)
         self.barrier = barrier
+        self._tables = None
 
-    def expert_destinations(self, plans: Sequence[dict]):
-        """Per expert e: the receive buffer of e's owner, the row where this rank's kept rows
-        of e start in it, and its size (host lists of E entries)."""
+    def expert_tables(self, plans: Sequence[dict]):
+        """Per expert e (host lists of E entries): the owner's receive and output buffers, the
+        row where this rank's kept rows of e start in them, and their size in rows."""
         L = self.layer
         E, rank = L.E, L.rank
-        base, row0, rows = [self._recv_base_host[rank]] * E, [0] * E, [0] * E
+        recv, out = [self._recv_base[rank]] * E, [self._out_base[rank]] * E
+        row0, rows = [0] * E, [0] * E
         for peer, e, _, n in plans[rank]["sends"]:
             dst = {(p, ex): r for p, ex, r, _ in plans[peer]["recvs"]}
-            base[e], row0[e], rows[e] = (self._recv_base_host[peer], dst[(rank, e)],
-                                         self._recv_rows_host[peer])
-        return base, row0, rows
+            recv[e], out[e] = self._recv_base[peer], self._out_base[peer]
+            row0[e], rows[e] = dst[(rank, e)], self._rows[peer]
+        return recv, out, row0, rows
+
+    def _device_tables(self, plans: Sequence[dict]):
+        dev = self.buf.device
+        recv, out, row0, rows = self.expert_tables(plans)
+        i64 = dict(dtype=torch.int64)
+        return (torch.tensor(recv, **i64).to(dev), torch.tensor(out, **i64).to(dev),
+                torch.tensor(row0, dtype=torch.int32).to(dev), torch.tensor(rows, **i64).to(dev))
 
     def dispatch_fused(self, x: torch.Tensor, plans: Sequence[dict]) -> torch.Tensor:
         """The dispatch passes with the kept rows written straight into their owners'
@@ -185,34 +194,31 @@ class PeerTransport:
         rows."""
         L = self.layer
         N = L.N
+        self._tables = self._device_tables(plans)
         if N > 0:
-            dev = x.device
-            base, row0, rows = self.expert_destinations(plans)
+            recv, _, row0, rows = self._tables
             nat.moe_permute_ep_p2p(
                 L.config(N), ids=L.ids[:N], cap=L.cap, x=x, offsets=L.offsets,
-                slot_row=L.slot_row[:N],
-                dst_base=torch.tensor(base, dtype=torch.int64).to(dev, non_blocking=True),
-                dst_row0=torch.tensor(row0, dtype=torch.int32).to(dev, non_blocking=True),
-                dst_rows=torch.tensor(rows, dtype=torch.int64).to(dev, non_blocking=True),
+                slot_row=L.slot_row[:N], dst_base=recv, dst_row0=row0, dst_rows=rows,
                 counts=L.counts, drop_mask=L.drop_mask[:N], ws=L.ws)
         self.barrier()
         return self.recv[:max(1, plans[L.rank]["rows_owned"])]
 
-    def dispatch(self, xp: torch.Tensor, plans: Sequence[dict]) -> torch.Tensor:
-        """The rows of a send buffer (moe_permute_ep's layout) copied into the owners' receive
-        buffers (moe_ep_copy_runs), then the barrier."""
-        L = self.layer
-        nat.moe_ep_copy_runs(xp, dst_base=self.recv_base, dst_rows=self.recv_rows,
-                             runs=peer_runs(L.rank, plans, "dispatch"), ws=L.ws)
-        self.barrier()
-        return self.recv[:max(1, plans[L.rank]["rows_owned"])]
+    def outputs(self, plans: Sequence[dict]) -> torch.Tensor:
+        """Where this rank's experts write their outputs (row i: the output of received row i)."""
+        return self.out[:max(1, plans[self.layer.rank]["rows_owned"])]
 
-    def give_back(self, ye: torch.Tensor, plans: Sequence[dict]) -> torch.Tensor:
+    def combine(self, y: torch.Tensor) -> torch.Tensor:
+        """The gate-weighted sum onto y, each slot's output read from its owner's output buffer
+        (moe_ep_combine_p2p); follows the barrier after the experts."""
         L = self.layer
-        nat.moe_ep_copy_runs(ye, dst_base=self.ret_base, dst_rows=self.ret_rows,
-                             runs=peer_runs(L.rank, plans, "return"), ws=L.ws)
-        self.barrier()
-        return self.ret[:max(1, plans[L.rank]["rows_kept"])]
+        N = L.N
+        if N > 0:
+            _, out, row0, rows = self._tables
+            nat.moe_ep_combine_p2p(L.config(N), ids=L.ids[:N], slot_row=L.slot_row[:N],
+                                   gates=L.gates[:N], offsets=L.offsets, src_base=out,
+                                   src_row0=row0, src_rows=rows, y=y, ws=L.ws)
+        return y
 
     def close(self):
         torch.cuda.synchronize(self.buf.device)
@@ -335,9 +341,12 @@ class EPMoELayer:
         return torch.empty((max(1, self.plan["rows_kept"]), self.d), dtype=torch.bfloat16,
                            device=self.xp.device)
 
-    def run_experts(self, xr: torch.Tensor, x: torch.Tensor, y: torch.Tensor) -> torch.Tensor:
-        """The owned experts on the received rows; the shared expert's rows go into y."""
-        ye = torch.empty_like(xr)
+    def run_experts(self, xr: torch.Tensor, x: torch.Tensor, y: torch.Tensor,
+                    ye: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """The owned experts on the received rows (outputs into ye, a new buffer by default);
+        the shared expert's rows go into y."""
+        if ye is None:
+            ye = torch.empty_like(xr)
         nat.moe_ep_expert_ffn(self.config(self.max_tokens), self.world, self.rank, self.N,
                               self.plan["rows_owned"], xr=xr, owned_offsets=self.owned_offsets,
                               x=x if self.N else None, W_gu=self.W_gu, W_down=self.W_down, ye=ye,
@@ -366,10 +375,13 @@ class EPMoELayer:
             dist.all_gather_into_tensor(gathered, demand.cpu(), group=self.group)
         plan = self.set_plan(gathered)
         if self.transport is not None:
-            # the dispatch passes write the kept rows straight into the owners' buffers
-            xr = self.transport.dispatch_fused(x, self.plans)
-            ye = self.run_experts(xr, x, y)
-            return self.combine(self.transport.give_back(ye, self.plans), y)
+            # the dispatch passes write the kept rows straight into the owners' buffers; the
+            # combine reads the outputs back from them
+            t = self.transport
+            xr = t.dispatch_fused(x, self.plans)
+            self.run_experts(xr, x, y, ye=t.outputs(self.plans))
+            t.barrier()
+            return t.combine(y)
         xp = self.permute(x)
         xr = self.new_recv_buffer()
         exchange_rows(xp, xr, plan["sends"], plan["recvs"], self.rank, self.group)

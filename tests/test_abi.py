@@ -257,3 +257,13 @@ def test_expert_parallel_entry_points_validate_on_host(nat):
                                  fake, fake, fake, None) == nat.MOE_ERR_UNSUPPORTED
     assert lib.moe_ep_combine(ctypes.byref(c), fake, None, fake, fake, None) == nat.MOE_ERR_INVALID_ARG
     assert lib.moe_ep_combine(ctypes.byref(f32), fake, fake, fake, fake, None) == nat.MOE_ERR_UNSUPPORTED
+    # the peer-memory dispatch and combine: the tables are required, bf16 only
+    assert lib.moe_permute_ep_p2p(ctypes.byref(c), fake, fake, fake, fake, fake, None, fake, fake,
+                                  None, None, fake, None) == nat.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute_ep_p2p(ctypes.byref(f32), fake, fake, fake, fake, fake, fake, fake,
+                                  fake, None, None, fake, None) == nat.MOE_ERR_UNSUPPORTED
+    p2p = lambda cfg, src_base, ws: lib.moe_ep_combine_p2p(
+        ctypes.byref(cfg), fake, fake, fake, fake, src_base, fake, fake, fake, ws, None)
+    assert p2p(c, None, fake) == nat.MOE_ERR_INVALID_ARG
+    assert p2p(c, fake, None) == nat.MOE_ERR_INVALID_ARG
+    assert p2p(f32, fake, fake) == nat.MOE_ERR_UNSUPPORTED

@@ -277,8 +277,9 @@ def _p2p_worker(rank, world, port, case, out_dir):
 def test_peer_transport_between_processes_equals_the_single_device_layer(case, tmp_path,
                                                                         monkeypatch):
     """Ranks as separate processes sharing the GPU: each maps the others' buffers with CUDA
-    IPC and writes its rows into them with moe_ep_copy_runs (no message passing for the rows;
-    host barriers between the phases, no kernel waiting on another).  Every rank's output, on
+    IPC, its dispatch passes write its rows into the owners' receive buffers and its combine
+    reads the outputs from the owners' output buffers (no message passing for the rows; host
+    barriers between the phases, no kernel waiting on another).  Every rank's output, on
     two consecutive calls, equals bit for bit the fused layer over the concatenated batch given
     the ranks' routing, and the drop masks equal the oracle's for it."""
     import torch.multiprocessing as tmp
@@ -384,3 +385,85 @@ def test_dispatch_passes_writing_into_the_owners_buffers(world, case):
         dst_row0=torch.tensor(row0, dtype=torch.int32, device="cuda"),
         dst_rows=torch.tensor(rows, dtype=torch.int64, device="cuda"), ws=L.ws)
     assert nat.moe_check_status(L.ws) == nat.MOE_ERR_INVALID_INPUT
+
+
+@pytest.mark.parametrize("world,case,sizes", [
+    (2, CASES[0], None), (3, CASES[2], None), (4, CASES[1], None), (2, CASES[3], None),
+    # 10000+ tokens a rank, 256-byte rows: the warp-per-token kernel
+    (2, ("switch-cf1", 21000, 128, 12, 128, 2, 1.25), (10000, 11000)),
+])
+def test_combine_reading_the_owners_outputs(world, case, sizes):
+    """moe_ep_combine_p2p: each rank's combine reads its slots' expert outputs where their
+    owners wrote them (per-expert sources from every rank's plan; local buffers here, one per
+    emulated rank), with no return trip.  y equals, bit for bit, the return exchange followed
+    by moe_ep_combine; a source one row too small drops that slot alone and is reported."""
+    from mixture_experts_layer_50_b200.ep import loopback_exchange
+    name, N, d, E, F, k, cf = case
+    shape = W.PRESETS[name].replace(N=N, d=d, E=E, F=F, k=k)
+    t = W.make_inputs(shape, device="cuda")
+    if sizes is None:
+        sizes = _split(N, world, seed=world * 13 + E)
+    sizes = np.asarray(sizes)
+    starts = np.r_[0, np.cumsum(sizes)]
+    xs = [t["x"][starts[r]:starts[r + 1]] for r in range(world)]
+    mod = t.get("modality")
+    mods = [None if mod is None else mod[starts[r]:starts[r + 1]] for r in range(world)]
+    layers = _layers(shape, t, world, int(sizes.max()), cf)
+    dem = [L.route(x, m) for L, x, m in zip(layers, xs, mods)]
+    gathered = torch.stack(dem).cpu()
+    plans = [L.set_plan(gathered) for L in layers]
+    sends = [L.permute(x) for L, x in zip(layers, xs)]
+    recv = [L.new_recv_buffer() for L in layers]
+    loopback_exchange(sends, recv, [p["sends"] for p in plans], [p["recvs"] for p in plans])
+    shared = [torch.empty_like(x) for x in xs]
+    outs = [L.run_experts(r, x, y) for L, r, x, y in zip(layers, recv, xs, shared)]
+    # the reference: the return exchange and the local combine
+    back = [L.new_return_buffer() for L in layers]
+    loopback_exchange(outs, back, [p["recvs"] for p in plans], [p["sends"] for p in plans])
+    want = [L.combine(b, s.clone()) for L, b, s in zip(layers, back, shared)]
+    addr = [o.data_ptr() for o in outs]
+    nrows = [o.shape[0] for o in outs]
+
+    def tables(r):
+        base, row0, rows = [addr[r]] * E, [0] * E, [0] * E
+        for peer, e, _, n in plans[r]["sends"]:
+            dst = {(p_, ex): rr for p_, ex, rr, _ in plans[peer]["recvs"]}
+            base[e], row0[e], rows[e] = addr[peer], dst[(r, e)], nrows[peer]
+        return base, row0, rows
+
+    def combine_p2p(L, y, base, row0, rows):
+        nat.moe_ep_combine_p2p(
+            L.config(L.N), ids=L.ids[:L.N], slot_row=L.slot_row[:L.N], gates=L.gates[:L.N],
+            offsets=L.offsets, src_base=torch.tensor(base, dtype=torch.int64, device="cuda"),
+            src_row0=torch.tensor(row0, dtype=torch.int32, device="cuda"),
+            src_rows=torch.tensor(rows, dtype=torch.int64, device="cuda"), y=y, ws=L.ws)
+
+    for r, L in enumerate(layers):
+        if L.N == 0:
+            continue
+        y = shared[r].clone()
+        combine_p2p(L, y, *tables(r))
+        check_status(L.ws)
+        assert torch.equal(y, want[r]), r
+    # a source one row too small: the slot of that last row contributes nothing
+    r = next(i for i, L in enumerate(layers) if plans[i]["sends"] and L.N > 0)
+    L = layers[r]
+    peer, e, _, n = plans[r]["sends"][-1]
+    base, row0, rows = tables(r)
+    rows[e] = row0[e] + n - 1
+    last = int(L.offsets[e].item()) + n - 1               # the send-layout row of that slot
+    slot = (L.slot_row[:L.N] == last).nonzero()
+    assert slot.shape[0] == 1
+    tok, j = int(slot[0, 0]), int(slot[0, 1])
+    y = shared[r].clone()
+    combine_p2p(L, y, base, row0, rows)
+    assert nat.moe_check_status(L.ws) == nat.MOE_ERR_INVALID_INPUT
+    others = torch.ones(L.N, dtype=torch.bool, device="cuda")
+    others[tok] = False
+    assert torch.equal(y[others], want[r][others])
+    # that token: the combine of its other slots alone
+    sr = L.slot_row[:L.N].clone()
+    sr[tok, j] = -1
+    y1 = shared[r].clone()
+    nat.moe_ep_combine(L.config(L.N), ye=back[r], slot_row=sr, gates=L.gates[:L.N], y=y1)
+    assert torch.equal(y[tok], y1[tok])

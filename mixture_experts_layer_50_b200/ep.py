@@ -116,6 +116,24 @@ def peer_runs(rank: int, plans: Sequence[dict], direction: str) -> list:
     return out
 
 
+def expert_tables(rank: int, plans: Sequence[dict], E: int, recv_base: Sequence[int],
+                  out_base: Sequence[int], rows: Sequence[int]):
+    """Where rank ``rank``'s kept rows of each expert go and come back from: per expert e, the
+    receive and output buffer of e's owner (``recv_base``/``out_base`` indexed by rank), the
+    row of the owner's buffers where this rank's rows of e start (the owner's receive run for
+    (rank, e)), and the owner's buffer size (``rows``).  An expert this rank keeps no row of
+    gets this rank's own buffers at row 0 (never read).  Host lists of E entries."""
+    recv, out = [recv_base[rank]] * E, [out_base[rank]] * E
+    row0, size = [0] * E, [0] * E
+    for peer, e, _, n in plans[rank]["sends"]:
+        dst = {(p, ex): r for p, ex, r, _ in plans[peer]["recvs"]}
+        if (rank, e) not in dst:
+            raise RuntimeError(f"rank {rank} -> {peer} expert {e}: no matching receive run")
+        recv[e], out[e] = recv_base[peer], out_base[peer]
+        row0[e], size[e] = dst[(rank, e)], rows[peer]
+    return recv, out, row0, size
+
+
 class PeerTransport:
     """The rows of an expert-parallel layer moved through peer memory (the peers' allocations
     mapped with CUDA IPC) instead of NCCL messages.  One allocation, made once, holds the
@@ -172,14 +190,7 @@ class PeerTransport:
         """Per expert e (host lists of E entries): the owner's receive and output buffers, the
         row where this rank's kept rows of e start in them, and their size in rows."""
         L = self.layer
-        E, rank = L.E, L.rank
-        recv, out = [self._recv_base[rank]] * E, [self._out_base[rank]] * E
-        row0, rows = [0] * E, [0] * E
-        for peer, e, _, n in plans[rank]["sends"]:
-            dst = {(p, ex): r for p, ex, r, _ in plans[peer]["recvs"]}
-            recv[e], out[e] = self._recv_base[peer], self._out_base[peer]
-            row0[e], rows[e] = dst[(rank, e)], self._rows[peer]
-        return recv, out, row0, rows
+        return expert_tables(L.rank, plans, L.E, self._recv_base, self._out_base, self._rows)
 
     def _device_tables(self, plans: Sequence[dict]):
         dev = self.buf.device
@@ -400,4 +411,4 @@ class EPMoELayer:
 
 
 __all__ = ["EPMoELayer", "PeerTransport", "shard_experts", "exchange_rows", "loopback_exchange",
-           "all_plans", "peer_runs"]
+           "all_plans", "peer_runs", "expert_tables"]

@@ -171,3 +171,40 @@ def test_peer_runs_move_the_rows_the_message_exchange_moves(seed, world, N, E, k
         assert torch.equal(g, w)
     kept = sum(p["rows_kept"] for p in plans)
     assert sum(n for r in range(world) for *_, n in peer_runs(r, plans, "dispatch")) == kept
+
+
+@pytest.mark.parametrize("seed,world,N,E,k,cf", [
+    (0, 2, 300, 8, 2, 1), (1, 3, 500, 7, 2, 1.25), (2, 4, 257, 16, 4, None), (5, 8, 64, 64, 8, 2)])
+def test_expert_tables_address_the_rows_the_message_exchange_moves(seed, world, N, E, k, cf):
+    """The per-expert tables of the fused peer-memory dispatch and combine (kept row i of
+    expert e goes to, and its output comes back from, row row0[e] + i of the owner's buffers):
+    writing every rank's tagged send rows through them leaves each owner's receive buffer as
+    the message exchange does, and reading the owners' outputs through them gives each rank
+    what the return exchange gives."""
+    import torch
+    from mixture_experts_layer_50_b200.ep import all_plans, expert_tables, loopback_exchange
+    ids, C, sizes, starts, demand = _case(seed, world, N, E, k, cf)
+    plans = all_plans(world, E, C, demand)
+    rows = lambda n: max(1, n)
+    sends = [torch.arange(rows(p["rows_kept"]) * 2, dtype=torch.float64).reshape(-1, 2) + 1000 * r
+             for r, p in enumerate(plans)]
+    want = [torch.full((rows(p["rows_owned"]), 2), -1.0, dtype=torch.float64) for p in plans]
+    loopback_exchange(sends, want, [p["sends"] for p in plans], [p["recvs"] for p in plans])
+    outs = [w + 0.5 for w in want]
+    want_back = [torch.full_like(s, -1.0) for s in sends]
+    loopback_exchange(outs, want_back, [p["recvs"] for p in plans], [p["sends"] for p in plans])
+    # the buffers' "addresses" are rank numbers here
+    ranks = list(range(world))
+    sizes_owned = [w.shape[0] for w in want]
+    got = [torch.full_like(w, -1.0) for w in want]
+    for r in range(world):
+        recv, out, row0, size = expert_tables(r, plans, E, ranks, ranks, sizes_owned)
+        back = torch.full_like(sends[r], -1.0)
+        for peer, e, row, n in plans[r]["sends"]:
+            assert recv[e] == out[e] == peer and size[e] == sizes_owned[peer]
+            assert 0 <= row0[e] and row0[e] + n <= size[e]
+            got[peer][row0[e]:row0[e] + n] = sends[r][row:row + n]
+            back[row:row + n] = outs[peer][row0[e]:row0[e] + n]
+        assert torch.equal(back, want_back[r])
+    for g, w in zip(got, want):
+        assert torch.equal(g, w)

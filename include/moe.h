@@ -65,7 +65,7 @@ typedef struct CUstream_st* moe_stream_t; /* identical to cudaStream_t */
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,   /* a host-checked argument is wrong; nothing was enqueued */
-  MOE_ERR_UNSUPPORTED = 2,   /* valid request outside what this build implements
+  MOE_ERR_UNSUPPORTED = 2,   /* valid request outside what the library implements
                                 (alignment, d or F not a multiple of 8, k > 32, ...) */
   MOE_ERR_CUDA = 3,          /* a CUDA call or launch failed; see moe_last_error() */
   MOE_ERR_INVALID_INPUT = 4, /* device-detected: expert id out of range or repeated in a

@@ -224,6 +224,8 @@ class PeerTransport:
         (moe_ep_combine_p2p); follows the barrier after the experts."""
         L = self.layer
         N = L.N
+        if self._tables is None:
+            raise RuntimeError("PeerTransport.combine before dispatch_fused: no expert tables")
         if N > 0:
             _, out, row0, rows = self._tables
             nat.moe_ep_combine_p2p(L.config(N), ids=L.ids[:N], slot_row=L.slot_row[:N],

@@ -151,9 +151,11 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def test_forward_over_a_one_rank_nccl_group():
-    """EPMoELayer.forward itself (NCCL all-gather of the demands, the row exchange) on a
-    one-rank NCCL group equals moe_forward bit for bit."""
+@pytest.mark.parametrize("transport", ["nccl", "p2p"])
+def test_forward_over_a_one_rank_nccl_group(transport):
+    """EPMoELayer.forward itself (NCCL all-gather of the demands, then the row exchange, or
+    with the peer-memory transport the fused dispatch and combine around its stream-ordered
+    NCCL barriers) on a one-rank NCCL group equals moe_forward bit for bit, twice in a row."""
     import torch.distributed as dist
     shape = W.PRESETS["v41flash-n64"].replace(N=300, d=256, E=16, F=128, k=4)
     t = W.make_inputs(shape, device="cuda")
@@ -163,9 +165,18 @@ def test_forward_over_a_one_rank_nccl_group():
                             timeout=datetime.timedelta(seconds=60),
                             device_id=torch.device("cuda", 0))
     try:
-        (L,) = _layers(shape, t, 1, shape.N, 1.25)
+        (L,) = [EPMoELayer.from_full_weights(
+            W_g=t["W_g"], W_gu=t["W_gu"], W_down=t["W_down"], k=shape.k, E=shape.E, world=1,
+            rank=0, n_shared=shape.n_shared, score_fn=shape.score_fn, renorm=shape.renorm,
+            act=shape.act, clamp=shape.clamp, bias=t.get("bias"),
+            logit_offset=t.get("logit_offset"), capacity_factor=1.25, max_tokens=shape.N,
+            transport=transport)]
+        y_first = L.forward(t["x"], modality=t["modality"]).clone()
         y_ep = L.forward(t["x"], modality=t["modality"])
+        torch.cuda.synchronize()
         assert L.check_status() == 0
+        assert torch.equal(y_first, y_ep)
+        L.close()
     finally:
         dist.destroy_process_group()
     C = O.capacity(shape.N, shape.k, shape.E, 1.25)

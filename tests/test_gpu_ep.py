@@ -400,8 +400,12 @@ def test_dispatch_passes_writing_into_the_owners_buffers(world, case):
 
 @pytest.mark.parametrize("world,case,sizes", [
     (2, CASES[0], None), (3, CASES[2], None), (4, CASES[1], None), (2, CASES[3], None),
-    # 10000+ tokens a rank, 256-byte rows: the warp-per-token kernel
+    # k = 8 and k = 12: the block-per-token kernel's 8-slot and any-k forms
+    (2, ("dsv3-n64", 400, 256, 32, 128, 8, None), None),
+    (3, ("dsv3-n64", 300, 256, 48, 128, 12, 1.25), None),
+    # 10000+ tokens a rank, 256-byte rows: the warp-per-token kernel (2 and 8 slots)
     (2, ("switch-cf1", 21000, 128, 12, 128, 2, 1.25), (10000, 11000)),
+    (2, ("switch-cf1", 21000, 128, 16, 128, 8, 1.25), (11000, 10000)),
 ])
 def test_combine_reading_the_owners_outputs(world, case, sizes):
     """moe_ep_combine_p2p: each rank's combine reads its slots' expert outputs where their

@@ -330,8 +330,14 @@ def test_peer_transport_between_processes_equals_the_single_device_layer(case, t
         assert torch.equal(y_ep, y), call
 
 
-@pytest.mark.parametrize("world,case", [(2, CASES[0]), (3, CASES[2]), (4, CASES[1])])
-def test_dispatch_passes_writing_into_the_owners_buffers(world, case):
+@pytest.mark.parametrize("world,case,sizes", [
+    (2, CASES[0], None), (3, CASES[2], None), (4, CASES[1], None),
+    # ranks of at most 64 tokens: the one-launch dispatch
+    (2, ("mixtral-n16", 64, 256, 8, 384, 2, None), (40, 24)),
+    # 10000+ tokens a rank: the warp-per-token scatter
+    (2, ("switch-cf1", 21000, 128, 12, 128, 2, 1.25), (10000, 11000)),
+])
+def test_dispatch_passes_writing_into_the_owners_buffers(world, case, sizes):
     """moe_permute_ep_p2p: the dispatch passes write each kept row straight into its owner's
     receive buffer (per-expert destinations from every rank's plan; local buffers here, one per
     emulated rank).  Receive buffers, slot rows, counts and drop masks equal moe_permute_ep
@@ -340,7 +346,9 @@ def test_dispatch_passes_writing_into_the_owners_buffers(world, case):
     name, N, d, E, F, k, cf = case
     shape = W.PRESETS[name].replace(N=N, d=d, E=E, F=F, k=k)
     t = W.make_inputs(shape, device="cuda")
-    sizes = _split(N, world, seed=world * 7 + E)
+    if sizes is None:
+        sizes = _split(N, world, seed=world * 7 + E)
+    sizes = np.asarray(sizes)
     starts = np.r_[0, np.cumsum(sizes)]
     xs = [t["x"][starts[r]:starts[r + 1]] for r in range(world)]
     mod = t.get("modality")
